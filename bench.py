@@ -1,0 +1,365 @@
+"""Benchmark of the MoE layer forward pass on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+                    [--workload 20b_decode|20b_prefill|131k_skewed|120b_sweep|tiny] [--T n]
+
+One step = one moe_forward call (router, top-k, histogram/scan/permutation, gate/up + SwiGLU,
+down + weighted combine) over one batch of seeded synthetic tokens of the named workload
+(default: the gpt-oss-20b layer in decode, T = 16, H = I = 2880, 32 experts, top-4).  Inputs
+are resident in HBM before the timed region; the touched expert weights (~1.4 GB) are larger
+than the 126 MB L2, so every step streams them from HBM.
+
+Prints one JSON line.  With N > 1 (torchrun, one process per GPU) every rank runs its own
+replica on its own tokens (the layer is token-wise, so there is no data-path collective);
+`value` is the tokens all ranks processed divided by the slowest rank's time.
+
+--impl reference times the fp64 CPU oracle (the deliberately slow reference) on the host cores
+on a bounded token sample of the same workload; only rank 0 works.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import moe_inputs as mi  # noqa: E402
+
+METRIC = "MoE layer tokens/s and µs/layer at 1 GPU; % of HBM or bf16 tensor roofline"
+UNIT = "tokens/s"
+PEAKS_FILE = os.path.join(ROOT, "MEASURED_PEAKS.json")
+TRAFFIC_FILE = os.path.join(ROOT, "profiles", "traffic.json")
+FALLBACK_HBM_GBS, FALLBACK_BF16_TFLOPS = 6650.0, 1590.0
+
+
+# ----------------------------------------------------------------------------------------
+# host-side helpers (CPU-testable)
+# ----------------------------------------------------------------------------------------
+def dist_env() -> tuple[int, int, int]:
+    return (int(os.environ.get("RANK", "0")), int(os.environ.get("WORLD_SIZE", "1")),
+            int(os.environ.get("LOCAL_RANK", "0")))
+
+
+def reduce_max(value: float, world: int) -> float:
+    """Max of a float over all ranks (identity for one rank)."""
+    if world == 1:
+        return value
+    import torch.distributed as dist
+    dev = "cuda" if dist.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([value], dtype=torch.float64, device=dev)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def aggregate(tokens_per_rank: int, world: int, max_seconds: float, steps: int) -> dict:
+    """Whole-job throughput: all ranks' tokens over the slowest rank's timed seconds."""
+    total = tokens_per_rank * world * steps
+    return dict(value=total / max_seconds, ms_per_step=1e3 * max_seconds / steps)
+
+
+def measured_peaks() -> tuple[float, float, float, str]:
+    try:
+        with open(PEAKS_FILE) as f:
+            p = json.load(f)
+        return float(p["hbm_gbs"]), float(p["bf16_tflops"]), float(p["bf16_tflops_sustained"]), "measured"
+    except (OSError, KeyError, ValueError):
+        return FALLBACK_HBM_GBS, FALLBACK_BF16_TFLOPS, 1400.0, "fallback"
+
+
+def source_digest(paths) -> str:
+    h = hashlib.sha256()
+    for p in paths:
+        with open(os.path.join(ROOT, p), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def ncu_traffic(kernel_key: str, workload: str) -> float | None:
+    """DRAM bytes per launch from the committed ncu summary, if the kernel is unchanged."""
+    try:
+        with open(TRAFFIC_FILE) as f:
+            t = json.load(f)[kernel_key]
+    except (OSError, KeyError, ValueError):
+        return None
+    if t.get("workload") != workload or t.get("sources_sha") != source_digest(t["sources"]):
+        return None
+    return float(t["dram_bytes_per_launch"])
+
+
+def parse_clocks(csv_text: str) -> dict:
+    """Median SM clock under load, max clock and the throttle reasons seen, from nvidia-smi CSV."""
+    rows = [r.split(",") for r in csv_text.strip().splitlines()[1:] if r.strip()]
+    sm, mx, reasons = [], [], set()
+    names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+    for r in rows:
+        r = [c.strip() for c in r]
+        try:
+            s, m, pw = float(r[1].split()[0]), float(r[2].split()[0]), float(r[3].split()[0])
+        except (ValueError, IndexError):
+            continue
+        if pw > 200.0:  # under load
+            sm.append(s)
+        mx.append(m)
+        for n, v in zip(names, r[5:9]):
+            if v.lower() == "active":
+                reasons.add(n)
+    return dict(sm_mhz=statistics.median(sm) if sm else None, sm_max_mhz=max(mx) if mx else None,
+                reasons=sorted(reasons), samples=len(rows), samples_under_load=len(sm))
+
+
+class ClockSampler:
+    QUERY = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index: int):
+        self.index, self.proc, self.path = index, None, None
+
+    def __enter__(self):
+        self.path = f"/tmp/moe_bench_clocks_{os.getpid()}.csv"
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.index), f"--query-gpu={self.QUERY}",
+                 "--format=csv", "-lms", "100"], stdout=open(self.path, "w"),
+                stderr=subprocess.DEVNULL)
+            time.sleep(0.3)
+        except OSError:
+            self.proc = None
+        return self
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+
+    def result(self) -> dict:
+        if self.proc is None:
+            return dict(sm_mhz=None, sm_max_mhz=None, reasons=["nvidia-smi unavailable"])
+        with open(self.path) as f:
+            return parse_clocks(f.read())
+
+
+# ----------------------------------------------------------------------------------------
+# algorithmic work (what the method must touch)
+# ----------------------------------------------------------------------------------------
+def algorithmic(T: int, H: int, E: int, k: int, I: int, counts) -> dict:
+    touched = int(sum(1 for c in counts if c > 0))
+    R = T * k
+    w_gate_up = touched * H * 2 * I * 2
+    w_down = touched * I * H * 2
+    gate_up_bytes = w_gate_up + T * H * 2 + R * I * 2          # weights + x read + h write
+    down_bytes = w_down + R * I * 2 + T * H * 4                 # weights + h read + out write
+    layer_bytes = w_gate_up + w_down + H * E * 2 + T * H * 2 + T * H * 4
+    flops = 2 * R * (H * 2 * I + I * H) + 2 * T * H * E
+    return dict(touched=touched, gate_up_bytes=gate_up_bytes, down_bytes=down_bytes,
+                layer_bytes=layer_bytes, flops=flops)
+
+
+# ----------------------------------------------------------------------------------------
+# the CPU oracle as a baseline (rank 0, N = 1 only; and the reference arm)
+# ----------------------------------------------------------------------------------------
+def blas_threads() -> int:
+    try:
+        from threadpoolctl import threadpool_info
+        n = [i.get("num_threads", 1) for i in threadpool_info() if i.get("user_api") == "blas"]
+        return max(n) if n else 1
+    except Exception:
+        return 1
+
+
+def oracle_time(h: dict, k: int, n_tokens: int, reps: int) -> float:
+    import oracle
+    x = h["x"][:n_tokens]
+    t0 = time.perf_counter()
+    for _ in range(reps):
+        oracle.moe_forward_ref(x, h["W_router"], h["b_router"], h["W_gate_up"], h["W_down"], k)
+    return time.perf_counter() - t0
+
+
+def cpu_baseline(h: dict, w: mi.Workload, T: int, budget_s: float = 20.0) -> dict:
+    t1 = oracle_time(h, w.k, T, 1)       # one full call, also the warm-up
+    reps = max(1, int(budget_s / max(t1, 1e-3)))
+    secs = oracle_time(h, w.k, T, reps)
+    return dict(value=reps * T / secs, unit=UNIT, cores=blas_threads(), kind="oracle",
+                sample=f"{reps} full oracle calls of the {w.name} layer at T={T} "
+                       f"(numpy float64, {os.cpu_count()} host cores)")
+
+
+def run_reference(args, w: mi.Workload, T: int) -> None:
+    rank, world, _ = dist_env()
+    if rank != 0:
+        return
+    h = mi.host_inputs(mi.make_inputs(T, w.H, w.E, w.k, w.I, w.seed, "cpu", zipf=w.zipf))
+    budget = 150.0 / (args.steps + args.warmup)          # whole run within a few minutes
+    t1 = oracle_time(h, w.k, 1, 1)
+    n = max(1, min(T, int(budget / max(t1, 1e-3))))
+    for _ in range(args.warmup):
+        oracle_time(h, w.k, n, 1)
+    secs = oracle_time(h, w.k, n, args.steps)
+    value = args.steps * n / secs
+    line = dict(metric=METRIC, value=value, unit=UNIT, n_gpus=args.gpus, steps=args.steps,
+                warmup=args.warmup, ms_per_step=1e3 * secs / args.steps, higher_is_better=True,
+                scaling="weak", vs_baseline=None, dtype="f64", data="synthetic",
+                impl="reference",
+                config=dict(workload=w.name, T=T, H=w.H, E=w.E, k=w.k, I=w.I, sample_tokens=n),
+                cpu_baseline=dict(value=value, unit=UNIT, cores=blas_threads(), kind="oracle",
+                                  sample=f"first {n} of {T} tokens per step, full layer"),
+                e2e=dict(value=value, unit=UNIT, h2d_bytes_per_step=0, d2h_bytes_per_step=0))
+    print(json.dumps(line), flush=True)
+
+
+# ----------------------------------------------------------------------------------------
+# our arm
+# ----------------------------------------------------------------------------------------
+def run_ours(args, w: mi.Workload, T: int) -> None:
+    rank, world, local = dist_env()
+    if not torch.cuda.is_available():
+        raise SystemExit("bench.py needs a CUDA device (the library has no CPU path)")
+    torch.cuda.set_device(local)
+    if world > 1:
+        import torch.distributed as dist
+        from datetime import timedelta
+        dist.init_process_group("nccl", timeout=timedelta(seconds=120))
+    import mixture_experts_layer_48_b200 as moe
+
+    seed = w.seed + 7919 * rank          # every rank its own tokens (weights identical)
+    d = mi.make_inputs(T, w.H, w.E, w.k, w.I, w.seed, "cuda", zipf=w.zipf)
+    if rank:
+        d["x"] = mi.draw_x(T, w.H, seed, "cuda")
+    layer = moe.Moe(w.E, w.H, w.I, w.k)
+    counts = torch.diff(layer.route(d["x"], d["W_router"], d["b_router"])["expert_offsets"]).cpu().tolist()
+    alg = algorithmic(T, w.H, w.E, w.k, w.I, counts)
+    out = torch.empty((T, w.H), dtype=torch.float32, device="cuda")
+    ws = torch.empty(layer.workspace_bytes(T), dtype=torch.uint8, device="cuda")
+    args_fwd = (d["x"], d["W_router"], d["b_router"], d["W_gate_up"], d["W_down"])
+    stream = torch.cuda.current_stream()
+
+    def step():
+        layer.forward(*args_fwd, out=out, workspace=ws)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    assert layer.sync_status() == moe.MOE_OK
+
+    # ---- timed region: device events on the launching stream, per-kernel events inside ----
+    layer.profile_begin(args.steps)
+    n_launch0 = layer.launch_count()
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with ClockSampler(torch.cuda.current_device()) as clk:
+        if world > 1:
+            torch.distributed.barrier()
+        torch.cuda.synchronize()
+        ev0.record(stream)
+        for _ in range(args.steps):
+            step()
+        ev1.record(stream)
+        torch.cuda.synchronize()
+        if world > 1:
+            torch.distributed.barrier()
+    gpu_launches = layer.launch_count() - n_launch0
+    prof = layer.profile_end()
+    secs = reduce_max(ev0.elapsed_time(ev1) / 1e3, world)
+    assert layer.sync_status() == moe.MOE_OK
+    agg = aggregate(T, world, secs, args.steps)
+
+    # ---- e2e: the same call with host buffers, copies inside the timed region ----
+    x_host = d["x"].cpu().pin_memory()
+    out_host = torch.empty((T, w.H), dtype=torch.float32).pin_memory()
+    x_dev = torch.empty_like(d["x"])
+
+    def e2e_step():
+        x_dev.copy_(x_host, non_blocking=True)
+        layer.forward(x_dev, *args_fwd[1:], out=out, workspace=ws)
+        out_host.copy_(out, non_blocking=True)
+
+    for _ in range(max(1, args.warmup)):
+        e2e_step()
+    torch.cuda.synchronize()
+    if world > 1:
+        torch.distributed.barrier()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(args.steps):
+        e2e_step()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    e2e_secs = reduce_max(e0.elapsed_time(e1) / 1e3, world)
+
+    # ---- roofline of the dominant kernel (gate/up + SwiGLU streams 2/3 of the bytes) ----
+    hbm, bf16, bf16_sus, peak_src = measured_peaks()
+    gu_ms, gu_n = prof["gate_up_swiglu"]
+    dn_ms, dn_n = prof["down_combine"]
+    gu_avg_s = gu_ms / 1e3 / max(gu_n, 1)
+    dn_avg_s = dn_ms / 1e3 / max(dn_n, 1)
+    achieved = alg["gate_up_bytes"] / gu_avg_s / 1e9
+    traffic = ncu_traffic("stream_gate_up_kernel", w.name)
+    layer_roof_s = max(alg["layer_bytes"] / (hbm * 1e9), alg["flops"] / (bf16 * 1e12))
+    kernels_ms = {k_: round(v[0] / max(v[1], 1), 4) for k_, v in prof.items() if v[1]}
+
+    line = dict(
+        metric=METRIC, value=agg["value"], unit=UNIT, n_gpus=world, steps=args.steps,
+        warmup=args.warmup, ms_per_step=agg["ms_per_step"], us_per_layer=agg["ms_per_step"] * 1e3,
+        higher_is_better=True, scaling="weak", vs_baseline=None, dtype="bf16",
+        data="synthetic (seeded N(0,1) tokens, N(0,1/fan_in) bf16 weights; no trained weights)",
+        config=dict(workload=w.name, T=T, H=w.H, E=w.E, k=w.k, I=w.I, path="stream",
+                    parallelism=f"replicas{world}" if world > 1 else "single",
+                    l2="inputs larger than L2: %.2f GB of touched expert weights per step vs 126 MB L2"
+                       % ((alg["layer_bytes"]) / 1e9)),
+        roofline=dict(bound="hbm", achieved=achieved, peak=hbm, unit="GB/s", frac=achieved / hbm,
+                      traffic=traffic, kernel="stream_gate_up_kernel",
+                      alg_bytes_per_launch=alg["gate_up_bytes"], avg_launch_ms=gu_avg_s * 1e3,
+                      peak_source=f"{peak_src} hbm_gbs (MEASURED_PEAKS.json)" if peak_src == "measured" else "fallback"),
+        layer_roofline=dict(touched_experts=alg["touched"], alg_bytes=alg["layer_bytes"],
+                            alg_flops=alg["flops"], roofline_us=layer_roof_s * 1e6,
+                            frac=layer_roof_s / (secs / args.steps),
+                            down_kernel_GBps=alg["down_bytes"] / dn_avg_s / 1e9),
+        kernel_avg_ms=kernels_ms,
+        e2e=dict(value=T * world * args.steps / e2e_secs, unit=UNIT,
+                 h2d_bytes_per_step=T * w.H * 2, d2h_bytes_per_step=T * w.H * 4),
+        gpu_launches=gpu_launches,
+        clocks=clk.result(),
+    )
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        h = mi.host_inputs(d)
+        line["cpu_baseline"] = cpu_baseline(h, w, T)
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        torch.distributed.destroy_process_group()
+
+
+def main(argv=None):
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default="20b_decode", choices=sorted(mi.WORKLOADS))
+    ap.add_argument("--T", type=int, default=None)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args(argv)
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+    w = mi.WORKLOADS[args.workload]
+    T = args.T or w.T
+    if args.impl == "reference":
+        run_reference(args, w, T)
+    else:
+        run_ours(args, w, T)
+
+
+if __name__ == "__main__":
+    main()

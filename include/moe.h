@@ -1,0 +1,178 @@
+/*
+ * moe.h -- C ABI of the B200 (sm_100a) top-k routed SwiGLU Mixture-of-Experts layer.
+ *
+ * The operation (forward pass of one MoE layer, T tokens, hidden H, E experts, top-k,
+ * expert intermediate I):
+ *
+ *   l[t,e]   = sum_h x[t,h] W_router[h,e] + b_router[e]                    router logits
+ *   S_t      = the k experts with the largest l[t,.], largest first, equal logits by
+ *              lower expert index                                          top-k
+ *   w[t,j]   = exp(l[t,S_tj] - l[t,S_t0]) / sum_j' exp(l[t,S_tj'] - l[t,S_t0])
+ *                                                                          softmax over the
+ *                                                                          selected logits
+ *   count[e] = #{(t,j) : S_tj = e};  offsets = exclusive prefix sum of count
+ *   perm     : rows of expert e are offsets[e] .. offsets[e+1]-1, holding the tokens routed
+ *              to e in ascending token order; inv_perm[t,j] = row of (t, S_tj)
+ *   g | u    = x[t] W_gate_up[e]   (gate = columns [0,I), up = columns [I,2I))
+ *   h        = silu(g) * u,  silu(z) = z / (1 + exp(-z))                    SwiGLU
+ *   out[t]   = sum_j w[t,j] * (h_(t,S_tj) W_down[S_tj])                     combine
+ *
+ * Source: the layer is the mixture of SwiGLU experts with top-4 routing over 32 experts and
+ * hidden size 2880 in the Persona Kappa forum post ("Architecture Summary" table, "Notable
+ * Details") and the kappa-20b-131k model card ("Model Details" table); 128 experts in the
+ * hearth-lean-loomed-v1 card (intro and "Why 12-16 streams can be slow on Vulkan", which also
+ * describes the few-tokens-per-expert decode regime).  bf16 operands with fp32 accumulation
+ * follow the forum post's "Techniques That Made It Fit" list.  The pages print no formula,
+ * no tie rule and no interface: the formulas above are the plain reading, ties go to the
+ * lower expert index, and the calls below are this library's own.
+ *
+ * Conventions for every call
+ * --------------------------
+ * - All tensors are row-major and live in device memory of the current CUDA device, owned
+ *   by the caller.  bf16 = IEEE bfloat16.  Every pointer must be 16-byte aligned.
+ *     x          [T, H]      bf16
+ *     W_router   [H, E]      bf16
+ *     b_router   [E]         fp32
+ *     W_gate_up  [E, H, 2I]  bf16   (per expert: gate columns [0,I), up columns [I,2I))
+ *     W_down     [E, I, H]   bf16
+ *     out        [T, H]      fp32   (fully overwritten)
+ * - Work is only enqueued on `stream` (a cudaStream_t; NULL = legacy default stream).  No
+ *   call below synchronises, allocates device memory or reads device memory on the host,
+ *   except moe_create / moe_destroy (allocate / free the handle's 4-byte device status word),
+ *   moe_sync_status and moe_tune (which synchronise) and moe_profile_* (events).
+ * - Errors are returned, never thrown or aborted on.  Argument errors are found on the host
+ *   before anything is enqueued and leave every buffer untouched.  A failed launch returns
+ *   MOE_ERR_CUDA.  Faults detected on the device (a bounded wait that ran out) set the
+ *   handle's status word, which moe_sync_status reports.
+ * - One handle may be used from one stream at a time; separate handles are independent.
+ * - H and I must be multiples of 64 (2880 = 45 * 64 is not a multiple of 128), 1 <= k <= E
+ *   <= 256, H, I <= 16384, 0 <= T <= 2^20 and T * k < 2^31.  NaN or infinite inputs give
+ *   undefined results.
+ */
+#ifndef MOE_H_
+#define MOE_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#if defined(__GNUC__)
+#define MOE_API __attribute__((visibility("default")))
+#else
+#define MOE_API
+#endif
+
+struct CUstream_st;
+typedef struct CUstream_st* moe_stream_t;  /* the same object as cudaStream_t */
+
+typedef struct moe_ctx* moe_t;             /* opaque handle: shapes, settings, status word */
+
+typedef enum {
+  MOE_OK = 0,
+  MOE_ERR_ARG = 1,          /* bad argument: null / misaligned pointer, size out of range */
+  MOE_ERR_UNSUPPORTED = 2,  /* valid request this build does not support on this device */
+  MOE_ERR_WORKSPACE = 3,    /* workspace pointer null or smaller than moe_workspace_bytes */
+  MOE_ERR_CUDA = 4,         /* a CUDA runtime call or kernel launch failed */
+  MOE_ERR_TIMEOUT = 5,      /* a bounded device-side wait gave up (reported by sync_status) */
+  MOE_ERR_DEVICE = 6        /* no usable sm_100 device */
+} moe_status;
+
+typedef enum {
+  MOE_PATH_AUTO = 0,    /* weight streaming for T <= crossover, grouped GEMM above it */
+  MOE_PATH_STREAM = 1,  /* always stream expert weights (CUDA-core split-K GEMV) */
+  MOE_PATH_GEMM = 2     /* always the tcgen05 grouped GEMM */
+} moe_path;
+
+/* Create a handle for a layer of shape (E, H, I, k) on the current device.  Validates the
+ * shape (see conventions; MOE_ERR_ARG otherwise), checks for an sm_100 device
+ * (MOE_ERR_DEVICE), allocates the 4-byte device status word.  *out receives the handle. */
+MOE_API moe_status moe_create(int E, int H, int I, int k, moe_t* out);
+
+/* Free the handle and its status word.  NULL is accepted.  Work still queued on a stream
+ * that uses the handle must have completed. */
+MOE_API moe_status moe_destroy(moe_t ctx);
+
+/* Bytes of device workspace that moe_forward needs for T tokens with the handle's current
+ * path setting (moe_set_path / moe_tune change it, so query after them).  moe_route needs
+ * moe_route_workspace_bytes.  Returns 0 for a NULL handle or T < 0. */
+MOE_API size_t moe_workspace_bytes(moe_t ctx, int T);
+MOE_API size_t moe_route_workspace_bytes(moe_t ctx, int T);
+
+/* Routing half of the layer: router logits, top-k, softmax over the selected logits,
+ * histogram, offsets and the stable permutation.  Outputs (caller-owned device memory):
+ *   topk_idx       [T, k] int32   selected experts, largest logit first
+ *   topk_w         [T, k] fp32    routing weights (sum to 1 per token)
+ *   expert_offsets [E + 1] int32  row offsets of the expert segments (offsets[E] = T*k)
+ *   perm           [T * k] int32  token of each row
+ *   inv_perm       [T, k] int32   row of each (token, slot)
+ * workspace: at least moe_route_workspace_bytes(ctx, T) bytes, 16-byte aligned.
+ * T = 0 writes expert_offsets = 0 and nothing else. */
+MOE_API moe_status moe_route(moe_t ctx, int T, const void* x_bf16, const void* W_router_bf16,
+                     const float* b_router, int32_t* topk_idx, float* topk_w,
+                     int32_t* expert_offsets, int32_t* perm, int32_t* inv_perm,
+                     void* workspace, size_t ws_bytes, moe_stream_t stream);
+
+/* The whole layer: writes out [T, H] fp32 (every element).  workspace: at least
+ * moe_workspace_bytes(ctx, T) bytes.  The path (streaming or grouped GEMM) is chosen on the
+ * host from T and the handle's setting, never from device data, so the call does not
+ * synchronise.  T = 0 is a no-op. */
+MOE_API moe_status moe_forward(moe_t ctx, int T, const void* x_bf16, const void* W_router_bf16,
+                       const float* b_router, const void* W_gate_up_bf16,
+                       const void* W_down_bf16, float* out, void* workspace, size_t ws_bytes,
+                       moe_stream_t stream);
+
+/* Choose the path.  crossover_T >= 0 sets the largest T that MOE_PATH_AUTO streams;
+ * crossover_T < 0 keeps the current one (the built-in default or the value moe_tune
+ * measured).  MOE_ERR_UNSUPPORTED if the path is not available on this device. */
+MOE_API moe_status moe_set_path(moe_t ctx, moe_path path, int crossover_T);
+
+/* Current path setting and crossover. */
+MOE_API moe_status moe_get_path(moe_t ctx, moe_path* path, int* crossover_T);
+
+/* Measure the crossover on this device with the caller's layer: times both paths at
+ * T = 1, 2, 4, ... up to T_max (x must hold T_max rows, out T_max rows, workspace
+ * moe_tune_workspace_bytes) and stores the largest T at which streaming is not slower.
+ * Synchronises the stream.  *crossover_out (may be NULL) receives the value. */
+MOE_API size_t moe_tune_workspace_bytes(moe_t ctx, int T_max);
+MOE_API moe_status moe_tune(moe_t ctx, int T_max, const void* x_bf16, const void* W_router_bf16,
+                    const float* b_router, const void* W_gate_up_bf16,
+                    const void* W_down_bf16, float* out, void* workspace, size_t ws_bytes,
+                    moe_stream_t stream, int* crossover_out);
+
+/* Synchronise `stream`, then read and clear the handle's device status word.  Returns
+ * MOE_ERR_TIMEOUT if a device-side bounded wait gave up since the last call, MOE_ERR_CUDA if
+ * the stream reports an error, MOE_OK otherwise. */
+MOE_API moe_status moe_sync_status(moe_t ctx, moe_stream_t stream);
+
+/* Static text for a status code ("unknown status" for values outside the enum). */
+MOE_API const char* moe_status_string(moe_status s);
+
+/* Number of kernels this handle has launched since it was created (host counter). */
+MOE_API uint64_t moe_launch_count(moe_t ctx);
+
+/* Kernel timing for benchmarks.  moe_profile_begin(ctx, max_calls) creates CUDA events for up
+ * to max_calls subsequent moe_forward calls; each of those records an event pair around every
+ * kernel it launches, on the call's stream.  moe_profile_end synchronises, and writes for
+ * each kernel kind i < n_kinds the total milliseconds into ms[i] and its launch count into
+ * launches[i], then frees the events.  Kinds: 0 router, 1 routing finalize / scan / scatter,
+ * 2 gather, 3 gate/up projection + SwiGLU, 4 down projection + combine, 5 zero fill.
+ * moe_profile_kind_name gives a kind's name. */
+#define MOE_PROFILE_KINDS 6
+MOE_API moe_status moe_profile_begin(moe_t ctx, int max_calls);
+MOE_API moe_status moe_profile_end(moe_t ctx, float* ms, int* launches, int n_kinds);
+MOE_API const char* moe_profile_kind_name(int kind);
+
+/* Self-test of the device timeout path: launches one kernel that waits on a barrier nothing
+ * completes, with a limit of `limit_us` microseconds (1..1000000), after which it sets the
+ * status word and returns.  The next moe_sync_status then returns MOE_ERR_TIMEOUT.  No memory
+ * is touched apart from the status word. */
+MOE_API moe_status moe_selftest_timeout(moe_t ctx, int limit_us, moe_stream_t stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MOE_H_ */

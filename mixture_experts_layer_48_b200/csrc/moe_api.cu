@@ -1,0 +1,544 @@
+// C ABI of the MoE layer library (declared in include/moe.h): argument checks, workspace
+// layout, path choice and kernel launches.  Host code only; kernels live in the .cuh files.
+#include <cuda_runtime.h>
+
+#include <algorithm>
+#include <climits>
+#include <cstdint>
+#include <cstring>
+#include <new>
+#include <vector>
+
+#include "moe.h"
+#include "common.cuh"
+#include "route.cuh"
+#include "stream.cuh"
+
+using namespace moe;
+
+namespace {
+
+constexpr int kMaxE = 256;
+constexpr int kMaxHI = 16384;
+constexpr int kMaxT = 1 << 20;
+constexpr int kDefaultCrossover = INT_MAX;  // until a measured value exists: always stream
+constexpr size_t kPartBudget = size_t(256) << 20;  // split-partial scratch of the gate/up kernel
+constexpr int kMaxKernelsPerCall = 8;
+
+enum Kind { kKindRouter = 0, kKindRouteFin = 1, kKindGather = 2, kKindGateUp = 3,
+            kKindDown = 4, kKindZero = 5 };
+
+}  // namespace
+
+struct moe_ctx {
+  int E, H, I, k;
+  int device = 0;
+  int num_sms = 148;
+  moe_path path = MOE_PATH_AUTO;
+  int crossover = kDefaultCrossover;
+  uint32_t* d_status = nullptr;
+  uint64_t launches = 0;
+  // profiling
+  int prof_max = 0, prof_calls = 0;
+  std::vector<cudaEvent_t> ev;   // pairs
+  std::vector<int> ev_kind;
+  size_t ev_used = 0;
+  bool in_call = false;
+};
+
+namespace {
+
+inline size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
+
+struct Carver {
+  size_t cur = 0;
+  size_t take(size_t bytes) {
+    const size_t at = cur;
+    cur = align_up(cur + bytes, 256);
+    return at;
+  }
+};
+
+bool shape_ok(int E, int H, int I, int k) {
+  return E >= 1 && E <= kMaxE && k >= 1 && k <= E && H >= 64 && H <= kMaxHI && H % 64 == 0 &&
+         I >= 64 && I <= kMaxHI && I % 64 == 0;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// ---- workspace layouts ---------------------------------------------------------------
+struct RouteTmp {
+  size_t partial = 0, block_counts = 0, totals = 0;
+};
+
+RouteTmp carve_route_tmp(Carver& cv, const moe_ctx* c, int T) {
+  RouteTmp r;
+  if (T <= kSmallT) {
+    r.partial = cv.take(sizeof(float) * (size_t)(c->H / kRouterHSlice) * T * c->E);
+  } else {
+    const size_t NB = (T + kRouteTile - 1) / kRouteTile;
+    r.block_counts = cv.take(sizeof(int32_t) * NB * c->E);
+    r.totals = cv.take(sizeof(int32_t) * c->E);
+  }
+  return r;
+}
+
+struct StreamLayout {
+  size_t topk_idx, topk_w, inv_perm, perm, row_w, offsets, sched, chunks, part, done, h;
+  RouteTmp rt;
+  int split_cap, max_chunks, n_done;
+  size_t total;
+};
+
+int stream_split_cap(const moe_ctx* c, int T) {
+  const size_t R = (size_t)T * c->k;
+  const size_t per = R * 2 * c->I * sizeof(float);
+  if (per == 0) return 1;
+  const size_t cap = kPartBudget / per;
+  return (int)std::max<size_t>(1, std::min<size_t>(kStreamSplitMax, cap));
+}
+
+StreamLayout stream_layout(const moe_ctx* c, int T) {
+  StreamLayout L{};
+  Carver cv;
+  const size_t R = (size_t)T * c->k;
+  L.max_chunks = (int)(R / kStreamRB) + c->E;
+  const int NT = (c->I + kStreamCols - 1) / kStreamCols;
+  L.n_done = L.max_chunks * NT;
+  L.split_cap = stream_split_cap(c, T);
+  L.topk_idx = cv.take(4 * R);
+  L.topk_w = cv.take(4 * R);
+  L.inv_perm = cv.take(4 * R);
+  L.perm = cv.take(4 * R);
+  L.row_w = cv.take(4 * R);
+  L.offsets = cv.take(4 * (size_t)(c->E + 1));
+  L.sched = cv.take(16);
+  L.chunks = cv.take(16 * (size_t)L.max_chunks);
+  L.done = cv.take(4 * (size_t)L.n_done);
+  L.h = cv.take(2 * R * c->I);
+  L.part = L.split_cap > 1 ? cv.take(sizeof(float) * L.split_cap * R * 2 * c->I) : 0;
+  L.rt = carve_route_tmp(cv, c, T);
+  L.total = cv.cur;
+  return L;
+}
+
+size_t route_ws_bytes(const moe_ctx* c, int T) {
+  Carver cv;
+  cv.take(16);  // sched
+  carve_route_tmp(cv, c, T);
+  return cv.cur;
+}
+
+bool use_stream(const moe_ctx* c, int T) {
+  // The grouped-GEMM path is not part of this build yet: every T streams.
+  (void)c;
+  (void)T;
+  return true;
+}
+
+// ---- launches ------------------------------------------------------------------------
+template <typename F>
+moe_status launch(moe_ctx* c, int kind, cudaStream_t st, F&& f) {
+  const bool prof = c->prof_max > 0 && c->in_call && c->ev_used + 2 <= c->ev.size();
+  if (prof) cudaEventRecord(c->ev[c->ev_used], st);
+  f();
+  const cudaError_t err = cudaGetLastError();
+  if (prof) {
+    cudaEventRecord(c->ev[c->ev_used + 1], st);
+    c->ev_kind[c->ev_used / 2] = kind;
+    c->ev_used += 2;
+  }
+  if (err != cudaSuccess) return MOE_ERR_CUDA;
+  ++c->launches;
+  return MOE_OK;
+}
+
+#define MOE_TRY(expr)                    \
+  do {                                   \
+    const moe_status _s = (expr);        \
+    if (_s != MOE_OK) return _s;         \
+  } while (0)
+
+moe_status launch_route(moe_ctx* c, int T, const uint16_t* x, const uint16_t* Wr,
+                        const float* b, const RouteOut& o, uint8_t* ws, const RouteTmp& rt,
+                        cudaStream_t st) {
+  const int E = c->E, H = c->H, k = c->k;
+  if (T <= kSmallT) {
+    const int S = H / kRouterHSlice;
+    float* partial = reinterpret_cast<float*>(ws + rt.partial);
+    const size_t smem_p = (size_t)(kRouteTile * kRouterHSlice + kRouterHSlice * E) * 2;
+    MOE_TRY(launch(c, kKindRouter, st, [&] {
+      router_partial_kernel<<<dim3(S, (T + kRouteTile - 1) / kRouteTile), 256, smem_p, st>>>(
+          x, Wr, T, H, E, partial);
+    }));
+    const size_t smem_f = (size_t)T * E * 4 + (size_t)T * k * 4 + (size_t)T * 8 * 4 +
+                          (256 + 257 + 257) * 4;
+    MOE_TRY(launch(c, kKindRouteFin, st, [&] {
+      route_small_finalize_kernel<<<1, 1024, smem_f, st>>>(partial, S, b, T, E, k, o);
+    }));
+    return MOE_OK;
+  }
+  const int NB = (T + kRouteTile - 1) / kRouteTile;
+  int32_t* block_counts = reinterpret_cast<int32_t*>(ws + rt.block_counts);
+  int32_t* totals = reinterpret_cast<int32_t*>(ws + rt.totals);
+  const int EPW = E <= 32 ? 4 : (E <= 128 ? 16 : 32);
+  const int EP = 8 * EPW;
+  const size_t smem_r = (size_t)kRouterHSlice * kRouteTile * 2 + (size_t)kRouterHSlice * EP * 2 +
+                        (size_t)kRouteTile * EP * 4 + (size_t)EP * 4 + (size_t)kRouteTile * k * 4;
+  MOE_TRY(launch(c, kKindRouter, st, [&] {
+    if (EPW == 4)
+      router_topk_kernel<4><<<NB, 256, smem_r, st>>>(x, Wr, b, T, H, E, k, o.topk_idx, o.topk_w,
+                                                      block_counts);
+    else if (EPW == 16)
+      router_topk_kernel<16><<<NB, 256, smem_r, st>>>(x, Wr, b, T, H, E, k, o.topk_idx, o.topk_w,
+                                                       block_counts);
+    else
+      router_topk_kernel<32><<<NB, 256, smem_r, st>>>(x, Wr, b, T, H, E, k, o.topk_idx, o.topk_w,
+                                                       block_counts);
+  }));
+  MOE_TRY(launch(c, kKindRouteFin, st, [&] {
+    route_scan_kernel<<<E, 256, 0, st>>>(block_counts, NB, E, totals);
+  }));
+  const size_t smem_s = (256 + 257 + 257) * 4 + (size_t)kRouteTile * 8 * 4 + (size_t)kRouteTile * E;
+  MOE_TRY(launch(c, kKindRouteFin, st, [&] {
+    route_scatter_kernel<<<NB, 256, smem_s, st>>>(o.topk_idx, o.topk_w, block_counts, totals, T,
+                                                  E, k, o);
+  }));
+  return MOE_OK;
+}
+
+bool set_smem_attrs() {
+  const int big = 227 * 1024;
+  bool ok = true;
+  ok &= cudaFuncSetAttribute(route_small_finalize_kernel,
+                             cudaFuncAttributeMaxDynamicSharedMemorySize, big) == cudaSuccess;
+  ok &= cudaFuncSetAttribute(router_topk_kernel<4>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             big) == cudaSuccess;
+  ok &= cudaFuncSetAttribute(router_topk_kernel<16>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             big) == cudaSuccess;
+  ok &= cudaFuncSetAttribute(router_topk_kernel<32>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             big) == cudaSuccess;
+  ok &= cudaFuncSetAttribute(router_partial_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             big) == cudaSuccess;
+  ok &= cudaFuncSetAttribute(stream_gate_up_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             kGateUpSmem) == cudaSuccess;
+  ok &= cudaFuncSetAttribute(stream_down_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             kDownSmem) == cudaSuccess;
+  return ok;
+}
+
+moe_status check_common(const moe_ctx* c, int T, const void* x, const void* Wr, const float* b) {
+  if (!c) return MOE_ERR_ARG;
+  if (T < 0 || T > kMaxT || (long long)T * c->k >= (1ll << 31)) return MOE_ERR_ARG;
+  if (T == 0) return MOE_OK;
+  if (!x || !Wr || !b) return MOE_ERR_ARG;
+  if (!aligned16(x) || !aligned16(Wr) || !aligned16(b)) return MOE_ERR_ARG;
+  return MOE_OK;
+}
+
+__global__ void selftest_timeout_kernel(uint32_t* status, uint64_t limit_ns) {
+  __shared__ uint64_t bar;
+  if (threadIdx.x == 0) {
+    mbar_init(&bar, 1);
+    fence_barrier_init();
+  }
+  __syncthreads();
+  // Nothing ever arrives on `bar`: the wait must run out and report it.
+  if (threadIdx.x == 0 && !mbar_wait_bounded(&bar, 0, limit_ns)) atomicOr(status, kStatusTimeout);
+}
+
+}  // namespace
+
+extern "C" {
+
+moe_status moe_create(int E, int H, int I, int k, moe_t* out) {
+  if (!out) return MOE_ERR_ARG;
+  *out = nullptr;
+  if (!shape_ok(E, H, I, k)) return MOE_ERR_ARG;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) {
+    cudaGetLastError();
+    return MOE_ERR_DEVICE;
+  }
+  cudaDeviceProp prop;
+  if (cudaGetDeviceProperties(&prop, dev) != cudaSuccess) {
+    cudaGetLastError();
+    return MOE_ERR_DEVICE;
+  }
+  if (prop.major != 10) return MOE_ERR_DEVICE;
+  if (!set_smem_attrs()) {
+    cudaGetLastError();
+    return MOE_ERR_CUDA;
+  }
+  moe_ctx* c = new (std::nothrow) moe_ctx();
+  if (!c) return MOE_ERR_ARG;
+  c->E = E;
+  c->H = H;
+  c->I = I;
+  c->k = k;
+  c->device = dev;
+  c->num_sms = prop.multiProcessorCount;
+  if (cudaMalloc(&c->d_status, sizeof(uint32_t)) != cudaSuccess ||
+      cudaMemset(c->d_status, 0, sizeof(uint32_t)) != cudaSuccess) {
+    cudaGetLastError();
+    if (c->d_status) cudaFree(c->d_status);
+    delete c;
+    return MOE_ERR_CUDA;
+  }
+  *out = c;
+  return MOE_OK;
+}
+
+moe_status moe_destroy(moe_t c) {
+  if (!c) return MOE_OK;
+  for (cudaEvent_t e : c->ev) cudaEventDestroy(e);
+  if (c->d_status) cudaFree(c->d_status);
+  delete c;
+  return MOE_OK;
+}
+
+size_t moe_route_workspace_bytes(moe_t c, int T) {
+  if (!c || T < 0 || T > kMaxT) return 0;
+  if (T == 0) return 0;
+  return route_ws_bytes(c, T);
+}
+
+size_t moe_workspace_bytes(moe_t c, int T) {
+  if (!c || T < 0 || T > kMaxT) return 0;
+  if (T == 0) return 0;
+  return stream_layout(c, T).total;
+}
+
+moe_status moe_route(moe_t c, int T, const void* x_bf16, const void* W_router_bf16,
+                     const float* b_router, int32_t* topk_idx, float* topk_w,
+                     int32_t* expert_offsets, int32_t* perm, int32_t* inv_perm, void* workspace,
+                     size_t ws_bytes, moe_stream_t stream) {
+  MOE_TRY(check_common(c, T, x_bf16, W_router_bf16, b_router));
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  if (!expert_offsets || !aligned16(expert_offsets)) return MOE_ERR_ARG;
+  if (T == 0) {
+    if (cudaMemsetAsync(expert_offsets, 0, sizeof(int32_t) * (c->E + 1), st) != cudaSuccess)
+      return MOE_ERR_CUDA;
+    return MOE_OK;
+  }
+  if (!topk_idx || !topk_w || !perm || !inv_perm) return MOE_ERR_ARG;
+  if (!aligned16(topk_idx) || !aligned16(topk_w) || !aligned16(perm) || !aligned16(inv_perm))
+    return MOE_ERR_ARG;
+  const size_t need = route_ws_bytes(c, T);
+  if (!workspace || !aligned16(workspace) || ws_bytes < need) return MOE_ERR_WORKSPACE;
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  Carver cv;
+  const size_t sched_at = cv.take(16);
+  const RouteTmp rt = carve_route_tmp(cv, c, T);
+  RouteOut o{};
+  o.topk_idx = topk_idx;
+  o.topk_w = topk_w;
+  o.offsets = expert_offsets;
+  o.perm = perm;
+  o.inv_perm = inv_perm;
+  o.row_w = nullptr;
+  o.chunks = nullptr;
+  o.sched = reinterpret_cast<int32_t*>(ws + sched_at);
+  o.chunk_rows = 1;
+  o.zero_i32 = nullptr;
+  o.n_zero = 0;
+  return launch_route(c, T, static_cast<const uint16_t*>(x_bf16),
+                      static_cast<const uint16_t*>(W_router_bf16), b_router, o, ws, rt, st);
+}
+
+moe_status moe_forward(moe_t c, int T, const void* x_bf16, const void* W_router_bf16,
+                       const float* b_router, const void* W_gate_up_bf16,
+                       const void* W_down_bf16, float* out, void* workspace, size_t ws_bytes,
+                       moe_stream_t stream) {
+  MOE_TRY(check_common(c, T, x_bf16, W_router_bf16, b_router));
+  if (T == 0) return MOE_OK;
+  if (!W_gate_up_bf16 || !W_down_bf16 || !out) return MOE_ERR_ARG;
+  if (!aligned16(W_gate_up_bf16) || !aligned16(W_down_bf16) || !aligned16(out))
+    return MOE_ERR_ARG;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  if (c->path == MOE_PATH_GEMM) return MOE_ERR_UNSUPPORTED;
+  (void)use_stream;
+  const StreamLayout L = stream_layout(c, T);
+  if (!workspace || !aligned16(workspace) || ws_bytes < L.total) return MOE_ERR_WORKSPACE;
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  const size_t R = (size_t)T * c->k;
+
+  c->in_call = c->prof_max > 0 && c->prof_calls < c->prof_max;
+  RouteOut o{};
+  o.topk_idx = reinterpret_cast<int32_t*>(ws + L.topk_idx);
+  o.topk_w = reinterpret_cast<float*>(ws + L.topk_w);
+  o.offsets = reinterpret_cast<int32_t*>(ws + L.offsets);
+  o.perm = reinterpret_cast<int32_t*>(ws + L.perm);
+  o.inv_perm = reinterpret_cast<int32_t*>(ws + L.inv_perm);
+  o.row_w = reinterpret_cast<float*>(ws + L.row_w);
+  o.chunks = reinterpret_cast<int4*>(ws + L.chunks);
+  o.sched = reinterpret_cast<int32_t*>(ws + L.sched);
+  o.chunk_rows = kStreamRB;
+  o.zero_i32 = reinterpret_cast<int32_t*>(ws + L.done);
+  o.n_zero = L.n_done;
+  const uint16_t* x = static_cast<const uint16_t*>(x_bf16);
+  moe_status s = launch_route(c, T, x, static_cast<const uint16_t*>(W_router_bf16), b_router, o,
+                              ws, L.rt, st);
+  if (s == MOE_OK) {
+    GateUpArgs ga{};
+    ga.x = x;
+    ga.Wgu = static_cast<const uint16_t*>(W_gate_up_bf16);
+    ga.H = c->H;
+    ga.I = c->I;
+    ga.R = (int)R;
+    ga.perm = o.perm;
+    ga.chunks = o.chunks;
+    ga.sched = o.sched;
+    ga.split_cap = L.split_cap;
+    ga.part = L.split_cap > 1 ? reinterpret_cast<float*>(ws + L.part) : nullptr;
+    ga.done = o.zero_i32;
+    ga.h = reinterpret_cast<uint16_t*>(ws + L.h);
+    ga.out = out;
+    ga.out_elems = (size_t)T * c->H;
+    ga.status = c->d_status;
+    s = launch(c, kKindGateUp, st, [&] {
+      stream_gate_up_kernel<<<c->num_sms, kStreamThreads, kGateUpSmem, st>>>(ga);
+    });
+  }
+  if (s == MOE_OK) {
+    DownArgs da{};
+    da.h = reinterpret_cast<const uint16_t*>(ws + L.h);
+    da.Wd = static_cast<const uint16_t*>(W_down_bf16);
+    da.H = c->H;
+    da.I = c->I;
+    da.R = (int)R;
+    da.perm = o.perm;
+    da.row_w = o.row_w;
+    da.chunks = o.chunks;
+    da.sched = o.sched;
+    da.out = out;
+    da.status = c->d_status;
+    s = launch(c, kKindDown, st, [&] {
+      stream_down_kernel<<<c->num_sms, kStreamThreads, kDownSmem, st>>>(da);
+    });
+  }
+  if (c->in_call) ++c->prof_calls;
+  c->in_call = false;
+  return s;
+}
+
+moe_status moe_set_path(moe_t c, moe_path path, int crossover_T) {
+  if (!c) return MOE_ERR_ARG;
+  if (path != MOE_PATH_AUTO && path != MOE_PATH_STREAM && path != MOE_PATH_GEMM)
+    return MOE_ERR_ARG;
+  if (path == MOE_PATH_GEMM) return MOE_ERR_UNSUPPORTED;
+  c->path = path;
+  if (crossover_T >= 0) c->crossover = crossover_T;
+  return MOE_OK;
+}
+
+moe_status moe_get_path(moe_t c, moe_path* path, int* crossover_T) {
+  if (!c) return MOE_ERR_ARG;
+  if (path) *path = c->path;
+  if (crossover_T) *crossover_T = c->crossover;
+  return MOE_OK;
+}
+
+size_t moe_tune_workspace_bytes(moe_t c, int T_max) { return moe_workspace_bytes(c, T_max); }
+
+moe_status moe_tune(moe_t c, int T_max, const void*, const void*, const float*, const void*,
+                    const void*, float*, void*, size_t, moe_stream_t, int* crossover_out) {
+  if (!c || T_max < 1) return MOE_ERR_ARG;
+  // Only the streaming path exists in this build, so it wins at every T.
+  c->crossover = INT_MAX;
+  if (crossover_out) *crossover_out = c->crossover;
+  return MOE_OK;
+}
+
+moe_status moe_sync_status(moe_t c, moe_stream_t stream) {
+  if (!c) return MOE_ERR_ARG;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  if (cudaStreamSynchronize(st) != cudaSuccess) return MOE_ERR_CUDA;
+  uint32_t word = 0;
+  if (cudaMemcpy(&word, c->d_status, sizeof(word), cudaMemcpyDeviceToHost) != cudaSuccess)
+    return MOE_ERR_CUDA;
+  if (word != 0) {
+    if (cudaMemset(c->d_status, 0, sizeof(word)) != cudaSuccess) return MOE_ERR_CUDA;
+    if (word & kStatusTimeout) return MOE_ERR_TIMEOUT;
+  }
+  return MOE_OK;
+}
+
+const char* moe_status_string(moe_status s) {
+  switch (s) {
+    case MOE_OK: return "ok";
+    case MOE_ERR_ARG: return "invalid argument";
+    case MOE_ERR_UNSUPPORTED: return "unsupported on this build or device";
+    case MOE_ERR_WORKSPACE: return "workspace missing or too small";
+    case MOE_ERR_CUDA: return "CUDA error";
+    case MOE_ERR_TIMEOUT: return "device-side wait timed out";
+    case MOE_ERR_DEVICE: return "no usable sm_100 device";
+  }
+  return "unknown status";
+}
+
+uint64_t moe_launch_count(moe_t c) { return c ? c->launches : 0; }
+
+moe_status moe_profile_begin(moe_t c, int max_calls) {
+  if (!c || max_calls < 1 || max_calls > (1 << 20)) return MOE_ERR_ARG;
+  for (cudaEvent_t e : c->ev) cudaEventDestroy(e);
+  c->ev.assign((size_t)max_calls * kMaxKernelsPerCall * 2, nullptr);
+  c->ev_kind.assign((size_t)max_calls * kMaxKernelsPerCall, -1);
+  for (auto& e : c->ev)
+    if (cudaEventCreate(&e) != cudaSuccess) {
+      cudaGetLastError();
+      return MOE_ERR_CUDA;
+    }
+  c->prof_max = max_calls;
+  c->prof_calls = 0;
+  c->ev_used = 0;
+  return MOE_OK;
+}
+
+moe_status moe_profile_end(moe_t c, float* ms, int* launches, int n_kinds) {
+  if (!c || n_kinds < 0) return MOE_ERR_ARG;
+  for (int i = 0; i < n_kinds; ++i) {
+    if (ms) ms[i] = 0.f;
+    if (launches) launches[i] = 0;
+  }
+  moe_status s = MOE_OK;
+  for (size_t p = 0; p + 1 < c->ev_used; p += 2) {
+    float t = 0.f;
+    if (cudaEventSynchronize(c->ev[p + 1]) != cudaSuccess ||
+        cudaEventElapsedTime(&t, c->ev[p], c->ev[p + 1]) != cudaSuccess) {
+      cudaGetLastError();
+      s = MOE_ERR_CUDA;
+      continue;
+    }
+    const int kind = c->ev_kind[p / 2];
+    if (kind >= 0 && kind < n_kinds) {
+      if (ms) ms[kind] += t;
+      if (launches) launches[kind] += 1;
+    }
+  }
+  for (cudaEvent_t e : c->ev) cudaEventDestroy(e);
+  c->ev.clear();
+  c->ev_kind.clear();
+  c->ev_used = 0;
+  c->prof_max = 0;
+  c->prof_calls = 0;
+  return s;
+}
+
+const char* moe_profile_kind_name(int kind) {
+  static const char* names[MOE_PROFILE_KINDS] = {"router", "route_finalize", "gather",
+                                                 "gate_up_swiglu", "down_combine", "zero_fill"};
+  if (kind < 0 || kind >= MOE_PROFILE_KINDS) return "unknown";
+  return names[kind];
+}
+
+moe_status moe_selftest_timeout(moe_t c, int limit_us, moe_stream_t stream) {
+  if (!c || limit_us < 1 || limit_us > 1000000) return MOE_ERR_ARG;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  selftest_timeout_kernel<<<1, 32, 0, st>>>(c->d_status, (uint64_t)limit_us * 1000ull);
+  if (cudaGetLastError() != cudaSuccess) return MOE_ERR_CUDA;
+  ++c->launches;
+  return MOE_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,142 @@
+"""GPU edge cases: ragged and tiny token counts around every tile boundary, degenerate
+expert counts, ties, one hot expert, the status codes of bad calls, the timeout path."""
+import ctypes
+
+import numpy as np
+import pytest
+import torch
+
+import moe_inputs as mi
+import oracle
+from parity_util import check_outputs, compare_routing, gpu_route, host_route, inputs_on_gpu
+
+pytestmark = pytest.mark.gpu
+
+if torch.cuda.is_available():
+    import mixture_experts_layer_48_b200 as moe
+
+
+def _check_layer(d, h, E, H, I, k, layer=None):
+    layer = layer or moe.Moe(E, H, I, k)
+    T = d["x"].shape[0]
+    ref_route = host_route(h, k)
+    g = gpu_route(layer, d)
+    compare_routing(g, ref_route, k, E)
+    out = layer.forward(d["x"], d["W_router"], d["b_router"], d["W_gate_up"], d["W_down"])
+    assert layer.sync_status() == moe.MOE_OK
+    ref = oracle.moe_forward_ref(h["x"], h["W_router"], h["b_router"], h["W_gate_up"],
+                                 h["W_down"], k, route=ref_route)
+    check_outputs(out.double().cpu().numpy(), np.arange(T), h, ref_route, g, ref)
+    return layer, g
+
+
+@pytest.mark.parametrize("T", [1, 2, 3, 15, 16, 17, 31, 33, 63, 64, 65, 96, 127, 129, 300])
+def test_ragged_token_counts(T):
+    d, h = inputs_on_gpu(T, 256, 8, 2, 320, seed=100 + T)
+    _check_layer(d, h, 8, 256, 320, 2)
+
+
+@pytest.mark.parametrize("E,k", [(1, 1), (2, 1), (2, 2), (8, 1), (8, 8), (5, 3)])
+def test_degenerate_expert_counts(E, k):
+    d, h = inputs_on_gpu(40, 128, E, k, 192, seed=200 + E * 10 + k)
+    _check_layer(d, h, E, 128, 192, k)
+
+
+@pytest.mark.parametrize("T", [7, 100])
+def test_k_equals_E_256(T):
+    d, h = inputs_on_gpu(T, 64, 256, 256, 64, seed=300 + T, experts=False)
+    layer = moe.Moe(256, 64, 64, 256)
+    compare_routing(gpu_route(layer, d), host_route(h, 256), 256, 256)
+
+
+@pytest.mark.parametrize("T", [5, 70])
+def test_all_equal_logits(T):
+    d, h = inputs_on_gpu(T, 128, 8, 3, 128, seed=400 + T)
+    d["W_router"].zero_()
+    d["b_router"].zero_()
+    h = mi.host_inputs(d)
+    layer, g = _check_layer(d, h, 8, 128, 128, 3)
+    assert np.all(g["topk_idx"] == np.array([0, 1, 2]))
+    np.testing.assert_allclose(g["topk_w"], 1 / 3, atol=1e-7)
+
+
+@pytest.mark.parametrize("T", [40, 200])
+def test_one_hot_expert(T):
+    d, h = inputs_on_gpu(T, 128, 16, 2, 128, seed=500 + T)
+    d["b_router"].zero_()
+    d["b_router"][11] = 1000.0       # every token picks expert 11 first
+    h = mi.host_inputs(d)
+    layer, g = _check_layer(d, h, 16, 128, 128, 2)
+    assert np.all(g["topk_idx"][:, 0] == 11)
+    assert np.diff(g["expert_offsets"])[11] == T
+
+
+def test_gpt_oss_shape_with_ragged_T():
+    d, h = inputs_on_gpu(37, 2880, 32, 4, 2880, seed=600)
+    _check_layer(d, h, 32, 2880, 2880, 4)
+
+
+def test_forward_is_repeatable_and_overwrites_out():
+    d, h = inputs_on_gpu(24, 256, 8, 2, 256, seed=700)
+    layer = moe.Moe(8, 256, 256, 2)
+    out = torch.full((24, 256), 12345.0, device="cuda")
+    a = layer.forward(d["x"], d["W_router"], d["b_router"], d["W_gate_up"], d["W_down"], out=out).clone()
+    b = layer.forward(d["x"], d["W_router"], d["b_router"], d["W_gate_up"], d["W_down"])
+    torch.cuda.synchronize()
+    assert torch.isfinite(a).all()
+    torch.testing.assert_close(a, b, atol=1e-5, rtol=1e-5)
+
+
+def test_zero_tokens():
+    layer = moe.Moe(8, 256, 256, 2)
+    x = torch.empty((0, 256), dtype=torch.bfloat16, device="cuda")
+    Wr = torch.zeros((256, 8), dtype=torch.bfloat16, device="cuda")
+    b = torch.zeros(8, device="cuda")
+    Wgu = torch.zeros((8, 256, 512), dtype=torch.bfloat16, device="cuda")
+    Wd = torch.zeros((8, 256, 256), dtype=torch.bfloat16, device="cuda")
+    out = layer.forward(x, Wr, b, Wgu, Wd)
+    assert out.shape == (0, 256)
+    r = layer.route(x, Wr, b)
+    assert r["expert_offsets"].cpu().tolist() == [0] * 9
+    assert layer.sync_status() == moe.MOE_OK
+
+
+def test_bad_calls_return_status_codes():
+    d, _ = inputs_on_gpu(8, 256, 8, 2, 256, seed=800)
+    layer = moe.Moe(8, 256, 256, 2)
+    ws = torch.empty(layer.workspace_bytes(8), dtype=torch.uint8, device="cuda")
+    out = torch.empty((8, 256), device="cuda")
+    p = [d[k].data_ptr() for k in ("x", "W_router", "b_router", "W_gate_up", "W_down")]
+    st = torch.cuda.current_stream().cuda_stream
+    f = moe.moe_forward
+    assert f(layer.handle, 8, *p, out.data_ptr(), ws.data_ptr(), ws.numel(), st) == moe.MOE_OK
+    assert f(layer.handle, 8, *p, out.data_ptr(), ws.data_ptr(), ws.numel() - 1, st) == moe.MOE_ERR_WORKSPACE
+    assert f(layer.handle, 8, *p, out.data_ptr(), 0, ws.numel(), st) == moe.MOE_ERR_WORKSPACE
+    bad = list(p)
+    bad[0] += 2  # misaligned x
+    assert f(layer.handle, 8, *bad, out.data_ptr(), ws.data_ptr(), ws.numel(), st) == moe.MOE_ERR_ARG
+    assert f(layer.handle, -1, *p, out.data_ptr(), ws.data_ptr(), ws.numel(), st) == moe.MOE_ERR_ARG
+    assert f(layer.handle, 8, *p, 0, ws.data_ptr(), ws.numel(), st) == moe.MOE_ERR_ARG
+    assert layer.sync_status() == moe.MOE_OK
+
+
+def test_timeout_is_reported_not_hung():
+    layer = moe.Moe(8, 256, 256, 2)
+    layer.selftest_timeout(2000)   # 2 ms bounded wait on a barrier nothing completes
+    assert layer.sync_status() == moe.MOE_ERR_TIMEOUT
+    assert layer.sync_status() == moe.MOE_OK   # the word is cleared by the read
+    d, h = inputs_on_gpu(16, 256, 8, 2, 256, seed=900)
+    _check_layer(d, h, 8, 256, 256, 2, layer=layer)   # the context is still usable
+
+
+def test_profile_counts_kernels():
+    d, _ = inputs_on_gpu(16, 256, 8, 2, 256, seed=901)
+    layer = moe.Moe(8, 256, 256, 2)
+    layer.profile_begin(3)
+    n0 = layer.launch_count()
+    for _ in range(3):
+        layer.forward(d["x"], d["W_router"], d["b_router"], d["W_gate_up"], d["W_down"])
+    prof = layer.profile_end()
+    assert layer.launch_count() - n0 == sum(v[1] for v in prof.values())
+    assert prof["gate_up_swiglu"][1] == 3 and prof["down_combine"][1] == 3
+    assert all(v[0] >= 0 for v in prof.values())

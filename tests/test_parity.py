@@ -1,0 +1,67 @@
+"""GPU parity: the CUDA library against the fp64 oracle on the five seeded workloads.
+
+Routing (expert indices, histogram, offsets, permutation) must be bit-exact apart from
+reported near ties; outputs must satisfy |gpu - oracle| <= 1e-2 + 2e-2 |oracle| per element.
+"""
+import json
+
+import numpy as np
+import pytest
+import torch
+
+import moe_inputs as mi
+import oracle
+from parity_util import check_outputs, compare_routing, gpu_route, host_route, inputs_on_gpu
+
+pytestmark = pytest.mark.gpu
+
+if torch.cuda.is_available():
+    import mixture_experts_layer_48_b200 as moe
+
+
+def _run(name, T=None, path=None, sample=None):
+    w = mi.WORKLOADS[name]
+    T = w.T if T is None else T
+    d, h = inputs_on_gpu(T, w.H, w.E, w.k, w.I, w.seed, zipf=w.zipf)
+    layer = moe.Moe(w.E, w.H, w.I, w.k)
+    if path is not None:
+        layer.set_path(path)
+    ref_route = host_route(h, w.k)
+    g = gpu_route(layer, d)
+    rep = compare_routing(g, ref_route, w.k, w.E)
+    out = layer.forward(d["x"], d["W_router"], d["b_router"], d["W_gate_up"], d["W_down"])
+    assert layer.sync_status() == moe.MOE_OK
+    tokens = np.arange(T) if not sample else mi.sample_tokens(T, sample, w.seed)
+    out_gpu = out[torch.from_numpy(tokens).cuda()].double().cpu().numpy()
+    ref_out = oracle.moe_forward_ref(h["x"], h["W_router"], h["b_router"], h["W_gate_up"],
+                                     h["W_down"], w.k, tokens=tokens, route=ref_route)
+    orep = check_outputs(out_gpu, tokens, h, ref_route, g, ref_out)
+    rep.update(orep)
+    print(name, T, json.dumps({k: v for k, v in rep.items() if k != "set_changed"}))
+    return rep, g
+
+
+def test_tiny():
+    _run("tiny")
+
+
+def test_20b_decode():
+    _run("20b_decode")
+
+
+@pytest.mark.parametrize("T", mi.WORKLOADS["120b_sweep"].sweep)
+def test_120b_sweep(T):
+    _run("120b_sweep", T=T)
+
+
+def test_20b_prefill():
+    _run("20b_prefill", sample=1024)
+
+
+def test_131k_skewed():
+    w = mi.WORKLOADS["131k_skewed"]
+    rep, g = _run("131k_skewed", sample=w.oracle_sample)
+    cnt = np.diff(g["expert_offsets"])
+    ratio = cnt.max() / cnt.mean()
+    print("131k max/mean expert load", ratio)
+    assert 3.5 <= ratio <= 4.5
