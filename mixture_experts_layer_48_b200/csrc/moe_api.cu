@@ -1,5 +1,7 @@
 // C ABI of the MoE layer library (declared in include/moe.h): argument checks, workspace
 // layout, path choice and kernel launches.  Host code only; kernels live in the .cuh files.
+#include <cuda.h>
+#include <cudaTypedefs.h>
 #include <cuda_runtime.h>
 
 #include <algorithm>
@@ -22,7 +24,6 @@ constexpr int kMaxE = 256;
 constexpr int kMaxHI = 16384;
 constexpr int kMaxT = 1 << 20;
 constexpr int kDefaultCrossover = INT_MAX;  // until a measured value exists: always stream
-constexpr size_t kPartBudget = size_t(256) << 20;  // split-partial scratch of the gate/up kernel
 constexpr int kMaxKernelsPerCall = 8;
 
 enum Kind { kKindRouter = 0, kKindRouteFin = 1, kKindGather = 2, kKindGateUp = 3,
@@ -30,8 +31,15 @@ enum Kind { kKindRouter = 0, kKindRouteFin = 1, kKindGather = 2, kKindGateUp = 3
 
 }  // namespace
 
+// A TMA descriptor for one weight tensor, re-encoded when the caller passes another pointer.
+struct MapCache {
+  const void* ptr = nullptr;
+  CUtensorMap map;
+};
+
 struct moe_ctx {
   int E, H, I, k;
+  MapCache gate_up_stream, down_stream;
   int device = 0;
   int num_sms = 148;
   moe_path path = MOE_PATH_AUTO;
@@ -66,6 +74,48 @@ bool shape_ok(int E, int H, int I, int k) {
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
+PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  static bool tried = false;
+  if (!tried) {
+    tried = true;
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+    else
+      cudaGetLastError();
+  }
+  return fn;
+}
+
+// 2D bf16 view [rows, cols] (row-major, contiguous) with a [box_rows, box_cols] box.
+bool encode_2d(CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols, uint32_t box_rows,
+               uint32_t box_cols, CUtensorMapSwizzle swizzle) {
+  auto enc = tensor_map_encoder();
+  if (!enc) return false;
+  cuuint64_t dims[2] = {cols, rows};
+  cuuint64_t strides[1] = {cols * 2};
+  cuuint32_t box[2] = {box_cols, box_rows};
+  cuuint32_t estr[2] = {1, 1};
+  return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box,
+             estr, CU_TENSOR_MAP_INTERLEAVE_NONE, swizzle,
+             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+const CUtensorMap* cached_map(MapCache& mc, const void* ptr, uint64_t rows, uint64_t cols,
+                              uint32_t box_rows, uint32_t box_cols,
+                              CUtensorMapSwizzle swizzle = CU_TENSOR_MAP_SWIZZLE_128B) {
+  if (mc.ptr != ptr) {
+    mc.ptr = nullptr;
+    if (!encode_2d(&mc.map, ptr, rows, cols, box_rows, box_cols, swizzle)) return nullptr;
+    mc.ptr = ptr;
+  }
+  return &mc.map;
+}
+
 // ---- workspace layouts ---------------------------------------------------------------
 struct RouteTmp {
   size_t partial = 0, block_counts = 0, totals = 0;
@@ -84,19 +134,11 @@ RouteTmp carve_route_tmp(Carver& cv, const moe_ctx* c, int T) {
 }
 
 struct StreamLayout {
-  size_t topk_idx, topk_w, inv_perm, perm, row_w, offsets, sched, chunks, part, done, h;
+  size_t topk_idx, topk_w, inv_perm, perm, row_w, offsets, sched, chunks, acc, done, h;
   RouteTmp rt;
-  int split_cap, max_chunks, n_done;
+  int max_chunks, n_done;
   size_t total;
 };
-
-int stream_split_cap(const moe_ctx* c, int T) {
-  const size_t R = (size_t)T * c->k;
-  const size_t per = R * 2 * c->I * sizeof(float);
-  if (per == 0) return 1;
-  const size_t cap = kPartBudget / per;
-  return (int)std::max<size_t>(1, std::min<size_t>(kStreamSplitMax, cap));
-}
 
 StreamLayout stream_layout(const moe_ctx* c, int T) {
   StreamLayout L{};
@@ -105,7 +147,6 @@ StreamLayout stream_layout(const moe_ctx* c, int T) {
   L.max_chunks = (int)(R / kStreamRB) + c->E;
   const int NT = (c->I + kStreamCols - 1) / kStreamCols;
   L.n_done = L.max_chunks * NT;
-  L.split_cap = stream_split_cap(c, T);
   L.topk_idx = cv.take(4 * R);
   L.topk_w = cv.take(4 * R);
   L.inv_perm = cv.take(4 * R);
@@ -116,7 +157,7 @@ StreamLayout stream_layout(const moe_ctx* c, int T) {
   L.chunks = cv.take(16 * (size_t)L.max_chunks);
   L.done = cv.take(4 * (size_t)L.n_done);
   L.h = cv.take(2 * R * c->I);
-  L.part = L.split_cap > 1 ? cv.take(sizeof(float) * L.split_cap * R * 2 * c->I) : 0;
+  L.acc = cv.take(sizeof(float) * R * 2 * c->I);
   L.rt = carve_route_tmp(cv, c, T);
   L.total = cv.cur;
   return L;
@@ -159,9 +200,12 @@ moe_status launch(moe_ctx* c, int kind, cudaStream_t st, F&& f) {
     if (_s != MOE_OK) return _s;         \
   } while (0)
 
+// Routing chain.  zero4/n_zero4: a float scratch region the router kernel zero-fills.
 moe_status launch_route(moe_ctx* c, int T, const uint16_t* x, const uint16_t* Wr,
                         const float* b, const RouteOut& o, uint8_t* ws, const RouteTmp& rt,
-                        cudaStream_t st) {
+                        cudaStream_t st, float* zero = nullptr, size_t n_zero_floats = 0) {
+  float4* zero4 = reinterpret_cast<float4*>(zero);
+  const size_t n_zero4 = n_zero_floats / 4;
   const int E = c->E, H = c->H, k = c->k;
   if (T <= kSmallT) {
     const int S = H / kRouterHSlice;
@@ -169,7 +213,7 @@ moe_status launch_route(moe_ctx* c, int T, const uint16_t* x, const uint16_t* Wr
     const size_t smem_p = (size_t)(kRouteTile * kRouterHSlice + kRouterHSlice * E) * 2;
     MOE_TRY(launch(c, kKindRouter, st, [&] {
       router_partial_kernel<<<dim3(S, (T + kRouteTile - 1) / kRouteTile), 256, smem_p, st>>>(
-          x, Wr, T, H, E, partial);
+          x, Wr, T, H, E, partial, zero4, n_zero4);
     }));
     const size_t smem_f = (size_t)T * E * 4 + (size_t)T * k * 4 + (size_t)T * 8 * 4 +
                           (256 + 257 + 257) * 4;
@@ -188,13 +232,13 @@ moe_status launch_route(moe_ctx* c, int T, const uint16_t* x, const uint16_t* Wr
   MOE_TRY(launch(c, kKindRouter, st, [&] {
     if (EPW == 4)
       router_topk_kernel<4><<<NB, 256, smem_r, st>>>(x, Wr, b, T, H, E, k, o.topk_idx, o.topk_w,
-                                                      block_counts);
+                                                      block_counts, zero4, n_zero4);
     else if (EPW == 16)
       router_topk_kernel<16><<<NB, 256, smem_r, st>>>(x, Wr, b, T, H, E, k, o.topk_idx, o.topk_w,
-                                                       block_counts);
+                                                       block_counts, zero4, n_zero4);
     else
       router_topk_kernel<32><<<NB, 256, smem_r, st>>>(x, Wr, b, T, H, E, k, o.topk_idx, o.topk_w,
-                                                       block_counts);
+                                                       block_counts, zero4, n_zero4);
   }));
   MOE_TRY(launch(c, kKindRouteFin, st, [&] {
     route_scan_kernel<<<E, 256, 0, st>>>(block_counts, NB, E, totals);
@@ -378,32 +422,33 @@ moe_status moe_forward(moe_t c, int T, const void* x_bf16, const void* W_router_
   o.n_zero = L.n_done;
   const uint16_t* x = static_cast<const uint16_t*>(x_bf16);
   moe_status s = launch_route(c, T, x, static_cast<const uint16_t*>(W_router_bf16), b_router, o,
-                              ws, L.rt, st);
+                              ws, L.rt, st, reinterpret_cast<float*>(ws + L.acc), R * 2 * c->I);
   if (s == MOE_OK) {
     GateUpArgs ga{};
     ga.x = x;
-    ga.Wgu = static_cast<const uint16_t*>(W_gate_up_bf16);
     ga.H = c->H;
     ga.I = c->I;
     ga.R = (int)R;
     ga.perm = o.perm;
     ga.chunks = o.chunks;
     ga.sched = o.sched;
-    ga.split_cap = L.split_cap;
-    ga.part = L.split_cap > 1 ? reinterpret_cast<float*>(ws + L.part) : nullptr;
+    ga.acc = reinterpret_cast<float*>(ws + L.acc);
     ga.done = o.zero_i32;
     ga.h = reinterpret_cast<uint16_t*>(ws + L.h);
     ga.out = out;
     ga.out_elems = (size_t)T * c->H;
     ga.status = c->d_status;
-    s = launch(c, kKindGateUp, st, [&] {
-      stream_gate_up_kernel<<<c->num_sms, kStreamThreads, kGateUpSmem, st>>>(ga);
-    });
+    const CUtensorMap* m = cached_map(c->gate_up_stream, W_gate_up_bf16, (uint64_t)c->E * c->H,
+                                      2ull * c->I, kGateUpKC, kBox);
+    if (!m) s = MOE_ERR_CUDA;
+    else
+      s = launch(c, kKindGateUp, st, [&] {
+        stream_gate_up_kernel<<<c->num_sms, kStreamThreads, kGateUpSmem, st>>>(ga, *m);
+      });
   }
   if (s == MOE_OK) {
     DownArgs da{};
     da.h = reinterpret_cast<const uint16_t*>(ws + L.h);
-    da.Wd = static_cast<const uint16_t*>(W_down_bf16);
     da.H = c->H;
     da.I = c->I;
     da.R = (int)R;
@@ -413,9 +458,13 @@ moe_status moe_forward(moe_t c, int T, const void* x_bf16, const void* W_router_
     da.sched = o.sched;
     da.out = out;
     da.status = c->d_status;
-    s = launch(c, kKindDown, st, [&] {
-      stream_down_kernel<<<c->num_sms, kStreamThreads, kDownSmem, st>>>(da);
-    });
+    const CUtensorMap* m = cached_map(c->down_stream, W_down_bf16, (uint64_t)c->E * c->I,
+                                      (uint64_t)c->H, kDownKC, kBox);
+    if (!m) s = MOE_ERR_CUDA;
+    else
+      s = launch(c, kKindDown, st, [&] {
+        stream_down_kernel<<<c->num_sms, kStreamThreads, kDownSmem, st>>>(da, *m);
+      });
   }
   if (c->in_call) ++c->prof_calls;
   c->in_call = false;

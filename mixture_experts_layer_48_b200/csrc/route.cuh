@@ -102,10 +102,20 @@ MOE_DEVINL float warp_softmax_denominator(const float* lg, int k) {
 // Small T: partial router logits over one 64-row slice of W_router.
 // grid (H/64, ceil(T/32)), block 256.  partial layout [H/64][T][E].
 // ---------------------------------------------------------------------------------------
+// Grid-stride zero fill of a scratch region by every block of the launching kernel.
+MOE_DEVINL void zero_fill_f4(float4* z, size_t n4) {
+  const size_t nthreads = (size_t)gridDim.x * gridDim.y * blockDim.x;
+  const size_t b = (size_t)blockIdx.y * gridDim.x + blockIdx.x;
+  for (size_t i = b * blockDim.x + threadIdx.x; i < n4; i += nthreads)
+    z[i] = make_float4(0.f, 0.f, 0.f, 0.f);
+}
+
 __global__ void __launch_bounds__(256) router_partial_kernel(const uint16_t* __restrict__ x,
                                                              const uint16_t* __restrict__ Wr,
                                                              int T, int H, int E,
-                                                             float* __restrict__ partial) {
+                                                             float* __restrict__ partial,
+                                                             float4* zero4, size_t n_zero4) {
+  zero_fill_f4(zero4, n_zero4);
   extern __shared__ __align__(128) uint8_t smem_raw[];
   uint16_t* xs = reinterpret_cast<uint16_t*>(smem_raw);  // [32][64]
   uint16_t* ws = xs + kRouteTile * kRouterHSlice;          // [64][E]
@@ -247,7 +257,8 @@ __global__ void __launch_bounds__(256)
     router_topk_kernel(const uint16_t* __restrict__ x, const uint16_t* __restrict__ Wr,
                        const float* __restrict__ b_router, int T, int H, int E, int k,
                        int32_t* __restrict__ topk_idx, float* __restrict__ topk_w,
-                       int32_t* __restrict__ block_counts) {
+                       int32_t* __restrict__ block_counts, float4* zero4, size_t n_zero4) {
+  zero_fill_f4(zero4, n_zero4);
   extern __shared__ __align__(128) uint8_t smem_raw[];
   uint16_t* xsT = reinterpret_cast<uint16_t*>(smem_raw);          // [64][32] (h-major)
   uint16_t* ws = xsT + kRouterHSlice * kRouteTile;                  // [64][8*EPW]

@@ -3,42 +3,57 @@
 // With a handful of tokens per step each expert sees about one token (the regime the
 // hearth-lean-loomed-v1 card describes in "Why 12-16 streams can be slow on Vulkan"), so
 // the expert matmuls are matrix-vector products whose cost is reading the touched experts'
-// weights once from HBM.  These kernels stream those weights through shared memory at full
-// HBM bandwidth and apply them to every row routed to the expert.
+// weights once from HBM.  These kernels stream those weights through shared memory at HBM
+// bandwidth and apply them to every row routed to the expert.
 //
-// Layout: a persistent grid (one CTA per SM).  Each CTA has one producer warp that issues
-// bulk async copies (cp.async.bulk, 16-byte aligned rows, no multicast) of [KC x 320] weight
-// tiles into a 4-stage shared-memory ring, and 5 consumer warps (160 threads, 2 columns each)
-// that multiply the tile with the expert's rows (<= 16 per work item) in fp32 using packed
-// FFMA2.  Work items are (row chunk of one expert, 320-column tile, K split); the number of
-// K splits is chosen on the device from the routing so that every SM gets the same share.
+// Layout: a persistent grid (one CTA per SM).  Each CTA has one producer warp and five
+// consumer warps around a 4-stage shared-memory ring.  The producer issues TMA tensor loads
+// (no multicast) of 64-column weight boxes with the 128-byte swizzle, and bulk copies of the
+// rows' activations.  Consumer warp w owns box w of a 320-column tile and multiplies it with
+// the expert's rows on the tensor cores: the weight block is the 16-row A operand (read with
+// ldmatrix.trans, since W is [K, N] with N contiguous), the <= 16 activation rows are the
+// 8-wide B operand (mma.sync m16n8k16, bf16 in, fp32 accumulate).  The arithmetic costs a few
+// instructions per 16 x 16 x 8 block, so the kernels stay bound by the weight stream.
+//
+// Work items are (row chunk of one expert, 320-column tile, K split); the number of K splits
+// is chosen on the device from the routing so that every SM gets the same share.
 //
 //   gate/up kernel: columns [c0, c0+320) of the gate half AND the same columns of the up half,
-//     so one item holds matching gate and up sums.  Split partial sums go to a scratch
-//     buffer; the last CTA of a (chunk, tile) -- found with a fenced counter -- reduces them
-//     and writes h = silu(g) * u as bf16.  It also zero-fills `out` for the next kernel.
+//     so a thread holds matching gate and up sums.  K splits add their partial sums into an
+//     fp32 accumulator (zero-filled by the router kernel) with atomics; the last CTA of a
+//     (chunk, tile) -- found with a fenced counter -- reads the totals and writes
+//     h = silu(g) * u as bf16.  The kernel also zero-fills `out`.
 //   down kernel: y = h W_down[e] per row, scaled by the row's routing weight, added into
-//     out[token] with fp32 vector atomics (the combine).
+//     out[token] with fp32 atomics (the combine).
 #pragma once
 
 #include "common.cuh"
 
 namespace moe {
 
-constexpr int kStreamRB = 16;            // rows per work-list chunk
-constexpr int kStreamConsumers = 160;    // consumer threads (5 warps)
-constexpr int kStreamThreads = 192;      // + 1 producer warp
-constexpr int kStreamCols = 320;         // columns per tile (2 per consumer thread)
+constexpr int kStreamRB = 16;                          // rows per work-list chunk (<= 2 n8 tiles)
+constexpr int kStreamWarps = 5;                        // consumer warps
+constexpr int kStreamConsumers = 32 * kStreamWarps;
+constexpr int kStreamThreads = kStreamConsumers + 32;  // + 1 producer warp
+constexpr int kBox = 64;                               // columns per TMA box (128 B)
+constexpr int kStreamCols = kBox * kStreamWarps;       // 320 columns per tile
 constexpr int kStreamStages = 4;
-constexpr int kGateUpKC = 32;            // W_gate_up rows per stage
-constexpr int kDownKC = 64;              // W_down rows per stage
+constexpr int kGateUpKC = 32;                          // W_gate_up rows per stage
+constexpr int kDownKC = 64;                            // W_down rows per stage
 constexpr int kStreamSplitMax = 16;
 
-constexpr int kGateUpStageBytes = 2 * kGateUpKC * kStreamCols * 2 + kStreamRB * kGateUpKC * 2;
-constexpr int kDownStageBytes = kDownKC * kStreamCols * 2 + kStreamRB * kDownKC * 2;
-constexpr int kGateUpSmem = kStreamStages * kGateUpStageBytes + 2 * kStreamStages * 8;
-constexpr int kDownSmem = kStreamStages * kDownStageBytes + 2 * kStreamStages * 8;
-static_assert(kGateUpStageBytes % 16 == 0 && kDownStageBytes % 16 == 0, "stage alignment");
+constexpr int kGUBoxBytes = kGateUpKC * kBox * 2;                  // 4 KB
+constexpr int kDNBoxBytes = kDownKC * kBox * 2;                    // 8 KB
+constexpr int kGUStageW = 2 * kStreamWarps * kGUBoxBytes;          // gate + up boxes, 40 KB
+constexpr int kDNStageW = kStreamWarps * kDNBoxBytes;              // 40 KB
+constexpr int kGUXPitch = kGateUpKC * 2 + 16;                      // activation row pitch (bytes)
+constexpr int kDNXPitch = kDownKC * 2 + 16;                        // padded: conflict-free ldmatrix
+constexpr int kGUStageX = kStreamRB * kGUXPitch;
+constexpr int kDNStageX = kStreamRB * kDNXPitch;
+constexpr int kGateUpSmem = 1024 + kStreamStages * (kGUStageW + kGUStageX) + 2 * kStreamStages * 8;
+constexpr int kDownSmem = 1024 + kStreamStages * (kDNStageW + kDNStageX) + 2 * kStreamStages * 8;
+static_assert(kGUStageW % 1024 == 0 && kDNStageW % 1024 == 0, "128B-swizzle atoms need 1 KB");
+static_assert(kGUXPitch % 16 == 0 && kDNXPitch % 16 == 0, "bulk copy alignment");
 
 struct SplitPlan {
   int S;   // number of K splits (every split non-empty)
@@ -66,13 +81,11 @@ MOE_DEVINL SplitPlan choose_splits(int units, int nk, int G, int smax) {
 
 struct GateUpArgs {
   const uint16_t* x;     // [T, H]
-  const uint16_t* Wgu;   // [E, H, 2I]
   int H, I, R;
   const int32_t* perm;   // [R]
   const int4* chunks;    // work list
   const int32_t* sched;  // [0] chunk count
-  int split_cap;         // largest K split count the scratch buffer holds
-  float* part;           // [split_cap, R, 2I] split partial sums (split_cap > 1)
+  float* acc;            // [R, 2I] gate | up sums, zero on entry
   int32_t* done;         // [chunks * tiles] completion counters, zero on entry
   uint16_t* h;           // [R, I] bf16 SwiGLU output
   float* out;            // [T, H] zero-filled here
@@ -82,7 +95,6 @@ struct GateUpArgs {
 
 struct DownArgs {
   const uint16_t* h;     // [R, I]
-  const uint16_t* Wd;    // [E, I, H]
   int H, I, R;
   const int32_t* perm;   // [R]
   const float* row_w;    // [R]
@@ -92,27 +104,77 @@ struct DownArgs {
   uint32_t* status;
 };
 
-// Ring bookkeeping shared by the producer and the consumers of one CTA.
-struct Ring {
-  uint64_t* full;
-  uint64_t* empty;
-};
-
 MOE_DEVINL void record_timeout(uint32_t* status) { atomicOr(status, kStatusTimeout); }
+
+MOE_DEVINL uint8_t* align1k(uint8_t* p) {
+  return reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(p) + 1023) & ~uintptr_t(1023));
+}
+
+// Byte offset, inside a [rows][64] bf16 box stored with the 128-byte swizzle, of the 16-byte
+// chunk that lane provides to ldmatrix.x4.trans for m-tile mt (16 columns) and k-step ks
+// (16 rows).  Matrices: 0 (cols 0-7, rows 0-7), 1 (cols 8-15, rows 0-7), 2 (cols 0-7,
+// rows 8-15), 3 (cols 8-15, rows 8-15) -- the order of the A fragment registers.
+MOE_DEVINL uint32_t a_frag_offset(int lane, int mt, int ks) {
+  const int i = lane >> 3, j = lane & 7;
+  const int krow = ks * 16 + (i >> 1) * 8 + j;
+  const int chunk = 2 * mt + (i & 1);
+  return (uint32_t)(krow * 128 + ((chunk ^ j) << 4));
+}
+
+// Byte offset of the 16-byte activation chunk lane provides to ldmatrix (B operand):
+// matrices 0/1 = rows 0-7 at k 0-7 / 8-15, matrices 2/3 = rows 8-15 likewise.
+MOE_DEVINL uint32_t b_frag_offset(int lane, int ks, int pitch) {
+  const int row = (lane & 7) + ((lane >> 4) << 3);
+  return (uint32_t)(row * pitch + (ks * 16 + ((lane >> 3) & 1) * 8) * 2);
+}
 
 // ------------------------------------------------------------------------------------------
 // gate/up projection + SwiGLU
 // ------------------------------------------------------------------------------------------
-__global__ void __launch_bounds__(kStreamThreads, 1) stream_gate_up_kernel(const GateUpArgs a) {
+template <int NB>
+MOE_DEVINL void gateup_stage_mma(uint32_t wbase, uint32_t xbase, int warp_c, int lane,
+                                 float (&accg)[4][2][4], float (&accu)[4][2][4]) {
+  const uint32_t gbox = wbase + warp_c * kGUBoxBytes;
+  const uint32_t ubox = wbase + (kStreamWarps + warp_c) * kGUBoxBytes;
+#pragma unroll
+  for (int ks = 0; ks < kGateUpKC / 16; ++ks) {
+    uint32_t b[2][2];
+    const uint32_t baddr = xbase + b_frag_offset(lane, ks, kGUXPitch);
+    if constexpr (NB == 1) {
+      ldsm_x2(baddr, b[0][0], b[0][1]);
+    } else {
+      ldsm_x4(baddr, b[0][0], b[0][1], b[1][0], b[1][1]);
+    }
+#pragma unroll
+    for (int mt = 0; mt < 4; ++mt) {
+      const uint32_t off = a_frag_offset(lane, mt, ks);
+      uint32_t a0, a1, a2, a3;
+      ldsm_x4_trans(gbox + off, a0, a1, a2, a3);
+#pragma unroll
+      for (int nb = 0; nb < NB; ++nb)
+        mma_bf16_16816(accg[mt][nb], a0, a1, a2, a3, b[nb][0], b[nb][1]);
+      ldsm_x4_trans(ubox + off, a0, a1, a2, a3);
+#pragma unroll
+      for (int nb = 0; nb < NB; ++nb)
+        mma_bf16_16816(accu[mt][nb], a0, a1, a2, a3, b[nb][0], b[nb][1]);
+    }
+  }
+}
+
+// The weight tensor map views W_gate_up as [E*H rows, 2I columns], box [32 x 64], 128B swizzle.
+__global__ void __launch_bounds__(kStreamThreads, 1)
+    stream_gate_up_kernel(const GateUpArgs a, const __grid_constant__ CUtensorMap wmap) {
   extern __shared__ __align__(128) uint8_t smem_raw[];
   __shared__ int s_last;
-  uint64_t* bars = reinterpret_cast<uint64_t*>(smem_raw + kStreamStages * kGateUpStageBytes);
-  Ring ring{bars, bars + kStreamStages};
+  uint8_t* wring = align1k(smem_raw);
+  uint8_t* xring = wring + kStreamStages * kGUStageW;
+  uint64_t* full = reinterpret_cast<uint64_t*>(xring + kStreamStages * kGUStageX);
+  uint64_t* empty = full + kStreamStages;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   if (tid == 0) {
     for (int s = 0; s < kStreamStages; ++s) {
-      mbar_init(&ring.full[s], 1);
-      mbar_init(&ring.empty[s], kStreamConsumers / 32);
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], kStreamWarps);
     }
     fence_barrier_init();
   }
@@ -122,11 +184,12 @@ __global__ void __launch_bounds__(kStreamThreads, 1) stream_gate_up_kernel(const
   const int NT = (a.I + kStreamCols - 1) / kStreamCols;
   const int units = a.sched[0] * NT;
   const int nk = a.H / kGateUpKC;
-  const SplitPlan plan = choose_splits(units, nk, gridDim.x, a.split_cap);
+  const SplitPlan plan = choose_splits(units, nk, gridDim.x, kStreamSplitMax);
   const int items = units * plan.S;
 
-  if (warp == 0) {
+  if (warp == kStreamWarps) {
     // ---------------- producer ----------------
+    if (lane == 0) tma_prefetch_desc(&wmap);
     bool aborted = false;
     uint32_t it = 0;
     int last_it[kStreamStages];
@@ -136,33 +199,30 @@ __global__ void __launch_bounds__(kStreamThreads, 1) stream_gate_up_kernel(const
       const int unit = id / plan.S, sp = id - unit * plan.S;
       const int4 ch = a.chunks[unit / NT];
       const int col0 = (unit % NT) * kStreamCols;
-      const int wg = min(kStreamCols, a.I - col0);
       const int kb = sp * plan.ks, ke = min(nk, kb + plan.ks);
       const int tok = (lane < ch.z) ? a.perm[ch.y + lane] : 0;
-      const uint32_t bytes = 2u * kGateUpKC * wg * 2u + (uint32_t)ch.z * kGateUpKC * 2u;
+      // lanes 0-4 load gate boxes, lanes 5-9 the matching up boxes
+      const int box_col = lane < kStreamWarps ? col0 + kBox * lane
+                                              : a.I + col0 + kBox * (lane - kStreamWarps);
+      const uint32_t bytes = (uint32_t)kGUStageW + (uint32_t)ch.z * kGateUpKC * 2u;
       for (int kst = kb; kst < ke; ++kst, ++it) {
         const int slot = it % kStreamStages;
         const uint32_t ph = (it / kStreamStages) & 1u;
-        if (!aborted && lane == 0 &&
-            !mbar_wait_bounded(&ring.empty[slot], ph ^ 1u, kWaitLimitNs)) {
+        if (!aborted && lane == 0 && !mbar_wait_bounded(&empty[slot], ph ^ 1u, kWaitLimitNs)) {
           aborted = true;
           record_timeout(a.status);
         }
         aborted = __shfl_sync(0xffffffffu, aborted, 0);
         if (aborted) continue;
-        uint8_t* stage = smem_raw + slot * kGateUpStageBytes;
-        uint16_t* Wg_s = reinterpret_cast<uint16_t*>(stage);
-        uint16_t* Wu_s = Wg_s + kGateUpKC * kStreamCols;
-        uint16_t* X_s = Wu_s + kGateUpKC * kStreamCols;
-        if (lane == 0) mbar_arrive_expect_tx(&ring.full[slot], bytes);
+        if (lane == 0) mbar_arrive_expect_tx(&full[slot], bytes);
         __syncwarp();
         const int k0 = kst * kGateUpKC;
-        const uint16_t* src = a.Wgu + ((size_t)ch.x * a.H + k0 + lane) * I2 + col0;
-        bulk_g2s(Wg_s + lane * kStreamCols, src, wg * 2, &ring.full[slot]);
-        bulk_g2s(Wu_s + lane * kStreamCols, src + a.I, wg * 2, &ring.full[slot]);
+        if (lane < 2 * kStreamWarps)
+          tma_load_2d(wring + slot * kGUStageW + lane * kGUBoxBytes, &wmap, box_col,
+                      ch.x * a.H + k0, &full[slot]);
         if (lane < ch.z)
-          bulk_g2s(X_s + lane * kGateUpKC, a.x + (size_t)tok * a.H + k0, kGateUpKC * 2,
-                   &ring.full[slot]);
+          bulk_g2s(xring + slot * kGUStageX + lane * kGUXPitch, a.x + (size_t)tok * a.H + k0,
+                   kGateUpKC * 2, &full[slot]);
         last_it[slot] = it;
       }
     }
@@ -170,14 +230,14 @@ __global__ void __launch_bounds__(kStreamThreads, 1) stream_gate_up_kernel(const
     if (lane == 0) {
       for (int s = 0; s < kStreamStages; ++s)
         if (last_it[s] >= 0 &&
-            !mbar_wait_bounded(&ring.full[s], (last_it[s] / kStreamStages) & 1u, kWaitLimitNs))
+            !mbar_wait_bounded(&full[s], (last_it[s] / kStreamStages) & 1u, kWaitLimitNs))
           record_timeout(a.status);
     }
     return;
   }
 
   // ---------------- consumers ----------------
-  const int ctid = tid - 32;
+  const int ctid = tid;  // 0..159; warp = box index
   {
     float4* o4 = reinterpret_cast<float4*>(a.out);
     const size_t n4 = a.out_elems / 4;
@@ -185,9 +245,9 @@ __global__ void __launch_bounds__(kStreamThreads, 1) stream_gate_up_kernel(const
          i += (size_t)gridDim.x * kStreamConsumers)
       o4[i] = make_float4(0.f, 0.f, 0.f, 0.f);
   }
+  const uint32_t wring_s = smem_u32(wring), xring_s = smem_u32(xring);
   bool aborted = false;
   uint32_t it = 0;
-  const int c = 2 * ctid;
   for (int id = blockIdx.x; id < items; id += gridDim.x) {
     const int unit = id / plan.S, sp = id - unit * plan.S;
     const int4 ch = a.chunks[unit / NT];
@@ -195,89 +255,82 @@ __global__ void __launch_bounds__(kStreamThreads, 1) stream_gate_up_kernel(const
     const int wg = min(kStreamCols, a.I - col0);
     const int kb = sp * plan.ks, ke = min(nk, kb + plan.ks);
     const int nrows = ch.z;
-    float2 accg[kStreamRB], accu[kStreamRB];
+    float accg[4][2][4], accu[4][2][4];
 #pragma unroll
-    for (int r = 0; r < kStreamRB; ++r) accg[r] = accu[r] = make_float2(0.f, 0.f);
+    for (int mt = 0; mt < 4; ++mt)
+#pragma unroll
+      for (int nb = 0; nb < 2; ++nb)
+#pragma unroll
+        for (int v = 0; v < 4; ++v) accg[mt][nb][v] = accu[mt][nb][v] = 0.f;
 
     for (int kst = kb; kst < ke; ++kst, ++it) {
       const int slot = it % kStreamStages;
       const uint32_t ph = (it / kStreamStages) & 1u;
-      if (!aborted && !mbar_wait_bounded(&ring.full[slot], ph, kWaitLimitNs)) {
+      if (!aborted && !mbar_wait_bounded(&full[slot], ph, kWaitLimitNs)) {
         aborted = true;
         record_timeout(a.status);
       }
       if (!aborted) {
-        const uint8_t* stage = smem_raw + slot * kGateUpStageBytes;
-        const uint32_t* Wg32 = reinterpret_cast<const uint32_t*>(stage);
-        const uint32_t* Wu32 = Wg32 + kGateUpKC * kStreamCols / 2;
-        const uint32_t* X32 = Wu32 + kGateUpKC * kStreamCols / 2;
-#pragma unroll 2
-        for (int kk = 0; kk < kGateUpKC; kk += 2) {
-          const uint32_t g0 = Wg32[kk * (kStreamCols / 2) + ctid];
-          const uint32_t g1 = Wg32[(kk + 1) * (kStreamCols / 2) + ctid];
-          const uint32_t u0 = Wu32[kk * (kStreamCols / 2) + ctid];
-          const uint32_t u1 = Wu32[(kk + 1) * (kStreamCols / 2) + ctid];
-          const float2 G0 = make_float2(bf16lo(g0), bf16hi(g0));
-          const float2 G1 = make_float2(bf16lo(g1), bf16hi(g1));
-          const float2 U0 = make_float2(bf16lo(u0), bf16hi(u0));
-          const float2 U1 = make_float2(bf16lo(u1), bf16hi(u1));
-#pragma unroll
-          for (int r = 0; r < kStreamRB; ++r) {
-            if (r < nrows) {
-              const uint32_t xv = X32[r * (kGateUpKC / 2) + (kk >> 1)];
-              const float2 x0 = make_float2(bf16lo(xv), bf16lo(xv));
-              const float2 x1 = make_float2(bf16hi(xv), bf16hi(xv));
-              accg[r] = __ffma2_rn(x0, G0, accg[r]);
-              accg[r] = __ffma2_rn(x1, G1, accg[r]);
-              accu[r] = __ffma2_rn(x0, U0, accu[r]);
-              accu[r] = __ffma2_rn(x1, U1, accu[r]);
-            }
-          }
-        }
+        const uint32_t wb = wring_s + slot * kGUStageW, xb = xring_s + slot * kGUStageX;
+        if (nrows <= 8)
+          gateup_stage_mma<1>(wb, xb, warp, lane, accg, accu);
+        else
+          gateup_stage_mma<2>(wb, xb, warp, lane, accg, accu);
       }
       __syncwarp();
-      if (lane == 0 && !aborted) mbar_arrive(&ring.empty[slot]);
+      if (lane == 0 && !aborted) mbar_arrive(&empty[slot]);
     }
 
-    // ---- epilogue ----
-    const bool mine = c < wg;
+    // ---- epilogue: C fragment (m = weight column, n = row) ----
+    // value v of tile (mt, nb): column 64*warp + 16*mt + (lane>>2) + 8*(v>>1),
+    //                           row nb*8 + 2*(lane&3) + (v&1)
     if (plan.S == 1) {
-      if (mine && !aborted) {
+      if (!aborted) {
 #pragma unroll
-        for (int r = 0; r < kStreamRB; ++r)
-          if (r < nrows) {
-            const float hx = silu_f32(accg[r].x) * accu[r].x;
-            const float hy = silu_f32(accg[r].y) * accu[r].y;
-            *reinterpret_cast<uint32_t*>(a.h + (size_t)(ch.y + r) * a.I + col0 + c) =
-                pack_bf16x2(hx, hy);
-          }
+        for (int mt = 0; mt < 4; ++mt)
+#pragma unroll
+          for (int nb = 0; nb < 2; ++nb)
+#pragma unroll
+            for (int v = 0; v < 4; ++v) {
+              const int cl = kBox * warp + 16 * mt + (lane >> 2) + 8 * (v >> 1);
+              const int r = nb * 8 + 2 * (lane & 3) + (v & 1);
+              if (r < nrows && cl < wg) {
+                const float hv = silu_f32(accg[mt][nb][v]) * accu[mt][nb][v];
+                a.h[(size_t)(ch.y + r) * a.I + col0 + cl] = (uint16_t)f32_to_bf16_bits(hv);
+              }
+            }
       }
       continue;
     }
-    if (mine) {
+    if (!aborted) {
 #pragma unroll
-      for (int r = 0; r < kStreamRB; ++r)
-        if (r < nrows) {
-          float* p = a.part + ((size_t)sp * a.R + ch.y + r) * I2 + col0 + c;
-          *reinterpret_cast<float2*>(p) = accg[r];
-          *reinterpret_cast<float2*>(p + a.I) = accu[r];
-        }
+      for (int mt = 0; mt < 4; ++mt)
+#pragma unroll
+        for (int nb = 0; nb < 2; ++nb)
+#pragma unroll
+          for (int v = 0; v < 4; ++v) {
+            const int cl = kBox * warp + 16 * mt + (lane >> 2) + 8 * (v >> 1);
+            const int r = nb * 8 + 2 * (lane & 3) + (v & 1);
+            if (r < nrows && cl < wg) {
+              float* p = a.acc + (size_t)(ch.y + r) * I2 + col0 + cl;
+              atomicAdd(p, accg[mt][nb][v]);
+              atomicAdd(p + a.I, accu[mt][nb][v]);
+            }
+          }
     }
     __threadfence();
     named_bar_sync(1, kStreamConsumers);
     if (ctid == 0) s_last = (atomicAdd(&a.done[unit], 1) == plan.S - 1);
     named_bar_sync(1, kStreamConsumers);
-    if (s_last && mine && !aborted) {
+    if (s_last && !aborted) {
       __threadfence();
-      for (int r = 0; r < nrows; ++r) {
-        float2 g = make_float2(0.f, 0.f), u = make_float2(0.f, 0.f);
-        for (int s = 0; s < plan.S; ++s) {
-          const float* p = a.part + ((size_t)s * a.R + ch.y + r) * I2 + col0 + c;
-          const float2 pg = ld_cg_f2(p), pu = ld_cg_f2(p + a.I);
-          g.x += pg.x; g.y += pg.y;
-          u.x += pu.x; u.y += pu.y;
-        }
-        *reinterpret_cast<uint32_t*>(a.h + (size_t)(ch.y + r) * a.I + col0 + c) =
+      // the last split of this (chunk, tile): totals are complete, apply SwiGLU
+      for (int i = ctid; i < nrows * (wg / 2); i += kStreamConsumers) {
+        const int r = i / (wg / 2), cl = 2 * (i - r * (wg / 2));
+        const float* p = a.acc + (size_t)(ch.y + r) * I2 + col0 + cl;
+        const float2 g = __ldcg(reinterpret_cast<const float2*>(p));
+        const float2 u = __ldcg(reinterpret_cast<const float2*>(p + a.I));
+        *reinterpret_cast<uint32_t*>(a.h + (size_t)(ch.y + r) * a.I + col0 + cl) =
             pack_bf16x2(silu_f32(g.x) * u.x, silu_f32(g.y) * u.y);
       }
     }
@@ -287,15 +340,43 @@ __global__ void __launch_bounds__(kStreamThreads, 1) stream_gate_up_kernel(const
 // ------------------------------------------------------------------------------------------
 // down projection + routing weight + combine
 // ------------------------------------------------------------------------------------------
-__global__ void __launch_bounds__(kStreamThreads, 1) stream_down_kernel(const DownArgs a) {
+template <int NB>
+MOE_DEVINL void down_stage_mma(uint32_t wbase, uint32_t xbase, int warp_c, int lane,
+                               float (&acc)[4][2][4]) {
+  const uint32_t box = wbase + warp_c * kDNBoxBytes;
+#pragma unroll
+  for (int ks = 0; ks < kDownKC / 16; ++ks) {
+    uint32_t b[2][2];
+    const uint32_t baddr = xbase + b_frag_offset(lane, ks, kDNXPitch);
+    if constexpr (NB == 1) {
+      ldsm_x2(baddr, b[0][0], b[0][1]);
+    } else {
+      ldsm_x4(baddr, b[0][0], b[0][1], b[1][0], b[1][1]);
+    }
+#pragma unroll
+    for (int mt = 0; mt < 4; ++mt) {
+      uint32_t a0, a1, a2, a3;
+      ldsm_x4_trans(box + a_frag_offset(lane, mt, ks), a0, a1, a2, a3);
+#pragma unroll
+      for (int nb = 0; nb < NB; ++nb)
+        mma_bf16_16816(acc[mt][nb], a0, a1, a2, a3, b[nb][0], b[nb][1]);
+    }
+  }
+}
+
+// The weight tensor map views W_down as [E*I rows, H columns], box [64 x 64], 128B swizzle.
+__global__ void __launch_bounds__(kStreamThreads, 1)
+    stream_down_kernel(const DownArgs a, const __grid_constant__ CUtensorMap wmap) {
   extern __shared__ __align__(128) uint8_t smem_raw[];
-  uint64_t* bars = reinterpret_cast<uint64_t*>(smem_raw + kStreamStages * kDownStageBytes);
-  Ring ring{bars, bars + kStreamStages};
+  uint8_t* wring = align1k(smem_raw);
+  uint8_t* xring = wring + kStreamStages * kDNStageW;
+  uint64_t* full = reinterpret_cast<uint64_t*>(xring + kStreamStages * kDNStageX);
+  uint64_t* empty = full + kStreamStages;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   if (tid == 0) {
     for (int s = 0; s < kStreamStages; ++s) {
-      mbar_init(&ring.full[s], 1);
-      mbar_init(&ring.empty[s], kStreamConsumers / 32);
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], kStreamWarps);
     }
     fence_barrier_init();
   }
@@ -307,7 +388,8 @@ __global__ void __launch_bounds__(kStreamThreads, 1) stream_down_kernel(const Do
   const SplitPlan plan = choose_splits(units, nk, gridDim.x, kStreamSplitMax);
   const int items = units * plan.S;
 
-  if (warp == 0) {
+  if (warp == kStreamWarps) {
+    if (lane == 0) tma_prefetch_desc(&wmap);
     bool aborted = false;
     uint32_t it = 0;
     int last_it[kStreamStages];
@@ -317,46 +399,39 @@ __global__ void __launch_bounds__(kStreamThreads, 1) stream_down_kernel(const Do
       const int unit = id / plan.S, sp = id - unit * plan.S;
       const int4 ch = a.chunks[unit / NT];
       const int col0 = (unit % NT) * kStreamCols;
-      const int wc = min(kStreamCols, a.H - col0);
       const int kb = sp * plan.ks, ke = min(nk, kb + plan.ks);
-      const uint32_t bytes = (uint32_t)kDownKC * wc * 2u + (uint32_t)ch.z * kDownKC * 2u;
+      const uint32_t bytes = (uint32_t)kDNStageW + (uint32_t)ch.z * kDownKC * 2u;
       for (int kst = kb; kst < ke; ++kst, ++it) {
         const int slot = it % kStreamStages;
         const uint32_t ph = (it / kStreamStages) & 1u;
-        if (!aborted && lane == 0 &&
-            !mbar_wait_bounded(&ring.empty[slot], ph ^ 1u, kWaitLimitNs)) {
+        if (!aborted && lane == 0 && !mbar_wait_bounded(&empty[slot], ph ^ 1u, kWaitLimitNs)) {
           aborted = true;
           record_timeout(a.status);
         }
         aborted = __shfl_sync(0xffffffffu, aborted, 0);
         if (aborted) continue;
-        uint8_t* stage = smem_raw + slot * kDownStageBytes;
-        uint16_t* W_s = reinterpret_cast<uint16_t*>(stage);
-        uint16_t* H_s = W_s + kDownKC * kStreamCols;
-        if (lane == 0) mbar_arrive_expect_tx(&ring.full[slot], bytes);
+        if (lane == 0) mbar_arrive_expect_tx(&full[slot], bytes);
         __syncwarp();
         const int k0 = kst * kDownKC;
-        const uint16_t* src = a.Wd + ((size_t)ch.x * a.I + k0) * a.H + col0;
-        bulk_g2s(W_s + lane * kStreamCols, src + (size_t)lane * a.H, wc * 2, &ring.full[slot]);
-        bulk_g2s(W_s + (lane + 32) * kStreamCols, src + (size_t)(lane + 32) * a.H, wc * 2,
-                 &ring.full[slot]);
+        if (lane < kStreamWarps)
+          tma_load_2d(wring + slot * kDNStageW + lane * kDNBoxBytes, &wmap, col0 + kBox * lane,
+                      ch.x * a.I + k0, &full[slot]);
         if (lane < ch.z)
-          bulk_g2s(H_s + lane * kDownKC, a.h + (size_t)(ch.y + lane) * a.I + k0, kDownKC * 2,
-                   &ring.full[slot]);
+          bulk_g2s(xring + slot * kDNStageX + lane * kDNXPitch,
+                   a.h + (size_t)(ch.y + lane) * a.I + k0, kDownKC * 2, &full[slot]);
         last_it[slot] = it;
       }
     }
     if (lane == 0) {
       for (int s = 0; s < kStreamStages; ++s)
         if (last_it[s] >= 0 &&
-            !mbar_wait_bounded(&ring.full[s], (last_it[s] / kStreamStages) & 1u, kWaitLimitNs))
+            !mbar_wait_bounded(&full[s], (last_it[s] / kStreamStages) & 1u, kWaitLimitNs))
           record_timeout(a.status);
     }
     return;
   }
 
-  const int ctid = tid - 32;
-  const int c = 2 * ctid;
+  const uint32_t wring_s = smem_u32(wring), xring_s = smem_u32(xring);
   bool aborted = false;
   uint32_t it = 0;
   for (int id = blockIdx.x; id < items; id += gridDim.x) {
@@ -366,49 +441,53 @@ __global__ void __launch_bounds__(kStreamThreads, 1) stream_down_kernel(const Do
     const int wc = min(kStreamCols, a.H - col0);
     const int kb = sp * plan.ks, ke = min(nk, kb + plan.ks);
     const int nrows = ch.z;
-    float2 acc[kStreamRB];
+    float acc[4][2][4];
 #pragma unroll
-    for (int r = 0; r < kStreamRB; ++r) acc[r] = make_float2(0.f, 0.f);
+    for (int mt = 0; mt < 4; ++mt)
+#pragma unroll
+      for (int nb = 0; nb < 2; ++nb)
+#pragma unroll
+        for (int v = 0; v < 4; ++v) acc[mt][nb][v] = 0.f;
     for (int kst = kb; kst < ke; ++kst, ++it) {
       const int slot = it % kStreamStages;
       const uint32_t ph = (it / kStreamStages) & 1u;
-      if (!aborted && !mbar_wait_bounded(&ring.full[slot], ph, kWaitLimitNs)) {
+      if (!aborted && !mbar_wait_bounded(&full[slot], ph, kWaitLimitNs)) {
         aborted = true;
         record_timeout(a.status);
       }
       if (!aborted) {
-        const uint8_t* stage = smem_raw + slot * kDownStageBytes;
-        const uint32_t* W32 = reinterpret_cast<const uint32_t*>(stage);
-        const uint32_t* H32 = W32 + kDownKC * kStreamCols / 2;
-#pragma unroll 4
-        for (int kk = 0; kk < kDownKC; kk += 2) {
-          const uint32_t w0 = W32[kk * (kStreamCols / 2) + ctid];
-          const uint32_t w1 = W32[(kk + 1) * (kStreamCols / 2) + ctid];
-          const float2 W0 = make_float2(bf16lo(w0), bf16hi(w0));
-          const float2 W1 = make_float2(bf16lo(w1), bf16hi(w1));
-#pragma unroll
-          for (int r = 0; r < kStreamRB; ++r) {
-            if (r < nrows) {
-              const uint32_t hv = H32[r * (kDownKC / 2) + (kk >> 1)];
-              acc[r] = __ffma2_rn(make_float2(bf16lo(hv), bf16lo(hv)), W0, acc[r]);
-              acc[r] = __ffma2_rn(make_float2(bf16hi(hv), bf16hi(hv)), W1, acc[r]);
-            }
-          }
-        }
+        const uint32_t wb = wring_s + slot * kDNStageW, xb = xring_s + slot * kDNStageX;
+        if (nrows <= 8)
+          down_stage_mma<1>(wb, xb, warp, lane, acc);
+        else
+          down_stage_mma<2>(wb, xb, warp, lane, acc);
       }
       __syncwarp();
-      if (lane == 0 && !aborted) mbar_arrive(&ring.empty[slot]);
+      if (lane == 0 && !aborted) mbar_arrive(&empty[slot]);
     }
-    if (c < wc && !aborted) {
+    if (aborted) continue;
+    // rows this thread holds: nb*8 + 2*(lane&3) + {0,1}
+    int tok[2][2];
+    float wt[2][2];
 #pragma unroll
-      for (int r = 0; r < kStreamRB; ++r)
-        if (r < nrows) {
-          const int row = ch.y + r;
-          const float w = a.row_w[row];
-          red_add_f32x2(a.out + (size_t)a.perm[row] * a.H + col0 + c, w * acc[r].x,
-                        w * acc[r].y);
+    for (int nb = 0; nb < 2; ++nb)
+#pragma unroll
+      for (int q = 0; q < 2; ++q) {
+        const int r = nb * 8 + 2 * (lane & 3) + q;
+        tok[nb][q] = r < nrows ? a.perm[ch.y + r] : -1;
+        wt[nb][q] = r < nrows ? a.row_w[ch.y + r] : 0.f;
+      }
+#pragma unroll
+    for (int mt = 0; mt < 4; ++mt)
+#pragma unroll
+      for (int nb = 0; nb < 2; ++nb)
+#pragma unroll
+        for (int v = 0; v < 4; ++v) {
+          const int cl = kBox * warp + 16 * mt + (lane >> 2) + 8 * (v >> 1);
+          const int t = tok[nb][v & 1];
+          if (t >= 0 && cl < wc)
+            atomicAdd(a.out + (size_t)t * a.H + col0 + cl, wt[nb][v & 1] * acc[mt][nb][v]);
         }
-    }
   }
 }
 
