@@ -159,6 +159,13 @@ MOE_DEVINL void red_add_f32x4(float* p, float a, float b, float c, float d) {
                : "memory");
 }
 
+// gpu-scope release / acquire-release atomics for cross-CTA completion counters.
+MOE_DEVINL int atom_add_acq_rel_gpu(int* p, int v) {
+  int old;
+  asm volatile("atom.acq_rel.gpu.global.add.s32 %0, [%1], %2;" : "=r"(old) : "l"(p), "r"(v) : "memory");
+  return old;
+}
+
 MOE_DEVINL float silu_f32(float z) { return z / (1.0f + expf(-z)); }
 
 }  // namespace moe

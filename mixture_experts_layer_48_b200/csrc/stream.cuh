@@ -15,14 +15,16 @@
 // 8-wide B operand (mma.sync m16n8k16, bf16 in, fp32 accumulate).  The arithmetic costs a few
 // instructions per 16 x 16 x 8 block, so the kernels stay bound by the weight stream.
 //
-// Work items are (row chunk of one expert, 320-column tile, K split); the number of K splits
-// is chosen on the device from the routing so that every SM gets the same share.
+// Work: tiles are (row chunk of one expert, 320-column block); the tiles' K stages form one
+// sequence that is cut into equal contiguous ranges, one per CTA (stream-K), so every SM
+// streams the same number of bytes whatever the routing.
 //
 //   gate/up kernel: columns [c0, c0+320) of the gate half AND the same columns of the up half,
-//     so a thread holds matching gate and up sums.  K splits add their partial sums into an
-//     fp32 accumulator (zero-filled by the router kernel) with atomics; the last CTA of a
-//     (chunk, tile) -- found with a fenced counter -- reads the totals and writes
-//     h = silu(g) * u as bf16.  The kernel also zero-fills `out`.
+//     so a thread holds matching gate and up sums.  A CTA that covers a tile's whole K range
+//     applies SwiGLU from registers; otherwise the pieces add their partial sums into an fp32
+//     accumulator (zero-filled by the router kernel) with atomics, and the piece that
+//     completes the tile's stage count (a release/acquire counter) writes h = silu(g) * u as
+//     bf16.  The kernel also zero-fills `out`.
 //   down kernel: y = h W_down[e] per row, scaled by the row's routing weight, added into
 //     out[token] with fp32 atomics (the combine).
 #pragma once
@@ -37,10 +39,9 @@ constexpr int kStreamConsumers = 32 * kStreamWarps;
 constexpr int kStreamThreads = kStreamConsumers + 32;  // + 1 producer warp
 constexpr int kBox = 64;                               // columns per TMA box (128 B)
 constexpr int kStreamCols = kBox * kStreamWarps;       // 320 columns per tile
-constexpr int kStreamStages = 4;
+constexpr int kStreamStages = 5;
 constexpr int kGateUpKC = 32;                          // W_gate_up rows per stage
 constexpr int kDownKC = 64;                            // W_down rows per stage
-constexpr int kStreamSplitMax = 16;
 
 constexpr int kGUBoxBytes = kGateUpKC * kBox * 2;                  // 4 KB
 constexpr int kDNBoxBytes = kDownKC * kBox * 2;                    // 8 KB
@@ -55,28 +56,16 @@ constexpr int kDownSmem = 1024 + kStreamStages * (kDNStageW + kDNStageX) + 2 * k
 static_assert(kGUStageW % 1024 == 0 && kDNStageW % 1024 == 0, "128B-swizzle atoms need 1 KB");
 static_assert(kGUXPitch % 16 == 0 && kDNXPitch % 16 == 0, "bulk copy alignment");
 
-struct SplitPlan {
-  int S;   // number of K splits (every split non-empty)
-  int ks;  // K stages per split (the last may have fewer)
+// Stream-K work split: the (tile, K stage) pairs of all tiles form one sequence of
+// units * nk stages; CTA b takes the contiguous range [b*total/G, (b+1)*total/G).  Every CTA
+// streams the same number of weight bytes (to one stage); a tile's K range may be shared by
+// two or three CTAs, whose partial sums meet in fp32 atomics.
+struct StreamKRange {
+  long long g0, g1;
 };
-
-// Split count minimising the per-CTA makespan ceil(units*S / G) * ks with ks = ceil(nk/S).
-MOE_DEVINL SplitPlan choose_splits(int units, int nk, int G, int smax) {
-  SplitPlan best{1, nk};
-  long long best_cost = -1;
-  const int top = min(smax, nk);
-  for (int S = 1; S <= top; ++S) {
-    const int ks = (nk + S - 1) / S;
-    const int Se = (nk + ks - 1) / ks;
-    if (Se != S) continue;  // an equivalent smaller S was already costed
-    const long long rounds = ((long long)units * S + G - 1) / G;
-    const long long cost = rounds * ks;
-    if (best_cost < 0 || cost < best_cost) {
-      best_cost = cost;
-      best = SplitPlan{S, ks};
-    }
-  }
-  return best;
+MOE_DEVINL StreamKRange stream_k_range(long long units, int nk) {
+  const long long total = units * nk;
+  return StreamKRange{total * blockIdx.x / gridDim.x, total * (blockIdx.x + 1) / gridDim.x};
 }
 
 struct GateUpArgs {
@@ -182,10 +171,8 @@ __global__ void __launch_bounds__(kStreamThreads, 1)
 
   const int I2 = 2 * a.I;
   const int NT = (a.I + kStreamCols - 1) / kStreamCols;
-  const int units = a.sched[0] * NT;
   const int nk = a.H / kGateUpKC;
-  const SplitPlan plan = choose_splits(units, nk, gridDim.x, kStreamSplitMax);
-  const int items = units * plan.S;
+  const StreamKRange rng = stream_k_range((long long)a.sched[0] * NT, nk);
 
   if (warp == kStreamWarps) {
     // ---------------- producer ----------------
@@ -195,11 +182,12 @@ __global__ void __launch_bounds__(kStreamThreads, 1)
     int last_it[kStreamStages];
 #pragma unroll
     for (int s = 0; s < kStreamStages; ++s) last_it[s] = -1;
-    for (int id = blockIdx.x; id < items; id += gridDim.x) {
-      const int unit = id / plan.S, sp = id - unit * plan.S;
+    for (long long g = rng.g0; g < rng.g1;) {
+      const int unit = (int)(g / nk), kb = (int)(g % nk);
+      const int ke = (int)min((long long)nk, kb + (rng.g1 - g));
+      g += ke - kb;
       const int4 ch = a.chunks[unit / NT];
       const int col0 = (unit % NT) * kStreamCols;
-      const int kb = sp * plan.ks, ke = min(nk, kb + plan.ks);
       const int tok = (lane < ch.z) ? a.perm[ch.y + lane] : 0;
       // lanes 0-4 load gate boxes, lanes 5-9 the matching up boxes
       const int box_col = lane < kStreamWarps ? col0 + kBox * lane
@@ -248,12 +236,13 @@ __global__ void __launch_bounds__(kStreamThreads, 1)
   const uint32_t wring_s = smem_u32(wring), xring_s = smem_u32(xring);
   bool aborted = false;
   uint32_t it = 0;
-  for (int id = blockIdx.x; id < items; id += gridDim.x) {
-    const int unit = id / plan.S, sp = id - unit * plan.S;
+  for (long long g = rng.g0; g < rng.g1;) {
+    const int unit = (int)(g / nk), kb = (int)(g % nk);
+    const int ke = (int)min((long long)nk, kb + (rng.g1 - g));
+    g += ke - kb;
     const int4 ch = a.chunks[unit / NT];
     const int col0 = (unit % NT) * kStreamCols;
     const int wg = min(kStreamCols, a.I - col0);
-    const int kb = sp * plan.ks, ke = min(nk, kb + plan.ks);
     const int nrows = ch.z;
     float accg[4][2][4], accu[4][2][4];
 #pragma unroll
@@ -280,29 +269,12 @@ __global__ void __launch_bounds__(kStreamThreads, 1)
       __syncwarp();
       if (lane == 0 && !aborted) mbar_arrive(&empty[slot]);
     }
+    if (aborted) continue;
 
     // ---- epilogue: C fragment (m = weight column, n = row) ----
     // value v of tile (mt, nb): column 64*warp + 16*mt + (lane>>2) + 8*(v>>1),
     //                           row nb*8 + 2*(lane&3) + (v&1)
-    if (plan.S == 1) {
-      if (!aborted) {
-#pragma unroll
-        for (int mt = 0; mt < 4; ++mt)
-#pragma unroll
-          for (int nb = 0; nb < 2; ++nb)
-#pragma unroll
-            for (int v = 0; v < 4; ++v) {
-              const int cl = kBox * warp + 16 * mt + (lane >> 2) + 8 * (v >> 1);
-              const int r = nb * 8 + 2 * (lane & 3) + (v & 1);
-              if (r < nrows && cl < wg) {
-                const float hv = silu_f32(accg[mt][nb][v]) * accu[mt][nb][v];
-                a.h[(size_t)(ch.y + r) * a.I + col0 + cl] = (uint16_t)f32_to_bf16_bits(hv);
-              }
-            }
-      }
-      continue;
-    }
-    if (!aborted) {
+    if (kb == 0 && ke == nk) {  // this CTA holds the whole K range: SwiGLU from registers
 #pragma unroll
       for (int mt = 0; mt < 4; ++mt)
 #pragma unroll
@@ -312,26 +284,40 @@ __global__ void __launch_bounds__(kStreamThreads, 1)
             const int cl = kBox * warp + 16 * mt + (lane >> 2) + 8 * (v >> 1);
             const int r = nb * 8 + 2 * (lane & 3) + (v & 1);
             if (r < nrows && cl < wg) {
-              float* p = a.acc + (size_t)(ch.y + r) * I2 + col0 + cl;
-              atomicAdd(p, accg[mt][nb][v]);
-              atomicAdd(p + a.I, accu[mt][nb][v]);
+              const float hv = silu_f32(accg[mt][nb][v]) * accu[mt][nb][v];
+              a.h[(size_t)(ch.y + r) * a.I + col0 + cl] = (uint16_t)f32_to_bf16_bits(hv);
             }
           }
+      continue;
     }
-    __threadfence();
+#pragma unroll
+    for (int mt = 0; mt < 4; ++mt)
+#pragma unroll
+      for (int nb = 0; nb < 2; ++nb)
+#pragma unroll
+        for (int v = 0; v < 4; ++v) {
+          const int cl = kBox * warp + 16 * mt + (lane >> 2) + 8 * (v >> 1);
+          const int r = nb * 8 + 2 * (lane & 3) + (v & 1);
+          if (r < nrows && cl < wg) {
+            float* p = a.acc + (size_t)(ch.y + r) * I2 + col0 + cl;
+            atomicAdd(p, accg[mt][nb][v]);
+            atomicAdd(p + a.I, accu[mt][nb][v]);
+          }
+        }
+    // Completion count in K stages: the piece that brings it to nk applies SwiGLU.  The
+    // barrier orders every thread's atomics before thread 0's release; thread 0's acquire
+    // and the second barrier order the last piece's reads after all other pieces' atomics.
     named_bar_sync(1, kStreamConsumers);
-    if (ctid == 0) s_last = (atomicAdd(&a.done[unit], 1) == plan.S - 1);
+    if (ctid == 0) s_last = (atom_add_acq_rel_gpu(&a.done[unit], ke - kb) + (ke - kb) == nk);
     named_bar_sync(1, kStreamConsumers);
-    if (s_last && !aborted) {
-      __threadfence();
-      // the last split of this (chunk, tile): totals are complete, apply SwiGLU
+    if (s_last) {
       for (int i = ctid; i < nrows * (wg / 2); i += kStreamConsumers) {
         const int r = i / (wg / 2), cl = 2 * (i - r * (wg / 2));
         const float* p = a.acc + (size_t)(ch.y + r) * I2 + col0 + cl;
-        const float2 g = __ldcg(reinterpret_cast<const float2*>(p));
-        const float2 u = __ldcg(reinterpret_cast<const float2*>(p + a.I));
+        const float2 gs = __ldcg(reinterpret_cast<const float2*>(p));
+        const float2 us = __ldcg(reinterpret_cast<const float2*>(p + a.I));
         *reinterpret_cast<uint32_t*>(a.h + (size_t)(ch.y + r) * a.I + col0 + cl) =
-            pack_bf16x2(silu_f32(g.x) * u.x, silu_f32(g.y) * u.y);
+            pack_bf16x2(silu_f32(gs.x) * us.x, silu_f32(gs.y) * us.y);
       }
     }
   }
@@ -383,10 +369,8 @@ __global__ void __launch_bounds__(kStreamThreads, 1)
   __syncthreads();
 
   const int NT = (a.H + kStreamCols - 1) / kStreamCols;
-  const int units = a.sched[0] * NT;
   const int nk = a.I / kDownKC;
-  const SplitPlan plan = choose_splits(units, nk, gridDim.x, kStreamSplitMax);
-  const int items = units * plan.S;
+  const StreamKRange rng = stream_k_range((long long)a.sched[0] * NT, nk);
 
   if (warp == kStreamWarps) {
     if (lane == 0) tma_prefetch_desc(&wmap);
@@ -395,11 +379,12 @@ __global__ void __launch_bounds__(kStreamThreads, 1)
     int last_it[kStreamStages];
 #pragma unroll
     for (int s = 0; s < kStreamStages; ++s) last_it[s] = -1;
-    for (int id = blockIdx.x; id < items; id += gridDim.x) {
-      const int unit = id / plan.S, sp = id - unit * plan.S;
+    for (long long g = rng.g0; g < rng.g1;) {
+      const int unit = (int)(g / nk), kb = (int)(g % nk);
+      const int ke = (int)min((long long)nk, kb + (rng.g1 - g));
+      g += ke - kb;
       const int4 ch = a.chunks[unit / NT];
       const int col0 = (unit % NT) * kStreamCols;
-      const int kb = sp * plan.ks, ke = min(nk, kb + plan.ks);
       const uint32_t bytes = (uint32_t)kDNStageW + (uint32_t)ch.z * kDownKC * 2u;
       for (int kst = kb; kst < ke; ++kst, ++it) {
         const int slot = it % kStreamStages;
@@ -434,12 +419,13 @@ __global__ void __launch_bounds__(kStreamThreads, 1)
   const uint32_t wring_s = smem_u32(wring), xring_s = smem_u32(xring);
   bool aborted = false;
   uint32_t it = 0;
-  for (int id = blockIdx.x; id < items; id += gridDim.x) {
-    const int unit = id / plan.S, sp = id - unit * plan.S;
+  for (long long g = rng.g0; g < rng.g1;) {
+    const int unit = (int)(g / nk), kb = (int)(g % nk);
+    const int ke = (int)min((long long)nk, kb + (rng.g1 - g));
+    g += ke - kb;
     const int4 ch = a.chunks[unit / NT];
     const int col0 = (unit % NT) * kStreamCols;
     const int wc = min(kStreamCols, a.H - col0);
-    const int kb = sp * plan.ks, ke = min(nk, kb + plan.ks);
     const int nrows = ch.z;
     float acc[4][2][4];
 #pragma unroll
