@@ -21,7 +21,7 @@ LIB_PATH = os.path.join(_HERE, "libmoe.so")
 
 if not os.path.exists(LIB_PATH):
     raise ImportError(
-        f"{LIB_PATH} is missing: build it with `python -m mixture_experts_layer_48_b200.build` "
+        f"{LIB_PATH} is missing: build it with `python mixture_experts_layer_48_b200/build.py` "
         "(or __graft_entry__.build()); this package has no fallback")
 
 _lib = ctypes.CDLL(LIB_PATH)

@@ -1,6 +1,9 @@
 """Build step of the CUDA library: compiles csrc/ into libmoe.so (sm_100a) in this folder.
 
-    python -m mixture_experts_layer_48_b200.build [--verbose]
+    python mixture_experts_layer_48_b200/build.py [--verbose] [--force]
+
+Run it by path (or load it with load_builder()): importing the package itself loads libmoe.so,
+which must not be required to build it.
 
 nvcc cross-compiles for sm_100a without a GPU.  --verbose adds ``-Xptxas -v`` (registers,
 spills, shared memory per kernel).

@@ -19,8 +19,8 @@ def declared_symbols():
 
 @pytest.fixture(scope="module")
 def lib():
-    from mixture_experts_layer_48_b200 import build
-    build.build()
+    import __graft_entry__
+    __graft_entry__.load_builder().build()
     import mixture_experts_layer_48_b200 as m
     return m
 
