@@ -165,6 +165,29 @@ MOE_API moe_status moe_profile_begin(moe_t ctx, int max_calls);
 MOE_API moe_status moe_profile_end(moe_t ctx, float* ms, int* launches, int n_kinds);
 MOE_API const char* moe_profile_kind_name(int kind);
 
+/* Routing into the library's own device scratch, for callers that cannot allocate.
+ *
+ * No counterpart on the source pages: this is an interface convenience of this library.
+ * moe_route needs a caller-allocated workspace; some callers cannot provide one because they
+ * may not allocate device memory at call time (every device byte belongs to another
+ * allocator or pool, or allocation after start-up is forbidden, or the caller is plain C
+ * without an allocator).  moe_route_static computes exactly what moe_route computes, with
+ * the same arguments minus the workspace, and allocates nothing: its scratch is a fixed
+ * array of moe_route_static_max_bytes() bytes (2 MiB) compiled into the library, which every
+ * device that loads the library keeps until the process exits.
+ *   - The handle's device must be the current device (MOE_ERR_ARG otherwise).
+ *   - If moe_route_workspace_bytes(ctx, T) exceeds the array, the call returns
+ *     MOE_ERR_WORKSPACE and enqueues nothing (for H = 2880, E = 32: every T up to 2^20).
+ *   - The first call on a device looks up the array's device address (a runtime call that
+ *     does not allocate); make that first call before any stream capture.
+ *   - All calls share the one array: two calls whose work overlaps on the GPU (different
+ *     streams, or different handles on one device) race and give undefined results. */
+MOE_API size_t moe_route_static_max_bytes(void);
+MOE_API moe_status moe_route_static(moe_t ctx, int T, const void* x_bf16,
+                                    const void* W_router_bf16, const float* b_router,
+                                    int32_t* topk_idx, float* topk_w, int32_t* expert_offsets,
+                                    int32_t* perm, int32_t* inv_perm, moe_stream_t stream);
+
 /* Self-test of the device timeout path: launches one kernel that waits on a barrier nothing
  * completes, with a limit of `limit_us` microseconds (1..1000000), after which it sets the
  * status word and returns.  The next moe_sync_status then returns MOE_ERR_TIMEOUT.  No memory

@@ -53,6 +53,8 @@ _SIGS = {
                                  _c_int]),
     "moe_profile_kind_name": (ctypes.c_char_p, [_c_int]),
     "moe_selftest_timeout": (_c_int, [_vp, _c_int, _vp]),
+    "moe_route_static_max_bytes": (_sz, []),
+    "moe_route_static": (_c_int, [_vp, _c_int, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp]),
 }
 for _name, (_res, _args) in _SIGS.items():
     _f = getattr(_lib, _name)

@@ -9,6 +9,7 @@
 #include <cstdint>
 #include <cstring>
 #include <new>
+#include <mutex>
 #include <vector>
 
 #include "moe.h"
@@ -588,6 +589,98 @@ moe_status moe_selftest_timeout(moe_t c, int limit_us, moe_stream_t stream) {
   if (cudaGetLastError() != cudaSuccess) return MOE_ERR_CUDA;
   ++c->launches;
   return MOE_OK;
+}
+
+}  // extern "C"
+
+// ------------------------------------------------------------------------------------------
+// Routing without caller-provided device memory.
+//
+// Some callers cannot hand the library a workspace: code that runs where device allocation is
+// not allowed or not wanted at call time (a host process whose device memory is owned
+// entirely by another allocator or memory pool, a latency-critical serving loop that
+// forbids allocation after start-up, a plain C caller with no allocator of its own).  For
+// them, moe_route_static uses this fixed array in the library's own device memory instead.
+// Its size is fixed at build time; every device that loads the library holds it until the
+// process exits.  Calls share it, so two of them that overlap on the GPU race.
+// ------------------------------------------------------------------------------------------
+namespace {
+constexpr size_t kRouteStaticScratchBytes = size_t(2) << 20;  // 2 MiB
+constexpr int kMaxDevices = 64;
+}  // namespace
+
+static __device__ __align__(256) uint8_t g_route_static_scratch[kRouteStaticScratchBytes];
+
+namespace {
+std::mutex g_static_scratch_mu;
+void* g_static_scratch_addr[kMaxDevices] = {};
+
+// Device address of g_route_static_scratch on the current device.  In host code the array's
+// name only stands for the symbol, so the address is looked up once per device and cached.
+moe_status static_scratch_address(int dev, void** out) {
+  if (dev < 0 || dev >= kMaxDevices) return MOE_ERR_DEVICE;
+  std::lock_guard<std::mutex> lock(g_static_scratch_mu);
+  if (!g_static_scratch_addr[dev]) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_route_static_scratch) != cudaSuccess || p == nullptr) {
+      cudaGetLastError();
+      return MOE_ERR_CUDA;
+    }
+    g_static_scratch_addr[dev] = p;
+  }
+  *out = g_static_scratch_addr[dev];
+  return MOE_OK;
+}
+}  // namespace
+
+extern "C" {
+
+size_t moe_route_static_max_bytes(void) { return kRouteStaticScratchBytes; }
+
+moe_status moe_route_static(moe_t c, int T, const void* x_bf16, const void* W_router_bf16,
+                            const float* b_router, int32_t* topk_idx, float* topk_w,
+                            int32_t* expert_offsets, int32_t* perm, int32_t* inv_perm,
+                            moe_stream_t stream) {
+  MOE_TRY(check_common(c, T, x_bf16, W_router_bf16, b_router));
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  if (!expert_offsets || !aligned16(expert_offsets)) return MOE_ERR_ARG;
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess) {
+    cudaGetLastError();
+    return MOE_ERR_DEVICE;
+  }
+  if (dev != c->device) return MOE_ERR_ARG;
+  if (T == 0) {
+    if (cudaMemsetAsync(expert_offsets, 0, sizeof(int32_t) * (c->E + 1), st) != cudaSuccess)
+      return MOE_ERR_CUDA;
+    return MOE_OK;
+  }
+  if (!topk_idx || !topk_w || !perm || !inv_perm) return MOE_ERR_ARG;
+  if (!aligned16(topk_idx) || !aligned16(topk_w) || !aligned16(perm) || !aligned16(inv_perm))
+    return MOE_ERR_ARG;
+  if (route_ws_bytes(c, T) > kRouteStaticScratchBytes) return MOE_ERR_WORKSPACE;
+  void* scratch = nullptr;
+  MOE_TRY(static_scratch_address(dev, &scratch));
+  uint8_t* ws = static_cast<uint8_t*>(scratch);
+  Carver cv;
+  const size_t sched_at = cv.take(16);
+  const RouteTmp rt = carve_route_tmp(cv, c, T);
+  RouteOut o{};
+  o.topk_idx = topk_idx;
+  o.topk_w = topk_w;
+  o.offsets = expert_offsets;
+  o.perm = perm;
+  o.inv_perm = inv_perm;
+  o.row_w = nullptr;
+  o.chunks = nullptr;
+  o.sched = reinterpret_cast<int32_t*>(ws + sched_at);
+  o.chunk_rows = 1;
+  o.zero_i32 = nullptr;
+  o.n_zero = 0;
+  // Every scratch word the routing kernels read is written earlier in the same call (the
+  // partial logits or the per-block counts and totals), so nothing needs clearing.
+  return launch_route(c, T, static_cast<const uint16_t*>(x_bf16),
+                      static_cast<const uint16_t*>(W_router_bf16), b_router, o, ws, rt, st);
 }
 
 }  // extern "C"

@@ -1,0 +1,72 @@
+"""moe_route_static: routing for callers that cannot allocate device memory.
+
+Such callers (a process whose device memory all belongs to another allocator, a serving loop
+that forbids allocation after start-up, a C caller without an allocator) cannot pass the
+workspace moe_route needs.  moe_route_static uses a fixed scratch array built into the
+library instead.  This test calls it through the C ABI twice in a row and checks each result
+against moe_route with a caller workspace, to the routing tolerances the parity tests use.
+"""
+import ctypes
+
+import numpy as np
+import pytest
+import torch
+
+import moe_inputs as mi
+from parity_util import W_TOL
+
+pytestmark = pytest.mark.gpu
+
+if torch.cuda.is_available():
+    import mixture_experts_layer_48_b200 as moe
+
+
+def _outputs(T, k, E):
+    dev = "cuda"
+    return dict(topk_idx=torch.empty((T, k), dtype=torch.int32, device=dev),
+                topk_w=torch.empty((T, k), dtype=torch.float32, device=dev),
+                expert_offsets=torch.empty((E + 1,), dtype=torch.int32, device=dev),
+                perm=torch.empty((T * k,), dtype=torch.int32, device=dev),
+                inv_perm=torch.empty((T, k), dtype=torch.int32, device=dev))
+
+
+def _call_static(layer, d, o):
+    st = torch.cuda.current_stream().cuda_stream
+    return moe.moe_route_static(layer.handle, d["x"].shape[0], d["x"].data_ptr(),
+                                d["W_router"].data_ptr(), d["b_router"].data_ptr(),
+                                o["topk_idx"].data_ptr(), o["topk_w"].data_ptr(),
+                                o["expert_offsets"].data_ptr(), o["perm"].data_ptr(),
+                                o["inv_perm"].data_ptr(), st)
+
+
+@pytest.mark.parametrize("T", [16, 300])   # the single-block and the multi-block routing chain
+def test_static_scratch_route_matches_workspace_route(T):
+    E, H, k = 32, 2880, 4
+    d = mi.make_inputs(T, H, E, k, 64, seed=1234 + T, device="cuda", experts=False)
+    layer = moe.Moe(E, H, 64, k)
+    ref = {key: v.cpu().numpy() for key, v in layer.route(d["x"], d["W_router"], d["b_router"]).items()}
+    for _ in range(2):                       # two calls in a row share the one scratch array
+        o = _outputs(T, k, E)
+        for v in o.values():
+            v.fill_(-7)
+        assert _call_static(layer, d, o) == moe.MOE_OK
+        torch.cuda.synchronize()
+        got = {key: v.cpu().numpy() for key, v in o.items()}
+        for key in ("topk_idx", "expert_offsets", "perm", "inv_perm"):
+            assert np.array_equal(got[key], ref[key]), key
+        assert np.abs(got["topk_w"] - ref["topk_w"]).max() <= W_TOL
+    assert layer.sync_status() == moe.MOE_OK
+
+
+def test_static_scratch_rejects_sizes_beyond_its_array():
+    # 128 experts x 64 tokens of partial logits over 45 hidden slices need 1.47 MB: fits;
+    # 256 experts need 2.95 MB: more than the 2 MiB array, refused before any launch.
+    assert moe.moe_route_static_max_bytes() == 2 << 20
+    for E, ok in ((128, True), (256, False)):
+        layer = moe.Moe(E, 2880, 64, 4)
+        d = mi.make_inputs(64, 2880, E, 4, 64, seed=7, device="cuda", experts=False)
+        o = _outputs(64, 4, E)
+        assert (layer.route_workspace_bytes(64) <= moe.moe_route_static_max_bytes()) == ok
+        st = _call_static(layer, d, o)
+        assert st == (moe.MOE_OK if ok else moe.MOE_ERR_WORKSPACE)
+    torch.cuda.synchronize()
