@@ -16,6 +16,7 @@
 #include "common.cuh"
 #include "route.cuh"
 #include "stream.cuh"
+#include "gemm.cuh"
 
 using namespace moe;
 
@@ -24,7 +25,7 @@ namespace {
 constexpr int kMaxE = 256;
 constexpr int kMaxHI = 16384;
 constexpr int kMaxT = 1 << 20;
-constexpr int kDefaultCrossover = INT_MAX;  // until a measured value exists: always stream
+constexpr int kDefaultCrossover = 64;  // largest T streamed until moe_tune measures one
 constexpr int kMaxKernelsPerCall = 8;
 
 enum Kind { kKindRouter = 0, kKindRouteFin = 1, kKindGather = 2, kKindGateUp = 3,
@@ -32,15 +33,20 @@ enum Kind { kKindRouter = 0, kKindRouteFin = 1, kKindGather = 2, kKindGateUp = 3
 
 }  // namespace
 
-// A TMA descriptor for one weight tensor, re-encoded when the caller passes another pointer.
+// A TMA descriptor for one tensor, re-encoded when the pointer or the row count changes.
 struct MapCache {
   const void* ptr = nullptr;
+  uint64_t rows = 0;
   CUtensorMap map;
 };
 
+// Grouped-GEMM configurations: <mode, MMAs per K step, N per MMA, smem stages>.
+#define MOE_GEMM_GATE_UP 0, 2, 128, 4
+#define MOE_GEMM_DOWN 1, 1, 192, 5
+
 struct moe_ctx {
   int E, H, I, k;
-  MapCache gate_up_stream, down_stream;
+  MapCache gate_up_stream, down_stream, gate_up_gemm, x_perm_map, h_map;
   int device = 0;
   int num_sms = 148;
   moe_path path = MOE_PATH_AUTO;
@@ -109,10 +115,11 @@ bool encode_2d(CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols, u
 const CUtensorMap* cached_map(MapCache& mc, const void* ptr, uint64_t rows, uint64_t cols,
                               uint32_t box_rows, uint32_t box_cols,
                               CUtensorMapSwizzle swizzle = CU_TENSOR_MAP_SWIZZLE_128B) {
-  if (mc.ptr != ptr) {
+  if (mc.ptr != ptr || mc.rows != rows) {
     mc.ptr = nullptr;
     if (!encode_2d(&mc.map, ptr, rows, cols, box_rows, box_cols, swizzle)) return nullptr;
     mc.ptr = ptr;
+    mc.rows = rows;
   }
   return &mc.map;
 }
@@ -164,6 +171,33 @@ StreamLayout stream_layout(const moe_ctx* c, int T) {
   return L;
 }
 
+struct GemmLayout {
+  size_t topk_idx, topk_w, inv_perm, perm, row_w, offsets, sched, chunks, x_perm, h;
+  RouteTmp rt;
+  int max_chunks;
+  size_t total;
+};
+
+GemmLayout gemm_layout(const moe_ctx* c, int T) {
+  GemmLayout L{};
+  Carver cv;
+  const size_t R = (size_t)T * c->k;
+  L.max_chunks = (int)(R / kGemmBM) + c->E;
+  L.topk_idx = cv.take(4 * R);
+  L.topk_w = cv.take(4 * R);
+  L.inv_perm = cv.take(4 * R);
+  L.perm = cv.take(4 * R);
+  L.row_w = cv.take(4 * R);
+  L.offsets = cv.take(4 * (size_t)(c->E + 1));
+  L.sched = cv.take(16);
+  L.chunks = cv.take(16 * (size_t)L.max_chunks);
+  L.x_perm = cv.take(2 * R * c->H);
+  L.h = cv.take(2 * R * c->I);
+  L.rt = carve_route_tmp(cv, c, T);
+  L.total = cv.cur;
+  return L;
+}
+
 size_t route_ws_bytes(const moe_ctx* c, int T) {
   Carver cv;
   cv.take(16);  // sched
@@ -171,11 +205,11 @@ size_t route_ws_bytes(const moe_ctx* c, int T) {
   return cv.cur;
 }
 
+// The path is chosen on the host from T alone, so no device data is read.
 bool use_stream(const moe_ctx* c, int T) {
-  // The grouped-GEMM path is not part of this build yet: every T streams.
-  (void)c;
-  (void)T;
-  return true;
+  if (c->path == MOE_PATH_STREAM) return true;
+  if (c->path == MOE_PATH_GEMM) return false;
+  return T <= c->crossover;
 }
 
 // ---- launches ------------------------------------------------------------------------
@@ -269,6 +303,12 @@ bool set_smem_attrs() {
                              kGateUpSmem) == cudaSuccess;
   ok &= cudaFuncSetAttribute(stream_down_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              kDownSmem) == cudaSuccess;
+  ok &= cudaFuncSetAttribute(grouped_gemm_kernel<MOE_GEMM_GATE_UP>,
+                             cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             GemmCfg<2, 128, 4>::kSmem) == cudaSuccess;
+  ok &= cudaFuncSetAttribute(grouped_gemm_kernel<MOE_GEMM_DOWN>,
+                             cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             GemmCfg<1, 192, 5>::kSmem) == cudaSuccess;
   return ok;
 }
 
@@ -279,6 +319,147 @@ moe_status check_common(const moe_ctx* c, int T, const void* x, const void* Wr, 
   if (!x || !Wr || !b) return MOE_ERR_ARG;
   if (!aligned16(x) || !aligned16(Wr) || !aligned16(b)) return MOE_ERR_ARG;
   return MOE_OK;
+}
+
+moe_status forward_stream(moe_ctx* c, int T, const void* x_bf16, const void* W_router_bf16,
+                          const float* b_router, const void* W_gate_up_bf16,
+                          const void* W_down_bf16, float* out, uint8_t* ws, size_t ws_bytes,
+                          cudaStream_t st) {
+  const StreamLayout L = stream_layout(c, T);
+  if (ws_bytes < L.total) return MOE_ERR_WORKSPACE;
+  const size_t R = (size_t)T * c->k;
+  RouteOut o{};
+  o.topk_idx = reinterpret_cast<int32_t*>(ws + L.topk_idx);
+  o.topk_w = reinterpret_cast<float*>(ws + L.topk_w);
+  o.offsets = reinterpret_cast<int32_t*>(ws + L.offsets);
+  o.perm = reinterpret_cast<int32_t*>(ws + L.perm);
+  o.inv_perm = reinterpret_cast<int32_t*>(ws + L.inv_perm);
+  o.row_w = reinterpret_cast<float*>(ws + L.row_w);
+  o.chunks = reinterpret_cast<int4*>(ws + L.chunks);
+  o.sched = reinterpret_cast<int32_t*>(ws + L.sched);
+  o.chunk_rows = kStreamRB;
+  o.zero_i32 = reinterpret_cast<int32_t*>(ws + L.done);
+  o.n_zero = L.n_done;
+  const uint16_t* x = static_cast<const uint16_t*>(x_bf16);
+  moe_status s = launch_route(c, T, x, static_cast<const uint16_t*>(W_router_bf16), b_router, o,
+                              ws, L.rt, st, reinterpret_cast<float*>(ws + L.acc), R * 2 * c->I);
+  if (s == MOE_OK) {
+    GateUpArgs ga{};
+    ga.x = x;
+    ga.H = c->H;
+    ga.I = c->I;
+    ga.R = (int)R;
+    ga.perm = o.perm;
+    ga.chunks = o.chunks;
+    ga.sched = o.sched;
+    ga.acc = reinterpret_cast<float*>(ws + L.acc);
+    ga.done = o.zero_i32;
+    ga.h = reinterpret_cast<uint16_t*>(ws + L.h);
+    ga.out = out;
+    ga.out_elems = (size_t)T * c->H;
+    ga.status = c->d_status;
+    const CUtensorMap* m = cached_map(c->gate_up_stream, W_gate_up_bf16, (uint64_t)c->E * c->H,
+                                      2ull * c->I, kGateUpKC, kBox);
+    if (!m) s = MOE_ERR_CUDA;
+    else
+      s = launch(c, kKindGateUp, st, [&] {
+        stream_gate_up_kernel<<<c->num_sms, kStreamThreads, kGateUpSmem, st>>>(ga, *m);
+      });
+  }
+  if (s == MOE_OK) {
+    DownArgs da{};
+    da.h = reinterpret_cast<const uint16_t*>(ws + L.h);
+    da.H = c->H;
+    da.I = c->I;
+    da.R = (int)R;
+    da.perm = o.perm;
+    da.row_w = o.row_w;
+    da.chunks = o.chunks;
+    da.sched = o.sched;
+    da.out = out;
+    da.status = c->d_status;
+    const CUtensorMap* m = cached_map(c->down_stream, W_down_bf16, (uint64_t)c->E * c->I,
+                                      (uint64_t)c->H, kDownKC, kBox);
+    if (!m) s = MOE_ERR_CUDA;
+    else
+      s = launch(c, kKindDown, st, [&] {
+        stream_down_kernel<<<c->num_sms, kStreamThreads, kDownSmem, st>>>(da, *m);
+      });
+  }
+  return s;
+}
+
+moe_status forward_gemm(moe_ctx* c, int T, const void* x_bf16, const void* W_router_bf16,
+                        const float* b_router, const void* W_gate_up_bf16,
+                        const void* W_down_bf16, float* out, uint8_t* ws, size_t ws_bytes,
+                        cudaStream_t st) {
+  const GemmLayout L = gemm_layout(c, T);
+  if (ws_bytes < L.total) return MOE_ERR_WORKSPACE;
+  const size_t R = (size_t)T * c->k;
+  RouteOut o{};
+  o.topk_idx = reinterpret_cast<int32_t*>(ws + L.topk_idx);
+  o.topk_w = reinterpret_cast<float*>(ws + L.topk_w);
+  o.offsets = reinterpret_cast<int32_t*>(ws + L.offsets);
+  o.perm = reinterpret_cast<int32_t*>(ws + L.perm);
+  o.inv_perm = reinterpret_cast<int32_t*>(ws + L.inv_perm);
+  o.row_w = reinterpret_cast<float*>(ws + L.row_w);
+  o.chunks = reinterpret_cast<int4*>(ws + L.chunks);
+  o.sched = reinterpret_cast<int32_t*>(ws + L.sched);
+  o.chunk_rows = kGemmBM;
+  o.zero_i32 = nullptr;
+  o.n_zero = 0;
+  const uint16_t* x = static_cast<const uint16_t*>(x_bf16);
+  uint16_t* x_perm = reinterpret_cast<uint16_t*>(ws + L.x_perm);
+  uint16_t* h = reinterpret_cast<uint16_t*>(ws + L.h);
+  // the router kernel zero-fills `out`, which the down projection accumulates into
+  MOE_TRY(launch_route(c, T, x, static_cast<const uint16_t*>(W_router_bf16), b_router, o, ws,
+                       L.rt, st, out, (size_t)T * c->H));
+  MOE_TRY(launch(c, kKindGather, st, [&] {
+    gather_rows_kernel<<<(unsigned)((R + 7) / 8), 256, 0, st>>>(x, o.perm, (int)R, c->H, x_perm);
+  }));
+  const CUtensorMap* am = cached_map(c->x_perm_map, x_perm, R, (uint64_t)c->H, kGemmBM, 64);
+  const CUtensorMap* bm = cached_map(c->gate_up_gemm, W_gate_up_bf16, (uint64_t)c->E * c->H,
+                                     2ull * c->I, kGemmBK, 64);
+  if (!am || !bm) return MOE_ERR_CUDA;
+  GemmArgs g{};
+  g.K = c->H;
+  g.Ncols = c->I;
+  g.sub_stride = c->I;
+  g.w_rows = c->H;
+  g.chunks = o.chunks;
+  g.sched = o.sched;
+  g.h = h;
+  g.H = c->H;
+  g.status = c->d_status;
+  MOE_TRY(launch(c, kKindGateUp, st, [&] {
+    grouped_gemm_kernel<MOE_GEMM_GATE_UP>
+        <<<c->num_sms, kGemmThreads, GemmCfg<2, 128, 4>::kSmem, st>>>(g, *am, *bm);
+  }));
+  const CUtensorMap* hm = cached_map(c->h_map, h, R, (uint64_t)c->I, kGemmBM, 64);
+  const CUtensorMap* dm = cached_map(c->down_stream, W_down_bf16, (uint64_t)c->E * c->I,
+                                     (uint64_t)c->H, kDownKC, kBox);
+  if (!hm || !dm) return MOE_ERR_CUDA;
+  GemmArgs d{};
+  d.K = c->I;
+  d.Ncols = c->H;
+  d.sub_stride = 0;
+  d.w_rows = c->I;
+  d.chunks = o.chunks;
+  d.sched = o.sched;
+  d.perm = o.perm;
+  d.row_w = o.row_w;
+  d.out = out;
+  d.H = c->H;
+  d.status = c->d_status;
+  MOE_TRY(launch(c, kKindDown, st, [&] {
+    grouped_gemm_kernel<MOE_GEMM_DOWN>
+        <<<c->num_sms, kGemmThreads, GemmCfg<1, 192, 5>::kSmem, st>>>(d, *hm, *dm);
+  }));
+  return MOE_OK;
+}
+
+size_t forward_ws_bytes(const moe_ctx* c, int T) {
+  return use_stream(c, T) ? stream_layout(c, T).total : gemm_layout(c, T).total;
 }
 
 __global__ void selftest_timeout_kernel(uint32_t* status, uint64_t limit_ns) {
@@ -351,7 +532,7 @@ size_t moe_route_workspace_bytes(moe_t c, int T) {
 size_t moe_workspace_bytes(moe_t c, int T) {
   if (!c || T < 0 || T > kMaxT) return 0;
   if (T == 0) return 0;
-  return stream_layout(c, T).total;
+  return forward_ws_bytes(c, T);
 }
 
 moe_status moe_route(moe_t c, int T, const void* x_bf16, const void* W_router_bf16,
@@ -400,73 +581,16 @@ moe_status moe_forward(moe_t c, int T, const void* x_bf16, const void* W_router_
   if (!W_gate_up_bf16 || !W_down_bf16 || !out) return MOE_ERR_ARG;
   if (!aligned16(W_gate_up_bf16) || !aligned16(W_down_bf16) || !aligned16(out))
     return MOE_ERR_ARG;
+  if (!workspace || !aligned16(workspace)) return MOE_ERR_WORKSPACE;
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
-  if (c->path == MOE_PATH_GEMM) return MOE_ERR_UNSUPPORTED;
-  (void)use_stream;
-  const StreamLayout L = stream_layout(c, T);
-  if (!workspace || !aligned16(workspace) || ws_bytes < L.total) return MOE_ERR_WORKSPACE;
   uint8_t* ws = static_cast<uint8_t*>(workspace);
-  const size_t R = (size_t)T * c->k;
-
   c->in_call = c->prof_max > 0 && c->prof_calls < c->prof_max;
-  RouteOut o{};
-  o.topk_idx = reinterpret_cast<int32_t*>(ws + L.topk_idx);
-  o.topk_w = reinterpret_cast<float*>(ws + L.topk_w);
-  o.offsets = reinterpret_cast<int32_t*>(ws + L.offsets);
-  o.perm = reinterpret_cast<int32_t*>(ws + L.perm);
-  o.inv_perm = reinterpret_cast<int32_t*>(ws + L.inv_perm);
-  o.row_w = reinterpret_cast<float*>(ws + L.row_w);
-  o.chunks = reinterpret_cast<int4*>(ws + L.chunks);
-  o.sched = reinterpret_cast<int32_t*>(ws + L.sched);
-  o.chunk_rows = kStreamRB;
-  o.zero_i32 = reinterpret_cast<int32_t*>(ws + L.done);
-  o.n_zero = L.n_done;
-  const uint16_t* x = static_cast<const uint16_t*>(x_bf16);
-  moe_status s = launch_route(c, T, x, static_cast<const uint16_t*>(W_router_bf16), b_router, o,
-                              ws, L.rt, st, reinterpret_cast<float*>(ws + L.acc), R * 2 * c->I);
-  if (s == MOE_OK) {
-    GateUpArgs ga{};
-    ga.x = x;
-    ga.H = c->H;
-    ga.I = c->I;
-    ga.R = (int)R;
-    ga.perm = o.perm;
-    ga.chunks = o.chunks;
-    ga.sched = o.sched;
-    ga.acc = reinterpret_cast<float*>(ws + L.acc);
-    ga.done = o.zero_i32;
-    ga.h = reinterpret_cast<uint16_t*>(ws + L.h);
-    ga.out = out;
-    ga.out_elems = (size_t)T * c->H;
-    ga.status = c->d_status;
-    const CUtensorMap* m = cached_map(c->gate_up_stream, W_gate_up_bf16, (uint64_t)c->E * c->H,
-                                      2ull * c->I, kGateUpKC, kBox);
-    if (!m) s = MOE_ERR_CUDA;
-    else
-      s = launch(c, kKindGateUp, st, [&] {
-        stream_gate_up_kernel<<<c->num_sms, kStreamThreads, kGateUpSmem, st>>>(ga, *m);
-      });
-  }
-  if (s == MOE_OK) {
-    DownArgs da{};
-    da.h = reinterpret_cast<const uint16_t*>(ws + L.h);
-    da.H = c->H;
-    da.I = c->I;
-    da.R = (int)R;
-    da.perm = o.perm;
-    da.row_w = o.row_w;
-    da.chunks = o.chunks;
-    da.sched = o.sched;
-    da.out = out;
-    da.status = c->d_status;
-    const CUtensorMap* m = cached_map(c->down_stream, W_down_bf16, (uint64_t)c->E * c->I,
-                                      (uint64_t)c->H, kDownKC, kBox);
-    if (!m) s = MOE_ERR_CUDA;
-    else
-      s = launch(c, kKindDown, st, [&] {
-        stream_down_kernel<<<c->num_sms, kStreamThreads, kDownSmem, st>>>(da, *m);
-      });
-  }
+  const moe_status s =
+      use_stream(c, T)
+          ? forward_stream(c, T, x_bf16, W_router_bf16, b_router, W_gate_up_bf16, W_down_bf16,
+                           out, ws, ws_bytes, st)
+          : forward_gemm(c, T, x_bf16, W_router_bf16, b_router, W_gate_up_bf16, W_down_bf16,
+                         out, ws, ws_bytes, st);
   if (c->in_call) ++c->prof_calls;
   c->in_call = false;
   return s;
@@ -476,7 +600,6 @@ moe_status moe_set_path(moe_t c, moe_path path, int crossover_T) {
   if (!c) return MOE_ERR_ARG;
   if (path != MOE_PATH_AUTO && path != MOE_PATH_STREAM && path != MOE_PATH_GEMM)
     return MOE_ERR_ARG;
-  if (path == MOE_PATH_GEMM) return MOE_ERR_UNSUPPORTED;
   c->path = path;
   if (crossover_T >= 0) c->crossover = crossover_T;
   return MOE_OK;

@@ -95,10 +95,6 @@ struct DownArgs {
 
 MOE_DEVINL void record_timeout(uint32_t* status) { atomicOr(status, kStatusTimeout); }
 
-MOE_DEVINL uint8_t* align1k(uint8_t* p) {
-  return reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(p) + 1023) & ~uintptr_t(1023));
-}
-
 // Byte offset, inside a [rows][64] bf16 box stored with the 128-byte swizzle, of the 16-byte
 // chunk that lane provides to ldmatrix.x4.trans for m-tile mt (16 columns) and k-step ks
 // (16 rows).  Matrices: 0 (cols 0-7, rows 0-7), 1 (cols 8-15, rows 0-7), 2 (cols 0-7,

@@ -16,8 +16,10 @@ if torch.cuda.is_available():
     import mixture_experts_layer_48_b200 as moe
 
 
-def _check_layer(d, h, E, H, I, k, layer=None):
+def _check_layer(d, h, E, H, I, k, layer=None, path=None):
     layer = layer or moe.Moe(E, H, I, k)
+    if path is not None:
+        layer.set_path(path)
     T = d["x"].shape[0]
     ref_route = host_route(h, k)
     g = gpu_route(layer, d)
@@ -142,3 +144,19 @@ def test_profile_counts_kernels():
     assert layer.launch_count() - n0 == sum(v[1] for v in prof.values())
     assert prof["gate_up_swiglu"][1] == 3 and prof["down_combine"][1] == 3
     assert all(v[0] >= 0 for v in prof.values())
+
+
+@pytest.mark.parametrize("T", [1, 5, 16, 64, 65, 200, 520])
+@pytest.mark.parametrize("path", ["stream", "gemm"])
+def test_both_paths_match_the_oracle(T, path):
+    """Either path at any T: the streaming kernels and the tcgen05 grouped GEMM."""
+    p = moe.MOE_PATH_STREAM if path == "stream" else moe.MOE_PATH_GEMM
+    d, h = inputs_on_gpu(T, 256, 8, 2, 320, seed=1000 + T)
+    _check_layer(d, h, 8, 256, 320, 2, path=p)
+
+
+@pytest.mark.parametrize("path", ["stream", "gemm"])
+def test_both_paths_gpt_oss_shape(path):
+    p = moe.MOE_PATH_STREAM if path == "stream" else moe.MOE_PATH_GEMM
+    d, h = inputs_on_gpu(300, 2880, 32, 4, 2880, seed=1100)
+    _check_layer(d, h, 32, 2880, 2880, 4, path=p)
