@@ -134,7 +134,7 @@ RouteTmp carve_route_tmp(Carver& cv, const moe_ctx* c, int T) {
   if (T <= kSmallT) {
     r.partial = cv.take(sizeof(float) * (size_t)(c->H / kRouterHSlice) * T * c->E);
   } else {
-    const size_t NB = (T + kRouteTile - 1) / kRouteTile;
+    const size_t NB = (T + kRouterTcTokens - 1) / kRouterTcTokens;
     r.block_counts = cv.take(sizeof(int32_t) * NB * c->E);
     r.totals = cv.take(sizeof(int32_t) * c->E);
   }
@@ -235,6 +235,14 @@ moe_status launch(moe_ctx* c, int kind, cudaStream_t st, F&& f) {
     if (_s != MOE_OK) return _s;         \
   } while (0)
 
+template <int NT8>
+void launch_router_tc(int NB, cudaStream_t st, const uint16_t* x, const uint16_t* Wr,
+                      const float* b, int T, int H, int E, int k, const RouteOut& o,
+                      int32_t* block_counts, float4* zero4, size_t n_zero4) {
+  router_topk_kernel<NT8><<<NB, 128, RouterTcCfg<NT8>::smem(k), st>>>(
+      x, Wr, b, T, H, E, k, o.topk_idx, o.topk_w, block_counts, zero4, n_zero4);
+}
+
 // Routing chain.  zero4/n_zero4: a float scratch region the router kernel zero-fills.
 moe_status launch_route(moe_ctx* c, int T, const uint16_t* x, const uint16_t* Wr,
                         const float* b, const RouteOut& o, uint8_t* ws, const RouteTmp& rt,
@@ -257,28 +265,23 @@ moe_status launch_route(moe_ctx* c, int T, const uint16_t* x, const uint16_t* Wr
     }));
     return MOE_OK;
   }
-  const int NB = (T + kRouteTile - 1) / kRouteTile;
+  const int NB = (T + kRouterTcTokens - 1) / kRouterTcTokens;
   int32_t* block_counts = reinterpret_cast<int32_t*>(ws + rt.block_counts);
   int32_t* totals = reinterpret_cast<int32_t*>(ws + rt.totals);
-  const int EPW = E <= 32 ? 4 : (E <= 128 ? 16 : 32);
-  const int EP = 8 * EPW;
-  const size_t smem_r = (size_t)kRouterHSlice * kRouteTile * 2 + (size_t)kRouterHSlice * EP * 2 +
-                        (size_t)kRouteTile * EP * 4 + (size_t)EP * 4 + (size_t)kRouteTile * k * 4;
+  const int nt8 = (E + 7) / 8;
   MOE_TRY(launch(c, kKindRouter, st, [&] {
-    if (EPW == 4)
-      router_topk_kernel<4><<<NB, 256, smem_r, st>>>(x, Wr, b, T, H, E, k, o.topk_idx, o.topk_w,
-                                                      block_counts, zero4, n_zero4);
-    else if (EPW == 16)
-      router_topk_kernel<16><<<NB, 256, smem_r, st>>>(x, Wr, b, T, H, E, k, o.topk_idx, o.topk_w,
-                                                       block_counts, zero4, n_zero4);
-    else
-      router_topk_kernel<32><<<NB, 256, smem_r, st>>>(x, Wr, b, T, H, E, k, o.topk_idx, o.topk_w,
-                                                       block_counts, zero4, n_zero4);
+    if (nt8 <= 1) launch_router_tc<1>(NB, st, x, Wr, b, T, H, E, k, o, block_counts, zero4, n_zero4);
+    else if (nt8 <= 2) launch_router_tc<2>(NB, st, x, Wr, b, T, H, E, k, o, block_counts, zero4, n_zero4);
+    else if (nt8 <= 4) launch_router_tc<4>(NB, st, x, Wr, b, T, H, E, k, o, block_counts, zero4, n_zero4);
+    else if (nt8 <= 8) launch_router_tc<8>(NB, st, x, Wr, b, T, H, E, k, o, block_counts, zero4, n_zero4);
+    else if (nt8 <= 16) launch_router_tc<16>(NB, st, x, Wr, b, T, H, E, k, o, block_counts, zero4, n_zero4);
+    else launch_router_tc<32>(NB, st, x, Wr, b, T, H, E, k, o, block_counts, zero4, n_zero4);
   }));
   MOE_TRY(launch(c, kKindRouteFin, st, [&] {
     route_scan_kernel<<<E, 256, 0, st>>>(block_counts, NB, E, totals);
   }));
-  const size_t smem_s = (256 + 257 + 257) * 4 + (size_t)kRouteTile * 8 * 4 + (size_t)kRouteTile * E;
+  const size_t smem_s = (256 + 257 + 257) * 4 + (size_t)kRouterTcTokens * 8 * 4 +
+                        (size_t)kRouterTcTokens * E;
   MOE_TRY(launch(c, kKindRouteFin, st, [&] {
     route_scatter_kernel<<<NB, 256, smem_s, st>>>(o.topk_idx, o.topk_w, block_counts, totals, T,
                                                   E, k, o);
@@ -291,7 +294,13 @@ bool set_smem_attrs() {
   bool ok = true;
   ok &= cudaFuncSetAttribute(route_small_finalize_kernel,
                              cudaFuncAttributeMaxDynamicSharedMemorySize, big) == cudaSuccess;
+  ok &= cudaFuncSetAttribute(router_topk_kernel<1>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             big) == cudaSuccess;
+  ok &= cudaFuncSetAttribute(router_topk_kernel<2>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             big) == cudaSuccess;
   ok &= cudaFuncSetAttribute(router_topk_kernel<4>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             big) == cudaSuccess;
+  ok &= cudaFuncSetAttribute(router_topk_kernel<8>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              big) == cudaSuccess;
   ok &= cudaFuncSetAttribute(router_topk_kernel<16>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              big) == cudaSuccess;
@@ -411,12 +420,19 @@ moe_status forward_gemm(moe_ctx* c, int T, const void* x_bf16, const void* W_rou
   const uint16_t* x = static_cast<const uint16_t*>(x_bf16);
   uint16_t* x_perm = reinterpret_cast<uint16_t*>(ws + L.x_perm);
   uint16_t* h = reinterpret_cast<uint16_t*>(ws + L.h);
+  if (T > kSmallT) {  // the large-T scatter also writes the rows in expert order
+    o.x = x;
+    o.x_perm = x_perm;
+    o.H = c->H;
+  }
   // the router kernel zero-fills `out`, which the down projection accumulates into
   MOE_TRY(launch_route(c, T, x, static_cast<const uint16_t*>(W_router_bf16), b_router, o, ws,
                        L.rt, st, out, (size_t)T * c->H));
-  MOE_TRY(launch(c, kKindGather, st, [&] {
-    gather_rows_kernel<<<(unsigned)((R + 7) / 8), 256, 0, st>>>(x, o.perm, (int)R, c->H, x_perm);
-  }));
+  if (T <= kSmallT)
+    MOE_TRY(launch(c, kKindGather, st, [&] {
+      gather_rows_kernel<<<(unsigned)((R + 7) / 8), 256, 0, st>>>(x, o.perm, (int)R, c->H,
+                                                                 x_perm);
+    }));
   const CUtensorMap* am = cached_map(c->x_perm_map, x_perm, R, (uint64_t)c->H, kGemmBM, 64);
   const CUtensorMap* bm = cached_map(c->gate_up_gemm, W_gate_up_bf16, (uint64_t)c->E * c->H,
                                      2ull * c->I, kGemmBK, 64);

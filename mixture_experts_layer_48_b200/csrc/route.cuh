@@ -9,9 +9,10 @@
 //   T <= kSmallT : router_partial_kernel (H/64 blocks, one 64-row slice of W_router each)
 //                  -> route_small_finalize_kernel (one block: sum, top-k, softmax,
 //                     histogram, scan, permutation, work list).
-//   T >  kSmallT : router_topk_kernel (32 tokens per block, all experts, full H; top-k and a
-//                  block histogram) -> route_scan_kernel (one block per expert: prefix over
-//                  blocks) -> route_scatter_kernel (32 tokens per block: permutation).
+//   T >  kSmallT : router_topk_kernel (64 tokens per block, all experts on the tensor cores;
+//                  top-k and a block histogram) -> route_scan_kernel (one block per expert:
+//                  prefix over blocks) -> route_scatter_kernel (permutation, 64 tokens per
+//                  block, two 32-token ballot passes).
 #pragma once
 
 #include "common.cuh"
@@ -35,6 +36,9 @@ struct RouteOut {
   int chunk_rows;      // rows per work-list entry
   int32_t* zero_i32;   // region zeroed by the chain (completion counters), may be null
   int n_zero;
+  const uint16_t* x;   // with x_perm non-null: copy token rows into expert order
+  uint16_t* x_perm;    // [T * k, H]
+  int H;
 };
 
 // ---------------------------------------------------------------------------------------
@@ -248,74 +252,143 @@ __global__ void __launch_bounds__(1024)
 }
 
 // ---------------------------------------------------------------------------------------
-// Large T, step 1: logits of 32 tokens x all E experts over the full H, then top-k,
-// softmax and the block's expert histogram.  grid ceil(T/32), block 256.
-// Thread (warp w, lane l) owns token l of the tile and experts [w*EPW, (w+1)*EPW).
+// Large T, step 1: logits of 64 tokens x all experts on the tensor cores, then top-k, softmax
+// and the block's expert histogram.  grid ceil(T/64), block 128 (4 warps x 16 tokens).
+// x[64 tokens x 64] and W_router[64 x E] chunks stream through a 4-deep cp.async ring; each warp multiplies its 16 tokens with all experts (mma.sync m16n8k16, bf16 in,
+// fp32 accumulate).  Reading x once is the cost, so the kernel runs at memory speed.
+// NT8 = experts / 8 rounded up to a power of two; padding experts are zero and never chosen.
 // ---------------------------------------------------------------------------------------
-template <int EPW>
-__global__ void __launch_bounds__(256)
+constexpr int kRouterTcTokens = 64;
+constexpr int kRouterTcXPitch = 72;  // elements; 144-byte rows keep ldmatrix conflict-free
+
+template <int NT8>
+struct RouterTcCfg {
+  // cp.async ring depth (chunks of 64 hidden rows); wide expert sets keep two to fit in smem
+  static constexpr int kStages = NT8 >= 16 ? 2 : 4;
+  static constexpr int EP = NT8 * 8;
+  static constexpr int WP = EP + 8;
+  static constexpr int kXBytes = kStages * kRouterTcTokens * kRouterTcXPitch * 2;
+  static constexpr int kWBytes = kStages * kRouterHSlice * WP * 2;
+  static constexpr int kLgBytes = kRouterTcTokens * (EP + 1) * 4;
+  static size_t smem(int k) { return kXBytes + kWBytes + kLgBytes + EP * 4 + (size_t)kRouterTcTokens * k * 4; }
+};
+
+MOE_DEVINL void cp_async16(void* smem_dst, const void* gsrc, bool valid) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(smem_u32(smem_dst)),
+               "l"(gsrc), "r"(valid ? 16 : 0)
+               : "memory");
+}
+MOE_DEVINL void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+template <int N>
+MOE_DEVINL void cp_async_wait() {
+  asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
+}
+
+template <int NT8>
+__global__ void __launch_bounds__(128)
     router_topk_kernel(const uint16_t* __restrict__ x, const uint16_t* __restrict__ Wr,
                        const float* __restrict__ b_router, int T, int H, int E, int k,
                        int32_t* __restrict__ topk_idx, float* __restrict__ topk_w,
                        int32_t* __restrict__ block_counts, float4* zero4, size_t n_zero4) {
-  zero_fill_f4(zero4, n_zero4);
+  using C = RouterTcCfg<NT8>;
+  constexpr int EP = C::EP, WP = C::WP, XP = kRouterTcXPitch, TT = kRouterTcTokens;
   extern __shared__ __align__(128) uint8_t smem_raw[];
-  uint16_t* xsT = reinterpret_cast<uint16_t*>(smem_raw);          // [64][32] (h-major)
-  uint16_t* ws = xsT + kRouterHSlice * kRouteTile;                  // [64][8*EPW]
-  const int EP = 8 * EPW;                                           // padded expert count
-  float* lg = reinterpret_cast<float*>(ws + kRouterHSlice * EP);    // [32][EP]
-  int32_t* cnt = reinterpret_cast<int32_t*>(lg + kRouteTile * EP);  // [EP]
-  int32_t* sel = cnt + EP;                                          // [32][k]
+  uint16_t* xs = reinterpret_cast<uint16_t*>(smem_raw);                // [stages][64][XP]
+  uint16_t* wsm = reinterpret_cast<uint16_t*>(smem_raw + C::kXBytes);   // [stages][64][WP]
+  float* lg = reinterpret_cast<float*>(smem_raw + C::kXBytes + C::kWBytes);  // [64][EP+1]
+  int32_t* cnt = reinterpret_cast<int32_t*>(lg + TT * (EP + 1));            // [EP]
+  int32_t* sel = cnt + EP;                                                   // [64][k]
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const int t0 = blockIdx.x * kRouteTile, nt = min(kRouteTile, T - t0);
+  const int t0 = blockIdx.x * TT, nt = min(TT, T - t0);
+  const int nk = H / kRouterHSlice;
+  const bool vec_w = (E % 8) == 0;
 
-  float acc[EPW];
-#pragma unroll
-  for (int m = 0; m < EPW; ++m) acc[m] = 0.f;
+  zero_fill_f4(zero4, n_zero4);
   for (int i = tid; i < EP; i += blockDim.x) cnt[i] = 0;
+  for (int i = tid; i < C::kStages * kRouterHSlice * WP; i += blockDim.x)
+    wsm[i] = 0;  // padding experts stay zero
+  __syncthreads();
 
-  for (int h0 = 0; h0 < H; h0 += kRouterHSlice) {
-    {  // x tile, transposed to [h][t]
-      const int r = tid >> 3, c = tid & 7;  // 32 tokens x 8 chunks of 8
-      uint4 v = make_uint4(0, 0, 0, 0);
-      if (r < nt) v = reinterpret_cast<const uint4*>(x + (size_t)(t0 + r) * H + h0)[c];
-      const uint16_t* pv = reinterpret_cast<const uint16_t*>(&v);
-#pragma unroll
-      for (int q = 0; q < 8; ++q) xsT[(c * 8 + q) * kRouteTile + r] = pv[q];
+  auto load_chunk = [&](int kc, int buf) {
+    const int h0 = kc * kRouterHSlice;
+    uint16_t* xb = xs + buf * TT * XP;
+    for (int i = tid; i < TT * 8; i += blockDim.x) {  // 64 rows x 8 pieces of 16 B
+      const int r = i >> 3, c = i & 7;
+      const bool ok = r < nt;
+      cp_async16(xb + r * XP + c * 8, x + (size_t)(t0 + (ok ? r : 0)) * H + h0 + c * 8, ok);
     }
-    for (int i = tid; i < kRouterHSlice * EP; i += blockDim.x) {
-      const int hh = i / EP, e = i - hh * EP;
-      ws[i] = (e < E) ? Wr[(size_t)(h0 + hh) * E + e] : uint16_t(0);
-    }
-    __syncthreads();
-#pragma unroll 4
-    for (int hh = 0; hh < kRouterHSlice; ++hh) {
-      const float xv = bf16_to_f32(xsT[hh * kRouteTile + lane]);
-      const uint16_t* wrow = ws + hh * EP + warp * EPW;
-      if constexpr (EPW % 4 == 0) {
-#pragma unroll
-        for (int m = 0; m < EPW; m += 4) {
-          const uint2 wv = *reinterpret_cast<const uint2*>(wrow + m);
-          acc[m + 0] = fmaf(xv, bf16lo(wv.x), acc[m + 0]);
-          acc[m + 1] = fmaf(xv, bf16hi(wv.x), acc[m + 1]);
-          acc[m + 2] = fmaf(xv, bf16lo(wv.y), acc[m + 2]);
-          acc[m + 3] = fmaf(xv, bf16hi(wv.y), acc[m + 3]);
-        }
-      } else {
-#pragma unroll
-        for (int m = 0; m < EPW; ++m) acc[m] = fmaf(xv, bf16_to_f32(wrow[m]), acc[m]);
+    uint16_t* wb = wsm + buf * kRouterHSlice * WP;
+    if (vec_w) {
+      const int per_row = E / 8;
+      for (int i = tid; i < kRouterHSlice * per_row; i += blockDim.x) {
+        const int r = i / per_row, c = i - r * per_row;
+        cp_async16(wb + r * WP + c * 8, Wr + (size_t)(h0 + r) * E + c * 8, true);
+      }
+    } else {
+      for (int i = tid; i < kRouterHSlice * E; i += blockDim.x) {
+        const int r = i / E, c = i - r * E;
+        wb[r * WP + c] = Wr[(size_t)(h0 + r) * E + c];
       }
     }
-    __syncthreads();
-  }
+  };
+
+  float acc[NT8][4];
 #pragma unroll
-  for (int m = 0; m < EPW; ++m) {
-    const int e = warp * EPW + m;
-    if (e < E) lg[lane * EP + e] = acc[m] + b_router[e];
+  for (int n = 0; n < NT8; ++n) acc[n][0] = acc[n][1] = acc[n][2] = acc[n][3] = 0.f;
+
+  // prologue: stages-1 chunks in flight; every iteration commits one group (maybe empty)
+#pragma unroll
+  for (int p = 0; p < C::kStages - 1; ++p) {
+    if (p < nk) load_chunk(p, p);
+    cp_async_commit();
   }
+  for (int kc = 0; kc < nk; ++kc) {
+    const int buf = kc % C::kStages;
+    cp_async_wait<C::kStages - 2>();       // chunk kc has landed
+    __syncthreads();                       // ... for every thread; buffer kc-1 is free again
+    {
+      const int nx = kc + C::kStages - 1;
+      if (nx < nk) load_chunk(nx, nx % C::kStages);
+      cp_async_commit();
+    }
+    const uint32_t xb = smem_u32(xs + buf * TT * XP);
+    const uint32_t wb = smem_u32(wsm + buf * kRouterHSlice * WP);
+#pragma unroll
+    for (int k16 = 0; k16 < kRouterHSlice / 16; ++k16) {
+      const int i = lane >> 3, j = lane & 7;
+      uint32_t a0, a1, a2, a3;
+      ldsm_x4(xb + ((16 * warp + (i & 1) * 8 + j) * XP + k16 * 16 + (i >> 1) * 8) * 2, a0, a1, a2,
+              a3);
+#pragma unroll
+      for (int n = 0; n < NT8; n += 2) {
+        // matrices 0/1: experts [8n, 8n+8) at k 0-7 / 8-15; 2/3: experts [8n+8, 8n+16)
+        const int krow = k16 * 16 + (i & 1) * 8 + j;
+        const int ncol = 8 * n + ((i >> 1) & 1) * 8;
+        uint32_t b0, b1, b2, b3;
+        if constexpr (NT8 == 1) {
+          ldsm_x2_trans(wb + (krow * WP + ncol) * 2, b0, b1);
+          mma_bf16_16816(acc[n], a0, a1, a2, a3, b0, b1);
+        } else {
+          ldsm_x4_trans(wb + (krow * WP + ncol) * 2, b0, b1, b2, b3);
+          mma_bf16_16816(acc[n], a0, a1, a2, a3, b0, b1);
+          mma_bf16_16816(acc[n + 1], a0, a1, a2, a3, b2, b3);
+        }
+      }
+    }
+  }
+  cp_async_wait<0>();
+  // C fragment: c0,c1 -> token 16w + lane/4, experts 8n + 2(lane%4) + {0,1}; c2,c3 -> token + 8
+#pragma unroll
+  for (int n = 0; n < NT8; ++n)
+#pragma unroll
+    for (int v = 0; v < 4; ++v) {
+      const int tt = 16 * warp + (lane >> 2) + 8 * (v >> 1);
+      const int e = 8 * n + 2 * (lane & 3) + (v & 1);
+      if (e < E) lg[tt * (EP + 1) + e] = acc[n][v] + b_router[e];
+    }
   __syncthreads();
-  for (int tt = warp; tt < nt; tt += 8) {
-    float* row = lg + tt * EP;
+  for (int tt = warp; tt < nt; tt += 4) {
+    float* row = lg + tt * (EP + 1);
     int32_t* srow = sel + tt * k;
     warp_topk(row, E, k, srow);
     const float denom = warp_softmax_denominator(row, k);
@@ -365,25 +438,27 @@ __global__ void __launch_bounds__(256) route_scan_kernel(int32_t* __restrict__ b
 }
 
 // ---------------------------------------------------------------------------------------
-// Large T, step 3: stable scatter.  Block b handles tokens [32b, 32b+32); warp w takes
-// experts w, w+8, ...; lane = token, so a ballot gives each token its rank among the block's
-// earlier tokens that chose the same expert.  block 256.
+// Large T, step 3: stable scatter.  Block b handles the router's tokens [64b, 64b+64); warp w
+// takes experts w, w+8, ...; in two passes lane = token (first and second 32 tokens), and a
+// ballot gives each token its rank among the block's earlier tokens that chose the expert.
+// block 256.
 // ---------------------------------------------------------------------------------------
 __global__ void __launch_bounds__(256)
     route_scatter_kernel(const int32_t* __restrict__ topk_idx, const float* __restrict__ topk_w,
                          const int32_t* __restrict__ block_base,
                          const int32_t* __restrict__ totals, int T, int E, int k, RouteOut o) {
+  constexpr int TT = kRouterTcTokens;
   extern __shared__ __align__(128) uint8_t smem_raw[];
   int32_t* cnt = reinterpret_cast<int32_t*>(smem_raw);  // [256]
   int32_t* off = cnt + 256;                             // [257]
   int32_t* scratch = off + 257;                         // [257]
-  uint32_t* bits = reinterpret_cast<uint32_t*>(scratch + 257);  // [32][8]
-  uint8_t* slot = reinterpret_cast<uint8_t*>(bits + kRouteTile * 8);  // [32][E] (k <= 256)
+  uint32_t* bits = reinterpret_cast<uint32_t*>(scratch + 257);  // [64][8]
+  uint8_t* slot = reinterpret_cast<uint8_t*>(bits + TT * 8);    // [64][E] (k <= 256)
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const int t0 = blockIdx.x * kRouteTile, nt = min(kRouteTile, T - t0);
+  const int t0 = blockIdx.x * TT, nt = min(TT, T - t0);
 
   for (int e = tid; e < E; e += blockDim.x) cnt[e] = totals[e];
-  for (int i = tid; i < kRouteTile * 8; i += blockDim.x) bits[i] = 0u;
+  for (int i = tid; i < TT * 8; i += blockDim.x) bits[i] = 0u;
   __syncthreads();
   if (tid == 0) {
     int run = 0;
@@ -403,24 +478,44 @@ __global__ void __launch_bounds__(256)
   if (blockIdx.x == 0)
     for (int e = tid; e <= E; e += blockDim.x) o.offsets[e] = off[e];
   for (int e = warp; e < E; e += 8) {
-    const bool chose = lane < nt && (bits[lane * 8 + (e >> 5)] & (1u << (e & 31)));
-    const uint32_t mask = __ballot_sync(0xffffffffu, chose);
-    if (chose) {
-      const int rank = __popc(mask & ((1u << lane) - 1u));
-      const int r = off[e] + block_base[(size_t)blockIdx.x * E + e] + rank;
-      const int t = t0 + lane;
-      const int j = slot[lane * E + e];
-      o.perm[r] = t;
-      o.inv_perm[(size_t)t * k + j] = r;
-      if (o.row_w) o.row_w[r] = topk_w[(size_t)t * k + j];
+    const int base = off[e] + block_base[(size_t)blockIdx.x * E + e];
+    int before = 0;  // tokens of the first pass that chose e
+#pragma unroll
+    for (int half = 0; half < 2; ++half) {
+      const int tt = half * 32 + lane;
+      const bool chose = tt < nt && (bits[tt * 8 + (e >> 5)] & (1u << (e & 31)));
+      const uint32_t mask = __ballot_sync(0xffffffffu, chose);
+      if (chose) {
+        const int r = base + before + __popc(mask & ((1u << lane) - 1u));
+        const int t = t0 + tt;
+        const int j = slot[tt * E + e];
+        o.perm[r] = t;
+        o.inv_perm[(size_t)t * k + j] = r;
+        if (o.row_w) o.row_w[r] = topk_w[(size_t)t * k + j];
+      }
+      before += __popc(mask);
     }
   }
   if (blockIdx.x == 0) build_work_list(cnt, off, E, o, scratch);
   for (int i = blockIdx.x * blockDim.x + tid; i < o.n_zero; i += gridDim.x * blockDim.x)
     o.zero_i32[i] = 0;
+  if (o.x_perm) {
+    // rows in expert order for the grouped GEMM: each token's row is read once and written to
+    // its k rows (inv_perm of this block's tokens was written above by this block)
+    __syncthreads();
+    const int n16 = o.H / 8;  // 16-byte pieces per row
+#pragma unroll 4
+    for (int i = tid; i < nt * n16; i += blockDim.x) {
+      const int tt = i / n16, c = i - tt * n16;
+      const size_t t = (size_t)(t0 + tt);
+      const uint4 v = reinterpret_cast<const uint4*>(o.x + t * o.H)[c];
+      for (int j = 0; j < k; ++j)
+        reinterpret_cast<uint4*>(o.x_perm + (size_t)o.inv_perm[t * k + j] * o.H)[c] = v;
+    }
+  }
 }
 
-// Gather of token rows into expert order for the grouped GEMM: x_perm[r] = x[perm[r]].
+// Rows in expert order for the grouped GEMM when T is small: x_perm[r] = x[perm[r]].
 // One warp per row, 16-byte copies.  grid ceil(R/8), block 256.
 __global__ void __launch_bounds__(256) gather_rows_kernel(const uint16_t* __restrict__ x,
                                                           const int32_t* __restrict__ perm,
