@@ -82,7 +82,7 @@ MOE_DEVINL bool mbar_wait_bounded(uint64_t* bar, uint32_t parity, uint64_t limit
   }
 }
 
-// ---- bulk async copy global -> shared (no multicast) ---------------------------------
+// ---- bulk async copy global -> shared (one destination CTA) ---------------------------------
 // Both addresses 16-byte aligned, bytes a multiple of 16.  Completion is counted on `bar`.
 MOE_DEVINL void bulk_g2s(void* smem_dst, const void* gsrc, uint32_t bytes, uint64_t* bar) {
   asm volatile(
@@ -92,7 +92,7 @@ MOE_DEVINL void bulk_g2s(void* smem_dst, const void* gsrc, uint32_t bytes, uint6
       : "memory");
 }
 
-// ---- TMA tensor copy global -> shared (2D tile, no multicast) ---------------------------
+// ---- TMA tensor copy global -> shared (2D tile, one destination CTA) ---------------------------
 // c0 is the innermost (column) coordinate; c0 * element size must be a multiple of 16 bytes.
 // Parts of the box outside the tensor are zero-filled and still counted on `bar`.
 MOE_DEVINL void tma_load_2d(void* smem_dst, const CUtensorMap* map, int c0, int c1,
@@ -193,6 +193,68 @@ MOE_DEVINL void tmem_ld32(uint32_t taddr, float (&v)[32]) {
   for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
 }
 
+// ---- CTA pairs (cluster of 2) for the 2-SM tensor-core MMA ------------------------------------
+MOE_DEVINL uint32_t cluster_ctarank() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %cluster_ctarank;" : "=r"(r));
+  return r;
+}
+MOE_DEVINL void cluster_sync_all() {  // every thread of both CTAs
+  asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::
+                   : "memory");
+}
+// Address in CTA `rank` of the cluster of the same shared-memory offset as local address a.
+MOE_DEVINL uint32_t mapa_shared(uint32_t a, uint32_t rank) {
+  uint32_t r;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(a), "r"(rank));
+  return r;
+}
+MOE_DEVINL void mbar_arrive_cluster(uint32_t cluster_addr) {
+  asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr)
+               : "memory");
+}
+MOE_DEVINL void tmem_alloc_2sm(uint32_t* smem_dst, uint32_t ncols) {  // whole warp, both CTAs
+  asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+                   smem_u32(smem_dst)),
+               "r"(ncols)
+               : "memory");
+}
+MOE_DEVINL void tmem_relinquish_2sm() {
+  asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;" ::: "memory");
+}
+MOE_DEVINL void tmem_dealloc_2sm(uint32_t taddr, uint32_t ncols) {
+  asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols)
+               : "memory");
+}
+// One MMA over the CTA pair: A rows split (each CTA its 128 rows), B columns split (each CTA
+// its N/2 columns), D = 128 rows x N in each CTA's tensor memory.  Issued by the even CTA.
+MOE_DEVINL void tc_mma_bf16_2sm(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
+                                uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::2.kind::f16 [%0], %1, %2, %3, p;\n\t}"
+      ::"r"(d_tmem), "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+// Arrive once on the barrier at shared::cluster address `bar` (this CTA's or the peer's) when
+// the pair-wide tcgen05 operations issued so far by this thread have completed.
+MOE_DEVINL void tc_commit_2sm(uint32_t bar) {
+  asm volatile("tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
+                   bar)
+               : "memory");
+}
+// TMA 2D tile load into this CTA's shared memory whose completion is counted on a barrier that
+// may live in the peer CTA of the pair (one destination CTA).
+MOE_DEVINL void tma_load_2d_pair(void* smem_dst, const CUtensorMap* map, int c0, int c1,
+                                 uint32_t bar_cluster_addr) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%2, %3}], [%4];" ::"r"(smem_u32(smem_dst)),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(c0), "r"(c1), "r"(bar_cluster_addr)
+      : "memory");
+}
+
 // Shared-memory matrix descriptor for tcgen05.mma (sm_100 layout): start address, leading
 // and stride byte offsets (all >> 4), version 1, 128-byte swizzle.
 MOE_DEVINL uint64_t smem_desc_sw128(uint32_t saddr, uint32_t lbo_bytes, uint32_t sbo_bytes) {
@@ -248,5 +310,8 @@ MOE_DEVINL int atom_add_acq_rel_gpu(int* p, int v) {
 }
 
 MOE_DEVINL float silu_f32(float z) { return z / (1.0f + expf(-z)); }
+// SiLU with the fast exp / divide intrinsics (relative error ~1e-6, far below the bf16 step of the
+// value it feeds); for z -> -inf the denominator overflows to inf and the result goes to -0.
+MOE_DEVINL float silu_fast(float z) { return __fdividef(z, 1.0f + __expf(-z)); }
 
 }  // namespace moe

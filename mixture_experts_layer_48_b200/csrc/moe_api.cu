@@ -40,9 +40,11 @@ struct MapCache {
   CUtensorMap map;
 };
 
-// Grouped-GEMM configurations: <mode, MMAs per K step, N per MMA, smem stages>.
-#define MOE_GEMM_GATE_UP 0, 2, 128, 4
-#define MOE_GEMM_DOWN 1, 1, 192, 5
+// Grouped-GEMM configurations (CTA pairs): <mode, shared-memory stages>.
+constexpr int kGemmStages = 6;
+#define MOE_GEMM_GATE_UP 0, kGemmStages
+#define MOE_GEMM_DOWN 1, kGemmStages
+constexpr int kGemmChunkRows = 2 * kGemmBM;  // rows per tile: one 256-row MMA over a CTA pair
 
 struct moe_ctx {
   int E, H, I, k;
@@ -182,7 +184,7 @@ GemmLayout gemm_layout(const moe_ctx* c, int T) {
   GemmLayout L{};
   Carver cv;
   const size_t R = (size_t)T * c->k;
-  L.max_chunks = (int)(R / kGemmBM) + c->E;
+  L.max_chunks = (int)(R / kGemmChunkRows) + c->E;
   L.topk_idx = cv.take(4 * R);
   L.topk_w = cv.take(4 * R);
   L.inv_perm = cv.take(4 * R);
@@ -312,12 +314,12 @@ bool set_smem_attrs() {
                              kGateUpSmem) == cudaSuccess;
   ok &= cudaFuncSetAttribute(stream_down_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              kDownSmem) == cudaSuccess;
-  ok &= cudaFuncSetAttribute(grouped_gemm_kernel<MOE_GEMM_GATE_UP>,
+  ok &= cudaFuncSetAttribute(grouped_gemm_2sm_kernel<MOE_GEMM_GATE_UP>,
                              cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             GemmCfg<2, 128, 4>::kSmem) == cudaSuccess;
-  ok &= cudaFuncSetAttribute(grouped_gemm_kernel<MOE_GEMM_DOWN>,
+                             Gemm2Cfg<kGemmStages>::kSmem) == cudaSuccess;
+  ok &= cudaFuncSetAttribute(grouped_gemm_2sm_kernel<MOE_GEMM_DOWN>,
                              cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             GemmCfg<1, 192, 5>::kSmem) == cudaSuccess;
+                             Gemm2Cfg<kGemmStages>::kSmem) == cudaSuccess;
   return ok;
 }
 
@@ -414,7 +416,7 @@ moe_status forward_gemm(moe_ctx* c, int T, const void* x_bf16, const void* W_rou
   o.row_w = reinterpret_cast<float*>(ws + L.row_w);
   o.chunks = reinterpret_cast<int4*>(ws + L.chunks);
   o.sched = reinterpret_cast<int32_t*>(ws + L.sched);
-  o.chunk_rows = kGemmBM;
+  o.chunk_rows = kGemmChunkRows;
   o.zero_i32 = nullptr;
   o.n_zero = 0;
   const uint16_t* x = static_cast<const uint16_t*>(x_bf16);
@@ -447,9 +449,10 @@ moe_status forward_gemm(moe_ctx* c, int T, const void* x_bf16, const void* W_rou
   g.h = h;
   g.H = c->H;
   g.status = c->d_status;
+  const int grid = c->num_sms & ~1;  // whole CTA pairs
   MOE_TRY(launch(c, kKindGateUp, st, [&] {
-    grouped_gemm_kernel<MOE_GEMM_GATE_UP>
-        <<<c->num_sms, kGemmThreads, GemmCfg<2, 128, 4>::kSmem, st>>>(g, *am, *bm);
+    grouped_gemm_2sm_kernel<MOE_GEMM_GATE_UP>
+        <<<grid, kGemmThreads, Gemm2Cfg<kGemmStages>::kSmem, st>>>(g, *am, *bm);
   }));
   const CUtensorMap* hm = cached_map(c->h_map, h, R, (uint64_t)c->I, kGemmBM, 64);
   const CUtensorMap* dm = cached_map(c->down_stream, W_down_bf16, (uint64_t)c->E * c->I,
@@ -468,8 +471,8 @@ moe_status forward_gemm(moe_ctx* c, int T, const void* x_bf16, const void* W_rou
   d.H = c->H;
   d.status = c->d_status;
   MOE_TRY(launch(c, kKindDown, st, [&] {
-    grouped_gemm_kernel<MOE_GEMM_DOWN>
-        <<<c->num_sms, kGemmThreads, GemmCfg<1, 192, 5>::kSmem, st>>>(d, *hm, *dm);
+    grouped_gemm_2sm_kernel<MOE_GEMM_DOWN>
+        <<<grid, kGemmThreads, Gemm2Cfg<kGemmStages>::kSmem, st>>>(d, *hm, *dm);
   }));
   return MOE_OK;
 }

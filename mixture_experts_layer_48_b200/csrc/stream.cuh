@@ -8,7 +8,7 @@
 //
 // Layout: a persistent grid (one CTA per SM).  Each CTA has one producer warp and five
 // consumer warps around a 4-stage shared-memory ring.  The producer issues TMA tensor loads
-// (no multicast) of 64-column weight boxes with the 128-byte swizzle, and bulk copies of the
+// (one destination CTA) of 64-column weight boxes with the 128-byte swizzle, and bulk copies of the
 // rows' activations.  Consumer warp w owns box w of a 320-column tile and multiplies it with
 // the expert's rows on the tensor cores: the weight block is the 16-row A operand (read with
 // ldmatrix.trans, since W is [K, N] with N contiguous), the <= 16 activation rows are the
