@@ -132,10 +132,12 @@ MOE_API moe_status moe_set_path(moe_t ctx, moe_path path, int crossover_T);
 /* Current path setting and crossover. */
 MOE_API moe_status moe_get_path(moe_t ctx, moe_path* path, int* crossover_T);
 
-/* Measure the crossover on this device with the caller's layer: times both paths at
- * T = 1, 2, 4, ... up to T_max (x must hold T_max rows, out T_max rows, workspace
- * moe_tune_workspace_bytes) and stores the largest T at which streaming is not slower.
- * Synchronises the stream.  *crossover_out (may be NULL) receives the value. */
+/* Measure the crossover on this device with the caller's layer: times both paths (median of
+ * 5 calls after 2 warm-ups) at T = 1, 2, 4, 8, 12, 16, 24, 32, 48, 64, ... up to T_max, stops
+ * once the grouped GEMM has been faster for a doubling of T, and stores the largest T at which
+ * streaming was not slower (0 if never) as the handle's crossover.  x must hold T_max rows,
+ * out T_max rows; workspace at least moe_tune_workspace_bytes(ctx, T_max).  Synchronises
+ * `stream`; the path setting is left as it was.  *crossover_out (may be NULL) receives it. */
 MOE_API size_t moe_tune_workspace_bytes(moe_t ctx, int T_max);
 MOE_API moe_status moe_tune(moe_t ctx, int T_max, const void* x_bf16, const void* W_router_bf16,
                     const float* b_router, const void* W_gate_up_bf16,

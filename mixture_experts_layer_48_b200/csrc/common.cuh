@@ -277,6 +277,13 @@ MOE_DEVINL uint8_t* align1k(uint8_t* p) {
   return reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(p) + 1023) & ~uintptr_t(1023));
 }
 
+// ---- programmatic dependent launch ------------------------------------------------------------
+// Every kernel of the layer first waits for the kernel before it on the stream (a no-op when it
+// was launched without the programmatic-serialisation attribute), then lets the next kernel
+// launch.  Work placed before pdl_wait() may only touch memory no earlier kernel still uses.
+MOE_DEVINL void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+MOE_DEVINL void pdl_launch_next() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
 // ---- misc ----------------------------------------------------------------------------
 MOE_DEVINL void named_bar_sync(int id, int nthreads) {
   asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");

@@ -140,6 +140,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
   cluster_sync_all();
   tc_fence_after();
   const uint32_t tmem_base = s_tmem;
+  if (tid == 0) {
+    tma_prefetch_desc(&amap);
+    tma_prefetch_desc(&bmap);
+  }
+  pdl_wait();  // activations, work list and (down) h come from the previous kernels
+  pdl_launch_next();
 
   const int NT = (a.Ncols + TW - 1) / TW;
   const int tiles = a.sched[0] * NT;
@@ -150,8 +156,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
   if (warp == 0) {
     // ------------------------------ TMA producer (both CTAs) ------------------------------
     if (lane == 0) {
-      tma_prefetch_desc(&amap);
-      tma_prefetch_desc(&bmap);
       uint32_t it = 0;
       int last_it[STAGES];
 #pragma unroll

@@ -9,6 +9,7 @@
 #include <cstdint>
 #include <cstring>
 #include <new>
+#include <utility>
 #include <mutex>
 #include <vector>
 
@@ -48,7 +49,7 @@ constexpr int kGemmChunkRows = 2 * kGemmBM;  // rows per tile: one 256-row MMA o
 
 struct moe_ctx {
   int E, H, I, k;
-  MapCache gate_up_stream, down_stream, gate_up_gemm, x_perm_map, h_map;
+  MapCache gate_up_stream, down_stream, gate_up_gemm, down_gemm, x_perm_map, h_map;
   int device = 0;
   int num_sms = 148;
   moe_path path = MOE_PATH_AUTO;
@@ -101,8 +102,10 @@ PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
 }
 
 // 2D bf16 view [rows, cols] (row-major, contiguous) with a [box_rows, box_cols] box.
+// promote_256: let L2 fill 256-byte lines for each 128-byte box row (good when the neighbouring
+// 128 bytes are read by the same tile soon after; wasteful when they belong to another tile).
 bool encode_2d(CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols, uint32_t box_rows,
-               uint32_t box_cols, CUtensorMapSwizzle swizzle) {
+               uint32_t box_cols, CUtensorMapSwizzle swizzle, bool promote_256) {
   auto enc = tensor_map_encoder();
   if (!enc) return false;
   cuuint64_t dims[2] = {cols, rows};
@@ -111,15 +114,17 @@ bool encode_2d(CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols, u
   cuuint32_t estr[2] = {1, 1};
   return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box,
              estr, CU_TENSOR_MAP_INTERLEAVE_NONE, swizzle,
-             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+             promote_256 ? CU_TENSOR_MAP_L2_PROMOTION_L2_256B : CU_TENSOR_MAP_L2_PROMOTION_L2_128B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
 const CUtensorMap* cached_map(MapCache& mc, const void* ptr, uint64_t rows, uint64_t cols,
-                              uint32_t box_rows, uint32_t box_cols,
-                              CUtensorMapSwizzle swizzle = CU_TENSOR_MAP_SWIZZLE_128B) {
+                              uint32_t box_rows, uint32_t box_cols, bool promote_256 = true) {
   if (mc.ptr != ptr || mc.rows != rows) {
     mc.ptr = nullptr;
-    if (!encode_2d(&mc.map, ptr, rows, cols, box_rows, box_cols, swizzle)) return nullptr;
+    if (!encode_2d(&mc.map, ptr, rows, cols, box_rows, box_cols, CU_TENSOR_MAP_SWIZZLE_128B,
+                   promote_256))
+      return nullptr;
     mc.ptr = ptr;
     mc.rows = rows;
   }
@@ -215,12 +220,31 @@ bool use_stream(const moe_ctx* c, int T) {
 }
 
 // ---- launches ------------------------------------------------------------------------
+// Launch with programmatic stream serialisation: the kernel may start (and run the part before
+// its pdl_wait()) while the previous kernel on the stream finishes.
+template <typename... KArgs, typename... Args>
+cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem,
+                       cudaStream_t st, Args&&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
+}
+
 template <typename F>
 moe_status launch(moe_ctx* c, int kind, cudaStream_t st, F&& f) {
   const bool prof = c->prof_max > 0 && c->in_call && c->ev_used + 2 <= c->ev.size();
   if (prof) cudaEventRecord(c->ev[c->ev_used], st);
-  f();
-  const cudaError_t err = cudaGetLastError();
+  cudaError_t err = f();
+  if (err == cudaSuccess) err = cudaGetLastError();
+  else cudaGetLastError();
   if (prof) {
     cudaEventRecord(c->ev[c->ev_used + 1], st);
     c->ev_kind[c->ev_used / 2] = kind;
@@ -238,11 +262,11 @@ moe_status launch(moe_ctx* c, int kind, cudaStream_t st, F&& f) {
   } while (0)
 
 template <int NT8>
-void launch_router_tc(int NB, cudaStream_t st, const uint16_t* x, const uint16_t* Wr,
-                      const float* b, int T, int H, int E, int k, const RouteOut& o,
-                      int32_t* block_counts, float4* zero4, size_t n_zero4) {
-  router_topk_kernel<NT8><<<NB, 128, RouterTcCfg<NT8>::smem(k), st>>>(
-      x, Wr, b, T, H, E, k, o.topk_idx, o.topk_w, block_counts, zero4, n_zero4);
+cudaError_t launch_router_tc(int NB, cudaStream_t st, const uint16_t* x, const uint16_t* Wr,
+                             const float* b, int T, int H, int E, int k, const RouteOut& o,
+                             int32_t* block_counts, float4* zero4, size_t n_zero4) {
+  return launch_pdl(router_topk_kernel<NT8>, dim3(NB), dim3(128), RouterTcCfg<NT8>::smem(k), st,
+                    x, Wr, b, T, H, E, k, o.topk_idx, o.topk_w, block_counts, zero4, n_zero4);
 }
 
 // Routing chain.  zero4/n_zero4: a float scratch region the router kernel zero-fills.
@@ -257,13 +281,14 @@ moe_status launch_route(moe_ctx* c, int T, const uint16_t* x, const uint16_t* Wr
     float* partial = reinterpret_cast<float*>(ws + rt.partial);
     const size_t smem_p = (size_t)(kRouteTile * kRouterHSlice + kRouterHSlice * E) * 2;
     MOE_TRY(launch(c, kKindRouter, st, [&] {
-      router_partial_kernel<<<dim3(S, (T + kRouteTile - 1) / kRouteTile), 256, smem_p, st>>>(
-          x, Wr, T, H, E, partial, zero4, n_zero4);
+      return launch_pdl(router_partial_kernel, dim3(S, (T + kRouteTile - 1) / kRouteTile),
+                        dim3(256), smem_p, st, x, Wr, T, H, E, partial, zero4, n_zero4);
     }));
     const size_t smem_f = (size_t)T * E * 4 + (size_t)T * k * 4 + (size_t)T * 8 * 4 +
                           (256 + 257 + 257) * 4;
     MOE_TRY(launch(c, kKindRouteFin, st, [&] {
-      route_small_finalize_kernel<<<1, 1024, smem_f, st>>>(partial, S, b, T, E, k, o);
+      return launch_pdl(route_small_finalize_kernel, dim3(1), dim3(1024), smem_f, st,
+                        (const float*)partial, S, b, T, E, k, o);
     }));
     return MOE_OK;
   }
@@ -272,21 +297,22 @@ moe_status launch_route(moe_ctx* c, int T, const uint16_t* x, const uint16_t* Wr
   int32_t* totals = reinterpret_cast<int32_t*>(ws + rt.totals);
   const int nt8 = (E + 7) / 8;
   MOE_TRY(launch(c, kKindRouter, st, [&] {
-    if (nt8 <= 1) launch_router_tc<1>(NB, st, x, Wr, b, T, H, E, k, o, block_counts, zero4, n_zero4);
-    else if (nt8 <= 2) launch_router_tc<2>(NB, st, x, Wr, b, T, H, E, k, o, block_counts, zero4, n_zero4);
-    else if (nt8 <= 4) launch_router_tc<4>(NB, st, x, Wr, b, T, H, E, k, o, block_counts, zero4, n_zero4);
-    else if (nt8 <= 8) launch_router_tc<8>(NB, st, x, Wr, b, T, H, E, k, o, block_counts, zero4, n_zero4);
-    else if (nt8 <= 16) launch_router_tc<16>(NB, st, x, Wr, b, T, H, E, k, o, block_counts, zero4, n_zero4);
-    else launch_router_tc<32>(NB, st, x, Wr, b, T, H, E, k, o, block_counts, zero4, n_zero4);
+    if (nt8 <= 1) return launch_router_tc<1>(NB, st, x, Wr, b, T, H, E, k, o, block_counts, zero4, n_zero4);
+    if (nt8 <= 2) return launch_router_tc<2>(NB, st, x, Wr, b, T, H, E, k, o, block_counts, zero4, n_zero4);
+    if (nt8 <= 4) return launch_router_tc<4>(NB, st, x, Wr, b, T, H, E, k, o, block_counts, zero4, n_zero4);
+    if (nt8 <= 8) return launch_router_tc<8>(NB, st, x, Wr, b, T, H, E, k, o, block_counts, zero4, n_zero4);
+    if (nt8 <= 16) return launch_router_tc<16>(NB, st, x, Wr, b, T, H, E, k, o, block_counts, zero4, n_zero4);
+    return launch_router_tc<32>(NB, st, x, Wr, b, T, H, E, k, o, block_counts, zero4, n_zero4);
   }));
   MOE_TRY(launch(c, kKindRouteFin, st, [&] {
-    route_scan_kernel<<<E, 256, 0, st>>>(block_counts, NB, E, totals);
+    return launch_pdl(route_scan_kernel, dim3(E), dim3(256), 0, st, block_counts, NB, E, totals);
   }));
   const size_t smem_s = (256 + 257 + 257) * 4 + (size_t)kRouterTcTokens * 8 * 4 +
                         (size_t)kRouterTcTokens * E;
   MOE_TRY(launch(c, kKindRouteFin, st, [&] {
-    route_scatter_kernel<<<NB, 256, smem_s, st>>>(o.topk_idx, o.topk_w, block_counts, totals, T,
-                                                  E, k, o);
+    return launch_pdl(route_scatter_kernel, dim3(NB), dim3(256), smem_s, st,
+                      (const int32_t*)o.topk_idx, (const float*)o.topk_w,
+                      (const int32_t*)block_counts, (const int32_t*)totals, T, E, k, o);
   }));
   return MOE_OK;
 }
@@ -370,11 +396,12 @@ moe_status forward_stream(moe_ctx* c, int T, const void* x_bf16, const void* W_r
     ga.out_elems = (size_t)T * c->H;
     ga.status = c->d_status;
     const CUtensorMap* m = cached_map(c->gate_up_stream, W_gate_up_bf16, (uint64_t)c->E * c->H,
-                                      2ull * c->I, kGateUpKC, kBox);
+                                      2ull * c->I, kGateUpKC, kBox, /*promote_256=*/false);
     if (!m) s = MOE_ERR_CUDA;
     else
       s = launch(c, kKindGateUp, st, [&] {
-        stream_gate_up_kernel<<<c->num_sms, kStreamThreads, kGateUpSmem, st>>>(ga, *m);
+        return launch_pdl(stream_gate_up_kernel, dim3(c->num_sms), dim3(kStreamThreads),
+                          kGateUpSmem, st, ga, *m);
       });
   }
   if (s == MOE_OK) {
@@ -390,11 +417,12 @@ moe_status forward_stream(moe_ctx* c, int T, const void* x_bf16, const void* W_r
     da.out = out;
     da.status = c->d_status;
     const CUtensorMap* m = cached_map(c->down_stream, W_down_bf16, (uint64_t)c->E * c->I,
-                                      (uint64_t)c->H, kDownKC, kBox);
+                                      (uint64_t)c->H, kDownKC, kBox, /*promote_256=*/false);
     if (!m) s = MOE_ERR_CUDA;
     else
       s = launch(c, kKindDown, st, [&] {
-        stream_down_kernel<<<c->num_sms, kStreamThreads, kDownSmem, st>>>(da, *m);
+        return launch_pdl(stream_down_kernel, dim3(c->num_sms), dim3(kStreamThreads), kDownSmem,
+                          st, da, *m);
       });
   }
   return s;
@@ -432,8 +460,8 @@ moe_status forward_gemm(moe_ctx* c, int T, const void* x_bf16, const void* W_rou
                        L.rt, st, out, (size_t)T * c->H));
   if (T <= kSmallT)
     MOE_TRY(launch(c, kKindGather, st, [&] {
-      gather_rows_kernel<<<(unsigned)((R + 7) / 8), 256, 0, st>>>(x, o.perm, (int)R, c->H,
-                                                                 x_perm);
+      return launch_pdl(gather_rows_kernel, dim3((unsigned)((R + 7) / 8)), dim3(256), 0, st, x,
+                        (const int32_t*)o.perm, (int)R, c->H, x_perm);
     }));
   const CUtensorMap* am = cached_map(c->x_perm_map, x_perm, R, (uint64_t)c->H, kGemmBM, 64);
   const CUtensorMap* bm = cached_map(c->gate_up_gemm, W_gate_up_bf16, (uint64_t)c->E * c->H,
@@ -451,12 +479,12 @@ moe_status forward_gemm(moe_ctx* c, int T, const void* x_bf16, const void* W_rou
   g.status = c->d_status;
   const int grid = c->num_sms & ~1;  // whole CTA pairs
   MOE_TRY(launch(c, kKindGateUp, st, [&] {
-    grouped_gemm_2sm_kernel<MOE_GEMM_GATE_UP>
-        <<<grid, kGemmThreads, Gemm2Cfg<kGemmStages>::kSmem, st>>>(g, *am, *bm);
+    return launch_pdl(grouped_gemm_2sm_kernel<MOE_GEMM_GATE_UP>, dim3(grid), dim3(kGemmThreads),
+                      Gemm2Cfg<kGemmStages>::kSmem, st, g, *am, *bm);
   }));
   const CUtensorMap* hm = cached_map(c->h_map, h, R, (uint64_t)c->I, kGemmBM, 64);
-  const CUtensorMap* dm = cached_map(c->down_stream, W_down_bf16, (uint64_t)c->E * c->I,
-                                     (uint64_t)c->H, kDownKC, kBox);
+  const CUtensorMap* dm = cached_map(c->down_gemm, W_down_bf16, (uint64_t)c->E * c->I,
+                                     (uint64_t)c->H, kGemmBK, 64);
   if (!hm || !dm) return MOE_ERR_CUDA;
   GemmArgs d{};
   d.K = c->I;
@@ -471,8 +499,8 @@ moe_status forward_gemm(moe_ctx* c, int T, const void* x_bf16, const void* W_rou
   d.H = c->H;
   d.status = c->d_status;
   MOE_TRY(launch(c, kKindDown, st, [&] {
-    grouped_gemm_2sm_kernel<MOE_GEMM_DOWN>
-        <<<grid, kGemmThreads, Gemm2Cfg<kGemmStages>::kSmem, st>>>(d, *hm, *dm);
+    return launch_pdl(grouped_gemm_2sm_kernel<MOE_GEMM_DOWN>, dim3(grid), dim3(kGemmThreads),
+                      Gemm2Cfg<kGemmStages>::kSmem, st, d, *hm, *dm);
   }));
   return MOE_OK;
 }
@@ -631,14 +659,68 @@ moe_status moe_get_path(moe_t c, moe_path* path, int* crossover_T) {
   return MOE_OK;
 }
 
-size_t moe_tune_workspace_bytes(moe_t c, int T_max) { return moe_workspace_bytes(c, T_max); }
+size_t moe_tune_workspace_bytes(moe_t c, int T_max) {
+  if (!c || T_max < 1 || T_max > kMaxT) return 0;
+  return std::max(stream_layout(c, T_max).total, gemm_layout(c, T_max).total);
+}
 
-moe_status moe_tune(moe_t c, int T_max, const void*, const void*, const float*, const void*,
-                    const void*, float*, void*, size_t, moe_stream_t, int* crossover_out) {
-  if (!c || T_max < 1) return MOE_ERR_ARG;
-  // Only the streaming path exists in this build, so it wins at every T.
-  c->crossover = INT_MAX;
-  if (crossover_out) *crossover_out = c->crossover;
+moe_status moe_tune(moe_t c, int T_max, const void* x_bf16, const void* W_router_bf16,
+                    const float* b_router, const void* W_gate_up_bf16, const void* W_down_bf16,
+                    float* out, void* workspace, size_t ws_bytes, moe_stream_t stream,
+                    int* crossover_out) {
+  if (!c || T_max < 1 || T_max > kMaxT) return MOE_ERR_ARG;
+  MOE_TRY(check_common(c, T_max, x_bf16, W_router_bf16, b_router));
+  if (!W_gate_up_bf16 || !W_down_bf16 || !out || !aligned16(out)) return MOE_ERR_ARG;
+  if (!workspace || ws_bytes < moe_tune_workspace_bytes(c, T_max)) return MOE_ERR_WORKSPACE;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  const moe_path saved_path = c->path;
+  const int saved_prof = c->prof_max;
+  c->prof_max = 0;  // tuning launches are not profiled
+  cudaEvent_t e0 = nullptr, e1 = nullptr;
+  if (cudaEventCreate(&e0) != cudaSuccess || cudaEventCreate(&e1) != cudaSuccess) {
+    cudaGetLastError();
+    if (e0) cudaEventDestroy(e0);
+    c->prof_max = saved_prof;
+    return MOE_ERR_CUDA;
+  }
+  // median of 5 timed calls after 2 warm-up calls, for one path at one token count
+  auto time_path = [&](moe_path p, int T, float* ms_out) -> moe_status {
+    c->path = p;
+    float v[5];
+    for (int rep = 0; rep < 7; ++rep) {
+      if (rep >= 2 && cudaEventRecord(e0, st) != cudaSuccess) return MOE_ERR_CUDA;
+      MOE_TRY(moe_forward(c, T, x_bf16, W_router_bf16, b_router, W_gate_up_bf16, W_down_bf16,
+                          out, workspace, ws_bytes, stream));
+      if (rep >= 2) {
+        if (cudaEventRecord(e1, st) != cudaSuccess || cudaEventSynchronize(e1) != cudaSuccess ||
+            cudaEventElapsedTime(&v[rep - 2], e0, e1) != cudaSuccess)
+          return MOE_ERR_CUDA;
+      }
+    }
+    std::sort(v, v + 5);
+    *ms_out = v[2];
+    return MOE_OK;
+  };
+  static const int kCandidates[] = {1, 2, 4, 8, 12, 16, 24, 32, 48, 64, 96, 128, 192, 256, 384,
+                                    512, 768, 1024};
+  int crossover = 0;
+  moe_status s = MOE_OK;
+  for (int T : kCandidates) {
+    if (T > T_max) break;
+    float ts = 0.f, tg = 0.f;
+    s = time_path(MOE_PATH_STREAM, T, &ts);
+    if (s == MOE_OK) s = time_path(MOE_PATH_GEMM, T, &tg);
+    if (s != MOE_OK) break;
+    if (ts <= tg) crossover = T;
+    else if (T >= 2 * std::max(crossover, 1)) break;  // the grouped GEMM has taken over
+  }
+  cudaEventDestroy(e0);
+  cudaEventDestroy(e1);
+  c->path = saved_path;
+  c->prof_max = saved_prof;
+  if (s != MOE_OK) return s;
+  c->crossover = crossover;
+  if (crossover_out) *crossover_out = crossover;
   return MOE_OK;
 }
 

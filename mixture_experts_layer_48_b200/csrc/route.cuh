@@ -119,6 +119,8 @@ __global__ void __launch_bounds__(256) router_partial_kernel(const uint16_t* __r
                                                              int T, int H, int E,
                                                              float* __restrict__ partial,
                                                              float4* zero4, size_t n_zero4) {
+  pdl_wait();
+  pdl_launch_next();
   zero_fill_f4(zero4, n_zero4);
   extern __shared__ __align__(128) uint8_t smem_raw[];
   uint16_t* xs = reinterpret_cast<uint16_t*>(smem_raw);  // [32][64]
@@ -130,8 +132,10 @@ __global__ void __launch_bounds__(256) router_partial_kernel(const uint16_t* __r
     reinterpret_cast<uint4*>(xs)[r * 8 + c] =
         reinterpret_cast<const uint4*>(x + (size_t)(t0 + r) * H + h0)[c];
   }
-  const uint16_t* wsrc = Wr + (size_t)h0 * E;
-  for (int i = threadIdx.x; i < kRouterHSlice * E; i += blockDim.x) ws[i] = wsrc[i];
+  // the slice is 64*E contiguous bf16 = 128*E bytes: whole 16-byte pieces at a 128-byte offset
+  const uint4* wsrc = reinterpret_cast<const uint4*>(Wr + (size_t)h0 * E);
+  for (int i = threadIdx.x; i < kRouterHSlice * E / 8; i += blockDim.x)
+    reinterpret_cast<uint4*>(ws)[i] = wsrc[i];
   __syncthreads();
   for (int o = threadIdx.x; o < nt * E; o += blockDim.x) {
     const int t = o / E, e = o - t * E;
@@ -188,11 +192,22 @@ __global__ void __launch_bounds__(1024)
   int32_t* off = cnt + 256;                                          // [257]
   int32_t* scratch = off + 257;                                      // [257]
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5, nwarps = blockDim.x >> 5;
+  pdl_wait();
+  pdl_launch_next();
 
   for (int i = tid; i < T * E; i += blockDim.x) {
     const int e = i % E;
+    // the S partial sums are independent loads: keep many in flight, add in slice order
     float v = 0.f;
-    for (int s = 0; s < S; ++s) v += partial[(size_t)s * T * E + i];
+    int s = 0;
+    for (; s + 8 <= S; s += 8) {
+      float p[8];
+#pragma unroll
+      for (int q = 0; q < 8; ++q) p[q] = partial[(size_t)(s + q) * T * E + i];
+#pragma unroll
+      for (int q = 0; q < 8; ++q) v += p[q];
+    }
+    for (; s < S; ++s) v += partial[(size_t)s * T * E + i];
     lg[i] = v + b_router[e];
   }
   for (int i = tid; i < T * 8; i += blockDim.x) bits[i] = 0u;
@@ -303,6 +318,8 @@ __global__ void __launch_bounds__(128)
   const int nk = H / kRouterHSlice;
   const bool vec_w = (E % 8) == 0;
 
+  pdl_wait();
+  pdl_launch_next();
   zero_fill_f4(zero4, n_zero4);
   for (int i = tid; i < EP; i += blockDim.x) cnt[i] = 0;
   for (int i = tid; i < C::kStages * kRouterHSlice * WP; i += blockDim.x)
@@ -413,6 +430,8 @@ __global__ void __launch_bounds__(256) route_scan_kernel(int32_t* __restrict__ b
                                                          int32_t* __restrict__ totals) {
   __shared__ int32_t part[256];
   const int e = blockIdx.x, tid = threadIdx.x;
+  pdl_wait();
+  pdl_launch_next();
   const int per = (NB + blockDim.x - 1) / blockDim.x;
   const int b0 = tid * per, b1 = min(NB, b0 + per);
   int s = 0;
@@ -456,6 +475,8 @@ __global__ void __launch_bounds__(256)
   uint8_t* slot = reinterpret_cast<uint8_t*>(bits + TT * 8);    // [64][E] (k <= 256)
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int t0 = blockIdx.x * TT, nt = min(TT, T - t0);
+  pdl_wait();
+  pdl_launch_next();
 
   for (int e = tid; e < E; e += blockDim.x) cnt[e] = totals[e];
   for (int i = tid; i < TT * 8; i += blockDim.x) bits[i] = 0u;
@@ -522,6 +543,8 @@ __global__ void __launch_bounds__(256) gather_rows_kernel(const uint16_t* __rest
                                                           int R, int H,
                                                           uint16_t* __restrict__ x_perm) {
   const int r = blockIdx.x * 8 + (threadIdx.x >> 5), lane = threadIdx.x & 31;
+  pdl_wait();
+  pdl_launch_next();
   if (r >= R) return;
   const uint4* src = reinterpret_cast<const uint4*>(x + (size_t)perm[r] * H);
   uint4* dst = reinterpret_cast<uint4*>(x_perm + (size_t)r * H);

@@ -24,7 +24,7 @@
 //     applies SwiGLU from registers; otherwise the pieces add their partial sums into an fp32
 //     accumulator (zero-filled by the router kernel) with atomics, and the piece that
 //     completes the tile's stage count (a release/acquire counter) writes h = silu(g) * u as
-//     bf16.  The kernel also zero-fills `out`.
+//     bf16.  The kernel also zero-fills `out` (before it waits for the routing kernels).
 //   down kernel: y = h W_down[e] per row, scaled by the row's routing weight, added into
 //     out[token] with fp32 atomics (the combine).
 #pragma once
@@ -165,6 +165,17 @@ __global__ void __launch_bounds__(kStreamThreads, 1)
   }
   __syncthreads();
 
+  if (tid == 32 * kStreamWarps) tma_prefetch_desc(&wmap);
+  // `out` is written only by this call's down kernel, which cannot start before this one
+  {
+    float4* o4 = reinterpret_cast<float4*>(a.out);
+    const size_t n4 = a.out_elems / 4;
+    for (size_t i = (size_t)blockIdx.x * blockDim.x + tid; i < n4; i += (size_t)gridDim.x * blockDim.x)
+      o4[i] = make_float4(0.f, 0.f, 0.f, 0.f);
+  }
+  pdl_wait();  // the routing results below come from the previous kernels
+  pdl_launch_next();
+
   const int I2 = 2 * a.I;
   const int NT = (a.I + kStreamCols - 1) / kStreamCols;
   const int nk = a.H / kGateUpKC;
@@ -172,7 +183,6 @@ __global__ void __launch_bounds__(kStreamThreads, 1)
 
   if (warp == kStreamWarps) {
     // ---------------- producer ----------------
-    if (lane == 0) tma_prefetch_desc(&wmap);
     bool aborted = false;
     uint32_t it = 0;
     int last_it[kStreamStages];
@@ -222,13 +232,6 @@ __global__ void __launch_bounds__(kStreamThreads, 1)
 
   // ---------------- consumers ----------------
   const int ctid = tid;  // 0..159; warp = box index
-  {
-    float4* o4 = reinterpret_cast<float4*>(a.out);
-    const size_t n4 = a.out_elems / 4;
-    for (size_t i = (size_t)blockIdx.x * kStreamConsumers + ctid; i < n4;
-         i += (size_t)gridDim.x * kStreamConsumers)
-      o4[i] = make_float4(0.f, 0.f, 0.f, 0.f);
-  }
   const uint32_t wring_s = smem_u32(wring), xring_s = smem_u32(xring);
   bool aborted = false;
   uint32_t it = 0;
@@ -364,12 +367,15 @@ __global__ void __launch_bounds__(kStreamThreads, 1)
   }
   __syncthreads();
 
+  if (tid == 32 * kStreamWarps) tma_prefetch_desc(&wmap);
+  pdl_wait();  // h and the work list come from the previous kernels
+  pdl_launch_next();
+
   const int NT = (a.H + kStreamCols - 1) / kStreamCols;
   const int nk = a.I / kDownKC;
   const StreamKRange rng = stream_k_range((long long)a.sched[0] * NT, nk);
 
   if (warp == kStreamWarps) {
-    if (lane == 0) tma_prefetch_desc(&wmap);
     bool aborted = false;
     uint32_t it = 0;
     int last_it[kStreamStages];

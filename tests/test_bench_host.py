@@ -1,0 +1,89 @@
+"""Host-side logic of bench.py, on CPU: max-over-ranks timing with 2 gloo ranks, whole-job
+aggregation, clock-sample parsing, algorithmic work counts, and the CLI guard rails."""
+import os
+import socket
+import subprocess
+import sys
+
+import pytest
+import torch
+import torch.distributed as dist
+import torch.multiprocessing as mp
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+sys.path.insert(0, ROOT)
+import bench  # noqa: E402
+
+
+def _free_port():
+    s = socket.socket()
+    s.bind(("127.0.0.1", 0))
+    p = s.getsockname()[1]
+    s.close()
+    return p
+
+
+def _rank_main(rank, world, port, q):
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port), RANK=str(rank),
+                      WORLD_SIZE=str(world), LOCAL_RANK=str(rank))
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    r, w, lr = bench.dist_env()
+    t = bench.reduce_max(0.25 + rank, w)          # rank 1 is the slow one
+    agg = bench.aggregate(16, w, t, 10)
+    q.put((r, w, lr, t, agg["value"]))
+    dist.barrier()
+    dist.destroy_process_group()
+
+
+def test_two_rank_max_over_ranks_and_aggregate():
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_rank_main, args=(r, 2, port, q)) for r in range(2)]
+    for p in procs:
+        p.start()
+    res = sorted(q.get(timeout=120) for _ in procs)
+    for p in procs:
+        p.join(timeout=60)
+        assert p.exitcode == 0
+    assert [r[0] for r in res] == [0, 1] and all(r[1] == 2 for r in res)
+    assert all(r[3] == pytest.approx(1.25) for r in res)          # both see the slowest rank
+    assert all(r[4] == pytest.approx(16 * 2 * 10 / 1.25) for r in res)
+
+
+def test_aggregate_single_rank():
+    a = bench.aggregate(16, 1, 0.5, 100)
+    assert a["value"] == pytest.approx(3200.0) and a["ms_per_step"] == pytest.approx(5.0)
+
+
+def test_parse_clocks():
+    csv = ("index, clocks.sm [MHz], clocks.max.sm [MHz], power.draw [W], clocks_event_reasons.active,"
+           " hw_slowdown, hw_thermal_slowdown, sw_thermal_slowdown, sw_power_cap\n"
+           "0, 1965 MHz, 1965 MHz, 850.1 W, 0x0, Not Active, Not Active, Not Active, Not Active\n"
+           "0, 1890 MHz, 1965 MHz, 998.0 W, 0x4, Not Active, Not Active, Not Active, Active\n"
+           "0, 345 MHz, 1965 MHz, 120.0 W, 0x0, Not Active, Not Active, Not Active, Not Active\n")
+    c = bench.parse_clocks(csv)
+    assert c["sm_mhz"] == pytest.approx((1965 + 1890) / 2)
+    assert c["sm_max_mhz"] == 1965 and c["reasons"] == ["sw_power_cap"]
+    assert c["samples"] == 3 and c["samples_under_load"] == 2
+
+
+def test_algorithmic_work_counts_only_touched_experts():
+    a = bench.algorithmic(T=16, H=2880, E=32, k=4, I=2880, counts=[2] * 24 + [0] * 8)
+    assert a["touched"] == 24
+    assert a["gate_up_bytes"] == 24 * 2880 * 5760 * 2 + 16 * 2880 * 2 + 64 * 2880 * 2
+    assert a["gate_up_flops"] == 2 * 64 * 2880 * 5760
+    assert a["down_flops"] == 2 * 64 * 2880 * 2880
+
+
+def test_cli_refuses_too_few_warmup_steps():
+    r = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--warmup", "2"],
+                       capture_output=True, text=True, timeout=120)
+    assert r.returncode != 0 and "warmup" in r.stderr
+
+
+@pytest.mark.skipif(torch.cuda.is_available(), reason="checks the no-GPU refusal")
+def test_bench_refuses_to_run_without_gpu():
+    r = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--steps", "1", "--warmup", "3"],
+                       capture_output=True, text=True, timeout=300)
+    assert r.returncode != 0 and "CUDA" in (r.stderr + r.stdout)

@@ -160,3 +160,15 @@ def test_both_paths_gpt_oss_shape(path):
     p = moe.MOE_PATH_STREAM if path == "stream" else moe.MOE_PATH_GEMM
     d, h = inputs_on_gpu(300, 2880, 32, 4, 2880, seed=1100)
     _check_layer(d, h, 32, 2880, 2880, 4, path=p)
+
+
+def test_tune_measures_a_crossover_and_auto_follows_it():
+    E, H, I, k = 32, 2880, 2880, 4
+    d, _ = inputs_on_gpu(256, H, E, k, I, seed=1200)
+    layer = moe.Moe(E, H, I, k)
+    c = layer.tune(d["x"], d["W_router"], d["b_router"], d["W_gate_up"], d["W_down"])
+    path, cross = layer.get_path()
+    assert path == moe.MOE_PATH_AUTO and cross == c
+    assert 0 <= c <= 256
+    print("measured crossover T* =", c)
+    assert layer.sync_status() == moe.MOE_OK
