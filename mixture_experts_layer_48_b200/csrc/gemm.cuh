@@ -82,6 +82,8 @@ MOE_DEVINL bool wait_or_abort(uint64_t* bar, uint32_t parity, volatile int* abor
 // ------------------------------------------------------------------------------------------------
 constexpr int kGemmN = 256;                                  // MMA N (columns of D per CTA)
 constexpr int kGemmHalf = kGemmN / 2;                        // weight columns staged per CTA
+constexpr int kEpiPitch = 36;                                // floats per staged row (16B-aligned)
+constexpr int kEpiStageBytes = 4 * 32 * kEpiPitch * 4;       // 4 epilogue warps x 32 x 32 fp32
 
 template <int STAGES>
 struct Gemm2Cfg {
@@ -92,7 +94,7 @@ struct Gemm2Cfg {
   static constexpr int kBAtoms = kGemmHalf / 64;
   static constexpr int kBBytes = kBAtoms * kBAtomBytes;
   static constexpr int kStageBytes = kABytes + kBBytes;
-  static constexpr int kSmem = 1024 + STAGES * kStageBytes + 256;
+  static constexpr int kSmem = 1024 + STAGES * kStageBytes + 256 + kEpiStageBytes;
   static_assert(kAccBufs * kGemmN <= kTmemCols, "tensor memory");
   static_assert(kSmem <= 227 * 1024, "shared memory");
 };
@@ -115,6 +117,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
   uint64_t* acc_full = empty + STAGES;
   uint64_t* acc_empty = acc_full + 2;
   uint64_t* drain = acc_empty + 2;
+  float* epi_stage = reinterpret_cast<float*>(ring + STAGES * C::kStageBytes + 256);
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const uint32_t rank = cluster_ctarank();
   const bool leader = rank == 0;
@@ -274,19 +277,28 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
           }
         }
       } else {
-        const int tok = valid ? a.perm[r0 + row] : 0;
+        // Each thread holds 32 columns of its own row; the atomics go out transposed through
+        // shared memory so that one instruction covers 4 rows x 128 contiguous bytes instead of
+        // 32 scattered rows.
+        const int tok = valid ? a.perm[r0 + row] : -1;
         const float w = valid ? a.row_w[r0 + row] : 0.f;
-        float* orow = a.out + (size_t)tok * a.H + n0;
+        float* stage = epi_stage + (warp - kGemmEpiWarp0) * 32 * kEpiPitch;
 #pragma unroll 1
         for (int c = 0; c < kGemmN; c += 32) {
           float y[32];
           tmem_ld32(taddr + c, y);
-          if (valid && n0 + c < a.Ncols) {
+          if (n0 + c >= a.Ncols) continue;  // whole chunk past H (warp-uniform)
 #pragma unroll
-            for (int i = 0; i < 8; ++i)
-              red_add_f32x4(orow + c + 4 * i, w * y[4 * i], w * y[4 * i + 1], w * y[4 * i + 2],
-                            w * y[4 * i + 3]);
+          for (int j = 0; j < 32; ++j) stage[lane * kEpiPitch + j] = w * y[j];
+          __syncwarp();
+#pragma unroll
+          for (int it = 0; it < 8; ++it) {
+            const int rr = 4 * it + (lane >> 3), cc = 4 * (lane & 7);
+            const int t = __shfl_sync(0xffffffffu, tok, rr);
+            const float4 v = *reinterpret_cast<const float4*>(stage + rr * kEpiPitch + cc);
+            if (t >= 0) red_add_f32x4(a.out + (size_t)t * a.H + n0 + c + cc, v.x, v.y, v.z, v.w);
           }
+          __syncwarp();
         }
       }
       tc_fence_before();

@@ -134,9 +134,21 @@ const CUtensorMap* cached_map(MapCache& mc, const void* ptr, uint64_t rows, uint
 // ---- workspace layouts ---------------------------------------------------------------
 struct RouteTmp {
   size_t partial = 0, block_counts = 0, totals = 0;
+  int splits = 1, kc_per_split = 0;  // large-T router: hidden-dimension slices per token block
 };
 
-RouteTmp carve_route_tmp(Carver& cv, const moe_ctx* c, int T) {
+// Large-T router split: enough (token block, hidden slice) blocks for about two per SM.
+void router_split(const moe_ctx* c, int T, int* splits, int* kc_per_split) {
+  const int NB = (T + kRouterTcTokens - 1) / kRouterTcTokens;
+  const int nk = c->H / kRouterHSlice;
+  int S = std::max(1, std::min(nk, (2 * c->num_sms + NB - 1) / NB));
+  const int kcps = (nk + S - 1) / S;
+  *kc_per_split = kcps;
+  *splits = (nk + kcps - 1) / kcps;
+}
+
+// allow_split = false keeps the large-T router unsplit (the fixed-scratch routing entry point).
+RouteTmp carve_route_tmp(Carver& cv, const moe_ctx* c, int T, bool allow_split = true) {
   RouteTmp r;
   if (T <= kSmallT) {
     r.partial = cv.take(sizeof(float) * (size_t)(c->H / kRouterHSlice) * T * c->E);
@@ -144,6 +156,11 @@ RouteTmp carve_route_tmp(Carver& cv, const moe_ctx* c, int T) {
     const size_t NB = (T + kRouterTcTokens - 1) / kRouterTcTokens;
     r.block_counts = cv.take(sizeof(int32_t) * NB * c->E);
     r.totals = cv.take(sizeof(int32_t) * c->E);
+    r.kc_per_split = c->H / kRouterHSlice;
+    if (allow_split) {
+      router_split(c, T, &r.splits, &r.kc_per_split);
+      if (r.splits > 1) r.partial = cv.take(sizeof(float) * (size_t)r.splits * T * c->E);
+    }
   }
   return r;
 }
@@ -205,10 +222,10 @@ GemmLayout gemm_layout(const moe_ctx* c, int T) {
   return L;
 }
 
-size_t route_ws_bytes(const moe_ctx* c, int T) {
+size_t route_ws_bytes(const moe_ctx* c, int T, bool allow_split = true) {
   Carver cv;
   cv.take(16);  // sched
-  carve_route_tmp(cv, c, T);
+  carve_route_tmp(cv, c, T, allow_split);
   return cv.cur;
 }
 
@@ -264,9 +281,11 @@ moe_status launch(moe_ctx* c, int kind, cudaStream_t st, F&& f) {
 template <int NT8>
 cudaError_t launch_router_tc(int NB, cudaStream_t st, const uint16_t* x, const uint16_t* Wr,
                              const float* b, int T, int H, int E, int k, const RouteOut& o,
-                             int32_t* block_counts, float4* zero4, size_t n_zero4) {
-  return launch_pdl(router_topk_kernel<NT8>, dim3(NB), dim3(128), RouterTcCfg<NT8>::smem(k), st,
-                    x, Wr, b, T, H, E, k, o.topk_idx, o.topk_w, block_counts, zero4, n_zero4);
+                             int32_t* block_counts, float4* zero4, size_t n_zero4,
+                             const RouteTmp& rt, float* partial) {
+  return launch_pdl(router_topk_kernel<NT8>, dim3(NB, rt.splits), dim3(128),
+                    RouterTcCfg<NT8>::smem(k), st, x, Wr, b, T, H, E, k, o.topk_idx, o.topk_w,
+                    block_counts, zero4, n_zero4, rt.kc_per_split, partial);
 }
 
 // Routing chain.  zero4/n_zero4: a float scratch region the router kernel zero-fills.
@@ -296,14 +315,29 @@ moe_status launch_route(moe_ctx* c, int T, const uint16_t* x, const uint16_t* Wr
   int32_t* block_counts = reinterpret_cast<int32_t*>(ws + rt.block_counts);
   int32_t* totals = reinterpret_cast<int32_t*>(ws + rt.totals);
   const int nt8 = (E + 7) / 8;
+  float* split_partial = rt.splits > 1 ? reinterpret_cast<float*>(ws + rt.partial) : nullptr;
   MOE_TRY(launch(c, kKindRouter, st, [&] {
-    if (nt8 <= 1) return launch_router_tc<1>(NB, st, x, Wr, b, T, H, E, k, o, block_counts, zero4, n_zero4);
-    if (nt8 <= 2) return launch_router_tc<2>(NB, st, x, Wr, b, T, H, E, k, o, block_counts, zero4, n_zero4);
-    if (nt8 <= 4) return launch_router_tc<4>(NB, st, x, Wr, b, T, H, E, k, o, block_counts, zero4, n_zero4);
-    if (nt8 <= 8) return launch_router_tc<8>(NB, st, x, Wr, b, T, H, E, k, o, block_counts, zero4, n_zero4);
-    if (nt8 <= 16) return launch_router_tc<16>(NB, st, x, Wr, b, T, H, E, k, o, block_counts, zero4, n_zero4);
-    return launch_router_tc<32>(NB, st, x, Wr, b, T, H, E, k, o, block_counts, zero4, n_zero4);
+    if (nt8 <= 1) return launch_router_tc<1>(NB, st, x, Wr, b, T, H, E, k, o, block_counts, zero4, n_zero4, rt, split_partial);
+    if (nt8 <= 2) return launch_router_tc<2>(NB, st, x, Wr, b, T, H, E, k, o, block_counts, zero4, n_zero4, rt, split_partial);
+    if (nt8 <= 4) return launch_router_tc<4>(NB, st, x, Wr, b, T, H, E, k, o, block_counts, zero4, n_zero4, rt, split_partial);
+    if (nt8 <= 8) return launch_router_tc<8>(NB, st, x, Wr, b, T, H, E, k, o, block_counts, zero4, n_zero4, rt, split_partial);
+    if (nt8 <= 16) return launch_router_tc<16>(NB, st, x, Wr, b, T, H, E, k, o, block_counts, zero4, n_zero4, rt, split_partial);
+    return launch_router_tc<32>(NB, st, x, Wr, b, T, H, E, k, o, block_counts, zero4, n_zero4, rt, split_partial);
   }));
+  if (split_partial) {
+    const int n = T * E;
+    MOE_TRY(launch(c, kKindRouter, st, [&] {
+      return launch_pdl(sum_partials_kernel, dim3((n + 255) / 256), dim3(256), 0, st,
+                        split_partial, rt.splits, n);
+    }));
+    const size_t smem_t = (size_t)kRouterTcTokens * (E + 1) * 4 + (size_t)E * 4 +
+                          (size_t)kRouterTcTokens * k * 4;
+    MOE_TRY(launch(c, kKindRouter, st, [&] {
+      return launch_pdl(topk_from_partials_kernel, dim3(NB), dim3(128), smem_t, st,
+                        (const float*)split_partial, 1, b, T, E, k, o.topk_idx, o.topk_w,
+                        block_counts);
+    }));
+  }
   MOE_TRY(launch(c, kKindRouteFin, st, [&] {
     return launch_pdl(route_scan_kernel, dim3(E), dim3(256), 0, st, block_counts, NB, E, totals);
   }));
@@ -334,6 +368,8 @@ bool set_smem_attrs() {
                              big) == cudaSuccess;
   ok &= cudaFuncSetAttribute(router_topk_kernel<32>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              big) == cudaSuccess;
+  ok &= cudaFuncSetAttribute(topk_from_partials_kernel,
+                             cudaFuncAttributeMaxDynamicSharedMemorySize, big) == cudaSuccess;
   ok &= cudaFuncSetAttribute(router_partial_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              big) == cudaSuccess;
   ok &= cudaFuncSetAttribute(stream_gate_up_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -450,7 +486,11 @@ moe_status forward_gemm(moe_ctx* c, int T, const void* x_bf16, const void* W_rou
   const uint16_t* x = static_cast<const uint16_t*>(x_bf16);
   uint16_t* x_perm = reinterpret_cast<uint16_t*>(ws + L.x_perm);
   uint16_t* h = reinterpret_cast<uint16_t*>(ws + L.h);
-  if (T > kSmallT) {  // the large-T scatter also writes the rows in expert order
+  // With enough 64-token blocks to cover the GPU the scatter also writes the rows in expert
+  // order (each token row read once); otherwise a wide gather kernel does it.
+  const int NB = (T + kRouterTcTokens - 1) / kRouterTcTokens;
+  const bool fused_copy = T > kSmallT && NB >= c->num_sms;
+  if (fused_copy) {
     o.x = x;
     o.x_perm = x_perm;
     o.H = c->H;
@@ -458,7 +498,7 @@ moe_status forward_gemm(moe_ctx* c, int T, const void* x_bf16, const void* W_rou
   // the router kernel zero-fills `out`, which the down projection accumulates into
   MOE_TRY(launch_route(c, T, x, static_cast<const uint16_t*>(W_router_bf16), b_router, o, ws,
                        L.rt, st, out, (size_t)T * c->H));
-  if (T <= kSmallT)
+  if (!fused_copy)
     MOE_TRY(launch(c, kKindGather, st, [&] {
       return launch_pdl(gather_rows_kernel, dim3((unsigned)((R + 7) / 8)), dim3(256), 0, st, x,
                         (const int32_t*)o.perm, (int)R, c->H, x_perm);
@@ -882,13 +922,14 @@ moe_status moe_route_static(moe_t c, int T, const void* x_bf16, const void* W_ro
   if (!topk_idx || !topk_w || !perm || !inv_perm) return MOE_ERR_ARG;
   if (!aligned16(topk_idx) || !aligned16(topk_w) || !aligned16(perm) || !aligned16(inv_perm))
     return MOE_ERR_ARG;
-  if (route_ws_bytes(c, T) > kRouteStaticScratchBytes) return MOE_ERR_WORKSPACE;
+  if (route_ws_bytes(c, T, /*allow_split=*/false) > kRouteStaticScratchBytes)
+    return MOE_ERR_WORKSPACE;
   void* scratch = nullptr;
   MOE_TRY(static_scratch_address(dev, &scratch));
   uint8_t* ws = static_cast<uint8_t*>(scratch);
   Carver cv;
   const size_t sched_at = cv.take(16);
-  const RouteTmp rt = carve_route_tmp(cv, c, T);
+  const RouteTmp rt = carve_route_tmp(cv, c, T, /*allow_split=*/false);
   RouteOut o{};
   o.topk_idx = topk_idx;
   o.topk_w = topk_w;

@@ -102,6 +102,29 @@ MOE_DEVINL float warp_softmax_denominator(const float* lg, int k) {
   return s;
 }
 
+// Top-k, softmax and the block's expert histogram for up to 64 tokens whose logits (bias added)
+// are in shared memory, row stride `ld`; one warp per token.  Ends with the block's counts.
+MOE_DEVINL void topk_block_epilogue(float* lg, int ld, int nt, int t0, int E, int k, int32_t* sel,
+                                    int32_t* cnt, int32_t* topk_idx, float* topk_w,
+                                    int32_t* block_counts) {
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5, nwarps = blockDim.x >> 5;
+  for (int tt = warp; tt < nt; tt += nwarps) {
+    float* row = lg + tt * ld;
+    int32_t* srow = sel + tt * k;
+    warp_topk(row, E, k, srow);
+    const float denom = warp_softmax_denominator(row, k);
+    const size_t t = (size_t)(t0 + tt);
+    for (int j = lane; j < k; j += 32) {
+      topk_idx[t * k + j] = srow[j];
+      topk_w[t * k + j] = expf(row[j] - row[0]) / denom;
+      atomicAdd(&cnt[srow[j]], 1);
+    }
+    __syncwarp();
+  }
+  __syncthreads();
+  for (int e = tid; e < E; e += blockDim.x) block_counts[(size_t)blockIdx.x * E + e] = cnt[e];
+}
+
 // ---------------------------------------------------------------------------------------
 // Small T: partial router logits over one 64-row slice of W_router.
 // grid (H/64, ceil(T/32)), block 256.  partial layout [H/64][T][E].
@@ -304,7 +327,8 @@ __global__ void __launch_bounds__(128)
     router_topk_kernel(const uint16_t* __restrict__ x, const uint16_t* __restrict__ Wr,
                        const float* __restrict__ b_router, int T, int H, int E, int k,
                        int32_t* __restrict__ topk_idx, float* __restrict__ topk_w,
-                       int32_t* __restrict__ block_counts, float4* zero4, size_t n_zero4) {
+                       int32_t* __restrict__ block_counts, float4* zero4, size_t n_zero4,
+                       int kc_per_split, float* __restrict__ partial) {
   using C = RouterTcCfg<NT8>;
   constexpr int EP = C::EP, WP = C::WP, XP = kRouterTcXPitch, TT = kRouterTcTokens;
   extern __shared__ __align__(128) uint8_t smem_raw[];
@@ -315,7 +339,9 @@ __global__ void __launch_bounds__(128)
   int32_t* sel = cnt + EP;                                                   // [64][k]
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int t0 = blockIdx.x * TT, nt = min(TT, T - t0);
-  const int nk = H / kRouterHSlice;
+  // this block's slice of the hidden dimension: chunks [kc0, kc0 + nk) of 64 rows
+  const int kc0 = blockIdx.y * kc_per_split;
+  const int nk = min(H / kRouterHSlice - kc0, kc_per_split);
   const bool vec_w = (E % 8) == 0;
 
   pdl_wait();
@@ -327,7 +353,7 @@ __global__ void __launch_bounds__(128)
   __syncthreads();
 
   auto load_chunk = [&](int kc, int buf) {
-    const int h0 = kc * kRouterHSlice;
+    const int h0 = (kc0 + kc) * kRouterHSlice;
     uint16_t* xb = xs + buf * TT * XP;
     for (int i = tid; i < TT * 8; i += blockDim.x) {  // 64 rows x 8 pieces of 16 B
       const int r = i >> 3, c = i & 7;
@@ -395,6 +421,17 @@ __global__ void __launch_bounds__(128)
   }
   cp_async_wait<0>();
   // C fragment: c0,c1 -> token 16w + lane/4, experts 8n + 2(lane%4) + {0,1}; c2,c3 -> token + 8
+  if (partial != nullptr) {  // one slice of the hidden dimension: partial logits, no bias
+#pragma unroll
+    for (int n = 0; n < NT8; ++n)
+#pragma unroll
+      for (int v = 0; v < 4; ++v) {
+        const int tt = 16 * warp + (lane >> 2) + 8 * (v >> 1);
+        const int e = 8 * n + 2 * (lane & 3) + (v & 1);
+        if (e < E && tt < nt) partial[((size_t)blockIdx.y * T + t0 + tt) * E + e] = acc[n][v];
+      }
+    return;
+  }
 #pragma unroll
   for (int n = 0; n < NT8; ++n)
 #pragma unroll
@@ -404,21 +441,65 @@ __global__ void __launch_bounds__(128)
       if (e < E) lg[tt * (EP + 1) + e] = acc[n][v] + b_router[e];
     }
   __syncthreads();
-  for (int tt = warp; tt < nt; tt += 4) {
-    float* row = lg + tt * (EP + 1);
-    int32_t* srow = sel + tt * k;
-    warp_topk(row, E, k, srow);
-    const float denom = warp_softmax_denominator(row, k);
-    const size_t t = (size_t)(t0 + tt);
-    for (int j = lane; j < k; j += 32) {
-      topk_idx[t * k + j] = srow[j];
-      topk_w[t * k + j] = expf(row[j] - row[0]) / denom;
-      atomicAdd(&cnt[srow[j]], 1);
+  topk_block_epilogue(lg, EP + 1, nt, t0, E, k, sel, cnt, topk_idx, topk_w, block_counts);
+}
+
+// Sum of the S partial-logit slices of every (token, expert), in slice order, written in place
+// into slice 0 (each thread owns one element).  grid ceil(n/256), block 256.
+__global__ void __launch_bounds__(256) sum_partials_kernel(float* __restrict__ partial, int S,
+                                                           int n) {
+  pdl_wait();
+  pdl_launch_next();
+  const int i = blockIdx.x * blockDim.x + threadIdx.x;
+  if (i >= n) return;
+  float v = 0.f;
+  int s = 0;
+  for (; s + 8 <= S; s += 8) {
+    float p[8];
+#pragma unroll
+    for (int q = 0; q < 8; ++q) p[q] = partial[(size_t)(s + q) * n + i];
+#pragma unroll
+    for (int q = 0; q < 8; ++q) v += p[q];
+  }
+  for (; s < S; ++s) v += partial[(size_t)s * n + i];
+  partial[i] = v;
+}
+
+// Large T with too few token blocks to fill the GPU: the router kernel runs split over the hidden
+// dimension and writes partial logits [S, T, E] (summed into slice 0 by sum_partials_kernel when
+// S > 1); this kernel sums what it is given in slice order, adds the bias and finishes the
+// 64-token block like the fused kernel.  grid ceil(T/64), block 128.
+__global__ void __launch_bounds__(128)
+    topk_from_partials_kernel(const float* __restrict__ partial, int S,
+                              const float* __restrict__ b_router, int T, int E, int k,
+                              int32_t* __restrict__ topk_idx, float* __restrict__ topk_w,
+                              int32_t* __restrict__ block_counts) {
+  extern __shared__ __align__(128) uint8_t smem_raw[];
+  float* lg = reinterpret_cast<float*>(smem_raw);           // [64][E+1]
+  int32_t* cnt = reinterpret_cast<int32_t*>(lg + kRouterTcTokens * (E + 1));  // [E]
+  int32_t* sel = cnt + E;                                    // [64][k]
+  const int tid = threadIdx.x;
+  const int t0 = blockIdx.x * kRouterTcTokens, nt = min(kRouterTcTokens, T - t0);
+  pdl_wait();
+  pdl_launch_next();
+  for (int i = tid; i < E; i += blockDim.x) cnt[i] = 0;
+  for (int i = tid; i < nt * E; i += blockDim.x) {
+    const int tt = i / E, e = i - tt * E;
+    const size_t at = (size_t)(t0 + tt) * E + e;
+    float v = 0.f;
+    int s = 0;
+    for (; s + 8 <= S; s += 8) {
+      float p[8];
+#pragma unroll
+      for (int q = 0; q < 8; ++q) p[q] = partial[(size_t)(s + q) * T * E + at];
+#pragma unroll
+      for (int q = 0; q < 8; ++q) v += p[q];
     }
-    __syncwarp();
+    for (; s < S; ++s) v += partial[(size_t)s * T * E + at];
+    lg[tt * (E + 1) + e] = v + b_router[e];
   }
   __syncthreads();
-  for (int e = tid; e < E; e += blockDim.x) block_counts[(size_t)blockIdx.x * E + e] = cnt[e];
+  topk_block_epilogue(lg, E + 1, nt, t0, E, k, sel, cnt, topk_idx, topk_w, block_counts);
 }
 
 // ---------------------------------------------------------------------------------------
