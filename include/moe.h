@@ -178,8 +178,11 @@ MOE_API const char* moe_profile_kind_name(int kind);
  * array of moe_route_static_max_bytes() bytes (2 MiB) compiled into the library, which every
  * device that loads the library keeps until the process exits.
  *   - The handle's device must be the current device (MOE_ERR_ARG otherwise).
- *   - If moe_route_workspace_bytes(ctx, T) exceeds the array, the call returns
- *     MOE_ERR_WORKSPACE and enqueues nothing (for H = 2880, E = 32: every T up to 2^20).
+ *   - If the routing scratch for T does not fit in the array, the call returns
+ *     MOE_ERR_WORKSPACE and enqueues nothing.  The scratch is (H/64)*T*E*4 bytes of partial
+ *     logits for T <= 64 and ceil(T/64)*E*4 bytes of per-block expert counts above that; with
+ *     H = 2880 it fits for E = 32 up to T = 1,048,320, for E = 128 up to T = 262,016, and for
+ *     E = 256 for T <= 45 and 65 <= T <= 130,944.
  *   - The first call on a device looks up the array's device address (a runtime call that
  *     does not allocate); make that first call before any stream capture.
  *   - All calls share the one array: two calls whose work overlaps on the GPU (different

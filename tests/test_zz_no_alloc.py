@@ -59,14 +59,16 @@ def test_static_scratch_route_matches_workspace_route(T):
 
 
 def test_static_scratch_rejects_sizes_beyond_its_array():
-    # 128 experts x 64 tokens of partial logits over 45 hidden slices need 1.47 MB: fits;
-    # 256 experts need 2.95 MB: more than the 2 MiB array, refused before any launch.
+    # Refused before anything is launched: 256 experts x 64 tokens need 45 x 64 x 256 x 4 B of
+    # partial logits (2.9 MB) and 131,008 tokens need 2047 blocks x 1 KB of per-block expert
+    # counts, both more than the 2 MiB array; 128 experts x 64 tokens (1.5 MB) and 256 experts
+    # x 130,944 tokens (2046 KB) fit.
     assert moe.moe_route_static_max_bytes() == 2 << 20
-    for E, ok in ((128, True), (256, False)):
-        layer = moe.Moe(E, 2880, 64, 4)
-        d = mi.make_inputs(64, 2880, E, 4, 64, seed=7, device="cuda", experts=False)
-        o = _outputs(64, 4, E)
-        assert (layer.route_workspace_bytes(64) <= moe.moe_route_static_max_bytes()) == ok
+    for E, T, H, ok in ((128, 64, 2880, True), (256, 64, 2880, False),
+                        (256, 130944, 64, True), (256, 131008, 64, False)):
+        layer = moe.Moe(E, H, 64, 4)
+        d = mi.make_inputs(T, H, E, 4, 64, seed=7, device="cuda", experts=False)
+        o = _outputs(T, 4, E)
         st = _call_static(layer, d, o)
-        assert st == (moe.MOE_OK if ok else moe.MOE_ERR_WORKSPACE)
+        assert st == (moe.MOE_OK if ok else moe.MOE_ERR_WORKSPACE), (E, T)
     torch.cuda.synchronize()
