@@ -172,3 +172,37 @@ def test_tune_measures_a_crossover_and_auto_follows_it():
     assert 0 <= c <= 256
     print("measured crossover T* =", c)
     assert layer.sync_status() == moe.MOE_OK
+
+
+@pytest.mark.parametrize("T,path", [(10, "stream"), (100, "gemm")])
+def test_forward_with_k_equal_E_256(T, path):
+    """Every token uses all 256 experts (the widest routing the ABI accepts)."""
+    p = moe.MOE_PATH_STREAM if path == "stream" else moe.MOE_PATH_GEMM
+    d, h = inputs_on_gpu(T, 64, 256, 256, 64, seed=1300 + T)
+    _check_layer(d, h, 256, 64, 64, 256, path=p)
+
+
+def test_largest_token_count():
+    """T = 2^20 (the largest T the ABI accepts) on a narrow layer; routing is checked on every
+    token, outputs on a seeded sample."""
+    T, H, E, k, I = 1 << 20, 64, 8, 2, 64
+    d, h = inputs_on_gpu(T, H, E, k, I, seed=1400)
+    layer = moe.Moe(E, H, I, k)
+    ref_route = host_route(h, k)
+    g = gpu_route(layer, d)
+    compare_routing(g, ref_route, k, E)
+    out = layer.forward(d["x"], d["W_router"], d["b_router"], d["W_gate_up"], d["W_down"])
+    assert layer.sync_status() == moe.MOE_OK
+    tokens = mi.sample_tokens(T, 2048, 1400)
+    got = out[torch.from_numpy(tokens).cuda()].double().cpu().numpy()
+    ref = oracle.moe_forward_ref(h["x"], h["W_router"], h["b_router"], h["W_gate_up"], h["W_down"],
+                                 k, tokens=tokens, route=ref_route)
+    check_outputs(got, tokens, h, ref_route, g, ref)
+
+
+@pytest.mark.parametrize("path", ["stream", "gemm"])
+def test_wide_hidden_and_intermediate(path):
+    """H = I = 8192: long K loops and many column tiles in both paths."""
+    p = moe.MOE_PATH_STREAM if path == "stream" else moe.MOE_PATH_GEMM
+    d, h = inputs_on_gpu(24, 8192, 2, 1, 8192, seed=1500)
+    _check_layer(d, h, 2, 8192, 8192, 1, path=p)
