@@ -45,6 +45,8 @@ struct GemmArgs {
   float* out;            // down: [T, H] fp32, zero on entry
   int H;
   uint32_t* status;
+  float4* zero4;         // gate/up: region its epilogue warps zero-fill (the down output), or null
+  size_t n_zero4;
 };
 
 MOE_DEVINL bool wait_or_abort(uint64_t* bar, uint32_t parity, volatile int* abort_flag,
@@ -248,6 +250,21 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
     // ------------------------------ epilogue (both CTAs) ------------------------------
     const int q = warp & 3;
     const int row = 32 * q + lane;
+    // gate/up: zero-fill this CTA's share of the down projection's output, one piece after
+    // each tile (the tensor cores run meanwhile; the rest of the share after the last tile)
+    size_t z_beg = 0, z_end = 0, z_piece = 0;
+    if (MODE == 0 && a.zero4 != nullptr) {
+      const size_t per = (a.n_zero4 + gridDim.x - 1) / gridDim.x;
+      z_beg = min(a.n_zero4, (size_t)blockIdx.x * per);
+      z_end = min(a.n_zero4, z_beg + per);
+      const int my_tiles = max(1, (tiles - pair + npairs - 1) / npairs);
+      z_piece = ((z_end - z_beg + my_tiles - 1) / my_tiles + 127) / 128 * 128;
+    }
+    const int et = tid - kGemmEpiWarp0 * 32;  // 0..127
+    auto zero_piece = [&](size_t stop) {
+      for (size_t i = z_beg + et; i < stop; i += 128) a.zero4[i] = make_float4(0.f, 0.f, 0.f, 0.f);
+      z_beg = stop;
+    };
     int tile_i = 0;
     for (int t = pair; t < tiles; t += npairs, ++tile_i) {
       const int buf = tile_i % C::kAccBufs;
@@ -303,7 +320,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
       }
       tc_fence_before();
       mbar_arrive_cluster(mapa_shared(smem_u32(&acc_empty[buf]), 0));
+      if (MODE == 0 && z_beg < z_end) zero_piece(min(z_end, z_beg + z_piece));
     }
+    if (MODE == 0 && z_beg < z_end) zero_piece(z_end);
   }
 
   tc_fence_before();

@@ -288,6 +288,8 @@ cudaError_t launch_router_tc(int NB, cudaStream_t st, const uint16_t* x, const u
                     block_counts, zero4, n_zero4, rt.kc_per_split, partial);
 }
 
+constexpr int kTopkMaxSlices = 8;  // partial-logit slices topk_from_partials sums itself
+
 // Routing chain.  zero4/n_zero4: a float scratch region the router kernel zero-fills.
 moe_status launch_route(moe_ctx* c, int T, const uint16_t* x, const uint16_t* Wr,
                         const float* b, const RouteOut& o, uint8_t* ws, const RouteTmp& rt,
@@ -325,17 +327,20 @@ moe_status launch_route(moe_ctx* c, int T, const uint16_t* x, const uint16_t* Wr
     return launch_router_tc<32>(NB, st, x, Wr, b, T, H, E, k, o, block_counts, zero4, n_zero4, rt, split_partial);
   }));
   if (split_partial) {
+    // a few slices are summed by the top-k kernel itself; many first by a wide kernel
+    const bool presum = rt.splits > kTopkMaxSlices;
     const int n = T * E;
-    MOE_TRY(launch(c, kKindRouter, st, [&] {
-      return launch_pdl(sum_partials_kernel, dim3((n + 255) / 256), dim3(256), 0, st,
-                        split_partial, rt.splits, n);
-    }));
+    if (presum)
+      MOE_TRY(launch(c, kKindRouter, st, [&] {
+        return launch_pdl(sum_partials_kernel, dim3((n + 255) / 256), dim3(256), 0, st,
+                          split_partial, rt.splits, n);
+      }));
     const size_t smem_t = (size_t)kRouterTcTokens * (E + 1) * 4 + (size_t)E * 4 +
                           (size_t)kRouterTcTokens * k * 4;
     MOE_TRY(launch(c, kKindRouter, st, [&] {
       return launch_pdl(topk_from_partials_kernel, dim3(NB), dim3(128), smem_t, st,
-                        (const float*)split_partial, 1, b, T, E, k, o.topk_idx, o.topk_w,
-                        block_counts);
+                        (const float*)split_partial, presum ? 1 : rt.splits, b, T, E, k,
+                        o.topk_idx, o.topk_w, block_counts);
     }));
   }
   MOE_TRY(launch(c, kKindRouteFin, st, [&] {
@@ -495,9 +500,8 @@ moe_status forward_gemm(moe_ctx* c, int T, const void* x_bf16, const void* W_rou
     o.x_perm = x_perm;
     o.H = c->H;
   }
-  // the router kernel zero-fills `out`, which the down projection accumulates into
   MOE_TRY(launch_route(c, T, x, static_cast<const uint16_t*>(W_router_bf16), b_router, o, ws,
-                       L.rt, st, out, (size_t)T * c->H));
+                       L.rt, st));
   if (!fused_copy)
     MOE_TRY(launch(c, kKindGather, st, [&] {
       return launch_pdl(gather_rows_kernel, dim3((unsigned)((R + 7) / 8)), dim3(256), 0, st, x,
@@ -517,6 +521,9 @@ moe_status forward_gemm(moe_ctx* c, int T, const void* x_bf16, const void* W_rou
   g.h = h;
   g.H = c->H;
   g.status = c->d_status;
+  // the gate/up epilogue zero-fills `out`, which the down projection accumulates into
+  g.zero4 = reinterpret_cast<float4*>(out);
+  g.n_zero4 = (size_t)T * c->H / 4;
   const int grid = c->num_sms & ~1;  // whole CTA pairs
   MOE_TRY(launch(c, kKindGateUp, st, [&] {
     return launch_pdl(grouped_gemm_2sm_kernel<MOE_GEMM_GATE_UP>, dim3(grid), dim3(kGemmThreads),

@@ -91,6 +91,70 @@ MOE_DEVINL void warp_topk(float* lg, int E, int k, int32_t* sel) {
   }
 }
 
+// ---------------------------------------------------------------------------------------
+// top-k of one token held by one thread (k <= K <= kThreadTopK): bv/be receive the k largest
+// of row[0..E) in descending order.  Experts are scanned in ascending order and a later expert
+// ranks above a held one only when strictly larger, so equal logits go to the lower expert
+// index, as in the warp version above.  Branch-free insertion, all slots in registers.
+// ---------------------------------------------------------------------------------------
+constexpr int kThreadTopK = 8;
+
+template <int K>
+MOE_DEVINL void thread_topk(const float* row, int E, int k, float (&bv)[K], int (&be)[K]) {
+#pragma unroll
+  for (int j = 0; j < K; ++j) {
+    bv[j] = -INFINITY;
+    be[j] = -1;  // empty slot
+  }
+  for (int e = 0; e < E; ++e) {
+    const float v = row[e];
+    bool gt[K];  // v ranks above slot j (slots past k never do)
+#pragma unroll
+    for (int j = 0; j < K; ++j) gt[j] = j < k && (be[j] < 0 || v > bv[j]);
+    // gt is monotone (gt[j-1] implies gt[j]): slot j takes slot j-1's entry when v ranks above
+    // j-1, else v itself when it ranks above j
+#pragma unroll
+    for (int j = K - 1; j > 0; --j) {
+      bv[j] = gt[j - 1] ? bv[j - 1] : (gt[j] ? v : bv[j]);
+      be[j] = gt[j - 1] ? be[j - 1] : (gt[j] ? e : be[j]);
+    }
+    bv[0] = gt[0] ? v : bv[0];
+    be[0] = gt[0] ? e : be[0];
+  }
+}
+
+// In place: the selected logits bv[0..k) (bv[0] the largest) become their softmax weights,
+// the denominator summed in slot order.
+template <int K>
+MOE_DEVINL void thread_softmax(int k, float (&bv)[K]) {
+  const float top = bv[0];
+  float denom = 0.f;
+#pragma unroll
+  for (int j = 0; j < K; ++j) {
+    bv[j] = (j < k) ? expf(bv[j] - top) : 0.f;
+    denom += bv[j];
+  }
+#pragma unroll
+  for (int j = 0; j < K; ++j) bv[j] = bv[j] / denom;
+}
+
+// One token per thread: top-k, weights, the token's outputs and the block histogram.
+template <int K>
+MOE_DEVINL void thread_route_token(const float* row, int E, int k, size_t t,
+                                   int32_t* topk_idx, float* topk_w, int32_t* cnt) {
+  float bv[K];
+  int be[K];
+  thread_topk<K>(row, E, k, bv, be);
+  thread_softmax<K>(k, bv);
+#pragma unroll
+  for (int j = 0; j < K; ++j)
+    if (j < k) {
+      topk_idx[t * k + j] = be[j];
+      topk_w[t * k + j] = bv[j];
+      atomicAdd(&cnt[be[j]], 1);
+    }
+}
+
 // Routing weights of one token (softmax over its k selected logits, lg[0] the largest).
 MOE_DEVINL float warp_softmax_denominator(const float* lg, int k) {
   const int lane = threadIdx.x & 31;
@@ -103,11 +167,24 @@ MOE_DEVINL float warp_softmax_denominator(const float* lg, int k) {
 }
 
 // Top-k, softmax and the block's expert histogram for up to 64 tokens whose logits (bias added)
-// are in shared memory, row stride `ld`; one warp per token.  Ends with the block's counts.
+// are in shared memory, row stride `ld` (odd, so one-thread-per-token reads are free of bank
+// conflicts); one thread per token for k <= kThreadTopK, else one warp.  Ends with the block's
+// counts.
 MOE_DEVINL void topk_block_epilogue(float* lg, int ld, int nt, int t0, int E, int k, int32_t* sel,
                                     int32_t* cnt, int32_t* topk_idx, float* topk_w,
                                     int32_t* block_counts) {
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5, nwarps = blockDim.x >> 5;
+  if (k <= kThreadTopK) {  // one thread per token (blockDim >= 64 >= nt)
+    if (tid < nt) {
+      if (k <= 4)
+        thread_route_token<4>(lg + tid * ld, E, k, (size_t)(t0 + tid), topk_idx, topk_w, cnt);
+      else
+        thread_route_token<8>(lg + tid * ld, E, k, (size_t)(t0 + tid), topk_idx, topk_w, cnt);
+    }
+    __syncthreads();
+    for (int e = tid; e < E; e += blockDim.x) block_counts[(size_t)blockIdx.x * E + e] = cnt[e];
+    return;
+  }
   for (int tt = warp; tt < nt; tt += nwarps) {
     float* row = lg + tt * ld;
     int32_t* srow = sel + tt * k;
@@ -466,40 +543,53 @@ __global__ void __launch_bounds__(256) sum_partials_kernel(float* __restrict__ p
 }
 
 // Large T with too few token blocks to fill the GPU: the router kernel runs split over the hidden
-// dimension and writes partial logits [S, T, E] (summed into slice 0 by sum_partials_kernel when
-// S > 1); this kernel sums what it is given in slice order, adds the bias and finishes the
-// 64-token block like the fused kernel.  grid ceil(T/64), block 128.
+// dimension and writes partial logits [S, T, E] (for many slices first summed into slice 0 by
+// sum_partials_kernel); this kernel sums the slices it is given in slice order, adds the bias and
+// finishes the 64-token block like the fused kernel.  grid ceil(T/64), block 128.
 __global__ void __launch_bounds__(128)
     topk_from_partials_kernel(const float* __restrict__ partial, int S,
                               const float* __restrict__ b_router, int T, int E, int k,
                               int32_t* __restrict__ topk_idx, float* __restrict__ topk_w,
                               int32_t* __restrict__ block_counts) {
   extern __shared__ __align__(128) uint8_t smem_raw[];
-  float* lg = reinterpret_cast<float*>(smem_raw);           // [64][E+1]
-  int32_t* cnt = reinterpret_cast<int32_t*>(lg + kRouterTcTokens * (E + 1));  // [E]
+  const int P = E | 1;                                       // odd row pitch
+  float* lg = reinterpret_cast<float*>(smem_raw);           // [64][P]
+  int32_t* cnt = reinterpret_cast<int32_t*>(lg + kRouterTcTokens * P);  // [E]
   int32_t* sel = cnt + E;                                    // [64][k]
   const int tid = threadIdx.x;
   const int t0 = blockIdx.x * kRouterTcTokens, nt = min(kRouterTcTokens, T - t0);
   pdl_wait();
   pdl_launch_next();
   for (int i = tid; i < E; i += blockDim.x) cnt[i] = 0;
-  for (int i = tid; i < nt * E; i += blockDim.x) {
-    const int tt = i / E, e = i - tt * E;
-    const size_t at = (size_t)(t0 + tt) * E + e;
-    float v = 0.f;
-    int s = 0;
-    for (; s + 8 <= S; s += 8) {
-      float p[8];
+  // this block's logits are one contiguous run of nt * E floats in every slice; eight
+  // independent loads per thread in flight, slices added in order
+  const int n = nt * E;
+  const float* src = partial + (size_t)t0 * E;
+  const size_t TE = (size_t)T * E;
+  for (int base = tid; base < n; base += 8 * blockDim.x) {
+    float v[8];
 #pragma unroll
-      for (int q = 0; q < 8; ++q) p[q] = partial[(size_t)(s + q) * T * E + at];
-#pragma unroll
-      for (int q = 0; q < 8; ++q) v += p[q];
+    for (int q = 0; q < 8; ++q) {
+      const int i = base + q * blockDim.x;
+      v[q] = i < n ? src[i] : 0.f;
     }
-    for (; s < S; ++s) v += partial[(size_t)s * T * E + at];
-    lg[tt * (E + 1) + e] = v + b_router[e];
+    for (int s = 1; s < S; ++s)
+#pragma unroll
+      for (int q = 0; q < 8; ++q) {
+        const int i = base + q * blockDim.x;
+        if (i < n) v[q] += src[s * TE + i];
+      }
+#pragma unroll
+    for (int q = 0; q < 8; ++q) {
+      const int i = base + q * blockDim.x;
+      if (i < n) {
+        const int tt = i / E, e = i - tt * E;
+        lg[tt * P + e] = v[q] + b_router[e];
+      }
+    }
   }
   __syncthreads();
-  topk_block_epilogue(lg, E + 1, nt, t0, E, k, sel, cnt, topk_idx, topk_w, block_counts);
+  topk_block_epilogue(lg, P, nt, t0, E, k, sel, cnt, topk_idx, topk_w, block_counts);
 }
 
 // ---------------------------------------------------------------------------------------
@@ -629,7 +719,16 @@ __global__ void __launch_bounds__(256) gather_rows_kernel(const uint16_t* __rest
   if (r >= R) return;
   const uint4* src = reinterpret_cast<const uint4*>(x + (size_t)perm[r] * H);
   uint4* dst = reinterpret_cast<uint4*>(x_perm + (size_t)r * H);
-  for (int c = lane; c < H / 8; c += 32) dst[c] = src[c];
+  const int n = H / 8;
+  int c = lane;
+  for (; c + 96 < n; c += 128) {  // four loads in flight before the stores
+    const uint4 v0 = src[c], v1 = src[c + 32], v2 = src[c + 64], v3 = src[c + 96];
+    dst[c] = v0;
+    dst[c + 32] = v1;
+    dst[c + 64] = v2;
+    dst[c + 96] = v3;
+  }
+  for (; c < n; c += 32) dst[c] = src[c];
 }
 
 }  // namespace moe
