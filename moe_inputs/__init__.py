@@ -14,6 +14,13 @@ here; these draws stand in for them with the same shapes):
   x ~ N(0, 1); W_router [H,E] and W_gate_up [E,H,2I] ~ N(0, 1/H); W_down [E,I,H] ~ N(0, 1/I);
   b_router ~ N(0, 0.1) kept in float32.  N(m, v) names the variance v;
 * W_gate_up and W_down are drawn one expert at a time (``[H,2I]`` then the next expert);
+* MXFP4 experts (``weights="mxfp4"``): ``gu_blocks [E, 2I, H/2]``, ``gu_scales [E, H/32, 2I]``,
+  ``dn_blocks [E, H, I/2]``, ``dn_scales [E, I/32, H]`` (uint8; the layout the oracle's
+  ``dequant_mxfp4`` reads).  Every block byte is uniform on 0..255 (two uniform 4-bit codes);
+  every scale byte is s0 + {-1, 0, +1} uniformly, with s0 = 127 + round(log2(1 / (4 *
+  sqrt(fan_in)))), which puts the dequantized weights' spread near 1/sqrt(fan_in) like the bf16
+  draws (0.8/sqrt(fan_in) at fan_in = 2880).  Slots 7 (gate/up) and 8 (down), drawn one expert
+  at a time (blocks, then scales);
 * skewed routing adds ``-c * s * ln(rank_e)`` to b_router, rank a seeded permutation of
   1..E and s = 1.1, so expert popularity falls off like a Zipf law.  c is the scale that gives
   a max/mean expert load of 4.0 on a 4096-token sample; it is computed by
@@ -48,6 +55,7 @@ class Workload:
     zipf: bool = False
     oracle_sample: int = 0          # 0: the oracle checks every token
     sweep: tuple = field(default=())  # token counts of a sweep (T is the largest)
+    weights: str = "bf16"             # expert weight format: "bf16" or "mxfp4"
 
 
 # The five workloads: a tiny layer; the 20b layer (H = I = 2880, 32 experts, top-4) in decode
@@ -61,6 +69,9 @@ WORKLOADS = {
                             zipf=True, oracle_sample=4096),
     "120b_sweep": Workload("120b_sweep", T=32, H=2880, E=128, k=4, I=2880, seed=4,
                            sweep=(1, 8, 12, 16, 32)),
+    # the 20b decode layer with its experts in their native MXFP4 format (W4A16)
+    "20b_decode_mxfp4": Workload("20b_decode_mxfp4", T=16, H=2880, E=32, k=4, I=2880, seed=5,
+                                 weights="mxfp4"),
 }
 
 
@@ -97,6 +108,30 @@ def draw_router(H: int, E: int, seed: int, device="cpu", zipf: bool = False,
     return W_router, b_router
 
 
+def _mx_scale_center(fan_in: int) -> int:
+    return 127 + int(round(math.log2(1.0 / (4.0 * math.sqrt(fan_in)))))
+
+
+def _draw_mx(E: int, N: int, K: int, seed: int, slot: int, device):
+    g = _gen(seed, slot, device)
+    blocks = torch.empty((E, N, K // 2), dtype=torch.uint8, device=device)
+    scales = torch.empty((E, K // 32, N), dtype=torch.uint8, device=device)
+    s0 = _mx_scale_center(K)
+    for e in range(E):
+        blocks[e] = torch.randint(0, 256, (N, K // 2), generator=g, device=device,
+                                  dtype=torch.int32).to(torch.uint8)
+        scales[e] = (torch.randint(-1, 2, (K // 32, N), generator=g, device=device,
+                                   dtype=torch.int32) + s0).to(torch.uint8)
+    return blocks, scales
+
+
+def draw_experts_mxfp4(E: int, H: int, I: int, seed: int, device="cpu"):
+    """MXFP4 experts: (gu_blocks, gu_scales, dn_blocks, dn_scales), see the module recipe."""
+    gu_blocks, gu_scales = _draw_mx(E, 2 * I, H, seed, 7, device)
+    dn_blocks, dn_scales = _draw_mx(E, H, I, seed, 8, device)
+    return gu_blocks, gu_scales, dn_blocks, dn_scales
+
+
 def draw_experts(E: int, H: int, I: int, seed: int, device="cpu"):
     W_gate_up = torch.empty((E, H, 2 * I), dtype=torch.bfloat16, device=device)
     g = _gen(seed, 3, device)
@@ -112,12 +147,18 @@ def draw_experts(E: int, H: int, I: int, seed: int, device="cpu"):
 
 
 def make_inputs(T: int, H: int, E: int, k: int, I: int, seed: int, device="cpu",
-                zipf: bool = False, experts: bool = True) -> dict:
-    """All inputs of one layer call as torch tensors on ``device`` (see the module recipe)."""
+                zipf: bool = False, experts: bool = True, weights: str = "bf16") -> dict:
+    """All inputs of one layer call as torch tensors on ``device`` (see the module recipe).
+
+    weights="bf16" gives W_gate_up / W_down; "mxfp4" gives gu_blocks, gu_scales, dn_blocks,
+    dn_scales instead."""
     x = draw_x(T, H, seed, device)
     W_router, b_router = draw_router(H, E, seed, device, zipf)
     d = dict(x=x, W_router=W_router, b_router=b_router, T=T, H=H, E=E, k=k, I=I)
-    if experts:
+    if experts and weights == "mxfp4":
+        (d["gu_blocks"], d["gu_scales"], d["dn_blocks"],
+         d["dn_scales"]) = draw_experts_mxfp4(E, H, I, seed, device)
+    elif experts:
         d["W_gate_up"], d["W_down"] = draw_experts(E, H, I, seed, device)
     return d
 
@@ -125,7 +166,7 @@ def make_inputs(T: int, H: int, E: int, k: int, I: int, seed: int, device="cpu",
 def workload_inputs(name: str, device="cpu", T: int | None = None, experts: bool = True) -> dict:
     w = WORKLOADS[name]
     return make_inputs(w.T if T is None else T, w.H, w.E, w.k, w.I, w.seed, device, w.zipf,
-                       experts)
+                       experts, w.weights)
 
 
 def sample_tokens(T: int, n: int, seed: int) -> np.ndarray:

@@ -25,6 +25,16 @@ each bf16 value widened exactly):
     SwiGLU expert but print no formula; this is its plain form.
 * combine             out[t] = sum_j w[t,j] * y_(t, S_j)   in float64.
 
+MXFP4 expert weights (W4A16).  The checkpoints' experts are natively MXFP4 with bf16
+activations (Persona Kappa forum post, "Quantization-Aware Training"; kappa-20b-131k card,
+"Architecture"); the pages name the format only.  This oracle reads it as the OCP Microscaling
+(MX) v1.0 FP4 format: E2M1 elements (sign, 2 exponent bits with bias 1, 1 mantissa bit;
+exponent 0 is subnormal) in blocks of 32 consecutive elements along the reduction dimension,
+each block sharing one E8M0 scale 2^(s-127) (s = 255 encodes NaN).  Storage of one expert's
+[K, N] matrix: ``blocks [N, K/2]`` uint8 (byte j of row n holds element k = 2j in bits 0-3 and
+k = 2j + 1 in bits 4-7) and ``scales [K/32, N]`` uint8.  The dequantized weights then enter the
+same float64 layer as the bf16 ones.
+
 Nothing is rounded between steps: the GPU rounds the SwiGLU output h to bf16 before the down
 projection and accumulates in fp32; those differences are what the tests' tolerance covers.
 
@@ -51,6 +61,10 @@ __all__ = [
     "moe_route_ref",
     "moe_forward_ref",
     "moe_token_output_ref",
+    "decode_e2m1",
+    "decode_e8m0",
+    "dequant_mxfp4",
+    "moe_forward_mxfp4_ref",
 ]
 
 
@@ -189,6 +203,20 @@ def moe_route_ref(x_bits, W_router_bits, b_router, k: int) -> dict:
                 inv_perm=inv_perm, gap_k=gap_k, gap_in=gap_in)
 
 
+def _layer_out(x_bits, route, tokens, gate_up_of, down_of) -> np.ndarray:
+    """out[t] = sum_j w[t,j] * expert_mlp(x[t], e = idx[t,j]); experts come from the getters."""
+    T, H = x_bits.shape
+    toks = np.arange(T) if tokens is None else np.asarray(tokens, dtype=np.int64)
+    idx, w = route["idx"][toks], route["w"][toks]
+    xs = decode_bf16(x_bits[toks])
+    out = np.zeros((toks.size, H), dtype=np.float64)
+    for e in np.unique(idx):
+        rows, slots = np.nonzero(idx == e)
+        y = expert_mlp(xs[rows], gate_up_of(e), down_of(e))
+        out[rows] += w[rows, slots][:, None] * y
+    return out
+
+
 def moe_forward_ref(x_bits, W_router_bits, b_router, W_gate_up_bits, W_down_bits, k: int,
                     tokens=None, route: dict | None = None) -> np.ndarray:
     """Whole layer: out[t] = sum_j w[t,j] * expert_mlp(x[t], e = idx[t,j]) in float64.
@@ -200,16 +228,49 @@ def moe_forward_ref(x_bits, W_router_bits, b_router, W_gate_up_bits, W_down_bits
     """
     if route is None:
         route = moe_route_ref(x_bits, W_router_bits, b_router, k)
-    T, H = x_bits.shape
-    toks = np.arange(T) if tokens is None else np.asarray(tokens, dtype=np.int64)
-    idx, w = route["idx"][toks], route["w"][toks]
-    xs = decode_bf16(x_bits[toks])
-    out = np.zeros((toks.size, H), dtype=np.float64)
-    for e in np.unique(idx):
-        rows, slots = np.nonzero(idx == e)
-        y = expert_mlp(xs[rows], decode_bf16(W_gate_up_bits[e]), decode_bf16(W_down_bits[e]))
-        out[rows] += w[rows, slots][:, None] * y
-    return out
+    return _layer_out(x_bits, route, tokens, lambda e: decode_bf16(W_gate_up_bits[e]),
+                      lambda e: decode_bf16(W_down_bits[e]))
+
+
+def decode_e2m1(codes) -> np.ndarray:
+    """FP4 E2M1 element codes (low 4 bits) to float64.
+
+    Bit 3 is the sign, bits 2-1 the exponent field e (bias 1), bit 0 the mantissa m:
+    e = 0 gives the subnormal m * 2^(1-1) * 0.5 = m / 2, otherwise 2^(e-1) * (1 + m / 2).
+    """
+    c = np.asarray(codes).astype(np.int64) & 0xF
+    sign, e, m = c >> 3, (c >> 1) & 3, c & 1
+    mag = np.where(e == 0, 0.5 * m, np.ldexp(1.0 + 0.5 * m, e - 1))
+    return np.where(sign == 1, -mag, mag)
+
+
+def decode_e8m0(s) -> np.ndarray:
+    """E8M0 shared scale codes to float64: 2^(s - 127), and NaN for s = 255."""
+    s = np.asarray(s).astype(np.int64)
+    return np.where(s == 255, np.nan, np.ldexp(1.0, np.minimum(s, 254) - 127))
+
+
+def dequant_mxfp4(blocks, scales) -> np.ndarray:
+    """MXFP4 matrices to float64: blocks [..., N, K/2] uint8, scales [..., K/32, N] uint8 ->
+    W [..., K, N] with W[k, n] = e2m1(element k of row n) * 2^(scales[k // 32, n] - 127)."""
+    b = np.asarray(blocks, dtype=np.uint8)
+    codes = np.stack([b & 0xF, b >> 4], axis=-1).reshape(*b.shape[:-1], 2 * b.shape[-1])
+    vals = np.swapaxes(decode_e2m1(codes), -1, -2)            # [..., K, N]
+    return vals * np.repeat(decode_e8m0(scales), 32, axis=-2)  # scale rows repeat per block
+
+
+def moe_forward_mxfp4_ref(x_bits, W_router_bits, b_router, gu_blocks, gu_scales, dn_blocks,
+                          dn_scales, k: int, tokens=None, route: dict | None = None) -> np.ndarray:
+    """Whole layer with MXFP4 experts: the bf16 layer above on the dequantized weights.
+
+    gu_blocks [E, 2I, H/2], gu_scales [E, H/32, 2I] hold W_gate_up [E, H, 2I] (gate columns
+    [0, I), up columns [I, 2I)); dn_blocks [E, H, I/2], dn_scales [E, I/32, H] hold W_down
+    [E, I, H].  Activations and the router stay bf16.
+    """
+    if route is None:
+        route = moe_route_ref(x_bits, W_router_bits, b_router, k)
+    return _layer_out(x_bits, route, tokens, lambda e: dequant_mxfp4(gu_blocks[e], gu_scales[e]),
+                      lambda e: dequant_mxfp4(dn_blocks[e], dn_scales[e]))
 
 
 def moe_token_output_ref(x_bits_t, logits_t, experts, W_gate_up_bits, W_down_bits) -> np.ndarray:
