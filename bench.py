@@ -154,11 +154,15 @@ class ClockSampler:
 # ----------------------------------------------------------------------------------------
 # algorithmic work (what the method must touch)
 # ----------------------------------------------------------------------------------------
-def algorithmic(T: int, H: int, E: int, k: int, I: int, counts) -> dict:
+def algorithmic(T: int, H: int, E: int, k: int, I: int, counts, weights: str = "bf16") -> dict:
     touched = int(sum(1 for c in counts if c > 0))
     R = T * k
-    w_gate_up = touched * H * 2 * I * 2
-    w_down = touched * I * H * 2
+    if weights == "mxfp4":   # 4-bit codes + one scale byte per 32 elements
+        w_gate_up = touched * (H * 2 * I // 2 + H // 32 * 2 * I)
+        w_down = touched * (I * H // 2 + I // 32 * H)
+    else:
+        w_gate_up = touched * H * 2 * I * 2
+        w_down = touched * I * H * 2
     gate_up_bytes = w_gate_up + T * H * 2 + R * I * 2          # weights + x read + h write
     down_bytes = w_down + R * I * 2 + T * H * 4                 # weights + h read + out write
     layer_bytes = w_gate_up + w_down + H * E * 2 + T * H * 2 + T * H * 4
@@ -187,7 +191,12 @@ def oracle_time(h: dict, k: int, n_tokens: int, reps: int) -> float:
     x = h["x"][:n_tokens]
     t0 = time.perf_counter()
     for _ in range(reps):
-        oracle.moe_forward_ref(x, h["W_router"], h["b_router"], h["W_gate_up"], h["W_down"], k)
+        if "gu_codes" in h:
+            oracle.moe_forward_mxfp4_ref(x, h["W_router"], h["b_router"], h["gu_codes"],
+                                         h["gu_scales"], h["dn_codes"], h["dn_scales"], k)
+        else:
+            oracle.moe_forward_ref(x, h["W_router"], h["b_router"], h["W_gate_up"], h["W_down"],
+                                   k)
     return time.perf_counter() - t0
 
 
@@ -204,7 +213,8 @@ def run_reference(args, w: mi.Workload, T: int) -> None:
     rank, world, _ = dist_env()
     if rank != 0:
         return
-    h = mi.host_inputs(mi.make_inputs(T, w.H, w.E, w.k, w.I, w.seed, "cpu", zipf=w.zipf))
+    h = mi.host_inputs(mi.make_inputs(T, w.H, w.E, w.k, w.I, w.seed, "cpu", zipf=w.zipf,
+                                      weights=w.weights))
     budget = 150.0 / (args.steps + args.warmup)          # whole run within a few minutes
     t1 = oracle_time(h, w.k, 1, 1)
     n = max(1, min(T, int(budget / max(t1, 1e-3))))
@@ -238,19 +248,27 @@ def run_ours(args, w: mi.Workload, T: int) -> None:
     import mixture_experts_layer_48_b200 as moe
 
     seed = w.seed + 7919 * rank          # every rank its own tokens (weights identical)
-    d = mi.make_inputs(T, w.H, w.E, w.k, w.I, w.seed, "cuda", zipf=w.zipf)
+    d = mi.make_inputs(T, w.H, w.E, w.k, w.I, w.seed, "cuda", zipf=w.zipf, weights=w.weights)
     if rank:
         d["x"] = mi.draw_x(T, w.H, seed, "cuda")
     layer = moe.Moe(w.E, w.H, w.I, w.k)
     counts = torch.diff(layer.route(d["x"], d["W_router"], d["b_router"])["expert_offsets"]).cpu().tolist()
-    alg = algorithmic(T, w.H, w.E, w.k, w.I, counts)
+    alg = algorithmic(T, w.H, w.E, w.k, w.I, counts, w.weights)
     out = torch.empty((T, w.H), dtype=torch.float32, device="cuda")
-    ws = torch.empty(layer.workspace_bytes(T), dtype=torch.uint8, device="cuda")
-    args_fwd = (d["x"], d["W_router"], d["b_router"], d["W_gate_up"], d["W_down"])
+    mx = w.weights == "mxfp4"
+    if mx:
+        fwd = layer.forward_mxfp4
+        ws = torch.empty(layer.workspace_bytes_mxfp4(T), dtype=torch.uint8, device="cuda")
+        args_fwd = (d["x"], d["W_router"], d["b_router"], d["gu_codes"], d["gu_scales"],
+                    d["dn_codes"], d["dn_scales"])
+    else:
+        fwd = layer.forward
+        ws = torch.empty(layer.workspace_bytes(T), dtype=torch.uint8, device="cuda")
+        args_fwd = (d["x"], d["W_router"], d["b_router"], d["W_gate_up"], d["W_down"])
     stream = torch.cuda.current_stream()
 
     def step():
-        layer.forward(*args_fwd, out=out, workspace=ws)
+        fwd(*args_fwd, out=out, workspace=ws)
 
     for _ in range(args.warmup):
         step()
@@ -291,7 +309,7 @@ def run_ours(args, w: mi.Workload, T: int) -> None:
 
     def e2e_step():
         x_dev.copy_(x_host, non_blocking=True)
-        layer.forward(x_dev, *args_fwd[1:], out=out, workspace=ws)
+        fwd(x_dev, *args_fwd[1:], out=out, workspace=ws)
         out_host.copy_(out, non_blocking=True)
 
     for _ in range(max(1, args.warmup)):
@@ -310,7 +328,7 @@ def run_ours(args, w: mi.Workload, T: int) -> None:
     # ---- roofline of the dominant kernel: the gate/up projection (2/3 of bytes and FLOPs) ----
     hbm, bf16, bf16_sus, peak_src = measured_peaks()
     path_setting, crossover = layer.get_path()
-    path = "stream" if (path_setting == moe.MOE_PATH_STREAM or
+    path = "stream" if (mx or path_setting == moe.MOE_PATH_STREAM or
                         (path_setting == moe.MOE_PATH_AUTO and T <= crossover)) else "gemm"
     gu_ms, gu_n = prof["gate_up_swiglu"]
     dn_ms, dn_n = prof["down_combine"]
@@ -320,7 +338,7 @@ def run_ours(args, w: mi.Workload, T: int) -> None:
     kernels_ms = {k_: round(v[0] / max(v[1], 1), 4) for k_, v in prof.items() if v[1]}
     src = f"{peak_src} %s (MEASURED_PEAKS.json)" if peak_src == "measured" else "fallback"
     if path == "stream":
-        kname = "stream_gate_up_kernel"
+        kname = "stream_gate_up_mx_kernel" if mx else "stream_gate_up_kernel"
         achieved = alg["gate_up_bytes"] / gu_avg_s / 1e9
         roof = dict(bound="hbm", achieved=achieved, peak=hbm, unit="GB/s", frac=achieved / hbm,
                     traffic=ncu_traffic(kname, w.name), kernel=kname,
@@ -340,9 +358,11 @@ def run_ours(args, w: mi.Workload, T: int) -> None:
     line = dict(
         metric=METRIC, value=agg["value"], unit=UNIT, n_gpus=world, steps=args.steps,
         warmup=args.warmup, ms_per_step=agg["ms_per_step"], us_per_layer=agg["ms_per_step"] * 1e3,
-        higher_is_better=True, scaling="weak", vs_baseline=None, dtype="bf16",
+        higher_is_better=True, scaling="weak", vs_baseline=None,
+        dtype="mxfp4 weights, bf16 activations" if mx else "bf16",
         data="synthetic (seeded N(0,1) tokens, N(0,1/fan_in) bf16 weights; no trained weights)",
         config=dict(workload=w.name, T=T, H=w.H, E=w.E, k=w.k, I=w.I, path=path,
+                    weights=w.weights,
                     parallelism=f"replicas{world}" if world > 1 else "single",
                     l2="inputs larger than L2: %.2f GB of touched expert weights and tokens per "
                        "step vs 126 MB L2" % ((alg["layer_bytes"]) / 1e9)),

@@ -124,6 +124,29 @@ MOE_API moe_status moe_forward(moe_t ctx, int T, const void* x_bf16, const void*
                        const void* W_down_bf16, float* out, void* workspace, size_t ws_bytes,
                        moe_stream_t stream);
 
+/* The whole layer with MXFP4 expert weights (W4A16): the experts' native format (Persona
+ * Kappa forum post, "Quantization-Aware Training": MXFP4 with bf16 activations), read as OCP
+ * Microscaling FP4 -- E2M1 codes, blocks of 32 consecutive K elements of one weight column
+ * sharing an E8M0 scale 2^(s - 127) (s = 255: NaN).  For a [K, N] expert matrix:
+ *   codes  [N, K/2] uint8  row n = column n of the matrix; byte j holds element k = 2j in
+ *                          bits 0-3 and k = 2j + 1 in bits 4-7
+ *   scales [K/32, N] uint8 scale of block k/32 of column n
+ * gu_codes [E, 2I, H/2] and gu_scales [E, H/32, 2I] hold W_gate_up [E, H, 2I] (gate columns
+ * [0, I), up columns [I, 2I)); dn_codes [E, H, I/2] and dn_scales [E, I/32, H] hold W_down
+ * [E, I, H].  x, W_router, b_router and out as in moe_forward; all pointers 16-byte aligned.
+ * Runs the streaming path at every T (there is no MXFP4 grouped GEMM): the weights stream
+ * at a quarter of the bf16 bytes.  The tensor-core products take the E2M1 values (exact in
+ * f16) and the activations converted from bf16 to f16, which is exact for magnitudes
+ * 2^-14 .. 65504 (larger ones overflow to infinity, smaller ones keep fewer bits); each
+ * 32-element block's fp32 result is scaled by its E8M0 factor in fp32.  workspace: at least
+ * moe_workspace_bytes_mxfp4(ctx, T) bytes.  T = 0 is a no-op. */
+MOE_API size_t moe_workspace_bytes_mxfp4(moe_t ctx, int T);
+MOE_API moe_status moe_forward_mxfp4(moe_t ctx, int T, const void* x_bf16,
+                                     const void* W_router_bf16, const float* b_router,
+                                     const void* gu_codes, const void* gu_scales,
+                                     const void* dn_codes, const void* dn_scales, float* out,
+                                     void* workspace, size_t ws_bytes, moe_stream_t stream);
+
 /* Choose the path.  crossover_T >= 0 sets the largest T that MOE_PATH_AUTO streams;
  * crossover_T < 0 keeps the current one (the built-in default or the value moe_tune
  * measured).  MOE_ERR_UNSUPPORTED if the path is not available on this device. */

@@ -40,6 +40,9 @@ _SIGS = {
     "moe_route_workspace_bytes": (_sz, [_vp, _c_int]),
     "moe_route": (_c_int, [_vp, _c_int, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _sz, _vp]),
     "moe_forward": (_c_int, [_vp, _c_int, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _sz, _vp]),
+    "moe_workspace_bytes_mxfp4": (_sz, [_vp, _c_int]),
+    "moe_forward_mxfp4": (_c_int, [_vp, _c_int, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp,
+                                   _sz, _vp]),
     "moe_set_path": (_c_int, [_vp, _c_int, _c_int]),
     "moe_get_path": (_c_int, [_vp, ctypes.POINTER(_c_int), ctypes.POINTER(_c_int)]),
     "moe_tune_workspace_bytes": (_sz, [_vp, _c_int]),
@@ -182,6 +185,30 @@ class Moe:
         return out
 
     __call__ = forward
+
+    def workspace_bytes_mxfp4(self, T: int) -> int:
+        return moe_workspace_bytes_mxfp4(self._h, T)
+
+    def forward_mxfp4(self, x, W_router, b_router, gu_codes, gu_scales, dn_codes, dn_scales,
+                      out=None, stream=None, workspace=None) -> torch.Tensor:
+        """The layer with MXFP4 experts (uint8 codes and E8M0 scales, see include/moe.h)."""
+        T = x.shape[0]
+        E, H, I = self.E, self.H, self.I
+        if out is None:
+            out = torch.empty((T, H), dtype=torch.float32, device=x.device)
+        need = self.workspace_bytes_mxfp4(T)
+        ws = self._workspace(need, x.device) if workspace is None else workspace
+        st = moe_forward_mxfp4(self._h, T, _ptr(x, torch.bfloat16, "x", (T, H)),
+                               _ptr(W_router, torch.bfloat16, "W_router", (H, E)),
+                               _ptr(b_router, torch.float32, "b_router", (E,)),
+                               _ptr(gu_codes, torch.uint8, "gu_codes", (E, 2 * I, H // 2)),
+                               _ptr(gu_scales, torch.uint8, "gu_scales", (E, H // 32, 2 * I)),
+                               _ptr(dn_codes, torch.uint8, "dn_codes", (E, H, I // 2)),
+                               _ptr(dn_scales, torch.uint8, "dn_scales", (E, I // 32, H)),
+                               _ptr(out, torch.float32, "out", (T, H)),
+                               ws.data_ptr(), ws.numel(), _stream(stream))
+        _check(st, "moe_forward_mxfp4")
+        return out
 
     def tune(self, x, W_router, b_router, W_gate_up, W_down, stream=None) -> int:
         T = x.shape[0]

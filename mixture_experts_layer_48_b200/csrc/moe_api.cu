@@ -17,6 +17,7 @@
 #include "common.cuh"
 #include "route.cuh"
 #include "stream.cuh"
+#include "stream_mx.cuh"
 #include "gemm.cuh"
 
 using namespace moe;
@@ -50,6 +51,7 @@ constexpr int kGemmChunkRows = 2 * kGemmBM;  // rows per tile: one 256-row MMA o
 struct moe_ctx {
   int E, H, I, k;
   MapCache gate_up_stream, down_stream, gate_up_gemm, down_gemm, x_perm_map, h_map;
+  MapCache gu_codes, gu_scales, dn_codes, dn_scales;  // MXFP4 weights (streaming path)
   int device = 0;
   int num_sms = 148;
   moe_path path = MOE_PATH_AUTO;
@@ -118,6 +120,32 @@ bool encode_2d(CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols, u
              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// 2D map over a byte tensor [rows, cols] (cols bytes per row, a multiple of 16).
+bool encode_2d_u8(CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols,
+                  uint32_t box_rows, uint32_t box_cols, CUtensorMapSwizzle swizzle) {
+  auto enc = tensor_map_encoder();
+  if (!enc) return false;
+  cuuint64_t dims[2] = {cols, rows};
+  cuuint64_t strides[1] = {cols};
+  cuuint32_t box[2] = {box_cols, box_rows};
+  cuuint32_t estr[2] = {1, 1};
+  return enc(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims, strides, box,
+             estr, CU_TENSOR_MAP_INTERLEAVE_NONE, swizzle, CU_TENSOR_MAP_L2_PROMOTION_L2_128B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+const CUtensorMap* cached_map_u8(MapCache& mc, const void* ptr, uint64_t rows, uint64_t cols,
+                                 uint32_t box_rows, uint32_t box_cols,
+                                 CUtensorMapSwizzle swizzle) {
+  if (mc.ptr != ptr || mc.rows != rows) {
+    mc.ptr = nullptr;
+    if (!encode_2d_u8(&mc.map, ptr, rows, cols, box_rows, box_cols, swizzle)) return nullptr;
+    mc.ptr = ptr;
+    mc.rows = rows;
+  }
+  return &mc.map;
+}
+
 const CUtensorMap* cached_map(MapCache& mc, const void* ptr, uint64_t rows, uint64_t cols,
                               uint32_t box_rows, uint32_t box_cols, bool promote_256 = true) {
   if (mc.ptr != ptr || mc.rows != rows) {
@@ -177,7 +205,9 @@ StreamLayout stream_layout(const moe_ctx* c, int T) {
   Carver cv;
   const size_t R = (size_t)T * c->k;
   L.max_chunks = (int)(R / kStreamRB) + c->E;
-  const int NT = (c->I + kStreamCols - 1) / kStreamCols;
+  // one completion counter per (chunk, column tile); the MXFP4 kernels' tiles are narrower
+  const int tile_cols = std::min(kStreamCols, kMxTileCols);
+  const int NT = (c->I + tile_cols - 1) / tile_cols;
   L.n_done = L.max_chunks * NT;
   L.topk_idx = cv.take(4 * R);
   L.topk_w = cv.take(4 * R);
@@ -381,6 +411,11 @@ bool set_smem_attrs() {
                              kGateUpSmem) == cudaSuccess;
   ok &= cudaFuncSetAttribute(stream_down_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              kDownSmem) == cudaSuccess;
+  ok &= cudaFuncSetAttribute(stream_gate_up_mx_kernel,
+                             cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             kMxGateUpSmem) == cudaSuccess;
+  ok &= cudaFuncSetAttribute(stream_down_mx_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             kMxDownSmem) == cudaSuccess;
   ok &= cudaFuncSetAttribute(grouped_gemm_2sm_kernel<MOE_GEMM_GATE_UP>,
                              cudaFuncAttributeMaxDynamicSharedMemorySize,
                              Gemm2Cfg<kGemmStages>::kSmem) == cudaSuccess;
@@ -399,10 +434,15 @@ moe_status check_common(const moe_ctx* c, int T, const void* x, const void* Wr, 
   return MOE_OK;
 }
 
+// MXFP4 expert weights: codes and scales of W_gate_up and W_down (null: bf16 weights).
+struct MxWeights {
+  const void *gu_codes, *gu_scales, *dn_codes, *dn_scales;
+};
+
 moe_status forward_stream(moe_ctx* c, int T, const void* x_bf16, const void* W_router_bf16,
                           const float* b_router, const void* W_gate_up_bf16,
                           const void* W_down_bf16, float* out, uint8_t* ws, size_t ws_bytes,
-                          cudaStream_t st) {
+                          cudaStream_t st, const MxWeights* mx = nullptr) {
   const StreamLayout L = stream_layout(c, T);
   if (ws_bytes < L.total) return MOE_ERR_WORKSPACE;
   const size_t R = (size_t)T * c->k;
@@ -436,14 +476,30 @@ moe_status forward_stream(moe_ctx* c, int T, const void* x_bf16, const void* W_r
     ga.out = out;
     ga.out_elems = (size_t)T * c->H;
     ga.status = c->d_status;
-    const CUtensorMap* m = cached_map(c->gate_up_stream, W_gate_up_bf16, (uint64_t)c->E * c->H,
-                                      2ull * c->I, kGateUpKC, kBox, /*promote_256=*/false);
-    if (!m) s = MOE_ERR_CUDA;
-    else
-      s = launch(c, kKindGateUp, st, [&] {
-        return launch_pdl(stream_gate_up_kernel, dim3(c->num_sms), dim3(kStreamThreads),
-                          kGateUpSmem, st, ga, *m);
-      });
+    if (mx) {
+      const CUtensorMap* cm = cached_map_u8(c->gu_codes, mx->gu_codes, 2ull * c->I * c->E,
+                                            (uint64_t)c->H / 2, kMxBoxRows, kMxKC / 2,
+                                            CU_TENSOR_MAP_SWIZZLE_128B);
+      const CUtensorMap* sm = cached_map_u8(c->gu_scales, mx->gu_scales,
+                                            (uint64_t)c->E * (c->H / 32), 2ull * c->I,
+                                            kMxKC / 32, kMxBoxRows, CU_TENSOR_MAP_SWIZZLE_NONE);
+      if (!cm || !sm) s = MOE_ERR_CUDA;
+      else
+        s = launch(c, kKindGateUp, st, [&] {
+          return launch_pdl(stream_gate_up_mx_kernel, dim3(c->num_sms), dim3(kMxThreads),
+                            kMxGateUpSmem, st, ga, *cm, *sm);
+        });
+    } else {
+      const CUtensorMap* m = cached_map(c->gate_up_stream, W_gate_up_bf16,
+                                        (uint64_t)c->E * c->H, 2ull * c->I, kGateUpKC, kBox,
+                                        /*promote_256=*/false);
+      if (!m) s = MOE_ERR_CUDA;
+      else
+        s = launch(c, kKindGateUp, st, [&] {
+          return launch_pdl(stream_gate_up_kernel, dim3(c->num_sms), dim3(kStreamThreads),
+                            kGateUpSmem, st, ga, *m);
+        });
+    }
   }
   if (s == MOE_OK) {
     DownArgs da{};
@@ -457,14 +513,29 @@ moe_status forward_stream(moe_ctx* c, int T, const void* x_bf16, const void* W_r
     da.sched = o.sched;
     da.out = out;
     da.status = c->d_status;
-    const CUtensorMap* m = cached_map(c->down_stream, W_down_bf16, (uint64_t)c->E * c->I,
-                                      (uint64_t)c->H, kDownKC, kBox, /*promote_256=*/false);
-    if (!m) s = MOE_ERR_CUDA;
-    else
-      s = launch(c, kKindDown, st, [&] {
-        return launch_pdl(stream_down_kernel, dim3(c->num_sms), dim3(kStreamThreads), kDownSmem,
-                          st, da, *m);
-      });
+    if (mx) {
+      const CUtensorMap* cm = cached_map_u8(c->dn_codes, mx->dn_codes, (uint64_t)c->H * c->E,
+                                            (uint64_t)c->I / 2, kMxBoxRows, kMxKC / 2,
+                                            CU_TENSOR_MAP_SWIZZLE_128B);
+      const CUtensorMap* sm = cached_map_u8(c->dn_scales, mx->dn_scales,
+                                            (uint64_t)c->E * (c->I / 32), (uint64_t)c->H,
+                                            kMxKC / 32, kMxBoxRows, CU_TENSOR_MAP_SWIZZLE_NONE);
+      if (!cm || !sm) s = MOE_ERR_CUDA;
+      else
+        s = launch(c, kKindDown, st, [&] {
+          return launch_pdl(stream_down_mx_kernel, dim3(c->num_sms), dim3(kMxThreads),
+                            kMxDownSmem, st, da, *cm, *sm);
+        });
+    } else {
+      const CUtensorMap* m = cached_map(c->down_stream, W_down_bf16, (uint64_t)c->E * c->I,
+                                        (uint64_t)c->H, kDownKC, kBox, /*promote_256=*/false);
+      if (!m) s = MOE_ERR_CUDA;
+      else
+        s = launch(c, kKindDown, st, [&] {
+          return launch_pdl(stream_down_kernel, dim3(c->num_sms), dim3(kStreamThreads),
+                            kDownSmem, st, da, *m);
+        });
+    }
   }
   return s;
 }
@@ -685,6 +756,33 @@ moe_status moe_forward(moe_t c, int T, const void* x_bf16, const void* W_router_
                            out, ws, ws_bytes, st)
           : forward_gemm(c, T, x_bf16, W_router_bf16, b_router, W_gate_up_bf16, W_down_bf16,
                          out, ws, ws_bytes, st);
+  if (c->in_call) ++c->prof_calls;
+  c->in_call = false;
+  return s;
+}
+
+size_t moe_workspace_bytes_mxfp4(moe_t c, int T) {
+  if (!c || T < 0 || T > kMaxT || (long long)T * c->k >= (1ll << 31)) return 0;
+  if (T == 0) return 0;
+  return stream_layout(c, T).total;
+}
+
+moe_status moe_forward_mxfp4(moe_t c, int T, const void* x_bf16, const void* W_router_bf16,
+                             const float* b_router, const void* gu_codes, const void* gu_scales,
+                             const void* dn_codes, const void* dn_scales, float* out,
+                             void* workspace, size_t ws_bytes, moe_stream_t stream) {
+  MOE_TRY(check_common(c, T, x_bf16, W_router_bf16, b_router));
+  if (T == 0) return MOE_OK;
+  if (!gu_codes || !gu_scales || !dn_codes || !dn_scales || !out) return MOE_ERR_ARG;
+  if (!aligned16(gu_codes) || !aligned16(gu_scales) || !aligned16(dn_codes) ||
+      !aligned16(dn_scales) || !aligned16(out))
+    return MOE_ERR_ARG;
+  if (!workspace || !aligned16(workspace)) return MOE_ERR_WORKSPACE;
+  const MxWeights mx{gu_codes, gu_scales, dn_codes, dn_scales};
+  c->in_call = c->prof_max > 0 && c->prof_calls < c->prof_max;
+  const moe_status s = forward_stream(c, T, x_bf16, W_router_bf16, b_router, nullptr, nullptr,
+                                      out, static_cast<uint8_t*>(workspace), ws_bytes,
+                                      reinterpret_cast<cudaStream_t>(stream), &mx);
   if (c->in_call) ++c->prof_calls;
   c->in_call = false;
   return s;
