@@ -183,7 +183,8 @@ MOE_API uint64_t moe_launch_count(moe_t ctx);
  * kernel it launches, on the call's stream.  moe_profile_end synchronises, and writes for
  * each kernel kind i < n_kinds the total milliseconds into ms[i] and its launch count into
  * launches[i], then frees the events.  Kinds: 0 router, 1 routing finalize / scan / scatter,
- * 2 gather, 3 gate/up projection + SwiGLU, 4 down projection + combine, 5 zero fill.
+ * 2 gather, 3 gate/up projection + SwiGLU, 4 down projection + combine, 5 conversion of the
+ * input to f16 (MXFP4 path).
  * moe_profile_kind_name gives a kind's name. */
 #define MOE_PROFILE_KINDS 6
 MOE_API moe_status moe_profile_begin(moe_t ctx, int max_calls);

@@ -31,7 +31,7 @@ constexpr int kDefaultCrossover = 64;  // largest T streamed until moe_tune meas
 constexpr int kMaxKernelsPerCall = 8;
 
 enum Kind { kKindRouter = 0, kKindRouteFin = 1, kKindGather = 2, kKindGateUp = 3,
-            kKindDown = 4, kKindZero = 5 };
+            kKindDown = 4, kKindConvert = 5 };
 
 }  // namespace
 
@@ -194,7 +194,7 @@ RouteTmp carve_route_tmp(Carver& cv, const moe_ctx* c, int T, bool allow_split =
 }
 
 struct StreamLayout {
-  size_t topk_idx, topk_w, inv_perm, perm, row_w, offsets, sched, chunks, acc, done, h;
+  size_t topk_idx, topk_w, inv_perm, perm, row_w, offsets, sched, chunks, acc, done, h, x16;
   RouteTmp rt;
   int max_chunks, n_done;
   size_t total;
@@ -219,6 +219,7 @@ StreamLayout stream_layout(const moe_ctx* c, int T) {
   L.chunks = cv.take(16 * (size_t)L.max_chunks);
   L.done = cv.take(4 * (size_t)L.n_done);
   L.h = cv.take(2 * R * c->I);
+  L.x16 = cv.take(2 * (size_t)T * c->H);  // MXFP4 path: the layer input in f16
   L.acc = cv.take(sizeof(float) * R * 2 * c->I);
   L.rt = carve_route_tmp(cv, c, T);
   L.total = cv.cur;
@@ -459,11 +460,19 @@ moe_status forward_stream(moe_ctx* c, int T, const void* x_bf16, const void* W_r
   o.zero_i32 = reinterpret_cast<int32_t*>(ws + L.done);
   o.n_zero = L.n_done;
   const uint16_t* x = static_cast<const uint16_t*>(x_bf16);
+  uint16_t* x16 = reinterpret_cast<uint16_t*>(ws + L.x16);
+  if (mx) {  // the MXFP4 kernels take f16 activations
+    const size_t n = (size_t)T * c->H;
+    const int blocks = (int)std::min<size_t>((n / 8 + 255) / 256, (size_t)c->num_sms * 4);
+    MOE_TRY(launch(c, kKindConvert, st, [&] {
+      return launch_pdl(to_f16_kernel, dim3(blocks), dim3(256), 0, st, x, x16, n);
+    }));
+  }
   moe_status s = launch_route(c, T, x, static_cast<const uint16_t*>(W_router_bf16), b_router, o,
                               ws, L.rt, st, reinterpret_cast<float*>(ws + L.acc), R * 2 * c->I);
   if (s == MOE_OK) {
     GateUpArgs ga{};
-    ga.x = x;
+    ga.x = mx ? x16 : x;
     ga.H = c->H;
     ga.I = c->I;
     ga.R = (int)R;
@@ -946,7 +955,7 @@ moe_status moe_profile_end(moe_t c, float* ms, int* launches, int n_kinds) {
 
 const char* moe_profile_kind_name(int kind) {
   static const char* names[MOE_PROFILE_KINDS] = {"router", "route_finalize", "gather",
-                                                 "gate_up_swiglu", "down_combine", "zero_fill"};
+                                                 "gate_up_swiglu", "down_combine", "to_f16"};
   if (kind < 0 || kind >= MOE_PROFILE_KINDS) return "unknown";
   return names[kind];
 }

@@ -22,12 +22,13 @@
 //     holds elements 8t..8t+7 (the same permutation on the activation side, whose 8 values are
 //     one 16-byte load);
 //   * the hardware converts each code pair to f16 (cvt.rn.f16x2.e2m1x2, exact: E2M1 values
-//     are f16 numbers; there is no bf16 form), the activations' bf16 pairs are converted to f16
-//     the same way, and the products run as f16 MMAs: one block's two MMAs give an fp32 tile
-//     that is added to the accumulator times the block's E8M0 scale (fp32, exact for every
-//     scale).  Converting a bf16 activation to f16 is exact for magnitudes 2^-14 .. 65504 (f16
-//     keeps more mantissa bits than bf16); below that range f16 keeps fewer bits, above it the
-//     value overflows to infinity.  That range is the one departure from bf16 arithmetic.
+//     are f16 numbers; there is no bf16 form), and the products run as f16 MMAs: one block's
+//     two MMAs give an fp32 tile that is added to the accumulator times the block's E8M0 scale
+//     (fp32, exact for every scale).  The activations are therefore f16: the layer input is
+//     converted once per call (to_f16_kernel) and the gate/up kernel writes h in f16.
+//     Converting a bf16 value to f16 is exact for magnitudes 2^-14 .. 65504 (f16 keeps more
+//     mantissa bits than bf16); below that range f16 keeps fewer bits, above it the value
+//     overflows to infinity.  That range is the one departure from bf16 arithmetic.
 #pragma once
 
 #include "stream.cuh"
@@ -74,12 +75,30 @@ MOE_DEVINL void e2m1x8_to_f16x2(uint32_t w, uint32_t (&h)[4]) {
       : "r"(w));
 }
 
-// bf16 pair to f16 pair (round to nearest; exact for magnitudes 2^-14 .. 65504).
-MOE_DEVINL uint32_t bf16x2_to_f16x2(uint32_t v) {
-  const float lo = __uint_as_float(v << 16), hi = __uint_as_float(v & 0xffff0000u);
+// Two fp32 values to an f16 pair (round to nearest), first in the low half.
+MOE_DEVINL uint32_t pack_f16x2(float lo, float hi) {
   uint32_t r;
   asm("cvt.rn.f16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
   return r;
+}
+
+// The layer input in f16 for the MXFP4 kernels: x16[i] = f16(x[i]) for n elements (n even).
+// grid-stride, 8 elements per thread and step.
+__global__ void __launch_bounds__(256) to_f16_kernel(const uint16_t* __restrict__ x,
+                                                     uint16_t* __restrict__ x16, size_t n) {
+  pdl_wait();  // x16 may still be read by the previous call's gate/up kernel until it ends
+  pdl_launch_next();
+  const size_t n8 = n / 8;
+  for (size_t i = (size_t)blockIdx.x * blockDim.x + threadIdx.x; i < n8;
+       i += (size_t)gridDim.x * blockDim.x) {
+    const uint4 v = reinterpret_cast<const uint4*>(x)[i];
+    const uint32_t in[4] = {v.x, v.y, v.z, v.w};
+    uint32_t o[4];
+#pragma unroll
+    for (int j = 0; j < 4; ++j)
+      o[j] = pack_f16x2(__uint_as_float(in[j] << 16), __uint_as_float(in[j] & 0xffff0000u));
+    reinterpret_cast<uint4*>(x16)[i] = make_uint4(o[0], o[1], o[2], o[3]);
+  }
 }
 
 // d = A B (f16 in, fp32 out, zero accumulator in) and d += A B.
@@ -114,8 +133,8 @@ MOE_DEVINL uint32_t lds_u8(uint32_t addr) {
   return v;
 }
 
-// Activation fragments of one 32-element block for the permuted K order: rows g (n8 tile 0)
-// and 8 + g (tile 1), elements 8t..8t+7 as f16 pairs; [nb][step][reg].
+// Activation fragments (f16 rows) of one 32-element block for the permuted K order: rows g
+// (n8 tile 0) and 8 + g (tile 1), elements 8t..8t+7, one 16-byte load; [nb][step][reg].
 template <int NB>
 MOE_DEVINL void mx_b_frags(uint32_t xbase, int kb, int lane, uint32_t (&b)[2][2][2]) {
   const int g = lane >> 2, t = lane & 3;
@@ -125,10 +144,10 @@ MOE_DEVINL void mx_b_frags(uint32_t xbase, int kb, int lane, uint32_t (&b)[2][2]
     asm volatile("ld.shared.v4.b32 {%0,%1,%2,%3}, [%4];"
                  : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
                  : "r"(xbase + (uint32_t)((8 * nb + g) * kMxXPitch + (32 * kb + 8 * t) * 2)));
-    b[nb][0][0] = bf16x2_to_f16x2(v.x);
-    b[nb][0][1] = bf16x2_to_f16x2(v.y);
-    b[nb][1][0] = bf16x2_to_f16x2(v.z);
-    b[nb][1][1] = bf16x2_to_f16x2(v.w);
+    b[nb][0][0] = v.x;
+    b[nb][0][1] = v.y;
+    b[nb][1][0] = v.z;
+    b[nb][1][1] = v.w;
   }
 }
 
@@ -182,8 +201,8 @@ MOE_DEVINL void mx_stage(const uint32_t (&boxes)[NMAT], const uint32_t (&scs)[NM
 }
 
 // ------------------------------------------------------------------------------------------
-// gate/up projection + SwiGLU, MXFP4 weights.  Codes of W_gate_up: [E * 2I rows, H/2 bytes];
-// scales: [E * H/32 rows, 2I bytes].
+// gate/up projection + SwiGLU, MXFP4 weights; a.x is the f16 copy of the input, a.h receives
+// f16.  Codes of W_gate_up: [E * 2I rows, H/2 bytes]; scales: [E * H/32 rows, 2I bytes].
 // ------------------------------------------------------------------------------------------
 __global__ void __launch_bounds__(kMxThreads, 1)
     stream_gate_up_mx_kernel(const GateUpArgs a, const __grid_constant__ CUtensorMap cmap,
@@ -335,7 +354,7 @@ __global__ void __launch_bounds__(kMxThreads, 1)
           const int r = nb * 8 + 2 * (lane & 3) + (v & 1);
           if (r < nrows && cl < wg) {
             const float hv = silu_f32(acc[0][nb][v]) * acc[1][nb][v];
-            a.h[(size_t)(ch.y + r) * a.I + col0 + cl] = (uint16_t)f32_to_bf16_bits(hv);
+            a.h[(size_t)(ch.y + r) * a.I + col0 + cl] = (uint16_t)pack_f16x2(hv, 0.f);
           }
         }
       continue;
@@ -365,14 +384,14 @@ __global__ void __launch_bounds__(kMxThreads, 1)
         const float2 gs = __ldcg(reinterpret_cast<const float2*>(p));
         const float2 us = __ldcg(reinterpret_cast<const float2*>(p + a.I));
         *reinterpret_cast<uint32_t*>(a.h + (size_t)(ch.y + r) * a.I + col0 + cl) =
-            pack_bf16x2(silu_f32(gs.x) * us.x, silu_f32(gs.y) * us.y);
+            pack_f16x2(silu_f32(gs.x) * us.x, silu_f32(gs.y) * us.y);
       }
     }
   }
 }
 
 // ------------------------------------------------------------------------------------------
-// down projection + routing weight + combine, MXFP4 weights.  Codes of W_down:
+// down projection + routing weight + combine, MXFP4 weights (h in f16).  Codes of W_down:
 // [E * H rows, I/2 bytes]; scales: [E * I/32 rows, H bytes].
 // ------------------------------------------------------------------------------------------
 __global__ void __launch_bounds__(kMxThreads, 1)
