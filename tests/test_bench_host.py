@@ -87,3 +87,12 @@ def test_bench_refuses_to_run_without_gpu():
     r = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--steps", "1", "--warmup", "3"],
                        capture_output=True, text=True, timeout=300)
     assert r.returncode != 0 and "CUDA" in (r.stderr + r.stdout)
+
+
+def test_algorithmic_bytes_of_mxfp4_weights():
+    """MXFP4 streams half a byte per weight plus one scale byte per 32 weights."""
+    b = bench.algorithmic(16, 2880, 32, 4, 2880, [1] * 27, "mxfp4")
+    f = bench.algorithmic(16, 2880, 32, 4, 2880, [1] * 27)
+    per_expert_gu = 2880 * 5760 // 2 + 2880 // 32 * 5760
+    assert b["gate_up_bytes"] - f["gate_up_bytes"] == 27 * (per_expert_gu - 2880 * 5760 * 2)
+    assert b["flops"] == f["flops"]

@@ -103,3 +103,14 @@ def test_zero_tokens_and_bad_calls():
         layer.forward_mxfp4(d["x"], d["W_router"], d["b_router"], d["gu_scales"], d["gu_codes"],
                             d["dn_codes"], d["dn_scales"])
     assert layer.workspace_bytes_mxfp4(0) == 0 and layer.workspace_bytes_mxfp4(4) > 0
+
+
+def test_120b_shape_eight_tokens():
+    """128 experts: most touched experts see one row."""
+    _run_mx(8, 2880, 128, 4, 2880, 41)
+
+
+def test_many_chunks_and_split_k():
+    """300 tokens x 2 of 8 experts: tens of 16-row chunks per expert, stream-K pieces that share
+    a tile's K range meet in the fp32 accumulator."""
+    _run_mx(300, 512, 8, 2, 704, 42, sample=64)
