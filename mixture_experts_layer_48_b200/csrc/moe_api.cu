@@ -532,7 +532,7 @@ moe_status forward_stream(moe_ctx* c, int T, const void* x_bf16, const void* W_r
       if (!cm || !sm) s = MOE_ERR_CUDA;
       else
         s = launch(c, kKindDown, st, [&] {
-          return launch_pdl(stream_down_mx_kernel, dim3(c->num_sms), dim3(kMxThreads),
+          return launch_pdl(stream_down_mx_kernel, dim3(c->num_sms), dim3(kMxDnThreads),
                             kMxDownSmem, st, da, *cm, *sm);
         });
     } else {

@@ -46,15 +46,21 @@ constexpr int kMxBoxBytes = kMxBoxRows * kMxKC / 2;  // 4 KB of codes, 128-byte 
 constexpr int kMxScaleBytes = (kMxKC / 32) * kMxBoxRows;  // 256 B: [8 blocks][32 columns]
 constexpr int kMxXPitch = kMxKC * 2 + 64;           // 576 B per activation row (144 words): the
                                                     // 16-byte fragment loads hit no bank twice
+// The down kernel has one matrix, so it affords twice the tile width and twice the warps.
+constexpr int kMxDnWarps = 2 * kMxWarps;
+constexpr int kMxDnConsumers = 32 * kMxDnWarps;
+constexpr int kMxDnThreads = kMxDnConsumers + 32;
+constexpr int kMxDnTileCols = 2 * kMxTileCols;             // 320 columns of H
+constexpr int kMxDnBoxes = kMxDnTileCols / kMxBoxRows;     // 10
 constexpr int kMxGUW = 2 * kMxBoxes * kMxBoxBytes;         // gate + up codes, 40 KB
 constexpr int kMxGUS = 2 * kMxBoxes * kMxScaleBytes;       // 2.5 KB
-constexpr int kMxDNW = kMxBoxes * kMxBoxBytes;             // 20 KB
-constexpr int kMxDNS = kMxBoxes * kMxScaleBytes;           // 1.25 KB
+constexpr int kMxDNW = kMxDnBoxes * kMxBoxBytes;           // 40 KB
+constexpr int kMxDNS = kMxDnBoxes * kMxScaleBytes;         // 2.5 KB
 constexpr int kMxX = kStreamRB * kMxXPitch;                // 9 KB
 constexpr int kMxGUStage = (kMxGUW + kMxGUS + kMxX + 1023) / 1024 * 1024;  // 53 KB
-constexpr int kMxDNStage = (kMxDNW + kMxDNS + kMxX + 1023) / 1024 * 1024;  // 31 KB
+constexpr int kMxDNStage = (kMxDNW + kMxDNS + kMxX + 1023) / 1024 * 1024;  // 53 KB
 constexpr int kMxGUStages = 4;
-constexpr int kMxDNStages = 7;
+constexpr int kMxDNStages = 4;
 constexpr int kMxGateUpSmem = 1024 + kMxGUStages * kMxGUStage + 2 * kMxGUStages * 8;
 constexpr int kMxDownSmem = 1024 + kMxDNStages * kMxDNStage + 2 * kMxDNStages * 8;
 static_assert(kMxGateUpSmem <= 227 * 1024 && kMxDownSmem <= 227 * 1024, "shared memory");
@@ -394,7 +400,7 @@ __global__ void __launch_bounds__(kMxThreads, 1)
 // down projection + routing weight + combine, MXFP4 weights (h in f16).  Codes of W_down:
 // [E * H rows, I/2 bytes]; scales: [E * I/32 rows, H bytes].
 // ------------------------------------------------------------------------------------------
-__global__ void __launch_bounds__(kMxThreads, 1)
+__global__ void __launch_bounds__(kMxDnThreads, 1)
     stream_down_mx_kernel(const DownArgs a, const __grid_constant__ CUtensorMap cmap,
                           const __grid_constant__ CUtensorMap smap) {
   extern __shared__ __align__(128) uint8_t smem_raw[];
@@ -405,24 +411,24 @@ __global__ void __launch_bounds__(kMxThreads, 1)
   if (tid == 0) {
     for (int s = 0; s < kMxDNStages; ++s) {
       mbar_init(&full[s], 1);
-      mbar_init(&empty[s], kMxWarps);
+      mbar_init(&empty[s], kMxDnWarps);
     }
     fence_barrier_init();
   }
   __syncthreads();
 
-  if (tid == kMxConsumers) {
+  if (tid == kMxDnConsumers) {
     tma_prefetch_desc(&cmap);
     tma_prefetch_desc(&smap);
   }
   pdl_wait();  // h and the work list come from the previous kernels
   pdl_launch_next();
 
-  const int NT = (a.H + kMxTileCols - 1) / kMxTileCols;
+  const int NT = (a.H + kMxDnTileCols - 1) / kMxDnTileCols;
   const int nk = (a.I + kMxKC - 1) / kMxKC;
   const StreamKRange rng = stream_k_range((long long)a.sched[0] * NT, nk);
 
-  if (warp == kMxWarps) {
+  if (warp == kMxDnWarps) {
     bool aborted = false;
     uint32_t it = 0;
     int last_it[kMxDNStages];
@@ -433,8 +439,8 @@ __global__ void __launch_bounds__(kMxThreads, 1)
       const int ke = (int)min((long long)nk, kb + (rng.g1 - g));
       g += ke - kb;
       const int4 ch = a.chunks[unit / NT];
-      const int col0 = (unit % NT) * kMxTileCols;
-      const int j = lane % kMxBoxes;
+      const int col0 = (unit % NT) * kMxDnTileCols;
+      const int j = lane % kMxDnBoxes;
       const int box_col = col0 + kMxBoxRows * j;
       for (int kst = kb; kst < ke; ++kst, ++it) {
         const int slot = it % kMxDNStages;
@@ -451,9 +457,9 @@ __global__ void __launch_bounds__(kMxThreads, 1)
           mbar_arrive_expect_tx(&full[slot], (uint32_t)(kMxDNW + kMxDNS) + (uint32_t)ch.z * xbytes);
         __syncwarp();
         uint8_t* st = ring + slot * kMxDNStage;
-        if (lane < kMxBoxes)
+        if (lane < kMxDnBoxes)
           tma_load_2d(st + lane * kMxBoxBytes, &cmap, k0 / 2, ch.x * a.H + box_col, &full[slot]);
-        else if (lane < 2 * kMxBoxes)
+        else if (lane < 2 * kMxDnBoxes)
           tma_load_2d(st + kMxDNW + j * kMxScaleBytes, &smap, box_col,
                       ch.x * (a.I / 32) + k0 / 32, &full[slot]);
         if (lane < ch.z)
@@ -480,8 +486,8 @@ __global__ void __launch_bounds__(kMxThreads, 1)
     const int ke = (int)min((long long)nk, kb0 + (rng.g1 - g));
     g += ke - kb0;
     const int4 ch = a.chunks[unit / NT];
-    const int col0 = (unit % NT) * kMxTileCols;
-    const int wc = min(kMxTileCols, a.H - col0);
+    const int col0 = (unit % NT) * kMxDnTileCols;
+    const int wc = min(kMxDnTileCols, a.H - col0);
     const int nrows = ch.z;
     float acc[1][2][4];
 #pragma unroll
