@@ -14,13 +14,13 @@ here; these draws stand in for them with the same shapes):
   x ~ N(0, 1); W_router [H,E] and W_gate_up [E,H,2I] ~ N(0, 1/H); W_down [E,I,H] ~ N(0, 1/I);
   b_router ~ N(0, 0.1) kept in float32.  N(m, v) names the variance v;
 * W_gate_up and W_down are drawn one expert at a time (``[H,2I]`` then the next expert);
-* MXFP4 experts (``weights="mxfp4"``): ``gu_blocks [E, 2I, H/2]``, ``gu_scales [E, H/32, 2I]``,
-  ``dn_blocks [E, H, I/2]``, ``dn_scales [E, I/32, H]`` (uint8; the layout the oracle's
+* MXFP4 experts (``weights="mxfp4"``): ``gu_codes [E, 2I, H/2]``, ``gu_scales [E, H/32, 2I]``,
+  ``dn_codes [E, H, I/2]``, ``dn_scales [E, I/32, H]`` (uint8; the layout the oracle's
   ``dequant_mxfp4`` reads).  Every block byte is uniform on 0..255 (two uniform 4-bit codes);
   every scale byte is s0 + {-1, 0, +1} uniformly, with s0 = 127 + round(log2(1 / (4 *
   sqrt(fan_in)))), which puts the dequantized weights' spread near 1/sqrt(fan_in) like the bf16
   draws (0.8/sqrt(fan_in) at fan_in = 2880).  Slots 7 (gate/up) and 8 (down), drawn one expert
-  at a time (blocks, then scales);
+  at a time (codes, then scales);
 * skewed routing adds ``-c * s * ln(rank_e)`` to b_router, rank a seeded permutation of
   1..E and s = 1.1, so expert popularity falls off like a Zipf law.  c is the scale that gives
   a max/mean expert load of 4.0 on a 4096-token sample; it is computed by
@@ -114,22 +114,22 @@ def _mx_scale_center(fan_in: int) -> int:
 
 def _draw_mx(E: int, N: int, K: int, seed: int, slot: int, device):
     g = _gen(seed, slot, device)
-    blocks = torch.empty((E, N, K // 2), dtype=torch.uint8, device=device)
+    codes = torch.empty((E, N, K // 2), dtype=torch.uint8, device=device)
     scales = torch.empty((E, K // 32, N), dtype=torch.uint8, device=device)
     s0 = _mx_scale_center(K)
     for e in range(E):
-        blocks[e] = torch.randint(0, 256, (N, K // 2), generator=g, device=device,
-                                  dtype=torch.int32).to(torch.uint8)
+        codes[e] = torch.randint(0, 256, (N, K // 2), generator=g, device=device,
+                                 dtype=torch.int32).to(torch.uint8)
         scales[e] = (torch.randint(-1, 2, (K // 32, N), generator=g, device=device,
                                    dtype=torch.int32) + s0).to(torch.uint8)
-    return blocks, scales
+    return codes, scales
 
 
 def draw_experts_mxfp4(E: int, H: int, I: int, seed: int, device="cpu"):
-    """MXFP4 experts: (gu_blocks, gu_scales, dn_blocks, dn_scales), see the module recipe."""
-    gu_blocks, gu_scales = _draw_mx(E, 2 * I, H, seed, 7, device)
-    dn_blocks, dn_scales = _draw_mx(E, H, I, seed, 8, device)
-    return gu_blocks, gu_scales, dn_blocks, dn_scales
+    """MXFP4 experts: (gu_codes, gu_scales, dn_codes, dn_scales), see the module recipe."""
+    gu_codes, gu_scales = _draw_mx(E, 2 * I, H, seed, 7, device)
+    dn_codes, dn_scales = _draw_mx(E, H, I, seed, 8, device)
+    return gu_codes, gu_scales, dn_codes, dn_scales
 
 
 def draw_experts(E: int, H: int, I: int, seed: int, device="cpu"):
@@ -150,13 +150,13 @@ def make_inputs(T: int, H: int, E: int, k: int, I: int, seed: int, device="cpu",
                 zipf: bool = False, experts: bool = True, weights: str = "bf16") -> dict:
     """All inputs of one layer call as torch tensors on ``device`` (see the module recipe).
 
-    weights="bf16" gives W_gate_up / W_down; "mxfp4" gives gu_blocks, gu_scales, dn_blocks,
+    weights="bf16" gives W_gate_up / W_down; "mxfp4" gives gu_codes, gu_scales, dn_codes,
     dn_scales instead."""
     x = draw_x(T, H, seed, device)
     W_router, b_router = draw_router(H, E, seed, device, zipf)
     d = dict(x=x, W_router=W_router, b_router=b_router, T=T, H=H, E=E, k=k, I=I)
     if experts and weights == "mxfp4":
-        (d["gu_blocks"], d["gu_scales"], d["dn_blocks"],
+        (d["gu_codes"], d["gu_scales"], d["dn_codes"],
          d["dn_scales"]) = draw_experts_mxfp4(E, H, I, seed, device)
     elif experts:
         d["W_gate_up"], d["W_down"] = draw_experts(E, H, I, seed, device)

@@ -31,7 +31,7 @@ activations (Persona Kappa forum post, "Quantization-Aware Training"; kappa-20b-
 (MX) v1.0 FP4 format: E2M1 elements (sign, 2 exponent bits with bias 1, 1 mantissa bit;
 exponent 0 is subnormal) in blocks of 32 consecutive elements along the reduction dimension,
 each block sharing one E8M0 scale 2^(s-127) (s = 255 encodes NaN).  Storage of one expert's
-[K, N] matrix: ``blocks [N, K/2]`` uint8 (byte j of row n holds element k = 2j in bits 0-3 and
+[K, N] matrix: ``codes [N, K/2]`` uint8 (byte j of row n holds element k = 2j in bits 0-3 and
 k = 2j + 1 in bits 4-7) and ``scales [K/32, N]`` uint8.  The dequantized weights then enter the
 same float64 layer as the bf16 ones.
 
@@ -250,27 +250,27 @@ def decode_e8m0(s) -> np.ndarray:
     return np.where(s == 255, np.nan, np.ldexp(1.0, np.minimum(s, 254) - 127))
 
 
-def dequant_mxfp4(blocks, scales) -> np.ndarray:
-    """MXFP4 matrices to float64: blocks [..., N, K/2] uint8, scales [..., K/32, N] uint8 ->
+def dequant_mxfp4(codes, scales) -> np.ndarray:
+    """MXFP4 matrices to float64: codes [..., N, K/2] uint8, scales [..., K/32, N] uint8 ->
     W [..., K, N] with W[k, n] = e2m1(element k of row n) * 2^(scales[k // 32, n] - 127)."""
-    b = np.asarray(blocks, dtype=np.uint8)
-    codes = np.stack([b & 0xF, b >> 4], axis=-1).reshape(*b.shape[:-1], 2 * b.shape[-1])
-    vals = np.swapaxes(decode_e2m1(codes), -1, -2)            # [..., K, N]
+    b = np.asarray(codes, dtype=np.uint8)
+    elems = np.stack([b & 0xF, b >> 4], axis=-1).reshape(*b.shape[:-1], 2 * b.shape[-1])
+    vals = np.swapaxes(decode_e2m1(elems), -1, -2)            # [..., K, N]
     return vals * np.repeat(decode_e8m0(scales), 32, axis=-2)  # scale rows repeat per block
 
 
-def moe_forward_mxfp4_ref(x_bits, W_router_bits, b_router, gu_blocks, gu_scales, dn_blocks,
+def moe_forward_mxfp4_ref(x_bits, W_router_bits, b_router, gu_codes, gu_scales, dn_codes,
                           dn_scales, k: int, tokens=None, route: dict | None = None) -> np.ndarray:
     """Whole layer with MXFP4 experts: the bf16 layer above on the dequantized weights.
 
-    gu_blocks [E, 2I, H/2], gu_scales [E, H/32, 2I] hold W_gate_up [E, H, 2I] (gate columns
-    [0, I), up columns [I, 2I)); dn_blocks [E, H, I/2], dn_scales [E, I/32, H] hold W_down
+    gu_codes [E, 2I, H/2], gu_scales [E, H/32, 2I] hold W_gate_up [E, H, 2I] (gate columns
+    [0, I), up columns [I, 2I)); dn_codes [E, H, I/2], dn_scales [E, I/32, H] hold W_down
     [E, I, H].  Activations and the router stay bf16.
     """
     if route is None:
         route = moe_route_ref(x_bits, W_router_bits, b_router, k)
-    return _layer_out(x_bits, route, tokens, lambda e: dequant_mxfp4(gu_blocks[e], gu_scales[e]),
-                      lambda e: dequant_mxfp4(dn_blocks[e], dn_scales[e]))
+    return _layer_out(x_bits, route, tokens, lambda e: dequant_mxfp4(gu_codes[e], gu_scales[e]),
+                      lambda e: dequant_mxfp4(dn_codes[e], dn_scales[e]))
 
 
 def moe_token_output_ref(x_bits_t, logits_t, experts, W_gate_up_bits, W_down_bits) -> np.ndarray:

@@ -88,7 +88,7 @@ def test_dequant_matches_elementwise_python():
 
 def test_dequantized_values_are_exact_in_bf16():
     d = mi.make_inputs(3, 64, 4, 2, 64, 11, weights="mxfp4")
-    W = moe_ref.dequant_mxfp4(d["gu_blocks"].numpy(), d["gu_scales"].numpy())
+    W = moe_ref.dequant_mxfp4(d["gu_codes"].numpy(), d["gu_scales"].numpy())
     back = torch.from_numpy(W).to(torch.bfloat16).double().numpy()
     np.testing.assert_array_equal(back, W)
 
@@ -98,10 +98,10 @@ def test_mxfp4_layer_equals_bf16_layer_on_dequantized_weights(T, E, k):
     H, I = 64, 64
     d = mi.make_inputs(T, H, E, k, I, 12 + T, weights="mxfp4")
     h = mi.host_inputs(d)
-    out_mx = moe_ref.moe_forward_mxfp4_ref(h["x"], h["W_router"], h["b_router"], h["gu_blocks"],
-                                           h["gu_scales"], h["dn_blocks"], h["dn_scales"], k)
-    Wgu = moe_ref.dequant_mxfp4(h["gu_blocks"], h["gu_scales"])
-    Wd = moe_ref.dequant_mxfp4(h["dn_blocks"], h["dn_scales"])
+    out_mx = moe_ref.moe_forward_mxfp4_ref(h["x"], h["W_router"], h["b_router"], h["gu_codes"],
+                                           h["gu_scales"], h["dn_codes"], h["dn_scales"], k)
+    Wgu = moe_ref.dequant_mxfp4(h["gu_codes"], h["gu_scales"])
+    Wd = moe_ref.dequant_mxfp4(h["dn_codes"], h["dn_scales"])
     bits = lambda W: mi.bf16_bits(torch.from_numpy(W).to(torch.bfloat16))
     out_bf = moe_ref.moe_forward_ref(h["x"], h["W_router"], h["b_router"], bits(Wgu), bits(Wd), k)
     np.testing.assert_array_equal(out_mx, out_bf)
@@ -110,7 +110,7 @@ def test_mxfp4_layer_equals_bf16_layer_on_dequantized_weights(T, E, k):
 
 def test_generated_weights_have_the_bf16_draws_spread():
     d = mi.make_inputs(1, 2880, 2, 1, 2880, 5, weights="mxfp4")
-    W = moe_ref.dequant_mxfp4(d["gu_blocks"][0].numpy(), d["gu_scales"][0].numpy())
+    W = moe_ref.dequant_mxfp4(d["gu_codes"][0].numpy(), d["gu_scales"][0].numpy())
     assert 0.5 < W.std() * math.sqrt(2880) < 1.5
 
 
