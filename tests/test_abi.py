@@ -28,7 +28,8 @@ def lib():
 def test_header_declares_the_boundary():
     syms = declared_symbols()
     for name in ("moe_create", "moe_destroy", "moe_route", "moe_forward", "moe_set_path",
-                 "moe_workspace_bytes", "moe_sync_status", "moe_status_string", "moe_tune"):
+                 "moe_workspace_bytes", "moe_sync_status", "moe_status_string", "moe_tune",
+                 "moe_forward_mxfp4", "moe_workspace_bytes_mxfp4", "moe_route_static"):
         assert name in syms
 
 
@@ -48,8 +49,11 @@ def test_status_strings(lib):
     for s in range(7):
         assert lib.moe_status_string(s).decode() not in ("", "unknown status")
     assert lib.moe_status_string(99).decode() == "unknown status"
-    assert lib.moe_profile_kind_name(3).decode() == "gate_up_swiglu"
+    names = [lib.moe_profile_kind_name(i).decode() for i in range(lib.MOE_PROFILE_KINDS)]
+    assert names == ["router", "route_finalize", "gather", "gate_up_swiglu", "down_combine",
+                     "to_f16"]
     assert lib.moe_profile_kind_name(-1).decode() == "unknown"
+    assert lib.moe_profile_kind_name(lib.MOE_PROFILE_KINDS).decode() == "unknown"
 
 
 @pytest.mark.parametrize("E,H,I,k", [
@@ -86,6 +90,9 @@ def test_null_handle_calls(lib):
     assert lib.moe_sync_status(None, None) == lib.MOE_ERR_ARG
     assert lib.moe_profile_begin(None, 4) == lib.MOE_ERR_ARG
     assert lib.moe_selftest_timeout(None, 10, None) == lib.MOE_ERR_ARG
+    assert lib.moe_workspace_bytes_mxfp4(None, 16) == 0
+    assert lib.moe_forward_mxfp4(None, 1, None, None, None, None, None, None, None, None, None,
+                                 0, None) == lib.MOE_ERR_ARG
 
 
 def test_no_closed_copy_calls_in_sources():
