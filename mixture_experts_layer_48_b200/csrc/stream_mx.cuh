@@ -3,20 +3,21 @@
 // The experts' native format (Persona Kappa forum post, "Quantization-Aware Training": MXFP4,
 // activations kept in bf16), read as OCP Microscaling FP4: E2M1 codes in blocks of 32 along the
 // reduction dimension K, each block of a weight column sharing one E8M0 scale 2^(s - 127).
-// Storage per expert of a [K, N] matrix: blocks [N, K/2] bytes (row n = weight column n; byte j
+// Storage per expert of a [K, N] matrix: codes [N, K/2] bytes (row n = weight column n; byte j
 // holds element 2j in bits 0-3 and 2j + 1 in bits 4-7) and scales [K/32, N] bytes.
 //
 // Same persistent, stream-K organisation as the bf16 streaming kernels (stream.cuh): one CTA
 // per SM, a producer warp and consumer warps around a shared-memory ring, tiles of (row chunk
-// of one expert, 160 weight columns), the same epilogues.  What changes is the weight stream,
-// a quarter of the bytes:
+// of one expert, 160 weight columns for gate/up, 320 for down), the same epilogues.  What
+// changes is the weight stream, a quarter of the bytes:
 //
 //   * per stage, 256 K (the last stage of a row holds what is left: H = 2880 is 11 * 256 + 64):
 //     one TMA box of [32 columns x 128 bytes] codes per 32-column group and matrix (128-byte
 //     swizzle; whole 128-byte rows, so a stage needs as few copy requests per byte as the bf16
 //     kernels), one box of [8 blocks x 32 columns] scales, and the rows' activations (bulk
 //     copies);
-//   * ten consumer warps, one 16-column m-tile of gate and up (or of W_down) each;
+//   * consumer warps own one 16-column m-tile each: ten for gate/up (gate and up of the same
+//     columns, for the SwiGLU), twenty for down (one matrix leaves room for both);
 //   * a thread's A fragment of mma.sync m16n8k16 comes from one 32-bit shared load per weight
 //     column: the K order inside each 32-element block is permuted so that thread t of a quad
 //     holds elements 8t..8t+7 (the same permutation on the activation side, whose 8 values are
