@@ -1,13 +1,16 @@
 """Benchmark of the MoE layer forward pass on B200.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
-                    [--workload 20b_decode|20b_prefill|131k_skewed|120b_sweep|tiny] [--T n]
+                    [--workload 131k_skewed|20b_decode|20b_prefill|120b_sweep|tiny|...] [--T n]
 
 One step = one moe_forward call (router, top-k, histogram/scan/permutation, gate/up + SwiGLU,
-down + weighted combine) over one batch of seeded synthetic tokens of the named workload
-(default: the gpt-oss-20b layer in decode, T = 16, H = I = 2880, 32 experts, top-4).  Inputs
-are resident in HBM before the timed region; the touched expert weights (~1.4 GB) are larger
-than the 126 MB L2, so every step streams them from HBM.
+down + weighted combine) over one batch of seeded synthetic tokens of the named workload.
+Default: the largest configuration that fits one GPU -- a packed 131,072-token sequence
+through the gpt-oss-20b-shaped layer (H = I = 2880, 32 experts, top-4) with Zipf-skewed
+routing (max/mean expert load 4).  Inputs are resident in HBM before the timed region; every
+step reads 0.75 GB of tokens and 1.6 GB of expert weights and writes 1.5 GB of output, far
+more than the 126 MB L2.  Without --steps, K is chosen from the warm-up timing so that the
+timed region lasts at least a second.
 
 Prints one JSON line.  With N > 1 (torchrun, one process per GPU) every rank runs its own
 replica on its own tokens (the layer is token-wise, so there is no data-path collective);
@@ -27,6 +30,7 @@ import subprocess
 import sys
 import time
 
+import numpy as np
 import torch
 
 ROOT = os.path.dirname(os.path.abspath(__file__))
@@ -129,7 +133,7 @@ class ClockSampler:
         try:
             self.proc = subprocess.Popen(
                 ["nvidia-smi", "-i", str(self.index), f"--query-gpu={self.QUERY}",
-                 "--format=csv", "-lms", "100"], stdout=open(self.path, "w"),
+                 "--format=csv", "-lms", "50"], stdout=open(self.path, "w"),
                 stderr=subprocess.DEVNULL)
             time.sleep(0.3)
         except OSError:
@@ -186,9 +190,11 @@ def blas_threads() -> int:
         return 1
 
 
-def oracle_time(h: dict, k: int, n_tokens: int, reps: int) -> float:
+def oracle_time(h: dict, k: int, tokens, reps: int) -> float:
+    """Seconds for `reps` oracle calls of the layer on the given token rows (the layer is
+    token-wise, so a subset of tokens gives the same rows as the whole batch)."""
     import oracle
-    x = h["x"][:n_tokens]
+    x = h["x"][np.asarray(tokens)]
     t0 = time.perf_counter()
     for _ in range(reps):
         if "gu_codes" in h:
@@ -200,13 +206,21 @@ def oracle_time(h: dict, k: int, n_tokens: int, reps: int) -> float:
     return time.perf_counter() - t0
 
 
+def baseline_tokens(w: mi.Workload, T: int) -> np.ndarray:
+    """Tokens the oracle baseline runs on: the workload's seeded sample, else all T."""
+    return mi.sample_tokens(T, w.oracle_sample, w.seed) if w.oracle_sample else np.arange(T)
+
+
 def cpu_baseline(h: dict, w: mi.Workload, T: int, budget_s: float = 20.0) -> dict:
-    t1 = oracle_time(h, w.k, T, 1)       # one full call, also the warm-up
+    toks = baseline_tokens(w, T)
+    t1 = oracle_time(h, w.k, toks, 1)       # one call, also the warm-up
     reps = max(1, int(budget_s / max(t1, 1e-3)))
-    secs = oracle_time(h, w.k, T, reps)
-    return dict(value=reps * T / secs, unit=UNIT, cores=blas_threads(), kind="oracle",
-                sample=f"{reps} full oracle calls of the {w.name} layer at T={T} "
-                       f"(numpy float64, {os.cpu_count()} host cores)")
+    secs = oracle_time(h, w.k, toks, reps)
+    what = (f"a seeded {toks.size}-token sample of the {w.name} layer (T={T})"
+            if toks.size < T else f"the {w.name} layer at T={T}")
+    return dict(value=reps * toks.size / secs, unit=UNIT, cores=blas_threads(), kind="oracle",
+                sample=f"{reps} oracle calls on {what}; numpy float64, "
+                       f"{blas_threads()} BLAS threads on {os.cpu_count()} host cores")
 
 
 def run_reference(args, w: mi.Workload, T: int) -> None:
@@ -215,20 +229,23 @@ def run_reference(args, w: mi.Workload, T: int) -> None:
         return
     h = mi.host_inputs(mi.make_inputs(T, w.H, w.E, w.k, w.I, w.seed, "cpu", zipf=w.zipf,
                                       weights=w.weights))
-    budget = 150.0 / (args.steps + args.warmup)          # whole run within a few minutes
-    t1 = oracle_time(h, w.k, 1, 1)
-    n = max(1, min(T, int(budget / max(t1, 1e-3))))
+    steps = args.steps or 10
+    budget = 150.0 / (steps + args.warmup)               # whole run within a few minutes
+    pool = baseline_tokens(w, T) if w.oracle_sample else mi.sample_tokens(T, T, w.seed)
+    t1 = oracle_time(h, w.k, pool[:1], 1)
+    n = max(1, min(pool.size, int(budget / max(t1, 1e-3))))
+    toks = np.sort(pool[:n]) if n < pool.size else pool
     for _ in range(args.warmup):
-        oracle_time(h, w.k, n, 1)
-    secs = oracle_time(h, w.k, n, args.steps)
-    value = args.steps * n / secs
-    line = dict(metric=METRIC, value=value, unit=UNIT, n_gpus=args.gpus, steps=args.steps,
-                warmup=args.warmup, ms_per_step=1e3 * secs / args.steps, higher_is_better=True,
+        oracle_time(h, w.k, toks, 1)
+    secs = oracle_time(h, w.k, toks, steps)
+    value = steps * n / secs
+    line = dict(metric=METRIC, value=value, unit=UNIT, n_gpus=args.gpus, steps=steps,
+                warmup=args.warmup, ms_per_step=1e3 * secs / steps, higher_is_better=True,
                 scaling="weak", vs_baseline=None, dtype="f64", data="synthetic",
                 impl="reference",
                 config=dict(workload=w.name, T=T, H=w.H, E=w.E, k=w.k, I=w.I, sample_tokens=n),
                 cpu_baseline=dict(value=value, unit=UNIT, cores=blas_threads(), kind="oracle",
-                                  sample=f"first {n} of {T} tokens per step, full layer"),
+                                  sample=f"{n} seeded tokens of {T} per step, full layer"),
                 e2e=dict(value=value, unit=UNIT, h2d_bytes_per_step=0, d2h_bytes_per_step=0))
     print(json.dumps(line), flush=True)
 
@@ -236,6 +253,26 @@ def run_reference(args, w: mi.Workload, T: int) -> None:
 # ----------------------------------------------------------------------------------------
 # our arm
 # ----------------------------------------------------------------------------------------
+MIN_TIMED_S = 1.2   # the timed region lasts at least this long (the clock sampler sees it)
+
+
+def steps_for(step_s: float, min_s: float = MIN_TIMED_S, lo: int = 10, hi: int = 200000) -> int:
+    """Steps that make the timed region last at least min_s, given one step's seconds."""
+    return int(min(hi, max(lo, -(-min_s // max(step_s, 1e-7)))))
+
+
+def default_steps(step, stream, world: int) -> int:
+    """K from three timed extra warm-up steps (same K on every rank: the max)."""
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(3):
+        step()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    k = steps_for(e0.elapsed_time(e1) / 3e3)
+    return int(reduce_max(float(k), world))
+
+
 def run_ours(args, w: mi.Workload, T: int) -> None:
     rank, world, local = dist_env()
     if not torch.cuda.is_available():
@@ -274,6 +311,7 @@ def run_ours(args, w: mi.Workload, T: int) -> None:
         step()
     torch.cuda.synchronize()
     assert layer.sync_status() == moe.MOE_OK
+    steps = args.steps or default_steps(step, stream, world)
 
     # ---- timed region: K calls between device events on the launching stream ----
     n_launch0 = layer.launch_count()
@@ -283,7 +321,7 @@ def run_ours(args, w: mi.Workload, T: int) -> None:
             torch.distributed.barrier()
         torch.cuda.synchronize()
         ev0.record(stream)
-        for _ in range(args.steps):
+        for _ in range(steps):
             step()
         ev1.record(stream)
         torch.cuda.synchronize()
@@ -292,13 +330,14 @@ def run_ours(args, w: mi.Workload, T: int) -> None:
     gpu_launches = layer.launch_count() - n_launch0
     secs = reduce_max(ev0.elapsed_time(ev1) / 1e3, world)
     assert layer.sync_status() == moe.MOE_OK
-    agg = aggregate(T, world, secs, args.steps)
+    agg = aggregate(T, world, secs, steps)
 
     # ---- second timed region: the same K calls with CUDA events around every kernel (on the
     # launching stream); these per-kernel times give the roofline.  The events stop successive
     # kernels from overlapping, so this pass is kept apart from the one that gives `value`.
-    layer.profile_begin(args.steps)
-    for _ in range(args.steps):
+    prof_steps = min(steps, 200)
+    layer.profile_begin(prof_steps)
+    for _ in range(prof_steps):
         step()
     prof = layer.profile_end()
     assert layer.sync_status() == moe.MOE_OK
@@ -319,7 +358,7 @@ def run_ours(args, w: mi.Workload, T: int) -> None:
         torch.distributed.barrier()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     e0.record(stream)
-    for _ in range(args.steps):
+    for _ in range(steps):
         e2e_step()
     e1.record(stream)
     torch.cuda.synchronize()
@@ -352,11 +391,12 @@ def run_ours(args, w: mi.Workload, T: int) -> None:
         roof = dict(bound="tensor", achieved=achieved, peak=bf16, unit="TFLOP/s",
                     frac=achieved / bf16, traffic=ncu_traffic(kname, w.name), kernel=kname,
                     alg_flops_per_launch=alg["gate_up_flops"], avg_launch_ms=gu_avg_s * 1e3,
-                    peak_source=src % "bf16_tflops (burst)")
+                    peak_source=src % "bf16_tflops (burst)",
+                    frac_of_sustained=achieved / bf16_sus, frac_of_nominal_2250=achieved / 2250.0)
         down_rate = dict(down_kernel_TFLOPs=alg["down_flops"] / dn_avg_s / 1e12)
 
     line = dict(
-        metric=METRIC, value=agg["value"], unit=UNIT, n_gpus=world, steps=args.steps,
+        metric=METRIC, value=agg["value"], unit=UNIT, n_gpus=world, steps=steps,
         warmup=args.warmup, ms_per_step=agg["ms_per_step"], us_per_layer=agg["ms_per_step"] * 1e3,
         higher_is_better=True, scaling="weak", vs_baseline=None,
         dtype="mxfp4 weights, bf16 activations" if mx else "bf16",
@@ -369,10 +409,10 @@ def run_ours(args, w: mi.Workload, T: int) -> None:
         roofline=roof,
         layer_roofline=dict(touched_experts=alg["touched"], alg_bytes=alg["layer_bytes"],
                             alg_flops=alg["flops"], roofline_us=layer_roof_s * 1e6,
-                            frac=layer_roof_s / (secs / args.steps), **down_rate),
+                            frac=layer_roof_s / (secs / steps), **down_rate),
         kernel_avg_ms=kernels_ms,
-        kernel_timing="per-kernel CUDA events over a second timed pass of the same K calls",
-        e2e=dict(value=T * world * args.steps / e2e_secs, unit=UNIT,
+        kernel_timing="per-kernel CUDA events over a second timed pass of min(K, 200) of the same calls",
+        e2e=dict(value=T * world * steps / e2e_secs, unit=UNIT,
                  h2d_bytes_per_step=T * w.H * 2, d2h_bytes_per_step=T * w.H * 4),
         gpu_launches=gpu_launches,
         clocks=clk.result(),
@@ -389,10 +429,11 @@ def run_ours(args, w: mi.Workload, T: int) -> None:
 def main(argv=None):
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--steps", type=int, default=None,
+                    help="timed steps (default: enough for a timed region of >= 1.2 s)")
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--workload", default="20b_decode", choices=sorted(mi.WORKLOADS))
+    ap.add_argument("--workload", default="131k_skewed", choices=sorted(mi.WORKLOADS))
     ap.add_argument("--T", type=int, default=None)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     args = ap.parse_args(argv)

@@ -88,7 +88,8 @@ typedef enum {
 
 /* Create a handle for a layer of shape (E, H, I, k) on the current device.  Validates the
  * shape (see conventions; MOE_ERR_ARG otherwise), checks for an sm_100 device
- * (MOE_ERR_DEVICE), allocates the 4-byte device status word.  *out receives the handle. */
+ * (MOE_ERR_DEVICE), allocates the 4-byte device status word and looks up the device address
+ * of the library's routing scratch array (moe_route_static).  *out receives the handle. */
 MOE_API moe_status moe_create(int E, int H, int I, int k, moe_t* out);
 
 /* Free the handle and its status word.  NULL is accepted.  Work still queued on a stream
@@ -197,20 +198,27 @@ MOE_API const char* moe_profile_kind_name(int kind);
  * moe_route needs a caller-allocated workspace; some callers cannot provide one because they
  * may not allocate device memory at call time (every device byte belongs to another
  * allocator or pool, or allocation after start-up is forbidden, or the caller is plain C
- * without an allocator).  moe_route_static computes exactly what moe_route computes, with
- * the same arguments minus the workspace, and allocates nothing: its scratch is a fixed
- * array of moe_route_static_max_bytes() bytes (2 MiB) compiled into the library, which every
- * device that loads the library keeps until the process exits.
+ * without an allocator).  moe_route_static takes moe_route's arguments minus the workspace
+ * and allocates nothing: its scratch is a fixed array of moe_route_static_max_bytes() bytes
+ * (2 MiB) compiled into the library, which every device that loads the library keeps until
+ * the process exits.  moe_create looks up the array's device address (a runtime call that
+ * allocates nothing) and keeps it in the handle.
+ *   - Results: for T <= 64 identical to moe_route.  For T > 64 the router is not split over
+ *     the hidden dimension (moe_route splits it when T is small enough to leave SMs idle), so
+ *     the fp32 logit sums run in another order: topk_w can differ in the last bits, and a
+ *     token whose k-th and (k+1)-th logits are within rounding of each other (a near tie)
+ *     can select differently.  For the same reason it is slower than moe_route for T between
+ *     65 and a few thousand (ceil(T/64) blocks each sum over all of H).
  *   - The handle's device must be the current device (MOE_ERR_ARG otherwise).
  *   - If the routing scratch for T does not fit in the array, the call returns
  *     MOE_ERR_WORKSPACE and enqueues nothing.  The scratch is (H/64)*T*E*4 bytes of partial
  *     logits for T <= 64 and ceil(T/64)*E*4 bytes of per-block expert counts above that; with
  *     H = 2880 it fits for E = 32 up to T = 1,048,320, for E = 128 up to T = 262,016, and for
  *     E = 256 for T <= 45 and 65 <= T <= 130,944.
- *   - The first call on a device looks up the array's device address (a runtime call that
- *     does not allocate); make that first call before any stream capture.
- *   - All calls share the one array: two calls whose work overlaps on the GPU (different
- *     streams, or different handles on one device) race and give undefined results. */
+ *   - Every scratch word a call reads is written earlier in the same call, so no clearing is
+ *     needed between calls.  All calls share the one array: two calls whose work overlaps on
+ *     the GPU (different streams, or different handles on one device) race and give undefined
+ *     results. */
 MOE_API size_t moe_route_static_max_bytes(void);
 MOE_API moe_status moe_route_static(moe_t ctx, int T, const void* x_bf16,
                                     const void* W_router_bf16, const float* b_router,

@@ -10,7 +10,6 @@
 #include <cstring>
 #include <new>
 #include <utility>
-#include <mutex>
 #include <vector>
 
 #include "moe.h"
@@ -29,6 +28,8 @@ constexpr int kMaxHI = 16384;
 constexpr int kMaxT = 1 << 20;
 constexpr int kDefaultCrossover = 64;  // largest T streamed until moe_tune measures one
 constexpr int kMaxKernelsPerCall = 8;
+
+moe_status static_scratch_address(void** out);  // defined beside the array, at the end
 
 enum Kind { kKindRouter = 0, kKindRouteFin = 1, kKindGather = 2, kKindGateUp = 3,
             kKindDown = 4, kKindConvert = 5 };
@@ -57,6 +58,7 @@ struct moe_ctx {
   moe_path path = MOE_PATH_AUTO;
   int crossover = kDefaultCrossover;
   uint32_t* d_status = nullptr;
+  void* static_scratch = nullptr;  // device address of the routing scratch array (moe_route_static)
   uint64_t launches = 0;
   // profiling
   int prof_max = 0, prof_calls = 0;
@@ -685,6 +687,12 @@ moe_status moe_create(int E, int H, int I, int k, moe_t* out) {
     delete c;
     return MOE_ERR_CUDA;
   }
+  // the routing scratch of moe_route_static, looked up with this handle's device current
+  if (static_scratch_address(&c->static_scratch) != MOE_OK) {
+    cudaFree(c->d_status);
+    delete c;
+    return MOE_ERR_CUDA;
+  }
   *out = c;
   return MOE_OK;
 }
@@ -984,29 +992,22 @@ moe_status moe_selftest_timeout(moe_t c, int limit_us, moe_stream_t stream) {
 // ------------------------------------------------------------------------------------------
 namespace {
 constexpr size_t kRouteStaticScratchBytes = size_t(2) << 20;  // 2 MiB
-constexpr int kMaxDevices = 64;
 }  // namespace
 
 static __device__ __align__(256) uint8_t g_route_static_scratch[kRouteStaticScratchBytes];
 
 namespace {
-std::mutex g_static_scratch_mu;
-void* g_static_scratch_addr[kMaxDevices] = {};
-
-// Device address of g_route_static_scratch on the current device.  In host code the array's
-// name only stands for the symbol, so the address is looked up once per device and cached.
-moe_status static_scratch_address(int dev, void** out) {
-  if (dev < 0 || dev >= kMaxDevices) return MOE_ERR_DEVICE;
-  std::lock_guard<std::mutex> lock(g_static_scratch_mu);
-  if (!g_static_scratch_addr[dev]) {
-    void* p = nullptr;
-    if (cudaGetSymbolAddress(&p, g_route_static_scratch) != cudaSuccess || p == nullptr) {
-      cudaGetLastError();
-      return MOE_ERR_CUDA;
-    }
-    g_static_scratch_addr[dev] = p;
+// Device address of g_route_static_scratch in the current device's context.  In host code the
+// array's name only stands for the symbol; its device address comes from the runtime, which
+// allocates nothing to answer.  moe_create calls this with the handle's device current and
+// keeps the answer in the handle, whose lifetime is bounded by that context's.
+moe_status static_scratch_address(void** out) {
+  void* p = nullptr;
+  if (cudaGetSymbolAddress(&p, g_route_static_scratch) != cudaSuccess || p == nullptr) {
+    cudaGetLastError();
+    return MOE_ERR_CUDA;
   }
-  *out = g_static_scratch_addr[dev];
+  *out = p;
   return MOE_OK;
 }
 }  // namespace
@@ -1038,9 +1039,8 @@ moe_status moe_route_static(moe_t c, int T, const void* x_bf16, const void* W_ro
     return MOE_ERR_ARG;
   if (route_ws_bytes(c, T, /*allow_split=*/false) > kRouteStaticScratchBytes)
     return MOE_ERR_WORKSPACE;
-  void* scratch = nullptr;
-  MOE_TRY(static_scratch_address(dev, &scratch));
-  uint8_t* ws = static_cast<uint8_t*>(scratch);
+  if (!c->static_scratch) return MOE_ERR_CUDA;
+  uint8_t* ws = static_cast<uint8_t*>(c->static_scratch);
   Carver cv;
   const size_t sched_at = cv.take(16);
   const RouteTmp rt = carve_route_tmp(cv, c, T, /*allow_split=*/false);

@@ -5,6 +5,7 @@ import socket
 import subprocess
 import sys
 
+import numpy as np
 import pytest
 import torch
 import torch.distributed as dist
@@ -96,3 +97,29 @@ def test_algorithmic_bytes_of_mxfp4_weights():
     per_expert_gu = 2880 * 5760 // 2 + 2880 // 32 * 5760
     assert b["gate_up_bytes"] - f["gate_up_bytes"] == 27 * (per_expert_gu - 2880 * 5760 * 2)
     assert b["flops"] == f["flops"]
+
+
+def test_default_steps_make_the_timed_region_last_a_second():
+    assert bench.steps_for(0.0204) * 0.0204 >= bench.MIN_TIMED_S          # 131K layer, ~20 ms
+    assert bench.steps_for(0.0002) * 0.0002 >= bench.MIN_TIMED_S          # decode, ~0.2 ms
+    assert bench.steps_for(5.0) == 10                                       # never fewer than 10
+    assert bench.steps_for(1e-9) == 200000                                  # bounded
+
+
+def test_cpu_baseline_runs_on_the_workloads_seeded_sample():
+    import moe_inputs as mi
+    w = mi.WORKLOADS["131k_skewed"]
+    toks = bench.baseline_tokens(w, w.T)
+    assert toks.size == w.oracle_sample == 4096
+    assert np.array_equal(toks, mi.sample_tokens(w.T, 4096, w.seed))
+    assert np.all(np.diff(toks) > 0) and toks[-1] < w.T
+    d = mi.WORKLOADS["20b_decode"]
+    assert np.array_equal(bench.baseline_tokens(d, d.T), np.arange(d.T))
+
+
+def test_default_workload_is_the_largest_single_gpu_config():
+    import moe_inputs as mi
+    ap_default = bench.main.__code__.co_consts
+    w = mi.WORKLOADS["131k_skewed"]
+    assert "131k_skewed" in ap_default
+    assert w.T == max(x.T for x in mi.WORKLOADS.values())

@@ -251,6 +251,40 @@ def test_routing_invariants(T, E, k):
         assert np.all(np.any(idx[seg] == e, axis=1))
 
 
+def _brute_logits(h, rows):
+    """Pure-Python logits of the given token rows (own bf16 decoding, plain loops)."""
+    x, Wr, br = h["x"], h["W_router"], h["b_router"]
+    H, E = Wr.shape
+    return [[sum(py_bf16(x[t][c]) * py_bf16(Wr[c][e]) for c in range(H)) + float(br[e])
+             for e in range(E)] for t in rows]
+
+
+def check_chunked_logits(orc=moe_ref):
+    """The oracle computes the router logits in token chunks; every chunk size, including ones
+    that leave a ragged last chunk, gives the brute-force logits for every row."""
+    h = tiny_case(17, 6, 4, 2, 4, 51)
+    brute = np.array(_brute_logits(h, range(17)))
+    for chunk in (1, 4, 5, 16, 17, 64):
+        got = orc._logits_chunked(h["x"], h["W_router"], h["b_router"], chunk=chunk)
+        np.testing.assert_allclose(got, brute, rtol=1e-13, atol=1e-14)
+    # the default chunk (8192 tokens): routing of the rows on both sides of the first boundary
+    # and of the one-row tail
+    T = 8192 + 1
+    h = mi.host_inputs(mi.make_inputs(T, 4, 3, 2, 4, 52, "cpu", experts=False))
+    r = orc.moe_route_ref(h["x"], h["W_router"], h["b_router"], 2)
+    rows = [0, 8190, 8191, 8192]
+    np.testing.assert_allclose(r["logits"][rows], np.array(_brute_logits(h, rows)),
+                               rtol=1e-13, atol=1e-14)
+    for i, t in enumerate(rows):
+        lg = r["logits"][t]
+        best = sorted(range(3), key=lambda e: (-lg[e], e))[:2]
+        assert r["idx"][t].tolist() == best
+
+
+def test_chunked_router_logits_across_chunk_boundaries():
+    check_chunked_logits()
+
+
 def test_token_subset_equals_full_rows():
     h = tiny_case(40, 32, 6, 2, 16, 41)
     args = (h["x"], h["W_router"], h["b_router"], h["W_gate_up"], h["W_down"], 2)
@@ -330,6 +364,37 @@ def _down_transposed(xrows, Wgu, Wd):
 
 
 _ORIG_PERM = moe_ref.permutation
+
+
+def _chunk_tail_dropped(x_bits, W_router_bits, b_router, chunk=8192):
+    Wr = moe_ref.decode_bf16(W_router_bits)
+    b = np.asarray(b_router, dtype=np.float32).astype(np.float64)
+    T = x_bits.shape[0]
+    out = np.zeros((T, Wr.shape[1]))
+    for t0 in range(0, T - T % chunk, chunk):        # the ragged last chunk is skipped
+        out[t0:t0 + chunk] = moe_ref.router_logits(moe_ref.decode_bf16(x_bits[t0:t0 + chunk]), Wr, b)
+    return out
+
+
+def _chunk_bias_once(x_bits, W_router_bits, b_router, chunk=8192):
+    Wr = moe_ref.decode_bf16(W_router_bits)
+    b = np.asarray(b_router, dtype=np.float32).astype(np.float64)
+    T = x_bits.shape[0]
+    out = np.empty((T, Wr.shape[1]))
+    for t0 in range(0, T, chunk):                     # bias added to the first chunk only
+        out[t0:t0 + chunk] = moe_ref.router_logits(moe_ref.decode_bf16(x_bits[t0:t0 + chunk]), Wr,
+                                                   b if t0 == 0 else 0 * b)
+    return out
+
+
+CHUNK_MUTANTS = {"chunk_tail_dropped": _chunk_tail_dropped, "chunk_bias_once": _chunk_bias_once}
+
+
+@pytest.mark.parametrize("name", sorted(CHUNK_MUTANTS))
+def test_planted_chunking_mistake_is_caught(name, monkeypatch):
+    monkeypatch.setattr(moe_ref, "_logits_chunked", CHUNK_MUTANTS[name])
+    with pytest.raises(AssertionError):
+        check_chunked_logits(moe_ref)
 
 MUTANTS = {
     "gate_up_swapped": ("expert_mlp", _gate_up_swapped),

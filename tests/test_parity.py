@@ -65,3 +65,35 @@ def test_131k_skewed():
     ratio = cnt.max() / cnt.mean()
     print("131k max/mean expert load", ratio)
     assert 3.5 <= ratio <= 4.5
+
+
+@pytest.fixture(scope="module")
+def layer_120b():
+    """The 120b-shaped layer (128 experts, top-4: hearth-lean-loomed-v1 card, intro) with 512
+    seeded tokens, drawn once on the GPU and copied to the host for the oracle."""
+    w = mi.WORKLOADS["120b_sweep"]
+    d, h = inputs_on_gpu(512, w.H, w.E, w.k, w.I, w.seed)
+    return w, d, h
+
+
+@pytest.mark.parametrize("T", [65, 97, 512])
+@pytest.mark.parametrize("path", ["gemm", "auto"])
+def test_120b_above_the_crossover(layer_120b, T, path):
+    """E = 128 at token counts where AUTO leaves the streaming path: the tcgen05 grouped GEMM
+    (forced, and as AUTO picks it), every token's routing and output against the oracle."""
+    w, d0, h0 = layer_120b
+    d = dict(d0, x=d0["x"][:T].contiguous())
+    h = dict(h0, x=h0["x"][:T])
+    layer = moe.Moe(w.E, w.H, w.I, w.k)
+    if path == "gemm":
+        layer.set_path(moe.MOE_PATH_GEMM)
+    ref_route = host_route(h, w.k)
+    g = gpu_route(layer, d)
+    rep = compare_routing(g, ref_route, w.k, w.E)
+    out = layer.forward(d["x"], d["W_router"], d["b_router"], d["W_gate_up"], d["W_down"])
+    assert layer.sync_status() == moe.MOE_OK
+    tokens = np.arange(T)
+    ref_out = oracle.moe_forward_ref(h["x"], h["W_router"], h["b_router"], h["W_gate_up"],
+                                     h["W_down"], w.k, route=ref_route)
+    rep.update(check_outputs(out.double().cpu().numpy(), tokens, h, ref_route, g, ref_out))
+    print("120b", path, T, json.dumps({k: v for k, v in rep.items() if k != "set_changed"}))

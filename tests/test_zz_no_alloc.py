@@ -4,7 +4,10 @@ Such callers (a process whose device memory all belongs to another allocator, a 
 that forbids allocation after start-up, a C caller without an allocator) cannot pass the
 workspace moe_route needs.  moe_route_static uses a fixed scratch array built into the
 library instead.  This test calls it through the C ABI twice in a row and checks each result
-against moe_route with a caller workspace, to the routing tolerances the parity tests use.
+against moe_route with a caller workspace, to the routing tolerances the parity tests use:
+above 64 tokens the static call's router sums the logits in another order, so a token may
+select differently only where the fp64 oracle's k-th / (k+1)-th logit gap is a near tie, and
+the permutation must then be the one of the static call's own selection.
 """
 import ctypes
 
@@ -13,7 +16,8 @@ import pytest
 import torch
 
 import moe_inputs as mi
-from parity_util import W_TOL
+import oracle
+from parity_util import NEAR_TIE, W_TOL, host_route
 
 pytestmark = pytest.mark.gpu
 
@@ -39,10 +43,29 @@ def _call_static(layer, d, o):
                                 o["inv_perm"].data_ptr(), st)
 
 
+def _check_against_workspace_route(got, ref, gaps, E):
+    """Routing of the static call against moe_route's, to the parity tests' tolerances."""
+    diff = np.nonzero(np.any(got["topk_idx"] != ref["topk_idx"], axis=1))[0]
+    for t in diff:                            # only near ties may select differently
+        assert min(gaps["gap_k"][t], gaps["gap_in"][t]) < NEAR_TIE, f"token {t}"
+    same = np.setdiff1d(np.arange(got["topk_idx"].shape[0]), diff)
+    assert np.abs(got["topk_w"][same] - ref["topk_w"][same]).max() <= W_TOL
+    # the permutation is unique given the selection: the static call's own, bit for bit
+    idx = got["topk_idx"].astype(np.int64)
+    perm, inv = oracle.permutation(idx, E)
+    assert np.array_equal(got["expert_offsets"], oracle.expert_offsets(oracle.expert_histogram(idx, E)))
+    assert np.array_equal(got["perm"], perm) and np.array_equal(got["inv_perm"], inv)
+    if diff.size == 0:
+        for key in ("expert_offsets", "perm", "inv_perm"):
+            assert np.array_equal(got[key], ref[key]), key
+    return int(diff.size)
+
+
 @pytest.mark.parametrize("T", [16, 300])   # the single-block and the multi-block routing chain
 def test_static_scratch_route_matches_workspace_route(T):
     E, H, k = 32, 2880, 4
     d = mi.make_inputs(T, H, E, k, 64, seed=1234 + T, device="cuda", experts=False)
+    gaps = host_route(mi.host_inputs(d), k)
     layer = moe.Moe(E, H, 64, k)
     ref = {key: v.cpu().numpy() for key, v in layer.route(d["x"], d["W_router"], d["b_router"]).items()}
     for _ in range(2):                       # two calls in a row share the one scratch array
@@ -52,9 +75,10 @@ def test_static_scratch_route_matches_workspace_route(T):
         assert _call_static(layer, d, o) == moe.MOE_OK
         torch.cuda.synchronize()
         got = {key: v.cpu().numpy() for key, v in o.items()}
-        for key in ("topk_idx", "expert_offsets", "perm", "inv_perm"):
-            assert np.array_equal(got[key], ref[key]), key
-        assert np.abs(got["topk_w"] - ref["topk_w"]).max() <= W_TOL
+        n_diff = _check_against_workspace_route(got, ref, gaps, E)
+        if T <= 64:                          # same kernels, same order: identical
+            assert n_diff == 0
+            assert np.array_equal(got["topk_w"], ref["topk_w"])
     assert layer.sync_status() == moe.MOE_OK
 
 
