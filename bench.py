@@ -79,6 +79,13 @@ def measured_peaks() -> tuple[float, float, float, str]:
         return FALLBACK_HBM_GBS, FALLBACK_BF16_TFLOPS, 1400.0, "fallback"
 
 
+def peak_label(source: str, key: str) -> str:
+    """Where a roofline denominator comes from, for the JSON line."""
+    if source == "measured":
+        return f"measured {key} (MEASURED_PEAKS.json)"
+    return f"fallback {key} (no MEASURED_PEAKS.json: 6650 GB/s, 1590 TFLOP/s burst, 1400 sustained)"
+
+
 def source_digest(paths) -> str:
     h = hashlib.sha256()
     for p in paths:
@@ -176,6 +183,68 @@ def algorithmic(T: int, H: int, E: int, k: int, I: int, counts, weights: str = "
     return dict(touched=touched, gate_up_bytes=gate_up_bytes, down_bytes=down_bytes,
                 layer_bytes=layer_bytes, flops=flops, gate_up_flops=gate_up_flops,
                 down_flops=down_flops)
+
+
+FAMILIES = ("stream", "tile", "gemm")
+KERNEL_NAMES = {  # the gate/up kernel of each family, as ncu lists it
+    "stream": "stream_gate_up_kernel", "tile": "expert_tile_kernel<0>",
+    "gemm": "grouped_gemm_kernel<gate_up>"}
+
+
+def split_families(counts, path: str, stream_rows: int, tile_rows: int) -> dict:
+    """Row counts of the experts each kernel family multiplies, as the library dispatches them
+    (moe_path in include/moe.h): with "auto", an expert with c rows streams if c <= stream_rows,
+    takes expert tiles if c <= tile_rows, else row tiles."""
+    out = {f: [] for f in FAMILIES}
+    for c in counts:
+        if c <= 0:
+            continue
+        if path in FAMILIES:
+            f = path
+        elif c <= stream_rows:
+            f = "stream"
+        elif c <= max(stream_rows, tile_rows):
+            f = "tile"
+        else:
+            f = "gemm"
+        out[f].append(int(c))
+    return out
+
+
+def family_work(counts, H: int, I: int, weights: str = "bf16") -> dict:
+    """Algorithmic work of one projection pair over the given experts (their row counts): the
+    touched experts' weights, the rows read and written, and the MMA FLOPs."""
+    n, rows = len(counts), int(sum(counts))
+    per_gu = H * 2 * I // 2 + H // 32 * 2 * I if weights == "mxfp4" else H * 2 * I * 2
+    per_dn = I * H // 2 + I // 32 * H if weights == "mxfp4" else I * H * 2
+    return dict(experts=n, rows=rows,
+                gate_up_bytes=n * per_gu + rows * H * 2 + rows * I * 2,
+                down_bytes=n * per_dn + rows * I * 2 + rows * H * 4,
+                gate_up_flops=2 * rows * H * 2 * I, down_flops=2 * rows * I * H)
+
+
+def dominant_roofline(work: dict, gate_up_ms: dict, hbm: float, bf16: float, bf16_sus: float,
+                      peak_src: str) -> dict:
+    """Roofline of the dominant kernel: the gate/up kernel of the family that spent the most
+    time per call.  Its bound is its own: weight bytes over HBM bandwidth, or FLOPs over the
+    tensor peak, whichever takes longer.  gate_up_ms: family -> ms per call (profiled)."""
+    fam = max((f for f in FAMILIES if gate_up_ms.get(f, 0) > 0), key=lambda f: gate_up_ms[f])
+    wk, secs = work[fam], gate_up_ms[fam] / 1e3
+    t_hbm = wk["gate_up_bytes"] / (hbm * 1e9)
+    t_tc = wk["gate_up_flops"] / (bf16 * 1e12)
+    base = dict(kernel=KERNEL_NAMES[fam], family=fam, experts=wk["experts"], rows=wk["rows"],
+                avg_launch_ms=gate_up_ms[fam])
+    if t_hbm >= t_tc:
+        ach = wk["gate_up_bytes"] / secs / 1e9
+        return dict(bound="hbm", achieved=ach, peak=hbm, unit="GB/s", frac=ach / hbm,
+                    alg_bytes_per_launch=wk["gate_up_bytes"],
+                    peak_source=peak_label(peak_src, "hbm_gbs"), **base)
+    # a launch well under a second is timed alone: the burst tensor peak applies
+    ach = wk["gate_up_flops"] / secs / 1e12
+    return dict(bound="tensor", achieved=ach, peak=bf16, unit="TFLOP/s", frac=ach / bf16,
+                alg_flops_per_launch=wk["gate_up_flops"],
+                peak_source=peak_label(peak_src, "bf16_tflops (burst)"),
+                frac_of_sustained=ach / bf16_sus, frac_of_nominal_2250=ach / 2250.0, **base)
 
 
 # ----------------------------------------------------------------------------------------
@@ -364,36 +433,28 @@ def run_ours(args, w: mi.Workload, T: int) -> None:
     torch.cuda.synchronize()
     e2e_secs = reduce_max(e0.elapsed_time(e1) / 1e3, world)
 
-    # ---- roofline of the dominant kernel: the gate/up projection (2/3 of bytes and FLOPs) ----
+    # ---- roofline of the dominant kernel: the gate/up projection (2/3 of bytes and FLOPs) of
+    # the kernel family that spent the most time ----
     hbm, bf16, bf16_sus, peak_src = measured_peaks()
-    path_setting, crossover = layer.get_path()
-    path = "stream" if (mx or path_setting == moe.MOE_PATH_STREAM or
-                        (path_setting == moe.MOE_PATH_AUTO and T <= crossover)) else "gemm"
-    gu_ms, gu_n = prof["gate_up_swiglu"]
-    dn_ms, dn_n = prof["down_combine"]
-    gu_avg_s = gu_ms / 1e3 / max(gu_n, 1)
-    dn_avg_s = dn_ms / 1e3 / max(dn_n, 1)
+    path_setting, _ = layer.get_path()
+    stream_rows, tile_rows = layer.get_dispatch()
+    path = "stream" if mx else {moe.MOE_PATH_STREAM: "stream", moe.MOE_PATH_GEMM: "gemm",
+                                moe.MOE_PATH_TILE: "tile"}.get(path_setting, "auto")
+    fams = split_families(counts, path, stream_rows, tile_rows)
+    work = {f: family_work(fams[f], w.H, w.I, w.weights) for f in FAMILIES}
+    n_prof = prof_steps
+    gu_ms = {f: prof["gate_up_" + f][0] / n_prof for f in FAMILIES}
+    dn_ms = {f: prof["down_" + f][0] / n_prof for f in FAMILIES}
     layer_roof_s = max(alg["layer_bytes"] / (hbm * 1e9), alg["flops"] / (bf16 * 1e12))
-    kernels_ms = {k_: round(v[0] / max(v[1], 1), 4) for k_, v in prof.items() if v[1]}
-    src = f"{peak_src} %s (MEASURED_PEAKS.json)" if peak_src == "measured" else "fallback"
-    if path == "stream":
-        kname = "stream_gate_up_mx_kernel" if mx else "stream_gate_up_kernel"
-        achieved = alg["gate_up_bytes"] / gu_avg_s / 1e9
-        roof = dict(bound="hbm", achieved=achieved, peak=hbm, unit="GB/s", frac=achieved / hbm,
-                    traffic=ncu_traffic(kname, w.name), kernel=kname,
-                    alg_bytes_per_launch=alg["gate_up_bytes"], avg_launch_ms=gu_avg_s * 1e3,
-                    peak_source=src % "hbm_gbs")
-        down_rate = dict(down_kernel_GBps=alg["down_bytes"] / dn_avg_s / 1e9)
-    else:
-        kname = "grouped_gemm_kernel<gate_up>"
-        # a launch well under a second is timed alone: the burst tensor peak applies
-        achieved = alg["gate_up_flops"] / gu_avg_s / 1e12
-        roof = dict(bound="tensor", achieved=achieved, peak=bf16, unit="TFLOP/s",
-                    frac=achieved / bf16, traffic=ncu_traffic(kname, w.name), kernel=kname,
-                    alg_flops_per_launch=alg["gate_up_flops"], avg_launch_ms=gu_avg_s * 1e3,
-                    peak_source=src % "bf16_tflops (burst)",
-                    frac_of_sustained=achieved / bf16_sus, frac_of_nominal_2250=achieved / 2250.0)
-        down_rate = dict(down_kernel_TFLOPs=alg["down_flops"] / dn_avg_s / 1e12)
+    kernels_ms = {k_: round(v[0] / n_prof, 4) for k_, v in prof.items() if v[1]}
+    roof = dominant_roofline(work, gu_ms, hbm, bf16, bf16_sus, peak_src)
+    if mx:
+        roof["kernel"] = "stream_gate_up_mx_kernel"
+    roof["traffic"] = ncu_traffic(roof["kernel"], w.name)
+    down_rate = {f"down_{f}_ms": round(dn_ms[f], 4) for f in FAMILIES if dn_ms[f] > 0}
+    dispatch = dict(stream_rows=stream_rows, tile_rows=tile_rows,
+                    experts={f: len(fams[f]) for f in FAMILIES},
+                    rows={f: int(sum(fams[f])) for f in FAMILIES})
 
     line = dict(
         metric=METRIC, value=agg["value"], unit=UNIT, n_gpus=world, steps=steps,
@@ -402,7 +463,7 @@ def run_ours(args, w: mi.Workload, T: int) -> None:
         dtype="mxfp4 weights, bf16 activations" if mx else "bf16",
         data="synthetic (seeded N(0,1) tokens, N(0,1/fan_in) bf16 weights; no trained weights)",
         config=dict(workload=w.name, T=T, H=w.H, E=w.E, k=w.k, I=w.I, path=path,
-                    weights=w.weights,
+                    weights=w.weights, dispatch=dispatch,
                     parallelism=f"replicas{world}" if world > 1 else "single",
                     l2="inputs larger than L2: %.2f GB of touched expert weights and tokens per "
                        "step vs 126 MB L2" % ((alg["layer_bytes"]) / 1e9)),
@@ -411,7 +472,8 @@ def run_ours(args, w: mi.Workload, T: int) -> None:
                             alg_flops=alg["flops"], roofline_us=layer_roof_s * 1e6,
                             frac=layer_roof_s / (secs / steps), **down_rate),
         kernel_avg_ms=kernels_ms,
-        kernel_timing="per-kernel CUDA events over a second timed pass of min(K, 200) of the same calls",
+        kernel_timing="per-kernel CUDA events over a second timed pass of min(K, 200) of the same "
+                      "calls (ms per call)",
         e2e=dict(value=T * world * steps / e2e_secs, unit=UNIT,
                  h2d_bytes_per_step=T * w.H * 2, d2h_bytes_per_step=T * w.H * 4),
         gpu_launches=gpu_launches,

@@ -80,10 +80,23 @@ typedef enum {
   MOE_ERR_DEVICE = 6        /* no usable sm_100 device */
 } moe_status;
 
+/* Which kernels multiply an expert's rows.  AUTO decides per expert, on the device, from the
+ * expert's row count in this call's routing (no host synchronisation):
+ *   rows <= stream_rows               weight streaming (tensor-core mma.sync, split over K
+ *                                     across all SMs): the decode regime, ~1 row per expert
+ *   stream_rows < rows <= tile_rows   expert tiles: tcgen05 MMAs with the expert's weight
+ *                                     columns as the M operand and its rows as N, each weight
+ *                                     block read once for up to 128 rows
+ *   rows > tile_rows                  row tiles: 2-SM tcgen05 grouped GEMM, 256 rows x 256
+ *                                     columns per CTA pair (prefill, long sequences)
+ * This is the per-expert mat-vec / mat-mat choice of the hearth-lean-loomed-v1 card ("Why
+ * 12-16 streams can be slow on Vulkan"), made per expert and per call.  The other values
+ * force one kernel family for every expert. */
 typedef enum {
-  MOE_PATH_AUTO = 0,    /* weight streaming for T <= crossover, grouped GEMM above it */
-  MOE_PATH_STREAM = 1,  /* always stream expert weights (CUDA-core split-K GEMV) */
-  MOE_PATH_GEMM = 2     /* always the tcgen05 grouped GEMM */
+  MOE_PATH_AUTO = 0,    /* per-expert choice among the three families below */
+  MOE_PATH_STREAM = 1,  /* every expert through the weight-streaming kernels */
+  MOE_PATH_GEMM = 2,    /* every expert through the 2-SM row-tile grouped GEMM */
+  MOE_PATH_TILE = 3     /* every expert through the expert-tile kernels */
 } moe_path;
 
 /* Create a handle for a layer of shape (E, H, I, k) on the current device.  Validates the
@@ -117,9 +130,9 @@ MOE_API moe_status moe_route(moe_t ctx, int T, const void* x_bf16, const void* W
                      void* workspace, size_t ws_bytes, moe_stream_t stream);
 
 /* The whole layer: writes out [T, H] fp32 (every element).  workspace: at least
- * moe_workspace_bytes(ctx, T) bytes.  The path (streaming or grouped GEMM) is chosen on the
- * host from T and the handle's setting, never from device data, so the call does not
- * synchronise.  T = 0 is a no-op. */
+ * moe_workspace_bytes(ctx, T) bytes.  The kernel family of each expert is chosen on the device
+ * (see moe_path); the host only leaves out families that no expert can reach (an expert holds
+ * at most T rows), so the call never synchronises.  T = 0 is a no-op. */
 MOE_API moe_status moe_forward(moe_t ctx, int T, const void* x_bf16, const void* W_router_bf16,
                        const float* b_router, const void* W_gate_up_bf16,
                        const void* W_down_bf16, float* out, void* workspace, size_t ws_bytes,
@@ -148,20 +161,30 @@ MOE_API moe_status moe_forward_mxfp4(moe_t ctx, int T, const void* x_bf16,
                                      const void* dn_codes, const void* dn_scales, float* out,
                                      void* workspace, size_t ws_bytes, moe_stream_t stream);
 
-/* Choose the path.  crossover_T >= 0 sets the largest T that MOE_PATH_AUTO streams;
- * crossover_T < 0 keeps the current one (the built-in default or the value moe_tune
- * measured).  MOE_ERR_UNSUPPORTED if the path is not available on this device. */
-MOE_API moe_status moe_set_path(moe_t ctx, moe_path path, int crossover_T);
+/* Choose the path.  stream_rows >= 0 also sets the AUTO threshold: experts with at most this
+ * many rows in a call stream their weights (the built-in default is 16, one streaming chunk;
+ * moe_tune measures it); stream_rows < 0 keeps the current one.  MOE_ERR_ARG for an unknown
+ * path. */
+MOE_API moe_status moe_set_path(moe_t ctx, moe_path path, int stream_rows);
 
-/* Current path setting and crossover. */
-MOE_API moe_status moe_get_path(moe_t ctx, moe_path* path, int* crossover_T);
+/* Current path setting and AUTO streaming threshold (rows per expert). */
+MOE_API moe_status moe_get_path(moe_t ctx, moe_path* path, int* stream_rows);
 
-/* Measure the crossover on this device with the caller's layer: times both paths (median of
- * 5 calls after 2 warm-ups) at T = 1, 2, 4, 8, 12, 16, 24, 32, 48, 64, ... up to T_max, stops
- * once the grouped GEMM has been faster for a doubling of T, and stores the largest T at which
- * streaming was not slower (0 if never) as the handle's crossover.  x must hold T_max rows,
- * out T_max rows; workspace at least moe_tune_workspace_bytes(ctx, T_max).  Synchronises
- * `stream`; the path setting is left as it was.  *crossover_out (may be NULL) receives it. */
+/* Both AUTO thresholds, in rows of one expert: stream_rows (see moe_set_path) and tile_rows
+ * (experts with more rows than stream_rows and at most tile_rows take expert tiles, more rows
+ * the row-tile GEMM; default 256).  A negative value keeps the current one. */
+MOE_API moe_status moe_set_dispatch(moe_t ctx, int stream_rows, int tile_rows);
+MOE_API moe_status moe_get_dispatch(moe_t ctx, int* stream_rows, int* tile_rows);
+
+/* Measure the AUTO thresholds on this device with the caller's layer: times the whole layer
+ * (median of 5 calls after 2 warm-ups) with every expert forced through each family, at
+ * T = 1, 2, 4, 8, 12, 16, 24, 32, 48, 64, ... up to T_max, streaming against expert tiles and
+ * expert tiles against row tiles.  For each pair it takes the largest T at which the lower
+ * family was not slower (stopping once the upper one has been faster for a doubling of T) and
+ * stores the mean rows per expert at that T, ceil(T * k / E), as the threshold.  x must hold
+ * T_max rows, out T_max rows; workspace at least moe_tune_workspace_bytes(ctx, T_max).
+ * Synchronises `stream`; the path setting is left as it was.  *crossover_out (may be NULL)
+ * receives stream_rows; moe_get_dispatch gives both. */
 MOE_API size_t moe_tune_workspace_bytes(moe_t ctx, int T_max);
 MOE_API moe_status moe_tune(moe_t ctx, int T_max, const void* x_bf16, const void* W_router_bf16,
                     const float* b_router, const void* W_gate_up_bf16,
@@ -184,10 +207,11 @@ MOE_API uint64_t moe_launch_count(moe_t ctx);
  * kernel it launches, on the call's stream.  moe_profile_end synchronises, and writes for
  * each kernel kind i < n_kinds the total milliseconds into ms[i] and its launch count into
  * launches[i], then frees the events.  Kinds: 0 router, 1 routing finalize / scan / scatter,
- * 2 gather, 3 gate/up projection + SwiGLU, 4 down projection + combine, 5 conversion of the
- * input to f16 (MXFP4 path).
+ * 2 gather of the rows into expert order, 3 / 4 gate/up projection + SwiGLU / down projection
+ * + combine on the weight-streaming kernels, 5 conversion of the input to f16 (MXFP4 path),
+ * 6 / 7 the same projections on the expert-tile kernels, 8 / 9 on the row-tile grouped GEMM.
  * moe_profile_kind_name gives a kind's name. */
-#define MOE_PROFILE_KINDS 6
+#define MOE_PROFILE_KINDS 10
 MOE_API moe_status moe_profile_begin(moe_t ctx, int max_calls);
 MOE_API moe_status moe_profile_end(moe_t ctx, float* ms, int* launches, int n_kinds);
 MOE_API const char* moe_profile_kind_name(int kind);

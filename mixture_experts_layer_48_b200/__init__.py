@@ -28,8 +28,8 @@ _lib = ctypes.CDLL(LIB_PATH)
 
 MOE_OK, MOE_ERR_ARG, MOE_ERR_UNSUPPORTED, MOE_ERR_WORKSPACE = 0, 1, 2, 3
 MOE_ERR_CUDA, MOE_ERR_TIMEOUT, MOE_ERR_DEVICE = 4, 5, 6
-MOE_PATH_AUTO, MOE_PATH_STREAM, MOE_PATH_GEMM = 0, 1, 2
-MOE_PROFILE_KINDS = 6
+MOE_PATH_AUTO, MOE_PATH_STREAM, MOE_PATH_GEMM, MOE_PATH_TILE = 0, 1, 2, 3
+MOE_PROFILE_KINDS = 10
 
 # Every entry point of include/moe.h: name -> (restype, argtypes)
 _c_int, _vp, _sz = ctypes.c_int, ctypes.c_void_p, ctypes.c_size_t
@@ -45,6 +45,8 @@ _SIGS = {
                                    _sz, _vp]),
     "moe_set_path": (_c_int, [_vp, _c_int, _c_int]),
     "moe_get_path": (_c_int, [_vp, ctypes.POINTER(_c_int), ctypes.POINTER(_c_int)]),
+    "moe_set_dispatch": (_c_int, [_vp, _c_int, _c_int]),
+    "moe_get_dispatch": (_c_int, [_vp, ctypes.POINTER(_c_int), ctypes.POINTER(_c_int)]),
     "moe_tune_workspace_bytes": (_sz, [_vp, _c_int]),
     "moe_tune": (_c_int, [_vp, _c_int, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _sz, _vp,
                           ctypes.POINTER(_c_int)]),
@@ -124,13 +126,22 @@ class Moe:
         return self._h
 
     # -- settings --------------------------------------------------------------------
-    def set_path(self, path: int, crossover: int = -1) -> None:
-        _check(moe_set_path(self._h, path, crossover), "moe_set_path")
+    def set_path(self, path: int, stream_rows: int = -1) -> None:
+        _check(moe_set_path(self._h, path, stream_rows), "moe_set_path")
 
     def get_path(self) -> tuple[int, int]:
         p, c = _c_int(), _c_int()
         _check(moe_get_path(self._h, ctypes.byref(p), ctypes.byref(c)), "moe_get_path")
         return p.value, c.value
+
+    def set_dispatch(self, stream_rows: int = -1, tile_rows: int = -1) -> None:
+        """AUTO thresholds in rows of one expert (negative: keep); see include/moe.h."""
+        _check(moe_set_dispatch(self._h, stream_rows, tile_rows), "moe_set_dispatch")
+
+    def get_dispatch(self) -> tuple[int, int]:
+        s_, t_ = _c_int(), _c_int()
+        _check(moe_get_dispatch(self._h, ctypes.byref(s_), ctypes.byref(t_)), "moe_get_dispatch")
+        return s_.value, t_.value
 
     def workspace_bytes(self, T: int) -> int:
         return moe_workspace_bytes(self._h, T)

@@ -18,6 +18,7 @@
 #include "stream.cuh"
 #include "stream_mx.cuh"
 #include "gemm.cuh"
+#include "expert_gemm.cuh"
 
 using namespace moe;
 
@@ -26,13 +27,19 @@ namespace {
 constexpr int kMaxE = 256;
 constexpr int kMaxHI = 16384;
 constexpr int kMaxT = 1 << 20;
-constexpr int kDefaultCrossover = 64;  // largest T streamed until moe_tune measures one
-constexpr int kMaxKernelsPerCall = 8;
+// Per-expert dispatch thresholds (rows of one expert) until moe_tune measures them: up to one
+// streaming chunk streams, up to two expert tiles take the expert-tile kernel, more rows the
+// row-tile grouped GEMM.
+constexpr int kDefaultStreamRows = 16;
+constexpr int kDefaultTileRows = 256;
+constexpr int kMaxKernelsPerCall = 12;
 
 moe_status static_scratch_address(void** out);  // defined beside the array, at the end
 
+// Profiled kernel kinds (moe_profile_end): one per kernel family and projection.
 enum Kind { kKindRouter = 0, kKindRouteFin = 1, kKindGather = 2, kKindGateUp = 3,
-            kKindDown = 4, kKindConvert = 5 };
+            kKindDown = 4, kKindConvert = 5, kKindGateUpTile = 6, kKindDownTile = 7,
+            kKindGateUpGemm = 8, kKindDownGemm = 9 };
 
 }  // namespace
 
@@ -52,11 +59,13 @@ constexpr int kGemmChunkRows = 2 * kGemmBM;  // rows per tile: one 256-row MMA o
 struct moe_ctx {
   int E, H, I, k;
   MapCache gate_up_stream, down_stream, gate_up_gemm, down_gemm, x_perm_map, h_map;
+  MapCache et_x_map, et_h_map;  // activation rows for the expert-tile kernel (16-row boxes)
   MapCache gu_codes, gu_scales, dn_codes, dn_scales;  // MXFP4 weights (streaming path)
   int device = 0;
   int num_sms = 148;
   moe_path path = MOE_PATH_AUTO;
-  int crossover = kDefaultCrossover;
+  int stream_rows = kDefaultStreamRows;  // AUTO: experts with at most this many rows stream
+  int tile_rows = kDefaultTileRows;      // ... up to this many take expert tiles; more: row tiles
   uint32_t* d_status = nullptr;
   void* static_scratch = nullptr;  // device address of the routing scratch array (moe_route_static)
   uint64_t launches = 0;
@@ -195,61 +204,103 @@ RouteTmp carve_route_tmp(Carver& cv, const moe_ctx* c, int T, bool allow_split =
   return r;
 }
 
-struct StreamLayout {
-  size_t topk_idx, topk_w, inv_perm, perm, row_w, offsets, sched, chunks, acc, done, h, x16;
-  RouteTmp rt;
-  int max_chunks, n_done;
-  size_t total;
+// ---- per-expert dispatch --------------------------------------------------------------
+// Three kernel families multiply an expert's rows, chosen per expert on the device from its
+// row count (the routing kernels build one work list per family):
+//   stream  rows <= stream_rows:      weight streaming on mma.sync, stream-K split (decode)
+//   tile    up to tile_rows:          tcgen05 expert tiles, weights as the M operand
+//   gemm    more than tile_rows:      2-SM tcgen05 row tiles (prefill, long sequences)
+// The host only decides which families may receive rows: an expert holds at most T rows (a
+// token picks an expert at most once), so families above T are not launched.
+enum Family { kFamStream = 0, kFamTile = 1, kFamGemm = 2, kFamilies = 3 };
+constexpr int kFamChunkRows[kFamilies] = {kStreamRB, kEtRows, kGemmChunkRows};
+
+struct Plan {
+  bool has[kFamilies] = {false, false, false};
+  int max_count[kFamilies] = {0, 0, 0};   // family f takes counts in (max_count[f-1], max_count[f]]
+  int min_count(int f) const {
+    int m = 0;
+    for (int g = 0; g < f; ++g)
+      if (has[g]) m = max_count[g];
+    return m;
+  }
 };
 
-StreamLayout stream_layout(const moe_ctx* c, int T) {
-  StreamLayout L{};
-  Carver cv;
-  const size_t R = (size_t)T * c->k;
-  L.max_chunks = (int)(R / kStreamRB) + c->E;
-  // one completion counter per (chunk, column tile); the MXFP4 kernels' tiles are narrower
-  const int tile_cols = std::min(kStreamCols, kMxTileCols);
-  const int NT = (c->I + tile_cols - 1) / tile_cols;
-  L.n_done = L.max_chunks * NT;
-  L.topk_idx = cv.take(4 * R);
-  L.topk_w = cv.take(4 * R);
-  L.inv_perm = cv.take(4 * R);
-  L.perm = cv.take(4 * R);
-  L.row_w = cv.take(4 * R);
-  L.offsets = cv.take(4 * (size_t)(c->E + 1));
-  L.sched = cv.take(16);
-  L.chunks = cv.take(16 * (size_t)L.max_chunks);
-  L.done = cv.take(4 * (size_t)L.n_done);
-  L.h = cv.take(2 * R * c->I);
-  L.x16 = cv.take(2 * (size_t)T * c->H);  // MXFP4 path: the layer input in f16
-  L.acc = cv.take(sizeof(float) * R * 2 * c->I);
-  L.rt = carve_route_tmp(cv, c, T);
-  L.total = cv.cur;
-  return L;
+Plan make_plan(const moe_ctx* c, int T, bool mx, moe_path path) {
+  Plan p;
+  auto only = [&](int f) {
+    p.has[f] = true;
+    p.max_count[f] = INT_MAX;
+  };
+  if (mx) {  // MXFP4 experts: streaming kernels only
+    only(kFamStream);
+    return p;
+  }
+  switch (path) {
+    case MOE_PATH_STREAM: only(kFamStream); break;
+    case MOE_PATH_GEMM: only(kFamGemm); break;
+    case MOE_PATH_TILE: only(kFamTile); break;
+    default: {
+      const int s = c->stream_rows, t = std::max(c->stream_rows, c->tile_rows);
+      p.has[kFamStream] = s > 0;
+      p.max_count[kFamStream] = s;
+      p.has[kFamTile] = T > s && t > s;
+      p.max_count[kFamTile] = t;
+      p.has[kFamGemm] = T > t;
+      p.max_count[kFamGemm] = INT_MAX;
+      if (!p.has[kFamTile] && !p.has[kFamGemm]) p.max_count[kFamStream] = INT_MAX;
+      else if (!p.has[kFamGemm]) p.max_count[kFamTile] = INT_MAX;
+    }
+  }
+  return p;
 }
 
-struct GemmLayout {
-  size_t topk_idx, topk_w, inv_perm, perm, row_w, offsets, sched, chunks, x_perm, h;
+// Work-list entries family f can need for T tokens.
+int max_chunks(const moe_ctx* c, int T, const Plan& p, int f) {
+  const long long R = (long long)T * c->k, rows = kFamChunkRows[f];
+  long long n = R / rows + c->E;
+  if (p.max_count[f] != INT_MAX)
+    n = std::min(n, (long long)c->E * ((p.max_count[f] + rows - 1) / rows));
+  return (int)n;
+}
+
+struct Layout {
+  size_t topk_idx, topk_w, inv_perm, perm, row_w, offsets;
+  size_t sched[kFamilies], chunks[kFamilies];
+  size_t done, acc, h, x16, x_perm;
+  size_t acc_floats;
+  int n_done;
   RouteTmp rt;
-  int max_chunks;
   size_t total;
 };
 
-GemmLayout gemm_layout(const moe_ctx* c, int T) {
-  GemmLayout L{};
+Layout make_layout(const moe_ctx* c, int T, const Plan& p, bool mx) {
+  Layout L{};
   Carver cv;
   const size_t R = (size_t)T * c->k;
-  L.max_chunks = (int)(R / kGemmChunkRows) + c->E;
   L.topk_idx = cv.take(4 * R);
   L.topk_w = cv.take(4 * R);
   L.inv_perm = cv.take(4 * R);
   L.perm = cv.take(4 * R);
   L.row_w = cv.take(4 * R);
   L.offsets = cv.take(4 * (size_t)(c->E + 1));
-  L.sched = cv.take(16);
-  L.chunks = cv.take(16 * (size_t)L.max_chunks);
-  L.x_perm = cv.take(2 * R * c->H);
+  for (int f = 0; f < kFamilies; ++f)
+    if (p.has[f]) {
+      L.sched[f] = cv.take(16);
+      L.chunks[f] = cv.take(16 * (size_t)max_chunks(c, T, p, f));
+    }
+  if (p.has[kFamStream]) {
+    const int n = max_chunks(c, T, p, kFamStream);
+    // one completion counter per (chunk, column tile); the MXFP4 kernels' tiles are narrower
+    const int tile_cols = std::min(kStreamCols, kMxTileCols);
+    L.n_done = n * ((c->I + tile_cols - 1) / tile_cols);
+    L.done = cv.take(4 * (size_t)L.n_done);
+    L.acc_floats = (size_t)n * kStreamRB * 2 * c->I;  // split-K sums per chunk row
+    L.acc = cv.take(sizeof(float) * L.acc_floats);
+  }
   L.h = cv.take(2 * R * c->I);
+  if (mx) L.x16 = cv.take(2 * (size_t)T * c->H);  // the layer input in f16
+  if (p.has[kFamTile] || p.has[kFamGemm]) L.x_perm = cv.take(2 * R * c->H);
   L.rt = carve_route_tmp(cv, c, T);
   L.total = cv.cur;
   return L;
@@ -260,13 +311,6 @@ size_t route_ws_bytes(const moe_ctx* c, int T, bool allow_split = true) {
   cv.take(16);  // sched
   carve_route_tmp(cv, c, T, allow_split);
   return cv.cur;
-}
-
-// The path is chosen on the host from T alone, so no device data is read.
-bool use_stream(const moe_ctx* c, int T) {
-  if (c->path == MOE_PATH_STREAM) return true;
-  if (c->path == MOE_PATH_GEMM) return false;
-  return T <= c->crossover;
 }
 
 // ---- launches ------------------------------------------------------------------------
@@ -425,6 +469,10 @@ bool set_smem_attrs() {
   ok &= cudaFuncSetAttribute(grouped_gemm_2sm_kernel<MOE_GEMM_DOWN>,
                              cudaFuncAttributeMaxDynamicSharedMemorySize,
                              Gemm2Cfg<kGemmStages>::kSmem) == cudaSuccess;
+  ok &= cudaFuncSetAttribute(expert_tile_kernel<0>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             kEtSmem) == cudaSuccess;
+  ok &= cudaFuncSetAttribute(expert_tile_kernel<1>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             kEtSmem) == cudaSuccess;
   return ok;
 }
 
@@ -442,11 +490,16 @@ struct MxWeights {
   const void *gu_codes, *gu_scales, *dn_codes, *dn_scales;
 };
 
-moe_status forward_stream(moe_ctx* c, int T, const void* x_bf16, const void* W_router_bf16,
-                          const float* b_router, const void* W_gate_up_bf16,
-                          const void* W_down_bf16, float* out, uint8_t* ws, size_t ws_bytes,
-                          cudaStream_t st, const MxWeights* mx = nullptr) {
-  const StreamLayout L = stream_layout(c, T);
+// The layer for one plan: routing (with one work list per family that may receive rows), the
+// rows in expert order for the tcgen05 families, then gate/up + SwiGLU and down + combine by
+// every family in the plan.  All kernels go on one stream with programmatic serialisation;
+// each family's kernel finds its own work list (possibly empty) on the device.
+moe_status forward_plan(moe_ctx* c, int T, const void* x_bf16, const void* W_router_bf16,
+                        const float* b_router, const void* W_gate_up_bf16,
+                        const void* W_down_bf16, float* out, uint8_t* ws, size_t ws_bytes,
+                        cudaStream_t st, const MxWeights* mx = nullptr) {
+  const Plan p = make_plan(c, T, mx != nullptr, c->path);
+  const Layout L = make_layout(c, T, p, mx != nullptr);
   if (ws_bytes < L.total) return MOE_ERR_WORKSPACE;
   const size_t R = (size_t)T * c->k;
   RouteOut o{};
@@ -456,13 +509,24 @@ moe_status forward_stream(moe_ctx* c, int T, const void* x_bf16, const void* W_r
   o.perm = reinterpret_cast<int32_t*>(ws + L.perm);
   o.inv_perm = reinterpret_cast<int32_t*>(ws + L.inv_perm);
   o.row_w = reinterpret_cast<float*>(ws + L.row_w);
-  o.chunks = reinterpret_cast<int4*>(ws + L.chunks);
-  o.sched = reinterpret_cast<int32_t*>(ws + L.sched);
-  o.chunk_rows = kStreamRB;
-  o.zero_i32 = reinterpret_cast<int32_t*>(ws + L.done);
-  o.n_zero = L.n_done;
+  for (int f = 0; f < kFamilies; ++f)
+    if (p.has[f]) {
+      WorkList& wl = o.wl[o.n_lists];
+      wl.chunks = reinterpret_cast<int4*>(ws + L.chunks[f]);
+      wl.sched = reinterpret_cast<int32_t*>(ws + L.sched[f]);
+      wl.chunk_rows = kFamChunkRows[f];
+      wl.min_count = p.min_count(f);
+      wl.max_count = p.max_count[f];
+      ++o.n_lists;
+    }
+  auto chunks_of = [&](int f) { return reinterpret_cast<const int4*>(ws + L.chunks[f]); };
+  auto sched_of = [&](int f) { return reinterpret_cast<const int32_t*>(ws + L.sched[f]); };
+  o.zero_i32 = p.has[kFamStream] ? reinterpret_cast<int32_t*>(ws + L.done) : nullptr;
+  o.n_zero = p.has[kFamStream] ? L.n_done : 0;
   const uint16_t* x = static_cast<const uint16_t*>(x_bf16);
-  uint16_t* x16 = reinterpret_cast<uint16_t*>(ws + L.x16);
+  uint16_t* x16 = mx ? reinterpret_cast<uint16_t*>(ws + L.x16) : nullptr;
+  uint16_t* h = reinterpret_cast<uint16_t*>(ws + L.h);
+  uint16_t* x_perm = L.x_perm ? reinterpret_cast<uint16_t*>(ws + L.x_perm) : nullptr;
   if (mx) {  // the MXFP4 kernels take f16 activations
     const size_t n = (size_t)T * c->H;
     const int blocks = (int)std::min<size_t>((n / 8 + 255) / 256, (size_t)c->num_sms * 4);
@@ -470,22 +534,44 @@ moe_status forward_stream(moe_ctx* c, int T, const void* x_bf16, const void* W_r
       return launch_pdl(to_f16_kernel, dim3(blocks), dim3(256), 0, st, x, x16, n);
     }));
   }
-  moe_status s = launch_route(c, T, x, static_cast<const uint16_t*>(W_router_bf16), b_router, o,
-                              ws, L.rt, st, reinterpret_cast<float*>(ws + L.acc), R * 2 * c->I);
-  if (s == MOE_OK) {
+  // With enough 64-token blocks to cover the GPU the scatter also writes the rows in expert
+  // order (each token row read once); otherwise a wide gather kernel does it.
+  const int NB = (T + kRouterTcTokens - 1) / kRouterTcTokens;
+  const bool fused_copy = x_perm && T > kSmallT && NB >= c->num_sms;
+  if (fused_copy) {
+    o.x = x;
+    o.x_perm = x_perm;
+    o.H = c->H;
+  }
+  float* acc = p.has[kFamStream] ? reinterpret_cast<float*>(ws + L.acc) : nullptr;
+  MOE_TRY(launch_route(c, T, x, static_cast<const uint16_t*>(W_router_bf16), b_router, o, ws,
+                       L.rt, st, acc, L.acc_floats));
+  if (x_perm && !fused_copy)
+    MOE_TRY(launch(c, kKindGather, st, [&] {
+      return launch_pdl(gather_rows_kernel, dim3((unsigned)((R + 7) / 8)), dim3(256), 0, st, x,
+                        (const int32_t*)o.perm, (int)R, c->H, x_perm);
+    }));
+
+  // `out` is zero-filled once, by one gate/up kernel: the row-tile GEMM's epilogue warps while
+  // its tensor cores run, else the first other gate/up kernel before its dependency wait.
+  const int zero_owner = p.has[kFamGemm] ? kFamGemm : p.has[kFamStream] ? kFamStream : kFamTile;
+  const int pair_grid = c->num_sms & ~1;  // whole CTA pairs
+
+  // ---------------------------- gate/up projection + SwiGLU ----------------------------
+  if (p.has[kFamStream]) {
     GateUpArgs ga{};
     ga.x = mx ? x16 : x;
     ga.H = c->H;
     ga.I = c->I;
     ga.R = (int)R;
     ga.perm = o.perm;
-    ga.chunks = o.chunks;
-    ga.sched = o.sched;
-    ga.acc = reinterpret_cast<float*>(ws + L.acc);
+    ga.chunks = chunks_of(kFamStream);
+    ga.sched = sched_of(kFamStream);
+    ga.acc = acc;
     ga.done = o.zero_i32;
-    ga.h = reinterpret_cast<uint16_t*>(ws + L.h);
+    ga.h = h;
     ga.out = out;
-    ga.out_elems = (size_t)T * c->H;
+    ga.out_elems = zero_owner == kFamStream ? (size_t)T * c->H : 0;
     ga.status = c->d_status;
     if (mx) {
       const CUtensorMap* cm = cached_map_u8(c->gu_codes, mx->gu_codes, 2ull * c->I * c->E,
@@ -494,34 +580,85 @@ moe_status forward_stream(moe_ctx* c, int T, const void* x_bf16, const void* W_r
       const CUtensorMap* sm = cached_map_u8(c->gu_scales, mx->gu_scales,
                                             (uint64_t)c->E * (c->H / 32), 2ull * c->I,
                                             kMxKC / 32, kMxBoxRows, CU_TENSOR_MAP_SWIZZLE_NONE);
-      if (!cm || !sm) s = MOE_ERR_CUDA;
-      else
-        s = launch(c, kKindGateUp, st, [&] {
-          return launch_pdl(stream_gate_up_mx_kernel, dim3(c->num_sms), dim3(kMxThreads),
-                            kMxGateUpSmem, st, ga, *cm, *sm);
-        });
+      if (!cm || !sm) return MOE_ERR_CUDA;
+      MOE_TRY(launch(c, kKindGateUp, st, [&] {
+        return launch_pdl(stream_gate_up_mx_kernel, dim3(c->num_sms), dim3(kMxThreads),
+                          kMxGateUpSmem, st, ga, *cm, *sm);
+      }));
     } else {
       const CUtensorMap* m = cached_map(c->gate_up_stream, W_gate_up_bf16,
                                         (uint64_t)c->E * c->H, 2ull * c->I, kGateUpKC, kBox,
                                         /*promote_256=*/false);
-      if (!m) s = MOE_ERR_CUDA;
-      else
-        s = launch(c, kKindGateUp, st, [&] {
-          return launch_pdl(stream_gate_up_kernel, dim3(c->num_sms), dim3(kStreamThreads),
-                            kGateUpSmem, st, ga, *m);
-        });
+      if (!m) return MOE_ERR_CUDA;
+      MOE_TRY(launch(c, kKindGateUp, st, [&] {
+        return launch_pdl(stream_gate_up_kernel, dim3(c->num_sms), dim3(kStreamThreads),
+                          kGateUpSmem, st, ga, *m);
+      }));
     }
   }
-  if (s == MOE_OK) {
+  const CUtensorMap* wgu = nullptr;
+  const CUtensorMap* wdn = nullptr;
+  if (p.has[kFamTile] || p.has[kFamGemm]) {
+    wgu = cached_map(c->gate_up_gemm, W_gate_up_bf16, (uint64_t)c->E * c->H, 2ull * c->I,
+                     kGemmBK, 64);
+    wdn = cached_map(c->down_gemm, W_down_bf16, (uint64_t)c->E * c->I, (uint64_t)c->H,
+                     kGemmBK, 64);
+    if (!wgu || !wdn) return MOE_ERR_CUDA;
+  }
+  if (p.has[kFamTile]) {
+    const CUtensorMap* xm = cached_map(c->et_x_map, x_perm, R, (uint64_t)c->H, kEtRowBox, 64);
+    if (!xm) return MOE_ERR_CUDA;
+    EtArgs e{};
+    e.K = c->H;
+    e.Ncols = c->I;
+    e.w_rows = c->H;
+    e.chunks = chunks_of(kFamTile);
+    e.sched = sched_of(kFamTile);
+    e.h = h;
+    e.H = c->H;
+    e.status = c->d_status;
+    if (zero_owner == kFamTile) {
+      e.zero4 = reinterpret_cast<float4*>(out);
+      e.n_zero4 = (size_t)T * c->H / 4;
+    }
+    MOE_TRY(launch(c, kKindGateUpTile, st, [&] {
+      return launch_pdl(expert_tile_kernel<0>, dim3(c->num_sms), dim3(kEtThreads), kEtSmem, st,
+                        e, *wgu, *xm);
+    }));
+  }
+  if (p.has[kFamGemm]) {
+    const CUtensorMap* am = cached_map(c->x_perm_map, x_perm, R, (uint64_t)c->H, kGemmBM, 64);
+    if (!am) return MOE_ERR_CUDA;
+    GemmArgs g{};
+    g.K = c->H;
+    g.Ncols = c->I;
+    g.sub_stride = c->I;
+    g.w_rows = c->H;
+    g.chunks = chunks_of(kFamGemm);
+    g.sched = sched_of(kFamGemm);
+    g.h = h;
+    g.H = c->H;
+    g.status = c->d_status;
+    // the epilogue warps zero-fill `out`, which the down projections accumulate into
+    g.zero4 = reinterpret_cast<float4*>(out);
+    g.n_zero4 = (size_t)T * c->H / 4;
+    MOE_TRY(launch(c, kKindGateUpGemm, st, [&] {
+      return launch_pdl(grouped_gemm_2sm_kernel<MOE_GEMM_GATE_UP>, dim3(pair_grid),
+                        dim3(kGemmThreads), Gemm2Cfg<kGemmStages>::kSmem, st, g, *am, *wgu);
+    }));
+  }
+
+  // ---------------------------- down projection + weighted combine ----------------------------
+  if (p.has[kFamStream]) {
     DownArgs da{};
-    da.h = reinterpret_cast<const uint16_t*>(ws + L.h);
+    da.h = h;
     da.H = c->H;
     da.I = c->I;
     da.R = (int)R;
     da.perm = o.perm;
     da.row_w = o.row_w;
-    da.chunks = o.chunks;
-    da.sched = o.sched;
+    da.chunks = chunks_of(kFamStream);
+    da.sched = sched_of(kFamStream);
     da.out = out;
     da.status = c->d_status;
     if (mx) {
@@ -531,111 +668,65 @@ moe_status forward_stream(moe_ctx* c, int T, const void* x_bf16, const void* W_r
       const CUtensorMap* sm = cached_map_u8(c->dn_scales, mx->dn_scales,
                                             (uint64_t)c->E * (c->I / 32), (uint64_t)c->H,
                                             kMxKC / 32, kMxBoxRows, CU_TENSOR_MAP_SWIZZLE_NONE);
-      if (!cm || !sm) s = MOE_ERR_CUDA;
-      else
-        s = launch(c, kKindDown, st, [&] {
-          return launch_pdl(stream_down_mx_kernel, dim3(c->num_sms), dim3(kMxDnThreads),
-                            kMxDownSmem, st, da, *cm, *sm);
-        });
+      if (!cm || !sm) return MOE_ERR_CUDA;
+      MOE_TRY(launch(c, kKindDown, st, [&] {
+        return launch_pdl(stream_down_mx_kernel, dim3(c->num_sms), dim3(kMxDnThreads),
+                          kMxDownSmem, st, da, *cm, *sm);
+      }));
     } else {
       const CUtensorMap* m = cached_map(c->down_stream, W_down_bf16, (uint64_t)c->E * c->I,
                                         (uint64_t)c->H, kDownKC, kBox, /*promote_256=*/false);
-      if (!m) s = MOE_ERR_CUDA;
-      else
-        s = launch(c, kKindDown, st, [&] {
-          return launch_pdl(stream_down_kernel, dim3(c->num_sms), dim3(kStreamThreads),
-                            kDownSmem, st, da, *m);
-        });
+      if (!m) return MOE_ERR_CUDA;
+      MOE_TRY(launch(c, kKindDown, st, [&] {
+        return launch_pdl(stream_down_kernel, dim3(c->num_sms), dim3(kStreamThreads),
+                          kDownSmem, st, da, *m);
+      }));
     }
   }
-  return s;
-}
-
-moe_status forward_gemm(moe_ctx* c, int T, const void* x_bf16, const void* W_router_bf16,
-                        const float* b_router, const void* W_gate_up_bf16,
-                        const void* W_down_bf16, float* out, uint8_t* ws, size_t ws_bytes,
-                        cudaStream_t st) {
-  const GemmLayout L = gemm_layout(c, T);
-  if (ws_bytes < L.total) return MOE_ERR_WORKSPACE;
-  const size_t R = (size_t)T * c->k;
-  RouteOut o{};
-  o.topk_idx = reinterpret_cast<int32_t*>(ws + L.topk_idx);
-  o.topk_w = reinterpret_cast<float*>(ws + L.topk_w);
-  o.offsets = reinterpret_cast<int32_t*>(ws + L.offsets);
-  o.perm = reinterpret_cast<int32_t*>(ws + L.perm);
-  o.inv_perm = reinterpret_cast<int32_t*>(ws + L.inv_perm);
-  o.row_w = reinterpret_cast<float*>(ws + L.row_w);
-  o.chunks = reinterpret_cast<int4*>(ws + L.chunks);
-  o.sched = reinterpret_cast<int32_t*>(ws + L.sched);
-  o.chunk_rows = kGemmChunkRows;
-  o.zero_i32 = nullptr;
-  o.n_zero = 0;
-  const uint16_t* x = static_cast<const uint16_t*>(x_bf16);
-  uint16_t* x_perm = reinterpret_cast<uint16_t*>(ws + L.x_perm);
-  uint16_t* h = reinterpret_cast<uint16_t*>(ws + L.h);
-  // With enough 64-token blocks to cover the GPU the scatter also writes the rows in expert
-  // order (each token row read once); otherwise a wide gather kernel does it.
-  const int NB = (T + kRouterTcTokens - 1) / kRouterTcTokens;
-  const bool fused_copy = T > kSmallT && NB >= c->num_sms;
-  if (fused_copy) {
-    o.x = x;
-    o.x_perm = x_perm;
-    o.H = c->H;
-  }
-  MOE_TRY(launch_route(c, T, x, static_cast<const uint16_t*>(W_router_bf16), b_router, o, ws,
-                       L.rt, st));
-  if (!fused_copy)
-    MOE_TRY(launch(c, kKindGather, st, [&] {
-      return launch_pdl(gather_rows_kernel, dim3((unsigned)((R + 7) / 8)), dim3(256), 0, st, x,
-                        (const int32_t*)o.perm, (int)R, c->H, x_perm);
+  if (p.has[kFamTile]) {
+    const CUtensorMap* hm = cached_map(c->et_h_map, h, R, (uint64_t)c->I, kEtRowBox, 64);
+    if (!hm) return MOE_ERR_CUDA;
+    EtArgs e{};
+    e.K = c->I;
+    e.Ncols = c->H;
+    e.w_rows = c->I;
+    e.chunks = chunks_of(kFamTile);
+    e.sched = sched_of(kFamTile);
+    e.perm = o.perm;
+    e.row_w = o.row_w;
+    e.out = out;
+    e.H = c->H;
+    e.status = c->d_status;
+    MOE_TRY(launch(c, kKindDownTile, st, [&] {
+      return launch_pdl(expert_tile_kernel<1>, dim3(c->num_sms), dim3(kEtThreads), kEtSmem, st,
+                        e, *wdn, *hm);
     }));
-  const CUtensorMap* am = cached_map(c->x_perm_map, x_perm, R, (uint64_t)c->H, kGemmBM, 64);
-  const CUtensorMap* bm = cached_map(c->gate_up_gemm, W_gate_up_bf16, (uint64_t)c->E * c->H,
-                                     2ull * c->I, kGemmBK, 64);
-  if (!am || !bm) return MOE_ERR_CUDA;
-  GemmArgs g{};
-  g.K = c->H;
-  g.Ncols = c->I;
-  g.sub_stride = c->I;
-  g.w_rows = c->H;
-  g.chunks = o.chunks;
-  g.sched = o.sched;
-  g.h = h;
-  g.H = c->H;
-  g.status = c->d_status;
-  // the gate/up epilogue zero-fills `out`, which the down projection accumulates into
-  g.zero4 = reinterpret_cast<float4*>(out);
-  g.n_zero4 = (size_t)T * c->H / 4;
-  const int grid = c->num_sms & ~1;  // whole CTA pairs
-  MOE_TRY(launch(c, kKindGateUp, st, [&] {
-    return launch_pdl(grouped_gemm_2sm_kernel<MOE_GEMM_GATE_UP>, dim3(grid), dim3(kGemmThreads),
-                      Gemm2Cfg<kGemmStages>::kSmem, st, g, *am, *bm);
-  }));
-  const CUtensorMap* hm = cached_map(c->h_map, h, R, (uint64_t)c->I, kGemmBM, 64);
-  const CUtensorMap* dm = cached_map(c->down_gemm, W_down_bf16, (uint64_t)c->E * c->I,
-                                     (uint64_t)c->H, kGemmBK, 64);
-  if (!hm || !dm) return MOE_ERR_CUDA;
-  GemmArgs d{};
-  d.K = c->I;
-  d.Ncols = c->H;
-  d.sub_stride = 0;
-  d.w_rows = c->I;
-  d.chunks = o.chunks;
-  d.sched = o.sched;
-  d.perm = o.perm;
-  d.row_w = o.row_w;
-  d.out = out;
-  d.H = c->H;
-  d.status = c->d_status;
-  MOE_TRY(launch(c, kKindDown, st, [&] {
-    return launch_pdl(grouped_gemm_2sm_kernel<MOE_GEMM_DOWN>, dim3(grid), dim3(kGemmThreads),
-                      Gemm2Cfg<kGemmStages>::kSmem, st, d, *hm, *dm);
-  }));
+  }
+  if (p.has[kFamGemm]) {
+    const CUtensorMap* hm = cached_map(c->h_map, h, R, (uint64_t)c->I, kGemmBM, 64);
+    if (!hm) return MOE_ERR_CUDA;
+    GemmArgs d{};
+    d.K = c->I;
+    d.Ncols = c->H;
+    d.sub_stride = 0;
+    d.w_rows = c->I;
+    d.chunks = chunks_of(kFamGemm);
+    d.sched = sched_of(kFamGemm);
+    d.perm = o.perm;
+    d.row_w = o.row_w;
+    d.out = out;
+    d.H = c->H;
+    d.status = c->d_status;
+    MOE_TRY(launch(c, kKindDownGemm, st, [&] {
+      return launch_pdl(grouped_gemm_2sm_kernel<MOE_GEMM_DOWN>, dim3(pair_grid),
+                        dim3(kGemmThreads), Gemm2Cfg<kGemmStages>::kSmem, st, d, *hm, *wdn);
+    }));
+  }
   return MOE_OK;
 }
 
-size_t forward_ws_bytes(const moe_ctx* c, int T) {
-  return use_stream(c, T) ? stream_layout(c, T).total : gemm_layout(c, T).total;
+size_t forward_ws_bytes(const moe_ctx* c, int T, bool mx, moe_path path) {
+  return make_layout(c, T, make_plan(c, T, mx, path), mx).total;
 }
 
 __global__ void selftest_timeout_kernel(uint32_t* status, uint64_t limit_ns) {
@@ -714,7 +805,7 @@ size_t moe_route_workspace_bytes(moe_t c, int T) {
 size_t moe_workspace_bytes(moe_t c, int T) {
   if (!c || T < 0 || T > kMaxT) return 0;
   if (T == 0) return 0;
-  return forward_ws_bytes(c, T);
+  return forward_ws_bytes(c, T, false, c->path);
 }
 
 moe_status moe_route(moe_t c, int T, const void* x_bf16, const void* W_router_bf16,
@@ -736,7 +827,7 @@ moe_status moe_route(moe_t c, int T, const void* x_bf16, const void* W_router_bf
   if (!workspace || !aligned16(workspace) || ws_bytes < need) return MOE_ERR_WORKSPACE;
   uint8_t* ws = static_cast<uint8_t*>(workspace);
   Carver cv;
-  const size_t sched_at = cv.take(16);
+  cv.take(16);  // the work-list word of the forward layouts (kept: same scratch size)
   const RouteTmp rt = carve_route_tmp(cv, c, T);
   RouteOut o{};
   o.topk_idx = topk_idx;
@@ -745,9 +836,7 @@ moe_status moe_route(moe_t c, int T, const void* x_bf16, const void* W_router_bf
   o.perm = perm;
   o.inv_perm = inv_perm;
   o.row_w = nullptr;
-  o.chunks = nullptr;
-  o.sched = reinterpret_cast<int32_t*>(ws + sched_at);
-  o.chunk_rows = 1;
+  o.n_lists = 0;  // routing only: no work lists
   o.zero_i32 = nullptr;
   o.n_zero = 0;
   return launch_route(c, T, static_cast<const uint16_t*>(x_bf16),
@@ -767,12 +856,8 @@ moe_status moe_forward(moe_t c, int T, const void* x_bf16, const void* W_router_
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   uint8_t* ws = static_cast<uint8_t*>(workspace);
   c->in_call = c->prof_max > 0 && c->prof_calls < c->prof_max;
-  const moe_status s =
-      use_stream(c, T)
-          ? forward_stream(c, T, x_bf16, W_router_bf16, b_router, W_gate_up_bf16, W_down_bf16,
-                           out, ws, ws_bytes, st)
-          : forward_gemm(c, T, x_bf16, W_router_bf16, b_router, W_gate_up_bf16, W_down_bf16,
-                         out, ws, ws_bytes, st);
+  const moe_status s = forward_plan(c, T, x_bf16, W_router_bf16, b_router, W_gate_up_bf16,
+                                    W_down_bf16, out, ws, ws_bytes, st);
   if (c->in_call) ++c->prof_calls;
   c->in_call = false;
   return s;
@@ -781,7 +866,7 @@ moe_status moe_forward(moe_t c, int T, const void* x_bf16, const void* W_router_
 size_t moe_workspace_bytes_mxfp4(moe_t c, int T) {
   if (!c || T < 0 || T > kMaxT || (long long)T * c->k >= (1ll << 31)) return 0;
   if (T == 0) return 0;
-  return stream_layout(c, T).total;
+  return forward_ws_bytes(c, T, /*mx=*/true, c->path);
 }
 
 moe_status moe_forward_mxfp4(moe_t c, int T, const void* x_bf16, const void* W_router_bf16,
@@ -797,7 +882,7 @@ moe_status moe_forward_mxfp4(moe_t c, int T, const void* x_bf16, const void* W_r
   if (!workspace || !aligned16(workspace)) return MOE_ERR_WORKSPACE;
   const MxWeights mx{gu_codes, gu_scales, dn_codes, dn_scales};
   c->in_call = c->prof_max > 0 && c->prof_calls < c->prof_max;
-  const moe_status s = forward_stream(c, T, x_bf16, W_router_bf16, b_router, nullptr, nullptr,
+  const moe_status s = forward_plan(c, T, x_bf16, W_router_bf16, b_router, nullptr, nullptr,
                                       out, static_cast<uint8_t*>(workspace), ws_bytes,
                                       reinterpret_cast<cudaStream_t>(stream), &mx);
   if (c->in_call) ++c->prof_calls;
@@ -805,25 +890,43 @@ moe_status moe_forward_mxfp4(moe_t c, int T, const void* x_bf16, const void* W_r
   return s;
 }
 
-moe_status moe_set_path(moe_t c, moe_path path, int crossover_T) {
+moe_status moe_set_path(moe_t c, moe_path path, int stream_rows) {
   if (!c) return MOE_ERR_ARG;
-  if (path != MOE_PATH_AUTO && path != MOE_PATH_STREAM && path != MOE_PATH_GEMM)
+  if (path != MOE_PATH_AUTO && path != MOE_PATH_STREAM && path != MOE_PATH_GEMM &&
+      path != MOE_PATH_TILE)
     return MOE_ERR_ARG;
   c->path = path;
-  if (crossover_T >= 0) c->crossover = crossover_T;
+  if (stream_rows >= 0) c->stream_rows = stream_rows;
   return MOE_OK;
 }
 
-moe_status moe_get_path(moe_t c, moe_path* path, int* crossover_T) {
+moe_status moe_get_path(moe_t c, moe_path* path, int* stream_rows) {
   if (!c) return MOE_ERR_ARG;
   if (path) *path = c->path;
-  if (crossover_T) *crossover_T = c->crossover;
+  if (stream_rows) *stream_rows = c->stream_rows;
+  return MOE_OK;
+}
+
+moe_status moe_set_dispatch(moe_t c, int stream_rows, int tile_rows) {
+  if (!c) return MOE_ERR_ARG;
+  if (stream_rows >= 0) c->stream_rows = stream_rows;
+  if (tile_rows >= 0) c->tile_rows = tile_rows;
+  return MOE_OK;
+}
+
+moe_status moe_get_dispatch(moe_t c, int* stream_rows, int* tile_rows) {
+  if (!c) return MOE_ERR_ARG;
+  if (stream_rows) *stream_rows = c->stream_rows;
+  if (tile_rows) *tile_rows = c->tile_rows;
   return MOE_OK;
 }
 
 size_t moe_tune_workspace_bytes(moe_t c, int T_max) {
   if (!c || T_max < 1 || T_max > kMaxT) return 0;
-  return std::max(stream_layout(c, T_max).total, gemm_layout(c, T_max).total);
+  size_t need = 0;
+  for (moe_path p : {MOE_PATH_STREAM, MOE_PATH_TILE, MOE_PATH_GEMM, MOE_PATH_AUTO})
+    need = std::max(need, forward_ws_bytes(c, T_max, false, p));
+  return need;
 }
 
 moe_status moe_tune(moe_t c, int T_max, const void* x_bf16, const void* W_router_bf16,
@@ -863,26 +966,42 @@ moe_status moe_tune(moe_t c, int T_max, const void* x_bf16, const void* W_router
     *ms_out = v[2];
     return MOE_OK;
   };
+  // Largest T at which family `lo` is not slower than family `hi` over the whole layer (0 if
+  // never); stops once `hi` has been faster for a doubling of T.
   static const int kCandidates[] = {1, 2, 4, 8, 12, 16, 24, 32, 48, 64, 96, 128, 192, 256, 384,
-                                    512, 768, 1024};
-  int crossover = 0;
-  moe_status s = MOE_OK;
-  for (int T : kCandidates) {
-    if (T > T_max) break;
-    float ts = 0.f, tg = 0.f;
-    s = time_path(MOE_PATH_STREAM, T, &ts);
-    if (s == MOE_OK) s = time_path(MOE_PATH_GEMM, T, &tg);
-    if (s != MOE_OK) break;
-    if (ts <= tg) crossover = T;
-    else if (T >= 2 * std::max(crossover, 1)) break;  // the grouped GEMM has taken over
-  }
+                                    512, 768, 1024, 1536, 2048, 3072, 4096};
+  auto crossover_T = [&](moe_path lo, moe_path hi, int* T_out) -> moe_status {
+    int cross = 0;
+    for (int T : kCandidates) {
+      if (T > T_max) break;
+      float tl = 0.f, th = 0.f;
+      MOE_TRY(time_path(lo, T, &tl));
+      MOE_TRY(time_path(hi, T, &th));
+      if (tl <= th) cross = T;
+      else if (T >= 2 * std::max(cross, 1)) break;
+    }
+    *T_out = cross;
+    return MOE_OK;
+  };
+  // A family boundary measured at T tokens becomes a per-expert row count: the mean rows per
+  // expert at that T (uniform routing: T*k/E), at least the token count itself when E <= k.
+  auto rows_at = [&](int T) {
+    return T == 0 ? 0 : std::max(1, (int)(((long long)T * c->k + c->E - 1) / c->E));
+  };
+  int Ts = 0, Tt = 0;
+  moe_status s = crossover_T(MOE_PATH_STREAM, MOE_PATH_TILE, &Ts);
+  if (s == MOE_OK) s = crossover_T(MOE_PATH_TILE, MOE_PATH_GEMM, &Tt);
   cudaEventDestroy(e0);
   cudaEventDestroy(e1);
   c->path = saved_path;
   c->prof_max = saved_prof;
   if (s != MOE_OK) return s;
-  c->crossover = crossover;
-  if (crossover_out) *crossover_out = crossover;
+  c->stream_rows = rows_at(Ts);
+  // the tile family ends where the row-tile GEMM wins; never below the streaming threshold,
+  // and where T_max never let the GEMM win the measured band is kept
+  c->tile_rows = std::max(c->stream_rows, Tt >= T_max ? std::max(c->tile_rows, rows_at(Tt))
+                                                       : rows_at(Tt));
+  if (crossover_out) *crossover_out = c->stream_rows;
   return MOE_OK;
 }
 
@@ -962,8 +1081,9 @@ moe_status moe_profile_end(moe_t c, float* ms, int* launches, int n_kinds) {
 }
 
 const char* moe_profile_kind_name(int kind) {
-  static const char* names[MOE_PROFILE_KINDS] = {"router", "route_finalize", "gather",
-                                                 "gate_up_swiglu", "down_combine", "to_f16"};
+  static const char* names[MOE_PROFILE_KINDS] = {
+      "router",       "route_finalize", "gather",  "gate_up_stream", "down_stream",
+      "to_f16",       "gate_up_tile",   "down_tile", "gate_up_gemm", "down_gemm"};
   if (kind < 0 || kind >= MOE_PROFILE_KINDS) return "unknown";
   return names[kind];
 }
@@ -1042,7 +1162,7 @@ moe_status moe_route_static(moe_t c, int T, const void* x_bf16, const void* W_ro
   if (!c->static_scratch) return MOE_ERR_CUDA;
   uint8_t* ws = static_cast<uint8_t*>(c->static_scratch);
   Carver cv;
-  const size_t sched_at = cv.take(16);
+  cv.take(16);  // the work-list word of the forward layouts (kept: same scratch size)
   const RouteTmp rt = carve_route_tmp(cv, c, T, /*allow_split=*/false);
   RouteOut o{};
   o.topk_idx = topk_idx;
@@ -1051,9 +1171,7 @@ moe_status moe_route_static(moe_t c, int T, const void* x_bf16, const void* W_ro
   o.perm = perm;
   o.inv_perm = inv_perm;
   o.row_w = nullptr;
-  o.chunks = nullptr;
-  o.sched = reinterpret_cast<int32_t*>(ws + sched_at);
-  o.chunk_rows = 1;
+  o.n_lists = 0;  // routing only: no work lists
   o.zero_i32 = nullptr;
   o.n_zero = 0;
   // Every scratch word the routing kernels read is written earlier in the same call (the

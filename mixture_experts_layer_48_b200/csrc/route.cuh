@@ -23,6 +23,18 @@ constexpr int kSmallT = 64;        // largest T handled by the single-block fina
 constexpr int kRouteTile = 32;     // tokens per block in the large-T chain
 constexpr int kRouterHSlice = 64;  // W_router rows per block in router_partial_kernel
 
+// One work list: the row segments of the experts whose row count lies in (min_count,
+// max_count], cut into chunks of at most chunk_rows rows.  Each expert kernel family walks
+// its own list, so the kernel that multiplies an expert's rows is chosen per expert on the
+// device, from the histogram.
+struct WorkList {
+  int4* chunks;        // {expert, first row, rows, 0}
+  int32_t* sched;      // [0] number of chunks
+  int chunk_rows;
+  int min_count, max_count;
+};
+constexpr int kMaxWorkLists = 3;
+
 // Outputs of routing, all in device memory.
 struct RouteOut {
   int32_t* topk_idx;   // [T, k]
@@ -31,9 +43,8 @@ struct RouteOut {
   int32_t* perm;       // [T * k]
   int32_t* inv_perm;   // [T, k]
   float* row_w;        // [T * k] routing weight of each row (may be null)
-  int4* chunks;        // work list: {expert, first row, rows, 0}; null = none
-  int32_t* sched;      // [0] number of chunks, [1] number of experts with rows
-  int chunk_rows;      // rows per work-list entry
+  WorkList wl[kMaxWorkLists];
+  int n_lists;         // work lists to build (0: routing only)
   int32_t* zero_i32;   // region zeroed by the chain (completion counters), may be null
   int n_zero;
   const uint16_t* x;   // with x_perm non-null: copy token rows into expert order
@@ -247,33 +258,40 @@ __global__ void __launch_bounds__(256) router_partial_kernel(const uint16_t* __r
   }
 }
 
-// Work list of one routing: expert e's rows split into entries of at most chunk_rows rows.
-// Called by all threads of a block with count/off in shared memory (E <= 256 entries).
-MOE_DEVINL void build_work_list(const int32_t* cnt, const int32_t* off, int E,
-                                const RouteOut& o, int32_t* scratch /* [256 + 1] smem */) {
+// Work lists of one routing: expert e (with count c > 0) belongs to the list whose
+// (min_count, max_count] holds c, and its rows are split there into entries of at most
+// chunk_rows rows, in expert order.  Called by all threads of a block with count/off in
+// shared memory (E <= 256 entries); scratch holds [256] ints of shared memory.
+MOE_DEVINL void build_work_lists(const int32_t* cnt, const int32_t* off, int E,
+                                 const RouteOut& o, int32_t* scratch) {
   const int tid = threadIdx.x;
-  if (o.chunks == nullptr) return;
-  // chunk counts per expert, exclusive scan by thread 0 (E <= 256)
-  for (int e = tid; e < E; e += blockDim.x)
-    scratch[e] = (cnt[e] + o.chunk_rows - 1) / o.chunk_rows;
-  __syncthreads();
-  if (tid == 0) {
-    int run = 0, active = 0;
+  if (o.n_lists == 0) return;
+  // thread i < n_lists: exclusive scan of list i's chunk counts, in expert order
+  if (tid < o.n_lists) {
+    const WorkList& L = o.wl[tid];
+    int run = 0;
     for (int e = 0; e < E; ++e) {
-      const int c = scratch[e];
-      scratch[e] = run;
-      run += c;
-      active += cnt[e] > 0;
+      const int c = cnt[e];
+      if (c > L.min_count && c <= L.max_count) {
+        scratch[e] = run;
+        run += (c + L.chunk_rows - 1) / L.chunk_rows;
+      }
     }
-    scratch[256] = run;
-    o.sched[0] = run;
-    o.sched[1] = active;
+    L.sched[0] = run;
   }
   __syncthreads();
   for (int e = tid; e < E; e += blockDim.x) {
-    int base = scratch[e];
-    for (int r0 = 0; r0 < cnt[e]; r0 += o.chunk_rows)
-      o.chunks[base++] = make_int4(e, off[e] + r0, min(o.chunk_rows, cnt[e] - r0), 0);
+    const int c = cnt[e];
+    if (c == 0) continue;
+    for (int i = 0; i < o.n_lists; ++i) {
+      const WorkList& L = o.wl[i];
+      if (c > L.min_count && c <= L.max_count) {
+        int base = scratch[e];
+        for (int r0 = 0; r0 < c; r0 += L.chunk_rows)
+          L.chunks[base++] = make_int4(e, off[e] + r0, min(L.chunk_rows, c - r0), 0);
+        break;
+      }
+    }
   }
 }
 
@@ -362,7 +380,7 @@ __global__ void __launch_bounds__(1024)
     if (o.row_w) o.row_w[r] = lg[t * E + (i - t * k)];
   }
   __syncthreads();
-  build_work_list(cnt, off, E, o, scratch);
+  build_work_lists(cnt, off, E, o, scratch);
   for (int i = tid; i < o.n_zero; i += blockDim.x) o.zero_i32[i] = 0;
 }
 
@@ -688,7 +706,7 @@ __global__ void __launch_bounds__(256)
       before += __popc(mask);
     }
   }
-  if (blockIdx.x == 0) build_work_list(cnt, off, E, o, scratch);
+  if (blockIdx.x == 0) build_work_lists(cnt, off, E, o, scratch);
   for (int i = blockIdx.x * blockDim.x + tid; i < o.n_zero; i += gridDim.x * blockDim.x)
     o.zero_i32[i] = 0;
   if (o.x_perm) {

@@ -29,7 +29,8 @@ def test_header_declares_the_boundary():
     syms = declared_symbols()
     for name in ("moe_create", "moe_destroy", "moe_route", "moe_forward", "moe_set_path",
                  "moe_workspace_bytes", "moe_sync_status", "moe_status_string", "moe_tune",
-                 "moe_forward_mxfp4", "moe_workspace_bytes_mxfp4", "moe_route_static"):
+                 "moe_forward_mxfp4", "moe_workspace_bytes_mxfp4", "moe_route_static",
+                 "moe_set_dispatch", "moe_get_dispatch"):
         assert name in syms
 
 
@@ -50,8 +51,8 @@ def test_status_strings(lib):
         assert lib.moe_status_string(s).decode() not in ("", "unknown status")
     assert lib.moe_status_string(99).decode() == "unknown status"
     names = [lib.moe_profile_kind_name(i).decode() for i in range(lib.MOE_PROFILE_KINDS)]
-    assert names == ["router", "route_finalize", "gather", "gate_up_swiglu", "down_combine",
-                     "to_f16"]
+    assert names == ["router", "route_finalize", "gather", "gate_up_stream", "down_stream",
+                     "to_f16", "gate_up_tile", "down_tile", "gate_up_gemm", "down_gemm"]
     assert lib.moe_profile_kind_name(-1).decode() == "unknown"
     assert lib.moe_profile_kind_name(lib.MOE_PROFILE_KINDS).decode() == "unknown"
 
@@ -87,6 +88,8 @@ def test_null_handle_calls(lib):
     assert lib.moe_forward(None, 1, None, None, None, None, None, None, None, 0, None) == lib.MOE_ERR_ARG
     assert lib.moe_route(None, 1, None, None, None, None, None, None, None, None, None, 0, None) == lib.MOE_ERR_ARG
     assert lib.moe_set_path(None, 0, -1) == lib.MOE_ERR_ARG
+    assert lib.moe_set_dispatch(None, 16, 256) == lib.MOE_ERR_ARG
+    assert lib.moe_get_dispatch(None, None, None) == lib.MOE_ERR_ARG
     assert lib.moe_sync_status(None, None) == lib.MOE_ERR_ARG
     assert lib.moe_profile_begin(None, 4) == lib.MOE_ERR_ARG
     assert lib.moe_selftest_timeout(None, 10, None) == lib.MOE_ERR_ARG

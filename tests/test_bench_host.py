@@ -123,3 +123,39 @@ def test_default_workload_is_the_largest_single_gpu_config():
     w = mi.WORKLOADS["131k_skewed"]
     assert "131k_skewed" in ap_default
     assert w.T == max(x.T for x in mi.WORKLOADS.values())
+
+
+def test_peak_labels_for_measured_and_fallback_peaks():
+    assert bench.peak_label("measured", "hbm_gbs") == "measured hbm_gbs (MEASURED_PEAKS.json)"
+    assert bench.peak_label("fallback", "bf16_tflops (burst)").startswith("fallback bf16_tflops")
+    hbm, bf16, sus, src = bench.measured_peaks()
+    assert src in ("measured", "fallback") and hbm > 0 and bf16 > sus > 0
+
+
+def test_family_split_follows_the_dispatch_thresholds():
+    f = bench.split_families([0, 3, 16, 17, 256, 257, 900], "auto", 16, 256)
+    assert f == {"stream": [3, 16], "tile": [17, 256], "gemm": [257, 900]}
+    assert bench.split_families([5, 40], "gemm", 16, 256) == {"stream": [], "tile": [], "gemm": [5, 40]}
+    # tile band empty when tile_rows <= stream_rows
+    assert bench.split_families([5, 40], "auto", 16, 8) == {"stream": [5], "tile": [], "gemm": [40]}
+
+
+def test_family_work_and_dominant_roofline():
+    w = bench.family_work([64, 64], 2880, 2880)
+    assert w["experts"] == 2 and w["rows"] == 128
+    assert w["gate_up_bytes"] == 2 * 2880 * 5760 * 2 + 128 * 2880 * 2 + 128 * 2880 * 2
+    assert w["gate_up_flops"] == 2 * 128 * 2880 * 5760
+    work = {"stream": bench.family_work([2] * 24, 2880, 2880), "tile": w,
+            "gemm": bench.family_work([4096] * 32, 2880, 2880)}
+    # the tile kernel dominates and is bandwidth-bound at 64 rows per expert
+    r = bench.dominant_roofline(work, {"stream": 0.05, "tile": 0.02, "gemm": 0.0}, 6548.8,
+                                1661.1, 1383.9, "measured")
+    assert r["family"] == "stream" and r["bound"] == "hbm"
+    r = bench.dominant_roofline(work, {"stream": 0.0, "tile": 0.02, "gemm": 0.0}, 6548.8,
+                                1661.1, 1383.9, "fallback")
+    assert r["bound"] == "hbm" and r["achieved"] == pytest.approx(w["gate_up_bytes"] / 2e-5 / 1e9)
+    assert r["kernel"] == "expert_tile_kernel<0>" and r["frac"] == pytest.approx(r["achieved"] / 6548.8)
+    r = bench.dominant_roofline(work, {"stream": 0.01, "tile": 0.02, "gemm": 12.0}, 6548.8,
+                                1661.1, 1383.9, "measured")
+    assert r["family"] == "gemm" and r["bound"] == "tensor" and r["unit"] == "TFLOP/s"
+    assert r["achieved"] == pytest.approx(2 * 4096 * 32 * 2880 * 5760 / 12e-3 / 1e12)

@@ -32,6 +32,13 @@ def _check_layer(d, h, E, H, I, k, layer=None, path=None):
     return layer, g
 
 
+_PATHS = {"stream": "MOE_PATH_STREAM", "gemm": "MOE_PATH_GEMM", "tile": "MOE_PATH_TILE"}
+
+
+def _path(name):
+    return getattr(moe, _PATHS[name])
+
+
 @pytest.mark.parametrize("T", [1, 2, 3, 15, 16, 17, 31, 33, 63, 64, 65, 96, 127, 129, 300])
 def test_ragged_token_counts(T):
     d, h = inputs_on_gpu(T, 256, 8, 2, 320, seed=100 + T)
@@ -142,42 +149,46 @@ def test_profile_counts_kernels():
         layer.forward(d["x"], d["W_router"], d["b_router"], d["W_gate_up"], d["W_down"])
     prof = layer.profile_end()
     assert layer.launch_count() - n0 == sum(v[1] for v in prof.values())
-    assert prof["gate_up_swiglu"][1] == 3 and prof["down_combine"][1] == 3
+    assert prof["gate_up_stream"][1] == 3 and prof["down_stream"][1] == 3
     assert all(v[0] >= 0 for v in prof.values())
 
 
 @pytest.mark.parametrize("T", [1, 5, 16, 64, 65, 200, 520])
-@pytest.mark.parametrize("path", ["stream", "gemm"])
-def test_both_paths_match_the_oracle(T, path):
-    """Either path at any T: the streaming kernels and the tcgen05 grouped GEMM."""
-    p = moe.MOE_PATH_STREAM if path == "stream" else moe.MOE_PATH_GEMM
+@pytest.mark.parametrize("path", ["stream", "gemm", "tile"])
+def test_every_path_matches_the_oracle(T, path):
+    """Each kernel family for every expert at any T: the streaming kernels, the 2-SM row-tile
+    grouped GEMM and the expert-tile kernels."""
     d, h = inputs_on_gpu(T, 256, 8, 2, 320, seed=1000 + T)
-    _check_layer(d, h, 8, 256, 320, 2, path=p)
+    _check_layer(d, h, 8, 256, 320, 2, path=_path(path))
 
 
-@pytest.mark.parametrize("path", ["stream", "gemm"])
-def test_both_paths_gpt_oss_shape(path):
-    p = moe.MOE_PATH_STREAM if path == "stream" else moe.MOE_PATH_GEMM
+@pytest.mark.parametrize("path", ["stream", "gemm", "tile"])
+def test_every_path_gpt_oss_shape(path):
     d, h = inputs_on_gpu(300, 2880, 32, 4, 2880, seed=1100)
-    _check_layer(d, h, 32, 2880, 2880, 4, path=p)
+    _check_layer(d, h, 32, 2880, 2880, 4, path=_path(path))
 
 
-def test_tune_measures_a_crossover_and_auto_follows_it():
+def test_tune_measures_the_dispatch_thresholds_and_auto_follows_them():
     E, H, I, k = 32, 2880, 2880, 4
-    d, _ = inputs_on_gpu(256, H, E, k, I, seed=1200)
+    d, h = inputs_on_gpu(1024, H, E, k, I, seed=1200)
     layer = moe.Moe(E, H, I, k)
     c = layer.tune(d["x"], d["W_router"], d["b_router"], d["W_gate_up"], d["W_down"])
-    path, cross = layer.get_path()
-    assert path == moe.MOE_PATH_AUTO and cross == c
-    assert 0 <= c <= 256
-    print("measured crossover T* =", c)
+    path, stream_rows = layer.get_path()
+    s, t = layer.get_dispatch()
+    assert path == moe.MOE_PATH_AUTO and stream_rows == c == s
+    assert 0 <= s <= t
+    print("measured dispatch thresholds: stream_rows", s, "tile_rows", t)
     assert layer.sync_status() == moe.MOE_OK
+    # the layer with the measured thresholds still matches the oracle
+    d2 = dict(d, x=d["x"][:300].contiguous())
+    h2 = dict(h, x=h["x"][:300])
+    _check_layer(d2, h2, E, H, I, k, layer=layer)
 
 
-@pytest.mark.parametrize("T,path", [(10, "stream"), (100, "gemm")])
+@pytest.mark.parametrize("T,path", [(10, "stream"), (100, "gemm"), (100, "tile"), (300, "auto")])
 def test_forward_with_k_equal_E_256(T, path):
     """Every token uses all 256 experts (the widest routing the ABI accepts)."""
-    p = moe.MOE_PATH_STREAM if path == "stream" else moe.MOE_PATH_GEMM
+    p = moe.MOE_PATH_AUTO if path == "auto" else _path(path)
     d, h = inputs_on_gpu(T, 64, 256, 256, 64, seed=1300 + T)
     _check_layer(d, h, 256, 64, 64, 256, path=p)
 
@@ -200,9 +211,8 @@ def test_largest_token_count():
     check_outputs(got, tokens, h, ref_route, g, ref)
 
 
-@pytest.mark.parametrize("path", ["stream", "gemm"])
+@pytest.mark.parametrize("path", ["stream", "gemm", "tile"])
 def test_wide_hidden_and_intermediate(path):
-    """H = I = 8192: long K loops and many column tiles in both paths."""
-    p = moe.MOE_PATH_STREAM if path == "stream" else moe.MOE_PATH_GEMM
+    """H = I = 8192: long K loops and many column tiles in every path."""
     d, h = inputs_on_gpu(24, 8192, 2, 1, 8192, seed=1500)
-    _check_layer(d, h, 2, 8192, 8192, 1, path=p)
+    _check_layer(d, h, 2, 8192, 8192, 1, path=_path(path))

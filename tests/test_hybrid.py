@@ -1,0 +1,90 @@
+"""Per-expert dispatch: in one call, each expert's rows go to the weight-streaming kernels, the
+expert-tile kernels or the row-tile grouped GEMM according to its row count (decided on the
+device).  The mid-token regime with skewed routing is where this matters: a few experts see
+hundreds of rows, many see tens, some a handful (hearth-lean-loomed-v1 card, "Why 12-16
+streams can be slow on Vulkan").  Every case is checked against the fp64 oracle on all tokens.
+"""
+import json
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from parity_util import check_outputs, compare_routing, gpu_route, host_route, inputs_on_gpu
+
+pytestmark = pytest.mark.gpu
+
+if torch.cuda.is_available():
+    import mixture_experts_layer_48_b200 as moe
+
+
+def _families(counts, stream_rows, tile_rows):
+    c = np.asarray(counts)
+    return (int(((c > 0) & (c <= stream_rows)).sum()),
+            int(((c > stream_rows) & (c <= tile_rows)).sum()), int((c > tile_rows).sum()))
+
+
+def _run(T, E, H, I, k, seed, zipf=False, path=None, dispatch=None):
+    d, h = inputs_on_gpu(T, H, E, k, I, seed, zipf=zipf)
+    layer = moe.Moe(E, H, I, k)
+    if path is not None:
+        layer.set_path(path)
+    if dispatch is not None:
+        layer.set_dispatch(*dispatch)
+    ref_route = host_route(h, k)
+    g = gpu_route(layer, d)
+    rep = compare_routing(g, ref_route, k, E)
+    out = layer.forward(d["x"], d["W_router"], d["b_router"], d["W_gate_up"], d["W_down"])
+    assert layer.sync_status() == moe.MOE_OK
+    ref = oracle.moe_forward_ref(h["x"], h["W_router"], h["b_router"], h["W_gate_up"],
+                                 h["W_down"], k, route=ref_route)
+    rep.update(check_outputs(out.double().cpu().numpy(), np.arange(T), h, ref_route, g, ref))
+    return layer, g, rep
+
+
+@pytest.mark.parametrize("T,dispatch", [(1024, None), (512, (16, 128)), (256, (8, 40))])
+def test_skewed_mid_T_mixes_all_three_families(T, dispatch):
+    """20b-shaped layer, Zipf-skewed routing: streaming, expert tiles and row tiles all take
+    experts in the same call."""
+    layer, g, rep = _run(T, 32, 2880, 2880, 4, seed=3, zipf=True, dispatch=dispatch)
+    s, t = layer.get_dispatch()
+    fam = _families(np.diff(g["expert_offsets"]), s, t)
+    print("hybrid T=%d thresholds=%s experts per family %s %s" % (T, (s, t), fam, json.dumps(
+        {k: v for k, v in rep.items() if k != "set_changed"})))
+    assert all(n > 0 for n in fam), fam
+
+
+@pytest.mark.parametrize("T", [17, 40, 129, 300, 777])
+def test_expert_tile_path_ragged(T):
+    """Every expert through the expert-tile kernels: rows 1..16 per box, 1 or 2 row chunks of
+    128, a half-filled last column block (I = 320: 128 + 128 + 64 gate/up columns)."""
+    _run(T, 8, 256, 320, 2, seed=2000 + T, path=moe.MOE_PATH_TILE)
+
+
+@pytest.mark.parametrize("T", [16, 96, 512])
+def test_expert_tile_path_gpt_oss_shape(T):
+    """H = I = 2880: 45 K stages, 23 gate/up column blocks (the last 64 wide), 12 down blocks
+    (the last 64 wide)."""
+    _run(T, 32, 2880, 2880, 4, seed=2100 + T, path=moe.MOE_PATH_TILE)
+
+
+def test_expert_tile_path_120b_shape():
+    _run(200, 128, 2880, 2880, 4, seed=2200, path=moe.MOE_PATH_TILE)
+
+
+@pytest.mark.parametrize("T", [96, 192, 512, 2048])
+def test_auto_20b_mid_T(T):
+    """The default per-expert thresholds across the mid-token band of the 20b layer."""
+    _run(T, 32, 2880, 2880, 4, seed=2300 + T)
+
+
+def test_thresholds_round_trip():
+    layer = moe.Moe(8, 256, 256, 2)
+    assert layer.get_dispatch() == (16, 256)
+    layer.set_dispatch(4, 100)
+    assert layer.get_dispatch() == (4, 100)
+    layer.set_dispatch(-1, 50)
+    assert layer.get_dispatch() == (4, 50)
+    layer.set_path(moe.MOE_PATH_AUTO, 9)
+    assert layer.get_path() == (moe.MOE_PATH_AUTO, 9) and layer.get_dispatch() == (9, 50)
