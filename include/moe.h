@@ -161,6 +161,44 @@ MOE_API moe_status moe_forward_mxfp4(moe_t ctx, int T, const void* x_bf16,
                                      const void* dn_codes, const void* dn_scales, float* out,
                                      void* workspace, size_t ws_bytes, moe_stream_t stream);
 
+/* ---- Expert parallelism: the device work on either side of the exchange ----------------
+ * With the E experts split over G GPUs (E/G each), every GPU routes its own tokens with
+ * moe_route (full E), puts the routed rows in expert order with moe_permute, sends each
+ * expert's rows to the GPU that owns it (an all-to-all over NVLink, sizes from the
+ * histogram: the rows of the owner's experts are one contiguous run of x_perm), runs
+ * moe_experts on what it received with a handle made for its E/G experts, sends the results
+ * back, and adds each token's k results with moe_combine.  The pages kept every expert on
+ * each GPU (Persona Kappa forum post, "The Config": expert-parallel degree 1); the split
+ * divides the expert weight bytes each GPU streams in decode by G.  The exchange is the
+ * caller's (NCCL all-to-all); these calls only enqueue kernels on `stream`.
+ *
+ * moe_permute: x_perm [T*k, H] bf16 = x[perm[r]] and row_w [T*k] fp32 = the routing weight
+ *   of row r (topk_w[t, j] where inv_perm[t, j] = r), from moe_route's perm, inv_perm and
+ *   topk_w.  A perm entry outside [0, T) skips its row and makes moe_sync_status return
+ *   MOE_ERR_ARG.
+ * moe_experts: the expert half of the layer on R rows that arrive as S*E segments (E = this
+ *   handle's experts): seg_counts [S, E] int32 in device memory holds the rows of expert e
+ *   from source s; rows are stored source-major, experts ascending inside a source (what an
+ *   all-to-all of per-owner runs of x_perm delivers).  Writes
+ *     y_rows[r] = row_w[r] * (swiglu(x_rows[r] W_gate_up[e]) W_down[e])   fp32 [R, H]
+ *   with e the expert of r's segment.  Each expert's kernel family follows the handle's
+ *   path setting, from its rows summed over the sources.  Counts that do not sum to R make
+ *   moe_sync_status return MOE_ERR_ARG (rows past R are never read or written).  S * E <=
+ *   4096.  workspace: moe_experts_workspace_bytes(ctx, R, S).
+ * moe_combine: out [T, H] fp32 = sum over j < k of y_rows[inv_perm[t, j]], in slot order
+ *   (y_rows in the row order of this GPU's x_perm, as the exchange back returns it). */
+MOE_API moe_status moe_permute(moe_t ctx, int T, const void* x_bf16, const int32_t* perm,
+                               const int32_t* inv_perm, const float* topk_w, void* x_perm_bf16,
+                               float* row_w, moe_stream_t stream);
+MOE_API size_t moe_experts_workspace_bytes(moe_t ctx, int R, int S);
+MOE_API moe_status moe_experts(moe_t ctx, int R, int S, const int32_t* seg_counts,
+                               const void* x_rows_bf16, const float* row_w,
+                               const void* W_gate_up_bf16, const void* W_down_bf16,
+                               float* y_rows, void* workspace, size_t ws_bytes,
+                               moe_stream_t stream);
+MOE_API moe_status moe_combine(moe_t ctx, int T, const int32_t* inv_perm, const float* y_rows,
+                               float* out, moe_stream_t stream);
+
 /* Choose the path.  stream_rows >= 0 also sets the AUTO threshold: experts with at most this
  * many rows in a call stream their weights (the built-in default is 16, one streaming chunk;
  * moe_tune measures it); stream_rows < 0 keeps the current one.  MOE_ERR_ARG for an unknown
@@ -192,8 +230,9 @@ MOE_API moe_status moe_tune(moe_t ctx, int T_max, const void* x_bf16, const void
                     moe_stream_t stream, int* crossover_out);
 
 /* Synchronise `stream`, then read and clear the handle's device status word.  Returns
- * MOE_ERR_TIMEOUT if a device-side bounded wait gave up since the last call, MOE_ERR_CUDA if
- * the stream reports an error, MOE_OK otherwise. */
+ * MOE_ERR_TIMEOUT if a device-side bounded wait gave up since the last call, MOE_ERR_ARG if a
+ * kernel met an index or count outside its buffers (moe_permute, moe_experts, moe_combine),
+ * MOE_ERR_CUDA if the stream reports an error, MOE_OK otherwise. */
 MOE_API moe_status moe_sync_status(moe_t ctx, moe_stream_t stream);
 
 /* Static text for a status code ("unknown status" for values outside the enum). */

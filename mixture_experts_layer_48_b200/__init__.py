@@ -58,6 +58,10 @@ _SIGS = {
                                  _c_int]),
     "moe_profile_kind_name": (ctypes.c_char_p, [_c_int]),
     "moe_selftest_timeout": (_c_int, [_vp, _c_int, _vp]),
+    "moe_permute": (_c_int, [_vp, _c_int, _vp, _vp, _vp, _vp, _vp, _vp, _vp]),
+    "moe_experts_workspace_bytes": (_sz, [_vp, _c_int, _c_int]),
+    "moe_experts": (_c_int, [_vp, _c_int, _c_int, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _sz, _vp]),
+    "moe_combine": (_c_int, [_vp, _c_int, _vp, _vp, _vp, _vp]),
     "moe_route_static_max_bytes": (_sz, []),
     "moe_route_static": (_c_int, [_vp, _c_int, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp]),
 }
@@ -196,6 +200,53 @@ class Moe:
         return out
 
     __call__ = forward
+
+    # -- expert parallelism: device work on either side of the exchange (include/moe.h) --
+    def permute(self, x, r: dict, stream=None) -> tuple[torch.Tensor, torch.Tensor]:
+        """Rows in expert order and their routing weights, from moe_route's outputs."""
+        T = x.shape[0]
+        R = T * self.k
+        x_perm = torch.empty((R, self.H), dtype=torch.bfloat16, device=x.device)
+        row_w = torch.empty((R,), dtype=torch.float32, device=x.device)
+        st = moe_permute(self._h, T, _ptr(x, torch.bfloat16, "x", (T, self.H)),
+                         _ptr(r["perm"], torch.int32, "perm", (R,)),
+                         _ptr(r["inv_perm"], torch.int32, "inv_perm", (T, self.k)),
+                         _ptr(r["topk_w"], torch.float32, "topk_w", (T, self.k)),
+                         x_perm.data_ptr(), row_w.data_ptr(), _stream(stream))
+        _check(st, "moe_permute")
+        return x_perm, row_w
+
+    def experts(self, x_rows, row_w, seg_counts, W_gate_up, W_down, stream=None,
+                workspace=None) -> torch.Tensor:
+        """The expert half on rows grouped as seg_counts [S, E] segments (source-major)."""
+        R = x_rows.shape[0]
+        S = seg_counts.shape[0]
+        y = torch.empty((R, self.H), dtype=torch.float32, device=x_rows.device)
+        if R == 0:
+            return y
+        need = moe_experts_workspace_bytes(self._h, R, S)
+        if need == 0:
+            raise ValueError("moe_experts: unsupported R or S")
+        ws = self._workspace(need, x_rows.device) if workspace is None else workspace
+        st = moe_experts(self._h, R, S, _ptr(seg_counts, torch.int32, "seg_counts", (S, self.E)),
+                         _ptr(x_rows, torch.bfloat16, "x_rows", (R, self.H)),
+                         _ptr(row_w, torch.float32, "row_w", (R,)),
+                         _ptr(W_gate_up, torch.bfloat16, "W_gate_up", (self.E, self.H, 2 * self.I)),
+                         _ptr(W_down, torch.bfloat16, "W_down", (self.E, self.I, self.H)),
+                         y.data_ptr(), ws.data_ptr(), ws.numel(), _stream(stream))
+        _check(st, "moe_experts")
+        return y
+
+    def combine(self, inv_perm, y_rows, out=None, stream=None) -> torch.Tensor:
+        """out[t] = sum_j y_rows[inv_perm[t, j]] (slot order)."""
+        T = inv_perm.shape[0]
+        if out is None:
+            out = torch.empty((T, self.H), dtype=torch.float32, device=y_rows.device)
+        st = moe_combine(self._h, T, _ptr(inv_perm, torch.int32, "inv_perm", (T, self.k)),
+                         _ptr(y_rows, torch.float32, "y_rows", (T * self.k, self.H)),
+                         _ptr(out, torch.float32, "out", (T, self.H)), _stream(stream))
+        _check(st, "moe_combine")
+        return out
 
     def workspace_bytes_mxfp4(self, T: int) -> int:
         return moe_workspace_bytes_mxfp4(self._h, T)

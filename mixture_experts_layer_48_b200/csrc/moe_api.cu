@@ -19,6 +19,7 @@
 #include "stream_mx.cuh"
 #include "gemm.cuh"
 #include "expert_gemm.cuh"
+#include "ep.cuh"
 
 using namespace moe;
 
@@ -306,6 +307,32 @@ Layout make_layout(const moe_ctx* c, int T, const Plan& p, bool mx) {
   return L;
 }
 
+// Workspace of the expert half alone (moe_experts): R received rows in S*E segments.
+Layout make_expert_layout(const moe_ctx* c, int R, int S, const Plan& p) {
+  Layout L{};
+  Carver cv;
+  for (int f = 0; f < kFamilies; ++f)
+    if (p.has[f]) {
+      const long long rows = kFamChunkRows[f], segs = (long long)S * c->E;
+      long long n = R / rows + segs;
+      if (p.max_count[f] != INT_MAX)  // every expert's segments together hold <= max_count rows
+        n = std::min(n, (long long)c->E * ((p.max_count[f] + rows - 1) / rows + S));
+      L.sched[f] = cv.take(16);
+      L.chunks[f] = cv.take(16 * (size_t)n);
+      if (f == kFamStream) {
+        const int tile_cols = std::min(kStreamCols, kMxTileCols);
+        L.n_done = (int)(n * ((c->I + tile_cols - 1) / tile_cols));
+        L.done = cv.take(4 * (size_t)L.n_done);
+        L.acc_floats = (size_t)n * kStreamRB * 2 * c->I;
+        L.acc = cv.take(sizeof(float) * L.acc_floats);
+      }
+    }
+  L.h = cv.take(2 * (size_t)R * c->I);
+  L.perm = cv.take(4 * (size_t)R);  // identity row map of the results
+  L.total = cv.cur;
+  return L;
+}
+
 size_t route_ws_bytes(const moe_ctx* c, int T, bool allow_split = true) {
   Carver cv;
   cv.take(16);  // sched
@@ -473,6 +500,9 @@ bool set_smem_attrs() {
                              kEtSmem) == cudaSuccess;
   ok &= cudaFuncSetAttribute(expert_tile_kernel<1>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              kEtSmem) == cudaSuccess;
+  ok &= cudaFuncSetAttribute(build_segment_lists_kernel,
+                             cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (3 * kMaxSegments + kMaxE) * 4) == cudaSuccess;
   return ok;
 }
 
@@ -490,68 +520,26 @@ struct MxWeights {
   const void *gu_codes, *gu_scales, *dn_codes, *dn_scales;
 };
 
-// The layer for one plan: routing (with one work list per family that may receive rows), the
-// rows in expert order for the tcgen05 families, then gate/up + SwiGLU and down + combine by
-// every family in the plan.  All kernels go on one stream with programmatic serialisation;
-// each family's kernel finds its own work list (possibly empty) on the device.
-moe_status forward_plan(moe_ctx* c, int T, const void* x_bf16, const void* W_router_bf16,
-                        const float* b_router, const void* W_gate_up_bf16,
-                        const void* W_down_bf16, float* out, uint8_t* ws, size_t ws_bytes,
-                        cudaStream_t st, const MxWeights* mx = nullptr) {
-  const Plan p = make_plan(c, T, mx != nullptr, c->path);
-  const Layout L = make_layout(c, T, p, mx != nullptr);
-  if (ws_bytes < L.total) return MOE_ERR_WORKSPACE;
-  const size_t R = (size_t)T * c->k;
-  RouteOut o{};
-  o.topk_idx = reinterpret_cast<int32_t*>(ws + L.topk_idx);
-  o.topk_w = reinterpret_cast<float*>(ws + L.topk_w);
-  o.offsets = reinterpret_cast<int32_t*>(ws + L.offsets);
-  o.perm = reinterpret_cast<int32_t*>(ws + L.perm);
-  o.inv_perm = reinterpret_cast<int32_t*>(ws + L.inv_perm);
-  o.row_w = reinterpret_cast<float*>(ws + L.row_w);
-  for (int f = 0; f < kFamilies; ++f)
-    if (p.has[f]) {
-      WorkList& wl = o.wl[o.n_lists];
-      wl.chunks = reinterpret_cast<int4*>(ws + L.chunks[f]);
-      wl.sched = reinterpret_cast<int32_t*>(ws + L.sched[f]);
-      wl.chunk_rows = kFamChunkRows[f];
-      wl.min_count = p.min_count(f);
-      wl.max_count = p.max_count[f];
-      ++o.n_lists;
-    }
-  auto chunks_of = [&](int f) { return reinterpret_cast<const int4*>(ws + L.chunks[f]); };
-  auto sched_of = [&](int f) { return reinterpret_cast<const int32_t*>(ws + L.sched[f]); };
-  o.zero_i32 = p.has[kFamStream] ? reinterpret_cast<int32_t*>(ws + L.done) : nullptr;
-  o.n_zero = p.has[kFamStream] ? L.n_done : 0;
-  const uint16_t* x = static_cast<const uint16_t*>(x_bf16);
-  uint16_t* x16 = mx ? reinterpret_cast<uint16_t*>(ws + L.x16) : nullptr;
-  uint16_t* h = reinterpret_cast<uint16_t*>(ws + L.h);
-  uint16_t* x_perm = L.x_perm ? reinterpret_cast<uint16_t*>(ws + L.x_perm) : nullptr;
-  if (mx) {  // the MXFP4 kernels take f16 activations
-    const size_t n = (size_t)T * c->H;
-    const int blocks = (int)std::min<size_t>((n / 8 + 255) / 256, (size_t)c->num_sms * 4);
-    MOE_TRY(launch(c, kKindConvert, st, [&] {
-      return launch_pdl(to_f16_kernel, dim3(blocks), dim3(256), 0, st, x, x16, n);
-    }));
-  }
-  // With enough 64-token blocks to cover the GPU the scatter also writes the rows in expert
-  // order (each token row read once); otherwise a wide gather kernel does it.
-  const int NB = (T + kRouterTcTokens - 1) / kRouterTcTokens;
-  const bool fused_copy = x_perm && T > kSmallT && NB >= c->num_sms;
-  if (fused_copy) {
-    o.x = x;
-    o.x_perm = x_perm;
-    o.H = c->H;
-  }
-  float* acc = p.has[kFamStream] ? reinterpret_cast<float*>(ws + L.acc) : nullptr;
-  MOE_TRY(launch_route(c, T, x, static_cast<const uint16_t*>(W_router_bf16), b_router, o, ws,
-                       L.rt, st, acc, L.acc_floats));
-  if (x_perm && !fused_copy)
-    MOE_TRY(launch(c, kKindGather, st, [&] {
-      return launch_pdl(gather_rows_kernel, dim3((unsigned)((R + 7) / 8)), dim3(256), 0, st, x,
-                        (const int32_t*)o.perm, (int)R, c->H, x_perm);
-    }));
+// The expert half of the layer for one plan: gate/up + SwiGLU, then down + weighted combine,
+// by every kernel family in the plan, each on its own work list (found on the device).
+struct ExpertIO {
+  int R;                              // rows
+  const uint16_t* x_tok;              // rows of the streaming family: x_tok[perm[r]]
+  const int32_t* perm;                // [R] row -> row of x_tok / of out
+  const uint16_t* x_perm;             // [R, H] rows in expert order (tcgen05 families), or null
+  const float* row_w;                 // [R] weight of each row's result
+  float* out;                         // [*, H] fp32, accumulated through perm
+  size_t out_elems;                   // elements of out this phase zero-fills first
+  const int4* chunks[kFamilies];
+  const int32_t* sched[kFamilies];
+  float* acc;                         // streaming family: split-K sums, zero on entry
+  int32_t* done;                      // streaming family: completion counters, zero on entry
+  uint16_t* h;                        // [R, I] SwiGLU output
+};
 
+moe_status expert_phase(moe_ctx* c, const Plan& p, const ExpertIO& io, const void* W_gate_up_bf16,
+                        const void* W_down_bf16, const MxWeights* mx, cudaStream_t st) {
+  const size_t R = (size_t)io.R;
   // `out` is zero-filled once, by one gate/up kernel: the row-tile GEMM's epilogue warps while
   // its tensor cores run, else the first other gate/up kernel before its dependency wait.
   const int zero_owner = p.has[kFamGemm] ? kFamGemm : p.has[kFamStream] ? kFamStream : kFamTile;
@@ -560,18 +548,18 @@ moe_status forward_plan(moe_ctx* c, int T, const void* x_bf16, const void* W_rou
   // ---------------------------- gate/up projection + SwiGLU ----------------------------
   if (p.has[kFamStream]) {
     GateUpArgs ga{};
-    ga.x = mx ? x16 : x;
+    ga.x = io.x_tok;
     ga.H = c->H;
     ga.I = c->I;
-    ga.R = (int)R;
-    ga.perm = o.perm;
-    ga.chunks = chunks_of(kFamStream);
-    ga.sched = sched_of(kFamStream);
-    ga.acc = acc;
-    ga.done = o.zero_i32;
-    ga.h = h;
-    ga.out = out;
-    ga.out_elems = zero_owner == kFamStream ? (size_t)T * c->H : 0;
+    ga.R = io.R;
+    ga.perm = io.perm;
+    ga.chunks = io.chunks[kFamStream];
+    ga.sched = io.sched[kFamStream];
+    ga.acc = io.acc;
+    ga.done = io.done;
+    ga.h = io.h;
+    ga.out = io.out;
+    ga.out_elems = zero_owner == kFamStream ? io.out_elems : 0;
     ga.status = c->d_status;
     if (mx) {
       const CUtensorMap* cm = cached_map_u8(c->gu_codes, mx->gu_codes, 2ull * c->I * c->E,
@@ -606,20 +594,20 @@ moe_status forward_plan(moe_ctx* c, int T, const void* x_bf16, const void* W_rou
     if (!wgu || !wdn) return MOE_ERR_CUDA;
   }
   if (p.has[kFamTile]) {
-    const CUtensorMap* xm = cached_map(c->et_x_map, x_perm, R, (uint64_t)c->H, kEtRowBox, 64);
+    const CUtensorMap* xm = cached_map(c->et_x_map, io.x_perm, R, (uint64_t)c->H, kEtRowBox, 64);
     if (!xm) return MOE_ERR_CUDA;
     EtArgs e{};
     e.K = c->H;
     e.Ncols = c->I;
     e.w_rows = c->H;
-    e.chunks = chunks_of(kFamTile);
-    e.sched = sched_of(kFamTile);
-    e.h = h;
+    e.chunks = io.chunks[kFamTile];
+    e.sched = io.sched[kFamTile];
+    e.h = io.h;
     e.H = c->H;
     e.status = c->d_status;
     if (zero_owner == kFamTile) {
-      e.zero4 = reinterpret_cast<float4*>(out);
-      e.n_zero4 = (size_t)T * c->H / 4;
+      e.zero4 = reinterpret_cast<float4*>(io.out);
+      e.n_zero4 = io.out_elems / 4;
     }
     MOE_TRY(launch(c, kKindGateUpTile, st, [&] {
       return launch_pdl(expert_tile_kernel<0>, dim3(c->num_sms), dim3(kEtThreads), kEtSmem, st,
@@ -627,21 +615,21 @@ moe_status forward_plan(moe_ctx* c, int T, const void* x_bf16, const void* W_rou
     }));
   }
   if (p.has[kFamGemm]) {
-    const CUtensorMap* am = cached_map(c->x_perm_map, x_perm, R, (uint64_t)c->H, kGemmBM, 64);
+    const CUtensorMap* am = cached_map(c->x_perm_map, io.x_perm, R, (uint64_t)c->H, kGemmBM, 64);
     if (!am) return MOE_ERR_CUDA;
     GemmArgs g{};
     g.K = c->H;
     g.Ncols = c->I;
     g.sub_stride = c->I;
     g.w_rows = c->H;
-    g.chunks = chunks_of(kFamGemm);
-    g.sched = sched_of(kFamGemm);
-    g.h = h;
+    g.chunks = io.chunks[kFamGemm];
+    g.sched = io.sched[kFamGemm];
+    g.h = io.h;
     g.H = c->H;
     g.status = c->d_status;
     // the epilogue warps zero-fill `out`, which the down projections accumulate into
-    g.zero4 = reinterpret_cast<float4*>(out);
-    g.n_zero4 = (size_t)T * c->H / 4;
+    g.zero4 = reinterpret_cast<float4*>(io.out);
+    g.n_zero4 = io.out_elems / 4;
     MOE_TRY(launch(c, kKindGateUpGemm, st, [&] {
       return launch_pdl(grouped_gemm_2sm_kernel<MOE_GEMM_GATE_UP>, dim3(pair_grid),
                         dim3(kGemmThreads), Gemm2Cfg<kGemmStages>::kSmem, st, g, *am, *wgu);
@@ -651,15 +639,15 @@ moe_status forward_plan(moe_ctx* c, int T, const void* x_bf16, const void* W_rou
   // ---------------------------- down projection + weighted combine ----------------------------
   if (p.has[kFamStream]) {
     DownArgs da{};
-    da.h = h;
+    da.h = io.h;
     da.H = c->H;
     da.I = c->I;
-    da.R = (int)R;
-    da.perm = o.perm;
-    da.row_w = o.row_w;
-    da.chunks = chunks_of(kFamStream);
-    da.sched = sched_of(kFamStream);
-    da.out = out;
+    da.R = io.R;
+    da.perm = io.perm;
+    da.row_w = io.row_w;
+    da.chunks = io.chunks[kFamStream];
+    da.sched = io.sched[kFamStream];
+    da.out = io.out;
     da.status = c->d_status;
     if (mx) {
       const CUtensorMap* cm = cached_map_u8(c->dn_codes, mx->dn_codes, (uint64_t)c->H * c->E,
@@ -684,17 +672,17 @@ moe_status forward_plan(moe_ctx* c, int T, const void* x_bf16, const void* W_rou
     }
   }
   if (p.has[kFamTile]) {
-    const CUtensorMap* hm = cached_map(c->et_h_map, h, R, (uint64_t)c->I, kEtRowBox, 64);
+    const CUtensorMap* hm = cached_map(c->et_h_map, io.h, R, (uint64_t)c->I, kEtRowBox, 64);
     if (!hm) return MOE_ERR_CUDA;
     EtArgs e{};
     e.K = c->I;
     e.Ncols = c->H;
     e.w_rows = c->I;
-    e.chunks = chunks_of(kFamTile);
-    e.sched = sched_of(kFamTile);
-    e.perm = o.perm;
-    e.row_w = o.row_w;
-    e.out = out;
+    e.chunks = io.chunks[kFamTile];
+    e.sched = io.sched[kFamTile];
+    e.perm = io.perm;
+    e.row_w = io.row_w;
+    e.out = io.out;
     e.H = c->H;
     e.status = c->d_status;
     MOE_TRY(launch(c, kKindDownTile, st, [&] {
@@ -703,18 +691,18 @@ moe_status forward_plan(moe_ctx* c, int T, const void* x_bf16, const void* W_rou
     }));
   }
   if (p.has[kFamGemm]) {
-    const CUtensorMap* hm = cached_map(c->h_map, h, R, (uint64_t)c->I, kGemmBM, 64);
+    const CUtensorMap* hm = cached_map(c->h_map, io.h, R, (uint64_t)c->I, kGemmBM, 64);
     if (!hm) return MOE_ERR_CUDA;
     GemmArgs d{};
     d.K = c->I;
     d.Ncols = c->H;
     d.sub_stride = 0;
     d.w_rows = c->I;
-    d.chunks = chunks_of(kFamGemm);
-    d.sched = sched_of(kFamGemm);
-    d.perm = o.perm;
-    d.row_w = o.row_w;
-    d.out = out;
+    d.chunks = io.chunks[kFamGemm];
+    d.sched = io.sched[kFamGemm];
+    d.perm = io.perm;
+    d.row_w = io.row_w;
+    d.out = io.out;
     d.H = c->H;
     d.status = c->d_status;
     MOE_TRY(launch(c, kKindDownGemm, st, [&] {
@@ -723,6 +711,85 @@ moe_status forward_plan(moe_ctx* c, int T, const void* x_bf16, const void* W_rou
     }));
   }
   return MOE_OK;
+}
+
+// Work lists of one plan inside a layout, as the routing (or segment) kernels fill them.
+void plan_lists(const Plan& p, const Layout& L, uint8_t* ws, RouteOut& o, ExpertIO& io) {
+  o.n_lists = 0;
+  for (int f = 0; f < kFamilies; ++f) {
+    io.chunks[f] = nullptr;
+    io.sched[f] = nullptr;
+    if (!p.has[f]) continue;
+    WorkList& wl = o.wl[o.n_lists++];
+    wl.chunks = reinterpret_cast<int4*>(ws + L.chunks[f]);
+    wl.sched = reinterpret_cast<int32_t*>(ws + L.sched[f]);
+    wl.chunk_rows = kFamChunkRows[f];
+    wl.min_count = p.min_count(f);
+    wl.max_count = p.max_count[f];
+    io.chunks[f] = wl.chunks;
+    io.sched[f] = wl.sched;
+  }
+  o.zero_i32 = p.has[kFamStream] ? reinterpret_cast<int32_t*>(ws + L.done) : nullptr;
+  o.n_zero = p.has[kFamStream] ? L.n_done : 0;
+  io.acc = p.has[kFamStream] ? reinterpret_cast<float*>(ws + L.acc) : nullptr;
+  io.done = o.zero_i32;
+  io.h = reinterpret_cast<uint16_t*>(ws + L.h);
+}
+
+// The whole layer for one plan: routing (with one work list per family that may receive
+// rows), the rows in expert order for the tcgen05 families, then the expert half.  All
+// kernels go on one stream with programmatic serialisation.
+moe_status forward_plan(moe_ctx* c, int T, const void* x_bf16, const void* W_router_bf16,
+                        const float* b_router, const void* W_gate_up_bf16,
+                        const void* W_down_bf16, float* out, uint8_t* ws, size_t ws_bytes,
+                        cudaStream_t st, const MxWeights* mx = nullptr) {
+  const Plan p = make_plan(c, T, mx != nullptr, c->path);
+  const Layout L = make_layout(c, T, p, mx != nullptr);
+  if (ws_bytes < L.total) return MOE_ERR_WORKSPACE;
+  const size_t R = (size_t)T * c->k;
+  RouteOut o{};
+  ExpertIO io{};
+  o.topk_idx = reinterpret_cast<int32_t*>(ws + L.topk_idx);
+  o.topk_w = reinterpret_cast<float*>(ws + L.topk_w);
+  o.offsets = reinterpret_cast<int32_t*>(ws + L.offsets);
+  o.perm = reinterpret_cast<int32_t*>(ws + L.perm);
+  o.inv_perm = reinterpret_cast<int32_t*>(ws + L.inv_perm);
+  o.row_w = reinterpret_cast<float*>(ws + L.row_w);
+  plan_lists(p, L, ws, o, io);
+  const uint16_t* x = static_cast<const uint16_t*>(x_bf16);
+  uint16_t* x16 = mx ? reinterpret_cast<uint16_t*>(ws + L.x16) : nullptr;
+  uint16_t* x_perm = L.x_perm ? reinterpret_cast<uint16_t*>(ws + L.x_perm) : nullptr;
+  if (mx) {  // the MXFP4 kernels take f16 activations
+    const size_t n = (size_t)T * c->H;
+    const int blocks = (int)std::min<size_t>((n / 8 + 255) / 256, (size_t)c->num_sms * 4);
+    MOE_TRY(launch(c, kKindConvert, st, [&] {
+      return launch_pdl(to_f16_kernel, dim3(blocks), dim3(256), 0, st, x, x16, n);
+    }));
+  }
+  // With enough 64-token blocks to cover the GPU the scatter also writes the rows in expert
+  // order (each token row read once); otherwise a wide gather kernel does it.
+  const int NB = (T + kRouterTcTokens - 1) / kRouterTcTokens;
+  const bool fused_copy = x_perm && T > kSmallT && NB >= c->num_sms;
+  if (fused_copy) {
+    o.x = x;
+    o.x_perm = x_perm;
+    o.H = c->H;
+  }
+  MOE_TRY(launch_route(c, T, x, static_cast<const uint16_t*>(W_router_bf16), b_router, o, ws,
+                       L.rt, st, io.acc, L.acc_floats));
+  if (x_perm && !fused_copy)
+    MOE_TRY(launch(c, kKindGather, st, [&] {
+      return launch_pdl(gather_rows_kernel, dim3((unsigned)((R + 7) / 8)), dim3(256), 0, st, x,
+                        (const int32_t*)o.perm, (int)R, c->H, x_perm);
+    }));
+  io.R = (int)R;
+  io.x_tok = mx ? x16 : x;
+  io.perm = o.perm;
+  io.x_perm = x_perm;
+  io.row_w = o.row_w;
+  io.out = out;
+  io.out_elems = (size_t)T * c->H;
+  return expert_phase(c, p, io, W_gate_up_bf16, W_down_bf16, mx, st);
 }
 
 size_t forward_ws_bytes(const moe_ctx* c, int T, bool mx, moe_path path) {
@@ -890,6 +957,84 @@ moe_status moe_forward_mxfp4(moe_t c, int T, const void* x_bf16, const void* W_r
   return s;
 }
 
+moe_status moe_permute(moe_t c, int T, const void* x_bf16, const int32_t* perm,
+                       const int32_t* inv_perm, const float* topk_w, void* x_perm_bf16,
+                       float* row_w, moe_stream_t stream) {
+  if (!c || T < 0 || T > kMaxT || (long long)T * c->k >= (1ll << 31)) return MOE_ERR_ARG;
+  if (T == 0) return MOE_OK;
+  if (!x_bf16 || !perm || !inv_perm || !topk_w || !x_perm_bf16 || !row_w) return MOE_ERR_ARG;
+  if (!aligned16(x_bf16) || !aligned16(x_perm_bf16)) return MOE_ERR_ARG;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  const long long R = (long long)T * c->k;
+  return launch(c, kKindGather, st, [&] {
+    return launch_pdl(permute_rows_kernel, dim3((unsigned)((R + 7) / 8)), dim3(256), 0, st,
+                      static_cast<const uint16_t*>(x_bf16), perm, inv_perm, topk_w, T, c->k,
+                      c->H, static_cast<uint16_t*>(x_perm_bf16), row_w, c->d_status);
+  });
+}
+
+moe_status moe_combine(moe_t c, int T, const int32_t* inv_perm, const float* y_rows, float* out,
+                       moe_stream_t stream) {
+  if (!c || T < 0 || T > kMaxT || (long long)T * c->k >= (1ll << 31)) return MOE_ERR_ARG;
+  if (T == 0) return MOE_OK;
+  if (!inv_perm || !y_rows || !out || !aligned16(y_rows) || !aligned16(out)) return MOE_ERR_ARG;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  return launch(c, kKindDown, st, [&] {
+    return launch_pdl(combine_rows_kernel, dim3((unsigned)((T + 7) / 8)), dim3(256), 0, st,
+                      inv_perm, y_rows, T, c->k, c->H, out, c->d_status);
+  });
+}
+
+size_t moe_experts_workspace_bytes(moe_t c, int R, int S) {
+  if (!c || R < 0 || R > kMaxT * 256 || S < 1 || (long long)S * c->E > kMaxSegments) return 0;
+  if (R == 0) return 0;
+  return make_expert_layout(c, R, S, make_plan(c, R, false, c->path)).total;
+}
+
+moe_status moe_experts(moe_t c, int R, int S, const int32_t* seg_counts, const void* x_rows_bf16,
+                       const float* row_w, const void* W_gate_up_bf16, const void* W_down_bf16,
+                       float* y_rows, void* workspace, size_t ws_bytes, moe_stream_t stream) {
+  if (!c || R < 0 || R > kMaxT * 256 || S < 1 || (long long)S * c->E > kMaxSegments)
+    return MOE_ERR_ARG;
+  if (R == 0) return MOE_OK;
+  if (!seg_counts || !x_rows_bf16 || !row_w || !W_gate_up_bf16 || !W_down_bf16 || !y_rows)
+    return MOE_ERR_ARG;
+  if (!aligned16(x_rows_bf16) || !aligned16(W_gate_up_bf16) || !aligned16(W_down_bf16) ||
+      !aligned16(y_rows))
+    return MOE_ERR_ARG;
+  if (!workspace || !aligned16(workspace)) return MOE_ERR_WORKSPACE;
+  const Plan p = make_plan(c, R, false, c->path);
+  const Layout L = make_expert_layout(c, R, S, p);
+  if (ws_bytes < L.total) return MOE_ERR_WORKSPACE;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  c->in_call = c->prof_max > 0 && c->prof_calls < c->prof_max;
+  RouteOut o{};
+  ExpertIO io{};
+  plan_lists(p, L, ws, o, io);
+  int32_t* iota = reinterpret_cast<int32_t*>(ws + L.perm);
+  const int grid = (int)std::max<long long>(1, std::min<long long>(c->num_sms, (R + 1023) / 1024));
+  const size_t smem = (size_t)(3 * S * c->E + c->E) * 4;
+  moe_status s = launch(c, kKindRouteFin, st, [&] {
+    return launch_pdl(build_segment_lists_kernel, dim3(grid), dim3(1024), smem, st, seg_counts,
+                      S, c->E, R, o, iota, reinterpret_cast<float4*>(io.acc), L.acc_floats / 4,
+                      c->d_status);
+  });
+  if (s == MOE_OK) {
+    io.R = R;
+    io.x_tok = static_cast<const uint16_t*>(x_rows_bf16);
+    io.perm = iota;
+    io.x_perm = static_cast<const uint16_t*>(x_rows_bf16);
+    io.row_w = row_w;
+    io.out = y_rows;
+    io.out_elems = (size_t)R * c->H;
+    s = expert_phase(c, p, io, W_gate_up_bf16, W_down_bf16, nullptr, st);
+  }
+  if (c->in_call) ++c->prof_calls;
+  c->in_call = false;
+  return s;
+}
+
 moe_status moe_set_path(moe_t c, moe_path path, int stream_rows) {
   if (!c) return MOE_ERR_ARG;
   if (path != MOE_PATH_AUTO && path != MOE_PATH_STREAM && path != MOE_PATH_GEMM &&
@@ -1015,6 +1160,7 @@ moe_status moe_sync_status(moe_t c, moe_stream_t stream) {
   if (word != 0) {
     if (cudaMemset(c->d_status, 0, sizeof(word)) != cudaSuccess) return MOE_ERR_CUDA;
     if (word & kStatusTimeout) return MOE_ERR_TIMEOUT;
+    if (word & (kStatusBadIndex | kStatusBadCounts)) return MOE_ERR_ARG;
   }
   return MOE_OK;
 }
