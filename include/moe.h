@@ -274,10 +274,10 @@ MOE_API const char* moe_profile_kind_name(int kind);
  *     65 and a few thousand (ceil(T/64) blocks each sum over all of H).
  *   - The handle's device must be the current device (MOE_ERR_ARG otherwise).
  *   - If the routing scratch for T does not fit in the array, the call returns
- *     MOE_ERR_WORKSPACE and enqueues nothing.  The scratch is (H/64)*T*E*4 bytes of partial
- *     logits for T <= 64 and ceil(T/64)*E*4 bytes of per-block expert counts above that; with
- *     H = 2880 it fits for E = 32 up to T = 1,048,320, for E = 128 up to T = 262,016, and for
- *     E = 256 for T <= 45 and 65 <= T <= 130,944.
+ *     MOE_ERR_WORKSPACE and enqueues nothing.  The scratch is ceil(H/256)*T*E*4 bytes of
+ *     partial logits for T <= 64 and ceil(T/64)*E*4 bytes of per-block expert counts above
+ *     that; with H = 2880 every T <= 64 fits for any E, and larger T fits for E = 32 up to
+ *     T = 1,048,320, for E = 128 up to T = 262,016 and for E = 256 up to T = 130,944.
  *   - Every scratch word a call reads is written earlier in the same call, so no clearing is
  *     needed between calls.  All calls share the one array: two calls whose work overlaps on
  *     the GPU (different streams, or different handles on one device) race and give undefined

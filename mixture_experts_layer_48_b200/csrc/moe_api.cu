@@ -191,7 +191,11 @@ void router_split(const moe_ctx* c, int T, int* splits, int* kc_per_split) {
 RouteTmp carve_route_tmp(Carver& cv, const moe_ctx* c, int T, bool allow_split = true) {
   RouteTmp r;
   if (T <= kSmallT) {
-    r.partial = cv.take(sizeof(float) * (size_t)(c->H / kRouterHSlice) * T * c->E);
+    // partial logits of each group of kSmallTChunks 64-row slices of W_router
+    const int nk = c->H / kRouterHSlice;
+    r.kc_per_split = kSmallTChunks;
+    r.splits = (nk + kSmallTChunks - 1) / kSmallTChunks;
+    r.partial = cv.take(sizeof(float) * (size_t)r.splits * T * c->E);
   } else {
     const size_t NB = (T + kRouterTcTokens - 1) / kRouterTcTokens;
     r.block_counts = cv.take(sizeof(int32_t) * NB * c->E);
@@ -401,26 +405,30 @@ moe_status launch_route(moe_ctx* c, int T, const uint16_t* x, const uint16_t* Wr
   float4* zero4 = reinterpret_cast<float4*>(zero);
   const size_t n_zero4 = n_zero_floats / 4;
   const int E = c->E, H = c->H, k = c->k;
+  const int nt8 = (E + 7) / 8;
   if (T <= kSmallT) {
-    const int S = H / kRouterHSlice;
+    // one token block, the hidden dimension split over rt.splits blocks: partial logits on the
+    // tensor cores, then one block finishes the routing
     float* partial = reinterpret_cast<float*>(ws + rt.partial);
-    const size_t smem_p = (size_t)(kRouteTile * kRouterHSlice + kRouterHSlice * E) * 2;
     MOE_TRY(launch(c, kKindRouter, st, [&] {
-      return launch_pdl(router_partial_kernel, dim3(S, (T + kRouteTile - 1) / kRouteTile),
-                        dim3(256), smem_p, st, x, Wr, T, H, E, partial, zero4, n_zero4);
+      if (nt8 <= 1) return launch_router_tc<1>(1, st, x, Wr, b, T, H, E, k, o, nullptr, zero4, n_zero4, rt, partial);
+      if (nt8 <= 2) return launch_router_tc<2>(1, st, x, Wr, b, T, H, E, k, o, nullptr, zero4, n_zero4, rt, partial);
+      if (nt8 <= 4) return launch_router_tc<4>(1, st, x, Wr, b, T, H, E, k, o, nullptr, zero4, n_zero4, rt, partial);
+      if (nt8 <= 8) return launch_router_tc<8>(1, st, x, Wr, b, T, H, E, k, o, nullptr, zero4, n_zero4, rt, partial);
+      if (nt8 <= 16) return launch_router_tc<16>(1, st, x, Wr, b, T, H, E, k, o, nullptr, zero4, n_zero4, rt, partial);
+      return launch_router_tc<32>(1, st, x, Wr, b, T, H, E, k, o, nullptr, zero4, n_zero4, rt, partial);
     }));
     const size_t smem_f = (size_t)T * E * 4 + (size_t)T * k * 4 + (size_t)T * 8 * 4 +
                           (256 + 257 + 257) * 4;
     MOE_TRY(launch(c, kKindRouteFin, st, [&] {
       return launch_pdl(route_small_finalize_kernel, dim3(1), dim3(1024), smem_f, st,
-                        (const float*)partial, S, b, T, E, k, o);
+                        (const float*)partial, rt.splits, b, T, E, k, o);
     }));
     return MOE_OK;
   }
   const int NB = (T + kRouterTcTokens - 1) / kRouterTcTokens;
   int32_t* block_counts = reinterpret_cast<int32_t*>(ws + rt.block_counts);
   int32_t* totals = reinterpret_cast<int32_t*>(ws + rt.totals);
-  const int nt8 = (E + 7) / 8;
   float* split_partial = rt.splits > 1 ? reinterpret_cast<float*>(ws + rt.partial) : nullptr;
   MOE_TRY(launch(c, kKindRouter, st, [&] {
     if (nt8 <= 1) return launch_router_tc<1>(NB, st, x, Wr, b, T, H, E, k, o, block_counts, zero4, n_zero4, rt, split_partial);
@@ -479,8 +487,6 @@ bool set_smem_attrs() {
                              big) == cudaSuccess;
   ok &= cudaFuncSetAttribute(topk_from_partials_kernel,
                              cudaFuncAttributeMaxDynamicSharedMemorySize, big) == cudaSuccess;
-  ok &= cudaFuncSetAttribute(router_partial_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             big) == cudaSuccess;
   ok &= cudaFuncSetAttribute(stream_gate_up_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              kGateUpSmem) == cudaSuccess;
   ok &= cudaFuncSetAttribute(stream_down_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,

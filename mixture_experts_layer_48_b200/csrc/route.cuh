@@ -6,9 +6,10 @@
 // card).  Ties go to the lower expert index; inside an expert's row segment tokens ascend.
 //
 // Two chains:
-//   T <= kSmallT : router_partial_kernel (H/64 blocks, one 64-row slice of W_router each)
-//                  -> route_small_finalize_kernel (one block: sum, top-k, softmax,
-//                     histogram, scan, permutation, work list).
+//   T <= kSmallT : router_topk_kernel split over the hidden dimension (one block per
+//                  kSmallTChunks 64-row slices of W_router, partial logits on the tensor cores)
+//                  -> route_small_finalize_kernel (one block: sum of the slices, top-k,
+//                     softmax, histogram, scan, permutation, work lists).
 //   T >  kSmallT : router_topk_kernel (64 tokens per block, all experts on the tensor cores;
 //                  top-k and a block histogram) -> route_scan_kernel (one block per expert:
 //                  prefix over blocks) -> route_scatter_kernel (permutation, 64 tokens per
@@ -20,8 +21,37 @@
 namespace moe {
 
 constexpr int kSmallT = 64;        // largest T handled by the single-block finalize
-constexpr int kRouteTile = 32;     // tokens per block in the large-T chain
-constexpr int kRouterHSlice = 64;  // W_router rows per block in router_partial_kernel
+constexpr int kRouterHSlice = 64;  // W_router rows per router pipeline stage
+constexpr int kSmallTChunks = 4;   // T <= kSmallT: 64-row slices of W_router per router block
+
+// Exclusive prefix sum over n <= 256 values by one warp (lane l holds entries 8l .. 8l+7):
+// val(e) gives entry e, put(e, prefix) receives its exclusive prefix.  Returns the total on
+// every lane.
+template <typename Val, typename Put>
+MOE_DEVINL int warp_exclusive_scan(int n, Val val, Put put) {
+  const int lane = threadIdx.x & 31;
+  int loc[8], sum = 0;
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    const int e = lane * 8 + i;
+    loc[i] = e < n ? val(e) : 0;
+    sum += loc[i];
+  }
+  int incl = sum;
+#pragma unroll
+  for (int off = 1; off < 32; off <<= 1) {
+    const int y = __shfl_up_sync(0xffffffffu, incl, off);
+    if (lane >= off) incl += y;
+  }
+  int run = incl - sum;
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    const int e = lane * 8 + i;
+    if (e < n) put(e, run);
+    run += loc[i];
+  }
+  return __shfl_sync(0xffffffffu, incl, 31);
+}
 
 // One work list: the row segments of the experts whose row count lies in (min_count,
 // max_count], cut into chunks of at most chunk_rows rows.  Each expert kernel family walks
@@ -213,49 +243,12 @@ MOE_DEVINL void topk_block_epilogue(float* lg, int ld, int nt, int t0, int E, in
   for (int e = tid; e < E; e += blockDim.x) block_counts[(size_t)blockIdx.x * E + e] = cnt[e];
 }
 
-// ---------------------------------------------------------------------------------------
-// Small T: partial router logits over one 64-row slice of W_router.
-// grid (H/64, ceil(T/32)), block 256.  partial layout [H/64][T][E].
-// ---------------------------------------------------------------------------------------
 // Grid-stride zero fill of a scratch region by every block of the launching kernel.
 MOE_DEVINL void zero_fill_f4(float4* z, size_t n4) {
   const size_t nthreads = (size_t)gridDim.x * gridDim.y * blockDim.x;
   const size_t b = (size_t)blockIdx.y * gridDim.x + blockIdx.x;
   for (size_t i = b * blockDim.x + threadIdx.x; i < n4; i += nthreads)
     z[i] = make_float4(0.f, 0.f, 0.f, 0.f);
-}
-
-__global__ void __launch_bounds__(256) router_partial_kernel(const uint16_t* __restrict__ x,
-                                                             const uint16_t* __restrict__ Wr,
-                                                             int T, int H, int E,
-                                                             float* __restrict__ partial,
-                                                             float4* zero4, size_t n_zero4) {
-  pdl_wait();
-  pdl_launch_next();
-  zero_fill_f4(zero4, n_zero4);
-  extern __shared__ __align__(128) uint8_t smem_raw[];
-  uint16_t* xs = reinterpret_cast<uint16_t*>(smem_raw);  // [32][64]
-  uint16_t* ws = xs + kRouteTile * kRouterHSlice;          // [64][E]
-  const int s = blockIdx.x, h0 = s * kRouterHSlice, t0 = blockIdx.y * kRouteTile;
-  const int nt = min(kRouteTile, T - t0);
-  for (int i = threadIdx.x; i < nt * 8; i += blockDim.x) {
-    const int r = i >> 3, c = i & 7;
-    reinterpret_cast<uint4*>(xs)[r * 8 + c] =
-        reinterpret_cast<const uint4*>(x + (size_t)(t0 + r) * H + h0)[c];
-  }
-  // the slice is 64*E contiguous bf16 = 128*E bytes: whole 16-byte pieces at a 128-byte offset
-  const uint4* wsrc = reinterpret_cast<const uint4*>(Wr + (size_t)h0 * E);
-  for (int i = threadIdx.x; i < kRouterHSlice * E / 8; i += blockDim.x)
-    reinterpret_cast<uint4*>(ws)[i] = wsrc[i];
-  __syncthreads();
-  for (int o = threadIdx.x; o < nt * E; o += blockDim.x) {
-    const int t = o / E, e = o - t * E;
-    float acc = 0.f;
-#pragma unroll 16
-    for (int h = 0; h < kRouterHSlice; ++h)
-      acc = fmaf(bf16_to_f32(xs[t * kRouterHSlice + h]), bf16_to_f32(ws[h * E + e]), acc);
-    partial[((size_t)s * T + t0 + t) * E + e] = acc;
-  }
 }
 
 // Work lists of one routing: expert e (with count c > 0) belongs to the list whose
@@ -266,18 +259,17 @@ MOE_DEVINL void build_work_lists(const int32_t* cnt, const int32_t* off, int E,
                                  const RouteOut& o, int32_t* scratch) {
   const int tid = threadIdx.x;
   if (o.n_lists == 0) return;
-  // thread i < n_lists: exclusive scan of list i's chunk counts, in expert order
-  if (tid < o.n_lists) {
-    const WorkList& L = o.wl[tid];
-    int run = 0;
-    for (int e = 0; e < E; ++e) {
-      const int c = cnt[e];
-      if (c > L.min_count && c <= L.max_count) {
-        scratch[e] = run;
-        run += (c + L.chunk_rows - 1) / L.chunk_rows;
-      }
-    }
-    L.sched[0] = run;
+  // warp l < n_lists: exclusive scan of list l's chunk counts, in expert order
+  const int warp = tid >> 5;
+  if (warp < o.n_lists) {
+    const WorkList& L = o.wl[warp];
+    auto member = [&](int e) { return cnt[e] > L.min_count && cnt[e] <= L.max_count; };
+    const int total = warp_exclusive_scan(
+        E, [&](int e) { return member(e) ? (cnt[e] + L.chunk_rows - 1) / L.chunk_rows : 0; },
+        [&](int e, int pre) {
+          if (member(e)) scratch[e] = pre;
+        });
+    if ((tid & 31) == 0) L.sched[0] = total;
   }
   __syncthreads();
   for (int e = tid; e < E; e += blockDim.x) {
@@ -357,13 +349,10 @@ __global__ void __launch_bounds__(1024)
     }
   }
   __syncthreads();
-  if (tid == 0) {
-    int run = 0;
-    for (int e = 0; e < E; ++e) {
-      off[e] = run;
-      run += cnt[e];
-    }
-    off[E] = run;
+  if (warp == 0) {
+    const int total = warp_exclusive_scan(E, [&](int e) { return cnt[e]; },
+                                          [&](int e, int pre) { off[e] = pre; });
+    if (lane == 0) off[E] = total;
   }
   __syncthreads();
   for (int e = tid; e <= E; e += blockDim.x) o.offsets[e] = off[e];
@@ -627,14 +616,10 @@ __global__ void __launch_bounds__(256) route_scan_kernel(int32_t* __restrict__ b
   for (int b = b0; b < b1; ++b) s += block_counts[(size_t)b * E + e];
   part[tid] = s;
   __syncthreads();
-  if (tid == 0) {
-    int run = 0;
-    for (int i = 0; i < (int)blockDim.x; ++i) {
-      const int v = part[i];
-      part[i] = run;
-      run += v;
-    }
-    totals[e] = run;
+  if (tid < 32) {  // blockDim.x == 256: one warp scans the 256 partial sums in place
+    const int total = warp_exclusive_scan(256, [&](int i) { return part[i]; },
+                                          [&](int i, int pre) { part[i] = pre; });
+    if (tid == 0) totals[e] = total;
   }
   __syncthreads();
   int run = part[tid];
@@ -670,13 +655,10 @@ __global__ void __launch_bounds__(256)
   for (int e = tid; e < E; e += blockDim.x) cnt[e] = totals[e];
   for (int i = tid; i < TT * 8; i += blockDim.x) bits[i] = 0u;
   __syncthreads();
-  if (tid == 0) {
-    int run = 0;
-    for (int e = 0; e < E; ++e) {
-      off[e] = run;
-      run += cnt[e];
-    }
-    off[E] = run;
+  if (warp == 0) {
+    const int total = warp_exclusive_scan(E, [&](int e) { return cnt[e]; },
+                                          [&](int e, int pre) { off[e] = pre; });
+    if (lane == 0) off[E] = total;
   }
   for (int i = tid; i < nt * k; i += blockDim.x) {
     const int tt = i / k, j = i - tt * k;

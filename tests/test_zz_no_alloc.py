@@ -83,12 +83,12 @@ def test_static_scratch_route_matches_workspace_route(T):
 
 
 def test_static_scratch_rejects_sizes_beyond_its_array():
-    # Refused before anything is launched: 256 experts x 64 tokens need 45 x 64 x 256 x 4 B of
-    # partial logits (2.9 MB) and 131,008 tokens need 2047 blocks x 1 KB of per-block expert
-    # counts, both more than the 2 MiB array; 128 experts x 64 tokens (1.5 MB) and 256 experts
-    # x 130,944 tokens (2046 KB) fit.
+    # Refused before anything is launched: 64 tokens with H = 16384 and 256 experts need
+    # 64 x 64 x 256 x 4 B of partial logits (4 MiB), and 131,008 tokens need 2047 blocks x 1 KB of
+    # per-block expert counts, both more than the 2 MiB array; 64 tokens with H = 2880 and
+    # 256 experts (12 slices: 768 KiB) and 130,944 tokens with 256 experts (2046 KiB) fit.
     assert moe.moe_route_static_max_bytes() == 2 << 20
-    for E, T, H, ok in ((128, 64, 2880, True), (256, 64, 2880, False),
+    for E, T, H, ok in ((256, 64, 2880, True), (256, 64, 16384, False),
                         (256, 130944, 64, True), (256, 131008, 64, False)):
         layer = moe.Moe(E, H, 64, 4)
         d = mi.make_inputs(T, H, E, 4, 64, seed=7, device="cuda", experts=False)
