@@ -148,12 +148,20 @@ MOE_API moe_status moe_forward(moe_t ctx, int T, const void* x_bf16, const void*
  * gu_codes [E, 2I, H/2] and gu_scales [E, H/32, 2I] hold W_gate_up [E, H, 2I] (gate columns
  * [0, I), up columns [I, 2I)); dn_codes [E, H, I/2] and dn_scales [E, I/32, H] hold W_down
  * [E, I, H].  x, W_router, b_router and out as in moe_forward; all pointers 16-byte aligned.
- * Runs the streaming path at every T (there is no MXFP4 grouped GEMM): the weights stream
- * at a quarter of the bf16 bytes.  The tensor-core products take the E2M1 values (exact in
- * f16) and the activations converted from bf16 to f16, which is exact for magnitudes
- * 2^-14 .. 65504 (larger ones overflow to infinity, smaller ones keep fewer bits); each
- * 32-element block's fp32 result is scaled by its E8M0 factor in fp32.  workspace: at least
- * moe_workspace_bytes_mxfp4(ctx, T) bytes.  T = 0 is a no-op. */
+ * Experts are dispatched like the bf16 layer's (moe_path), with two kernel families: up to
+ * stream_rows rows, the MXFP4 weight-streaming kernels; more rows, the MXFP4 expert-tile kernel
+ * (MOE_PATH_GEMM and MOE_PATH_TILE both force the latter; there is no MXFP4 row-tile GEMM).
+ *   - expert tiles: the codes are widened to bf16 weights in shared memory (exact: an E2M1 value
+ *     times 2^(s - 127) has two significant bits; bf16 holds it for 2 <= s <= 252, and for
+ *     smaller s as a subnormal down to 2^-133) and multiplied with the bf16 activations on
+ *     tcgen05 (fp32 accumulate): the pages' W4A16 as written.
+ *   - weight streaming: the products take the E2M1 values (exact in f16) and the activations
+ *     converted from bf16 to f16, exact for magnitudes 2^-14 .. 65504 (smaller ones keep fewer
+ *     bits); each 32-element block's fp32 result is scaled by its E8M0 factor in fp32.  An
+ *     input beyond 65504 in magnitude would become infinite there: the call then flags it and
+ *     the next moe_sync_status returns MOE_ERR_UNSUPPORTED (use MOE_PATH_TILE for such inputs).
+ * workspace: at least moe_workspace_bytes_mxfp4(ctx, T) bytes (it depends on the path setting).
+ * T = 0 is a no-op. */
 MOE_API size_t moe_workspace_bytes_mxfp4(moe_t ctx, int T);
 MOE_API moe_status moe_forward_mxfp4(moe_t ctx, int T, const void* x_bf16,
                                      const void* W_router_bf16, const float* b_router,
@@ -232,7 +240,8 @@ MOE_API moe_status moe_tune(moe_t ctx, int T_max, const void* x_bf16, const void
 /* Synchronise `stream`, then read and clear the handle's device status word.  Returns
  * MOE_ERR_TIMEOUT if a device-side bounded wait gave up since the last call, MOE_ERR_ARG if a
  * kernel met an index or count outside its buffers (moe_permute, moe_experts, moe_combine),
- * MOE_ERR_CUDA if the stream reports an error, MOE_OK otherwise. */
+ * MOE_ERR_UNSUPPORTED if an MXFP4 streaming call met an input beyond f16's range, MOE_ERR_CUDA if
+ * the stream reports an error, MOE_OK otherwise. */
 MOE_API moe_status moe_sync_status(moe_t ctx, moe_stream_t stream);
 
 /* Static text for a status code ("unknown status" for values outside the enum). */

@@ -12,6 +12,7 @@ namespace moe {
 
 // Device status word bits (the handle's status word).
 constexpr uint32_t kStatusTimeout = 1u;
+constexpr uint32_t kStatusF16Range = 8u;  // an MXFP4 streaming input beyond f16's range
 
 // A bounded wait gives up after this many nanoseconds of %globaltimer.
 constexpr uint64_t kWaitLimitNs = 2000000000ull;  // 2 s

@@ -81,6 +81,84 @@ MOE_DEVINL int et_boxes(int j, int n0, int Ncols) {
   return j == 0 ? min(2, vc) : max(0, vc - 2);
 }
 
+// Epilogue of the expert-tile kernels (warps 2-5, one TMEM lane quarter each): waits for each
+// tile's accumulators, writes h = silu(g) * u (gate/up) or adds w * y into out (down) through a
+// shared-memory transpose, and hands the accumulator buffer back.
+template <int MODE>
+MOE_DEVINL void et_epilogue(const EtArgs& a, uint32_t tmem_base, uint64_t* acc_full,
+                            uint64_t* acc_empty, float* epi, int tiles, int NT,
+                            volatile int* abort_flag) {
+  constexpr int TW = MODE == 0 ? kEtM : 2 * kEtM;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int q = warp & 3;                       // TMEM lanes 32q .. 32q + 31
+  float* stage = epi + (warp - 2) * 32 * kEtPitch;
+  int tile_i = 0;
+  for (int t = blockIdx.x; t < tiles; t += gridDim.x, ++tile_i) {
+    const int buf = tile_i & 1;
+    const uint32_t aph = (tile_i >> 1) & 1u;
+    if (!wait_or_abort(&acc_full[buf], aph, abort_flag, a.status)) break;
+    tc_fence_after();
+    const int4 ch = a.chunks[t / NT];
+    const int n0 = (t % NT) * TW;
+    const int nrows = ch.z;
+    const uint32_t tbase = tmem_base + ((uint32_t)(32 * q) << 16) + buf * 2 * kEtM;
+    if constexpr (MODE == 0) {
+      // this warp's 32 columns of gate and up: valid when the tile's last box is
+      const bool cols_ok = n0 + 32 * q < a.Ncols;  // warp-uniform
+      for (int r0 = 0; cols_ok && r0 < nrows; r0 += 32) {
+        float g[32], u[32];
+        tmem_ld32(tbase + r0, g);
+        tmem_ld32(tbase + kEtM + r0, u);
+#pragma unroll
+        for (int i = 0; i < 32; ++i) stage[i * kEtPitch + lane] = silu_fast(g[i]) * u[i];
+        __syncwarp();
+        // rows r0 + rr, 8 columns (16 bytes of h) per lane
+#pragma unroll
+        for (int it2 = 0; it2 < 4; ++it2) {
+          const int rr = (lane >> 2) + 8 * it2, cc = 8 * (lane & 3);
+          if (r0 + rr < nrows) {
+            const float* sp = stage + rr * kEtPitch + cc;
+            const uint4 v = make_uint4(pack_bf16x2(sp[0], sp[1]), pack_bf16x2(sp[2], sp[3]),
+                                       pack_bf16x2(sp[4], sp[5]), pack_bf16x2(sp[6], sp[7]));
+            *reinterpret_cast<uint4*>(a.h + (size_t)(ch.y + r0 + rr) * a.Ncols + n0 + 32 * q + cc) = v;
+          }
+        }
+        __syncwarp();
+      }
+    } else {
+#pragma unroll 1
+      for (int j = 0; j < 2; ++j) {
+        const int col0 = n0 + j * kEtM + 32 * q;
+        if (col0 >= a.Ncols) continue;  // warp-uniform: columns past H
+        for (int r0 = 0; r0 < nrows; r0 += 32) {
+          float y[32];
+          tmem_ld32(tbase + j * kEtM + r0, y);
+          const bool rv = r0 + lane < nrows;
+          const int tok = rv ? a.perm[ch.y + r0 + lane] : -1;
+          const float w = rv ? a.row_w[ch.y + r0 + lane] : 0.f;
+#pragma unroll
+          for (int i = 0; i < 32; ++i)
+            stage[i * kEtPitch + lane] = __shfl_sync(0xffffffffu, w, i) * y[i];
+          __syncwarp();
+          // rows r0 + rr, 4 columns (one 16-byte vector atomic) per lane
+#pragma unroll
+          for (int it2 = 0; it2 < 8; ++it2) {
+            const int rr = (lane >> 3) + 4 * it2, cc = 4 * (lane & 7);
+            const int tk = __shfl_sync(0xffffffffu, tok, rr);
+            if (tk >= 0) {
+              const float* sp = stage + rr * kEtPitch + cc;
+              red_add_f32x4(a.out + (size_t)tk * a.H + col0 + cc, sp[0], sp[1], sp[2], sp[3]);
+            }
+          }
+          __syncwarp();
+        }
+      }
+    }
+    tc_fence_before();
+    mbar_arrive(&acc_empty[buf]);
+  }
+}
+
 // MODE 0: gate/up projection with the SwiGLU epilogue.  MODE 1: down projection with the
 // routing-weight + combine epilogue.  wmap: the weights as [E*K rows, columns], box 64 x 64,
 // 128-byte swizzle.  xmap: the activation rows [R, K], box 16 x 64, 128-byte swizzle.
@@ -236,73 +314,7 @@ __global__ void __launch_bounds__(kEtThreads, 1)
     }
   } else {
     // ------------------------------ epilogue ------------------------------
-    const int q = warp & 3;                       // TMEM lanes 32q .. 32q + 31
-    float* stage = epi + (warp - 2) * 32 * kEtPitch;
-    int tile_i = 0;
-    for (int t = blockIdx.x; t < tiles; t += gridDim.x, ++tile_i) {
-      const int buf = tile_i & 1;
-      const uint32_t aph = (tile_i >> 1) & 1u;
-      if (!wait_or_abort(&acc_full[buf], aph, abort_flag, a.status)) break;
-      tc_fence_after();
-      const int4 ch = a.chunks[t / NT];
-      const int n0 = (t % NT) * TW;
-      const int nrows = ch.z;
-      const uint32_t tbase = tmem_base + ((uint32_t)(32 * q) << 16) + buf * 2 * kEtM;
-      if constexpr (MODE == 0) {
-        // this warp's 32 columns of gate and up: valid when the tile's last box is
-        const bool cols_ok = n0 + 32 * q < a.Ncols;  // warp-uniform
-        for (int r0 = 0; cols_ok && r0 < nrows; r0 += 32) {
-          float g[32], u[32];
-          tmem_ld32(tbase + r0, g);
-          tmem_ld32(tbase + kEtM + r0, u);
-#pragma unroll
-          for (int i = 0; i < 32; ++i) stage[i * kEtPitch + lane] = silu_fast(g[i]) * u[i];
-          __syncwarp();
-          // rows r0 + rr, 8 columns (16 bytes of h) per lane
-#pragma unroll
-          for (int it2 = 0; it2 < 4; ++it2) {
-            const int rr = (lane >> 2) + 8 * it2, cc = 8 * (lane & 3);
-            if (r0 + rr < nrows) {
-              const float* sp = stage + rr * kEtPitch + cc;
-              const uint4 v = make_uint4(pack_bf16x2(sp[0], sp[1]), pack_bf16x2(sp[2], sp[3]),
-                                         pack_bf16x2(sp[4], sp[5]), pack_bf16x2(sp[6], sp[7]));
-              *reinterpret_cast<uint4*>(a.h + (size_t)(ch.y + r0 + rr) * a.Ncols + n0 + 32 * q + cc) = v;
-            }
-          }
-          __syncwarp();
-        }
-      } else {
-#pragma unroll 1
-        for (int j = 0; j < 2; ++j) {
-          const int col0 = n0 + j * kEtM + 32 * q;
-          if (col0 >= a.Ncols) continue;  // warp-uniform: columns past H
-          for (int r0 = 0; r0 < nrows; r0 += 32) {
-            float y[32];
-            tmem_ld32(tbase + j * kEtM + r0, y);
-            const bool rv = r0 + lane < nrows;
-            const int tok = rv ? a.perm[ch.y + r0 + lane] : -1;
-            const float w = rv ? a.row_w[ch.y + r0 + lane] : 0.f;
-#pragma unroll
-            for (int i = 0; i < 32; ++i)
-              stage[i * kEtPitch + lane] = __shfl_sync(0xffffffffu, w, i) * y[i];
-            __syncwarp();
-            // rows r0 + rr, 4 columns (one 16-byte vector atomic) per lane
-#pragma unroll
-            for (int it2 = 0; it2 < 8; ++it2) {
-              const int rr = (lane >> 3) + 4 * it2, cc = 4 * (lane & 7);
-              const int tk = __shfl_sync(0xffffffffu, tok, rr);
-              if (tk >= 0) {
-                const float* sp = stage + rr * kEtPitch + cc;
-                red_add_f32x4(a.out + (size_t)tk * a.H + col0 + cc, sp[0], sp[1], sp[2], sp[3]);
-              }
-            }
-            __syncwarp();
-          }
-        }
-      }
-      tc_fence_before();
-      mbar_arrive(&acc_empty[buf]);
-    }
+    et_epilogue<MODE>(a, tmem_base, acc_full, acc_empty, epi, tiles, NT, abort_flag);
   }
 
   tc_fence_before();

@@ -19,6 +19,7 @@
 #include "stream_mx.cuh"
 #include "gemm.cuh"
 #include "expert_gemm.cuh"
+#include "expert_gemm_mx.cuh"
 #include "ep.cuh"
 
 using namespace moe;
@@ -62,6 +63,7 @@ struct moe_ctx {
   MapCache gate_up_stream, down_stream, gate_up_gemm, down_gemm, x_perm_map, h_map;
   MapCache et_x_map, et_h_map;  // activation rows for the expert-tile kernel (16-row boxes)
   MapCache gu_codes, gu_scales, dn_codes, dn_scales;  // MXFP4 weights (streaming path)
+  MapCache gu_codes_t, gu_scales_t, dn_codes_t, dn_scales_t;  // MXFP4 weights (expert tiles)
   int device = 0;
   int num_sms = 148;
   moe_path path = MOE_PATH_AUTO;
@@ -237,8 +239,18 @@ Plan make_plan(const moe_ctx* c, int T, bool mx, moe_path path) {
     p.has[f] = true;
     p.max_count[f] = INT_MAX;
   };
-  if (mx) {  // MXFP4 experts: streaming kernels only
-    only(kFamStream);
+  if (mx) {  // MXFP4 experts: weight streaming and expert tiles (no MXFP4 row-tile GEMM)
+    if (path == MOE_PATH_STREAM) {
+      only(kFamStream);
+    } else if (path == MOE_PATH_TILE || path == MOE_PATH_GEMM) {
+      only(kFamTile);
+    } else {
+      const int s = c->stream_rows;
+      p.has[kFamStream] = s > 0;
+      p.max_count[kFamStream] = T > s ? s : INT_MAX;
+      p.has[kFamTile] = T > s;
+      p.max_count[kFamTile] = INT_MAX;
+    }
     return p;
   }
   switch (path) {
@@ -506,6 +518,10 @@ bool set_smem_attrs() {
                              kEtSmem) == cudaSuccess;
   ok &= cudaFuncSetAttribute(expert_tile_kernel<1>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              kEtSmem) == cudaSuccess;
+  ok &= cudaFuncSetAttribute(expert_tile_mx_kernel<0>,
+                             cudaFuncAttributeMaxDynamicSharedMemorySize, kEmxSmem) == cudaSuccess;
+  ok &= cudaFuncSetAttribute(expert_tile_mx_kernel<1>,
+                             cudaFuncAttributeMaxDynamicSharedMemorySize, kEmxSmem) == cudaSuccess;
   ok &= cudaFuncSetAttribute(build_segment_lists_kernel,
                              cudaFuncAttributeMaxDynamicSharedMemorySize,
                              (3 * kMaxSegments + kMaxE) * 4) == cudaSuccess;
@@ -592,7 +608,7 @@ moe_status expert_phase(moe_ctx* c, const Plan& p, const ExpertIO& io, const voi
   }
   const CUtensorMap* wgu = nullptr;
   const CUtensorMap* wdn = nullptr;
-  if (p.has[kFamTile] || p.has[kFamGemm]) {
+  if (!mx && (p.has[kFamTile] || p.has[kFamGemm])) {
     wgu = cached_map(c->gate_up_gemm, W_gate_up_bf16, (uint64_t)c->E * c->H, 2ull * c->I,
                      kGemmBK, 64);
     wdn = cached_map(c->down_gemm, W_down_bf16, (uint64_t)c->E * c->I, (uint64_t)c->H,
@@ -602,6 +618,14 @@ moe_status expert_phase(moe_ctx* c, const Plan& p, const ExpertIO& io, const voi
   if (p.has[kFamTile]) {
     const CUtensorMap* xm = cached_map(c->et_x_map, io.x_perm, R, (uint64_t)c->H, kEtRowBox, 64);
     if (!xm) return MOE_ERR_CUDA;
+    const CUtensorMap *cm = nullptr, *sm = nullptr;
+    if (mx) {  // codes [E*2I, H/2] in 128 x 32-byte boxes, scales [E*H/32, 2I] in 2 x 128 boxes
+      cm = cached_map_u8(c->gu_codes_t, mx->gu_codes, 2ull * c->I * c->E, (uint64_t)c->H / 2,
+                         kEtM, kEtBK / 2, CU_TENSOR_MAP_SWIZZLE_NONE);
+      sm = cached_map_u8(c->gu_scales_t, mx->gu_scales, (uint64_t)c->E * (c->H / 32),
+                         2ull * c->I, kEtBK / 32, kEtM, CU_TENSOR_MAP_SWIZZLE_NONE);
+      if (!cm || !sm) return MOE_ERR_CUDA;
+    }
     EtArgs e{};
     e.K = c->H;
     e.Ncols = c->I;
@@ -616,6 +640,9 @@ moe_status expert_phase(moe_ctx* c, const Plan& p, const ExpertIO& io, const voi
       e.n_zero4 = io.out_elems / 4;
     }
     MOE_TRY(launch(c, kKindGateUpTile, st, [&] {
+      if (mx)
+        return launch_pdl(expert_tile_mx_kernel<0>, dim3(c->num_sms), dim3(kEmxThreads),
+                          kEmxSmem, st, e, *cm, *sm, *xm);
       return launch_pdl(expert_tile_kernel<0>, dim3(c->num_sms), dim3(kEtThreads), kEtSmem, st,
                         e, *wgu, *xm);
     }));
@@ -680,6 +707,14 @@ moe_status expert_phase(moe_ctx* c, const Plan& p, const ExpertIO& io, const voi
   if (p.has[kFamTile]) {
     const CUtensorMap* hm = cached_map(c->et_h_map, io.h, R, (uint64_t)c->I, kEtRowBox, 64);
     if (!hm) return MOE_ERR_CUDA;
+    const CUtensorMap *cm = nullptr, *sm = nullptr;
+    if (mx) {  // codes [E*H, I/2], scales [E*I/32, H]
+      cm = cached_map_u8(c->dn_codes_t, mx->dn_codes, (uint64_t)c->H * c->E, (uint64_t)c->I / 2,
+                         kEtM, kEtBK / 2, CU_TENSOR_MAP_SWIZZLE_NONE);
+      sm = cached_map_u8(c->dn_scales_t, mx->dn_scales, (uint64_t)c->E * (c->I / 32),
+                         (uint64_t)c->H, kEtBK / 32, kEtM, CU_TENSOR_MAP_SWIZZLE_NONE);
+      if (!cm || !sm) return MOE_ERR_CUDA;
+    }
     EtArgs e{};
     e.K = c->I;
     e.Ncols = c->H;
@@ -692,6 +727,9 @@ moe_status expert_phase(moe_ctx* c, const Plan& p, const ExpertIO& io, const voi
     e.H = c->H;
     e.status = c->d_status;
     MOE_TRY(launch(c, kKindDownTile, st, [&] {
+      if (mx)
+        return launch_pdl(expert_tile_mx_kernel<1>, dim3(c->num_sms), dim3(kEmxThreads),
+                          kEmxSmem, st, e, *cm, *sm, *hm);
       return launch_pdl(expert_tile_kernel<1>, dim3(c->num_sms), dim3(kEtThreads), kEtSmem, st,
                         e, *wdn, *hm);
     }));
@@ -765,11 +803,11 @@ moe_status forward_plan(moe_ctx* c, int T, const void* x_bf16, const void* W_rou
   const uint16_t* x = static_cast<const uint16_t*>(x_bf16);
   uint16_t* x16 = mx ? reinterpret_cast<uint16_t*>(ws + L.x16) : nullptr;
   uint16_t* x_perm = L.x_perm ? reinterpret_cast<uint16_t*>(ws + L.x_perm) : nullptr;
-  if (mx) {  // the MXFP4 kernels take f16 activations
+  if (mx && p.has[kFamStream]) {  // the MXFP4 streaming kernels take f16 activations
     const size_t n = (size_t)T * c->H;
     const int blocks = (int)std::min<size_t>((n / 8 + 255) / 256, (size_t)c->num_sms * 4);
     MOE_TRY(launch(c, kKindConvert, st, [&] {
-      return launch_pdl(to_f16_kernel, dim3(blocks), dim3(256), 0, st, x, x16, n);
+      return launch_pdl(to_f16_kernel, dim3(blocks), dim3(256), 0, st, x, x16, n, c->d_status);
     }));
   }
   // With enough 64-token blocks to cover the GPU the scatter also writes the rows in expert
@@ -1167,6 +1205,7 @@ moe_status moe_sync_status(moe_t c, moe_stream_t stream) {
     if (cudaMemset(c->d_status, 0, sizeof(word)) != cudaSuccess) return MOE_ERR_CUDA;
     if (word & kStatusTimeout) return MOE_ERR_TIMEOUT;
     if (word & (kStatusBadIndex | kStatusBadCounts)) return MOE_ERR_ARG;
+    if (word & kStatusF16Range) return MOE_ERR_UNSUPPORTED;
   }
   return MOE_OK;
 }

@@ -89,10 +89,12 @@ MOE_DEVINL uint32_t pack_f16x2(float lo, float hi) {
   return r;
 }
 
-// The layer input in f16 for the MXFP4 kernels: x16[i] = f16(x[i]) for n elements (n even).
-// grid-stride, 8 elements per thread and step.
+// The layer input in f16 for the MXFP4 streaming kernels: x16[i] = f16(x[i]) for n elements
+// (n even).  An input beyond f16's range sets kStatusF16Range in the status word (its f16 value
+// is infinite).  grid-stride, 8 elements per thread and step.
 __global__ void __launch_bounds__(256) to_f16_kernel(const uint16_t* __restrict__ x,
-                                                     uint16_t* __restrict__ x16, size_t n) {
+                                                     uint16_t* __restrict__ x16, size_t n,
+                                                     uint32_t* status) {
   pdl_wait();  // x16 may still be read by the previous call's gate/up kernel until it ends
   pdl_launch_next();
   const size_t n8 = n / 8;
@@ -101,9 +103,14 @@ __global__ void __launch_bounds__(256) to_f16_kernel(const uint16_t* __restrict_
     const uint4 v = reinterpret_cast<const uint4*>(x)[i];
     const uint32_t in[4] = {v.x, v.y, v.z, v.w};
     uint32_t o[4];
+    bool big = false;
 #pragma unroll
-    for (int j = 0; j < 4; ++j)
-      o[j] = pack_f16x2(__uint_as_float(in[j] << 16), __uint_as_float(in[j] & 0xffff0000u));
+    for (int j = 0; j < 4; ++j) {
+      const float lo = __uint_as_float(in[j] << 16), hi = __uint_as_float(in[j] & 0xffff0000u);
+      big |= fabsf(lo) > 65504.f || fabsf(hi) > 65504.f;   // beyond f16: would become inf
+      o[j] = pack_f16x2(lo, hi);
+    }
+    if (big) atomicOr(status, kStatusF16Range);
     reinterpret_cast<uint4*>(x16)[i] = make_uint4(o[0], o[1], o[2], o[3]);
   }
 }

@@ -1,4 +1,6 @@
-"""GPU parity of the MXFP4 (W4A16) streaming path against the oracle's dequantized layer.
+"""GPU parity of the MXFP4 (W4A16) layer against the oracle's dequantized layer: the weight-
+streaming kernels (f16 activations) and the expert-tile kernel (codes widened to bf16 weights on
+chip, bf16 activations), alone and mixed per expert.
 
 Routing must be bit-exact apart from reported near ties (it does not involve the expert
 weights); outputs must satisfy |gpu - oracle| <= 1e-2 + 2e-2 |oracle| per element, the bound
@@ -44,12 +46,14 @@ class _LazyWeights(dict):
         return self[key]
 
 
-def _run_mx(T, H, E, k, I, seed, sample=None, edit=None):
+def _run_mx(T, H, E, k, I, seed, sample=None, edit=None, path=None):
     d = mi.make_inputs(T, H, E, k, I, seed, device="cuda", weights="mxfp4")
     if edit is not None:
         edit(d)
     h = _LazyWeights(mi.host_inputs(d))
     layer = moe.Moe(E, H, I, k)
+    if path is not None:
+        layer.set_path(path)
     ref_route = host_route(h, k)
     g = gpu_route(layer, d)
     rep = compare_routing(g, ref_route, k, E)
@@ -82,15 +86,16 @@ def test_gpt_oss_shape_more_tokens():
 
 def test_extreme_scales():
     """E8M0 codes far from the others in some blocks (0 = 2^-127, an fp32 subnormal; 2^-37;
-    32 times the usual scale): the block scale is applied in fp32, after the tensor-core
-    products.  (Far larger scales make h so large that the bf16 rounding of h, which the
-    oracle does not do, shows through cancellation in the down projection.)"""
+    32 times the usual scale) on the streaming kernels: the block scale is applied in fp32,
+    after the tensor-core products.  (Far larger scales make h so large that its f16 rounding
+    on this path, which the oracle does not do, shows through cancellation in the down
+    projection.)"""
     def edit(d):
         s0 = int(d["gu_scales"].float().mean().round())
         d["gu_scales"][:, 0, :7] = 0
         d["gu_scales"][:, 1, 3:9] = s0 + 5
         d["dn_scales"][:, 2, :5] = 90
-    _run_mx(12, 256, 4, 2, 256, 300, edit=edit)
+    _run_mx(12, 256, 4, 2, 256, 300, edit=edit, path=moe.MOE_PATH_STREAM)
 
 
 def test_zero_tokens_and_bad_calls():
@@ -111,6 +116,54 @@ def test_120b_shape_eight_tokens():
 
 
 def test_many_chunks_and_split_k():
-    """300 tokens x 2 of 8 experts: tens of 16-row chunks per expert, stream-K pieces that share
-    a tile's K range meet in the fp32 accumulator."""
-    _run_mx(300, 512, 8, 2, 704, 42, sample=64)
+    """300 tokens x 2 of 8 experts on the streaming kernels: tens of 16-row chunks per expert,
+    stream-K pieces that share a tile's K range meet in the fp32 accumulator."""
+    _run_mx(300, 512, 8, 2, 704, 42, sample=64, path=moe.MOE_PATH_STREAM)
+
+
+@pytest.mark.parametrize("T", [1, 17, 40, 129, 300])
+def test_expert_tiles_ragged(T):
+    """Every expert on the MXFP4 expert-tile kernel: 1..16 rows per box, one or two 128-row
+    chunks, a 64-column last gate/up block (I = 320), scale blocks on both sides of each stage."""
+    _run_mx(T, 256, 8, 2, 320, 500 + T, path=moe.MOE_PATH_TILE)
+
+
+def test_expert_tiles_extreme_scales():
+    """The scales of test_extreme_scales on the expert-tile kernel: widened to bf16 exactly
+    (2^-127 times an E2M1 value is a bf16 subnormal)."""
+    def edit(d):
+        s0 = int(d["gu_scales"].float().mean().round())
+        d["gu_scales"][:, 0, :7] = 0
+        d["gu_scales"][:, 1, 3:9] = s0 + 5
+        d["dn_scales"][:, 2, :5] = 90
+    _run_mx(12, 256, 4, 2, 256, 300, edit=edit, path=moe.MOE_PATH_TILE)
+
+
+@pytest.mark.parametrize("T", [64, 512])
+def test_auto_mixes_streaming_and_expert_tiles_gpt_oss_shape(T):
+    """20b shape: at 64 tokens most experts stream and a few take tiles; at 512 all take tiles."""
+    _run_mx(T, 2880, 32, 4, 2880, 600 + T, sample=48)
+
+
+def test_gemm_path_means_expert_tiles_for_mxfp4():
+    _run_mx(100, 256, 8, 2, 256, 650, path=moe.MOE_PATH_GEMM)
+
+
+def test_inputs_beyond_f16_range():
+    """|x| > 65504: the streaming kernels' f16 activations cannot hold it; the call reports it
+    (moe_sync_status: MOE_ERR_UNSUPPORTED) and the expert-tile kernel, whose activations stay
+    bf16, computes the layer exactly as the oracle does."""
+    def edit(d):
+        d["x"][3, 5] = 1.0e5
+        d["x"][7, 100] = -3.0e6
+
+    E, H, I, k, T = 8, 256, 256, 2, 12
+    d = mi.make_inputs(T, H, E, k, I, 660, device="cuda", weights="mxfp4")
+    edit(d)
+    layer = moe.Moe(E, H, I, k)
+    layer.set_path(moe.MOE_PATH_STREAM)
+    layer.forward_mxfp4(d["x"], d["W_router"], d["b_router"], d["gu_codes"], d["gu_scales"],
+                        d["dn_codes"], d["dn_scales"])
+    assert layer.sync_status() == moe.MOE_ERR_UNSUPPORTED
+    assert layer.sync_status() == moe.MOE_OK
+    _run_mx(T, H, E, k, I, 660, edit=edit, path=moe.MOE_PATH_TILE)
