@@ -358,6 +358,8 @@ def run_ours(args, w: mi.Workload, T: int) -> None:
     if rank:
         d["x"] = mi.draw_x(T, w.H, seed, "cuda")
     layer = moe.Moe(w.E, w.H, w.I, w.k)
+    layer.set_path({"auto": moe.MOE_PATH_AUTO, "stream": moe.MOE_PATH_STREAM,
+                    "tile": moe.MOE_PATH_TILE, "gemm": moe.MOE_PATH_GEMM}[args.path])
     counts = torch.diff(layer.route(d["x"], d["W_router"], d["b_router"])["expert_offsets"]).cpu().tolist()
     alg = algorithmic(T, w.H, w.E, w.k, w.I, counts, w.weights)
     out = torch.empty((T, w.H), dtype=torch.float32, device="cuda")
@@ -498,6 +500,8 @@ def main(argv=None):
     ap.add_argument("--workload", default="131k_skewed", choices=sorted(mi.WORKLOADS))
     ap.add_argument("--T", type=int, default=None)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--path", default="auto", choices=["auto", "stream", "tile", "gemm"],
+                    help="kernel family for every expert (default: chosen per expert)")
     args = ap.parse_args(argv)
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")

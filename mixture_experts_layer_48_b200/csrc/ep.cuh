@@ -85,7 +85,7 @@ constexpr int kMaxSegments = 4096;  // sources x experts of one expert-half call
 // over all sources); every block writes part of the identity row map perm[r] = r and zeroes the
 // completion counters.  Counts that do not add up to R are reported in the status word; rows
 // past R are never listed.  Also zero-fills zero4[0, n_zero4).  block 1024; dynamic smem
-// (3*S*E + E) ints.
+// (4*S*E + E) ints.
 __global__ void __launch_bounds__(1024)
     build_segment_lists_kernel(const int32_t* __restrict__ seg_counts, int S, int E, int R,
                                RouteOut o, int32_t* __restrict__ perm_iota, float4* zero4,
@@ -95,7 +95,8 @@ __global__ void __launch_bounds__(1024)
   int32_t* seg_off = seg_smem;   // [n] first row of each segment
   int32_t* cnt = seg_off + n;    // [n] rows of each segment inside [0, R)
   int32_t* base = cnt + n;       // [n] first work-list entry of each segment
-  int32_t* total = base + n;     // [E] rows of each expert over all sources
+  int32_t* rbase = base + n;     // [n] first row of each segment among its list's rows
+  int32_t* total = rbase + n;    // [E] rows of each expert over all sources
   const int tid = threadIdx.x;
   pdl_wait();
   pdl_launch_next();
@@ -124,12 +125,14 @@ __global__ void __launch_bounds__(1024)
   // thread l < n_lists: exclusive scan of list l's entries over the segments in order
   if (tid < o.n_lists) {
     const WorkList& L = o.wl[tid];
-    int run = 0;
+    int run = 0, rows = 0;
     for (int i = 0; i < n; ++i) {
       const int tot = total[i % E];
       if (tot > L.min_count && tot <= L.max_count) {
         base[i] = run;
+        rbase[i] = rows;
         run += (cnt[i] + L.chunk_rows - 1) / L.chunk_rows;
+        rows += cnt[i];
       }
     }
     L.sched[0] = run;
@@ -143,7 +146,7 @@ __global__ void __launch_bounds__(1024)
       if (tot > L.min_count && tot <= L.max_count) {
         int b = base[i];
         for (int r0 = 0; r0 < c; r0 += L.chunk_rows)
-          L.chunks[b++] = make_int4(e, seg_off[i] + r0, min(L.chunk_rows, c - r0), 0);
+          L.chunks[b++] = make_int4(e, seg_off[i] + r0, min(L.chunk_rows, c - r0), rbase[i] + r0);
         break;
       }
     }

@@ -312,7 +312,11 @@ Layout make_layout(const moe_ctx* c, int T, const Plan& p, bool mx) {
     const int tile_cols = std::min(kStreamCols, kMxTileCols);
     L.n_done = n * ((c->I + tile_cols - 1) / tile_cols);
     L.done = cv.take(4 * (size_t)L.n_done);
-    L.acc_floats = (size_t)n * kStreamRB * 2 * c->I;  // split-K sums per chunk row
+    // split-K sums of the streaming family's rows (each entry carries its rows' first index)
+    const long long srows = p.max_count[kFamStream] == INT_MAX
+                                ? (long long)R
+                                : std::min((long long)R, (long long)c->E * p.max_count[kFamStream]);
+    L.acc_floats = (size_t)srows * 2 * c->I;
     L.acc = cv.take(sizeof(float) * L.acc_floats);
   }
   L.h = cv.take(2 * R * c->I);
@@ -339,7 +343,10 @@ Layout make_expert_layout(const moe_ctx* c, int R, int S, const Plan& p) {
         const int tile_cols = std::min(kStreamCols, kMxTileCols);
         L.n_done = (int)(n * ((c->I + tile_cols - 1) / tile_cols));
         L.done = cv.take(4 * (size_t)L.n_done);
-        L.acc_floats = (size_t)n * kStreamRB * 2 * c->I;
+        const long long srows = p.max_count[f] == INT_MAX
+                                    ? (long long)R
+                                    : std::min((long long)R, (long long)c->E * p.max_count[f]);
+        L.acc_floats = (size_t)srows * 2 * c->I;
         L.acc = cv.take(sizeof(float) * L.acc_floats);
       }
     }
@@ -431,7 +438,7 @@ moe_status launch_route(moe_ctx* c, int T, const uint16_t* x, const uint16_t* Wr
       return launch_router_tc<32>(1, st, x, Wr, b, T, H, E, k, o, nullptr, zero4, n_zero4, rt, partial);
     }));
     const size_t smem_f = (size_t)T * E * 4 + (size_t)T * k * 4 + (size_t)T * 8 * 4 +
-                          (256 + 257 + 257) * 4;
+                          (256 + 257 + 512) * 4;
     MOE_TRY(launch(c, kKindRouteFin, st, [&] {
       return launch_pdl(route_small_finalize_kernel, dim3(1), dim3(1024), smem_f, st,
                         (const float*)partial, rt.splits, b, T, E, k, o);
@@ -470,7 +477,7 @@ moe_status launch_route(moe_ctx* c, int T, const uint16_t* x, const uint16_t* Wr
   MOE_TRY(launch(c, kKindRouteFin, st, [&] {
     return launch_pdl(route_scan_kernel, dim3(E), dim3(256), 0, st, block_counts, NB, E, totals);
   }));
-  const size_t smem_s = (256 + 257 + 257) * 4 + (size_t)kRouterTcTokens * 8 * 4 +
+  const size_t smem_s = (256 + 257 + 512) * 4 + (size_t)kRouterTcTokens * 8 * 4 +
                         (size_t)kRouterTcTokens * E;
   MOE_TRY(launch(c, kKindRouteFin, st, [&] {
     return launch_pdl(route_scatter_kernel, dim3(NB), dim3(256), smem_s, st,
@@ -524,7 +531,7 @@ bool set_smem_attrs() {
                              cudaFuncAttributeMaxDynamicSharedMemorySize, kEmxSmem) == cudaSuccess;
   ok &= cudaFuncSetAttribute(build_segment_lists_kernel,
                              cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             (3 * kMaxSegments + kMaxE) * 4) == cudaSuccess;
+                             (4 * kMaxSegments + kMaxE) * 4) == cudaSuccess;
   return ok;
 }
 
@@ -1058,7 +1065,7 @@ moe_status moe_experts(moe_t c, int R, int S, const int32_t* seg_counts, const v
   plan_lists(p, L, ws, o, io);
   int32_t* iota = reinterpret_cast<int32_t*>(ws + L.perm);
   const int grid = (int)std::max<long long>(1, std::min<long long>(c->num_sms, (R + 1023) / 1024));
-  const size_t smem = (size_t)(3 * S * c->E + c->E) * 4;
+  const size_t smem = (size_t)(4 * S * c->E + c->E) * 4;
   moe_status s = launch(c, kKindRouteFin, st, [&] {
     return launch_pdl(build_segment_lists_kernel, dim3(grid), dim3(1024), smem, st, seg_counts,
                       S, c->E, R, o, iota, reinterpret_cast<float4*>(io.acc), L.acc_floats / 4,

@@ -253,13 +253,17 @@ MOE_DEVINL void zero_fill_f4(float4* z, size_t n4) {
 
 // Work lists of one routing: expert e (with count c > 0) belongs to the list whose
 // (min_count, max_count] holds c, and its rows are split there into entries of at most
-// chunk_rows rows, in expert order.  Called by all threads of a block with count/off in
-// shared memory (E <= 256 entries); scratch holds [256] ints of shared memory.
+// chunk_rows rows, in expert order.  Each entry is {expert, first row, rows, first row among
+// the list's rows} (the last field lets a kernel keep per-row scratch for its own rows only).
+// Called by all threads of a block with count/off in shared memory (E <= 256 entries);
+// scratch holds [512] ints of shared memory.
 MOE_DEVINL void build_work_lists(const int32_t* cnt, const int32_t* off, int E,
                                  const RouteOut& o, int32_t* scratch) {
   const int tid = threadIdx.x;
   if (o.n_lists == 0) return;
-  // warp l < n_lists: exclusive scan of list l's chunk counts, in expert order
+  int32_t* chunk_base = scratch;        // [256] first entry of each expert in its list
+  int32_t* row_base = scratch + 256;    // [256] first row of each expert among its list's rows
+  // warp l < n_lists: exclusive scans of list l's entries and rows, in expert order
   const int warp = tid >> 5;
   if (warp < o.n_lists) {
     const WorkList& L = o.wl[warp];
@@ -267,8 +271,12 @@ MOE_DEVINL void build_work_lists(const int32_t* cnt, const int32_t* off, int E,
     const int total = warp_exclusive_scan(
         E, [&](int e) { return member(e) ? (cnt[e] + L.chunk_rows - 1) / L.chunk_rows : 0; },
         [&](int e, int pre) {
-          if (member(e)) scratch[e] = pre;
+          if (member(e)) chunk_base[e] = pre;
         });
+    warp_exclusive_scan(E, [&](int e) { return member(e) ? cnt[e] : 0; },
+                        [&](int e, int pre) {
+                          if (member(e)) row_base[e] = pre;
+                        });
     if ((tid & 31) == 0) L.sched[0] = total;
   }
   __syncthreads();
@@ -278,9 +286,9 @@ MOE_DEVINL void build_work_lists(const int32_t* cnt, const int32_t* off, int E,
     for (int i = 0; i < o.n_lists; ++i) {
       const WorkList& L = o.wl[i];
       if (c > L.min_count && c <= L.max_count) {
-        int base = scratch[e];
+        int base = chunk_base[e];
         for (int r0 = 0; r0 < c; r0 += L.chunk_rows)
-          L.chunks[base++] = make_int4(e, off[e] + r0, min(L.chunk_rows, c - r0), 0);
+          L.chunks[base++] = make_int4(e, off[e] + r0, min(L.chunk_rows, c - r0), row_base[e] + r0);
         break;
       }
     }
@@ -300,7 +308,7 @@ __global__ void __launch_bounds__(1024)
   uint32_t* bits = reinterpret_cast<uint32_t*>(sel + T * k);         // [T][8]
   int32_t* cnt = reinterpret_cast<int32_t*>(bits + T * 8);           // [256]
   int32_t* off = cnt + 256;                                          // [257]
-  int32_t* scratch = off + 257;                                      // [257]
+  int32_t* scratch = off + 257;                                      // [512]
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5, nwarps = blockDim.x >> 5;
   pdl_wait();
   pdl_launch_next();
@@ -644,8 +652,8 @@ __global__ void __launch_bounds__(256)
   extern __shared__ __align__(128) uint8_t smem_raw[];
   int32_t* cnt = reinterpret_cast<int32_t*>(smem_raw);  // [256]
   int32_t* off = cnt + 256;                             // [257]
-  int32_t* scratch = off + 257;                         // [257]
-  uint32_t* bits = reinterpret_cast<uint32_t*>(scratch + 257);  // [64][8]
+  int32_t* scratch = off + 257;                         // [512]
+  uint32_t* bits = reinterpret_cast<uint32_t*>(scratch + 512);  // [64][8]
   uint8_t* slot = reinterpret_cast<uint8_t*>(bits + TT * 8);    // [64][E] (k <= 256)
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int t0 = blockIdx.x * TT, nt = min(TT, T - t0);

@@ -72,9 +72,9 @@ struct GateUpArgs {
   const uint16_t* x;     // [T, H]
   int H, I, R;
   const int32_t* perm;   // [R]
-  const int4* chunks;    // work list
+  const int4* chunks;    // work list {expert, first row, rows, first row among the list's rows}
   const int32_t* sched;  // [0] chunk count
-  float* acc;            // [chunks * 16, 2I] gate | up sums per chunk row, zero on entry
+  float* acc;            // [rows of the list, 2I] gate | up sums (row = entry .w + r), zero on entry
   int32_t* done;         // [chunks * tiles] completion counters, zero on entry
   uint16_t* h;           // [R, I] bf16 SwiGLU output
   float* out;            // [T, H] zero-filled here
@@ -298,7 +298,7 @@ __global__ void __launch_bounds__(kStreamThreads, 1)
           const int cl = kBox * warp + 16 * mt + (lane >> 2) + 8 * (v >> 1);
           const int r = nb * 8 + 2 * (lane & 3) + (v & 1);
           if (r < nrows && cl < wg) {
-            float* p = a.acc + ((size_t)(unit / NT) * kStreamRB + r) * I2 + col0 + cl;
+            float* p = a.acc + ((size_t)ch.w + r) * I2 + col0 + cl;
             atomicAdd(p, accg[mt][nb][v]);
             atomicAdd(p + a.I, accu[mt][nb][v]);
           }
@@ -312,7 +312,7 @@ __global__ void __launch_bounds__(kStreamThreads, 1)
     if (s_last) {
       for (int i = ctid; i < nrows * (wg / 2); i += kStreamConsumers) {
         const int r = i / (wg / 2), cl = 2 * (i - r * (wg / 2));
-        const float* p = a.acc + ((size_t)(unit / NT) * kStreamRB + r) * I2 + col0 + cl;
+        const float* p = a.acc + ((size_t)ch.w + r) * I2 + col0 + cl;
         const float2 gs = __ldcg(reinterpret_cast<const float2*>(p));
         const float2 us = __ldcg(reinterpret_cast<const float2*>(p + a.I));
         *reinterpret_cast<uint32_t*>(a.h + (size_t)(ch.y + r) * a.I + col0 + cl) =

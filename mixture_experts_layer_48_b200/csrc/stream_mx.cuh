@@ -380,7 +380,7 @@ __global__ void __launch_bounds__(kMxThreads, 1)
         const int cl = kMxBoxRows * box + 16 * mt + (lane >> 2) + 8 * (v >> 1);
         const int r = nb * 8 + 2 * (lane & 3) + (v & 1);
         if (r < nrows && cl < wg) {
-          float* p = a.acc + ((size_t)(unit / NT) * kStreamRB + r) * I2 + col0 + cl;
+          float* p = a.acc + ((size_t)ch.w + r) * I2 + col0 + cl;
           atomicAdd(p, acc[0][nb][v]);
           atomicAdd(p + a.I, acc[1][nb][v]);
         }
@@ -394,7 +394,7 @@ __global__ void __launch_bounds__(kMxThreads, 1)
     if (s_last) {
       for (int i = ctid; i < nrows * (wg / 2); i += kMxConsumers) {
         const int r = i / (wg / 2), cl = 2 * (i - r * (wg / 2));
-        const float* p = a.acc + ((size_t)(unit / NT) * kStreamRB + r) * I2 + col0 + cl;
+        const float* p = a.acc + ((size_t)ch.w + r) * I2 + col0 + cl;
         const float2 gs = __ldcg(reinterpret_cast<const float2*>(p));
         const float2 us = __ldcg(reinterpret_cast<const float2*>(p + a.I));
         *reinterpret_cast<uint32_t*>(a.h + (size_t)(ch.y + r) * a.I + col0 + cl) =
