@@ -7,6 +7,7 @@
 #include <algorithm>
 #include <climits>
 #include <cstdint>
+#include <cstdlib>
 #include <cstring>
 #include <new>
 #include <utility>
@@ -18,6 +19,7 @@
 #include "stream.cuh"
 #include "stream_mx.cuh"
 #include "gemm.cuh"
+#include "gemm_wide.cuh"
 #include "expert_gemm.cuh"
 #include "expert_gemm_mx.cuh"
 #include "ep.cuh"
@@ -69,6 +71,7 @@ struct moe_ctx {
   moe_path path = MOE_PATH_AUTO;
   int stream_rows = kDefaultStreamRows;  // AUTO: experts with at most this many rows stream
   int tile_rows = kDefaultTileRows;      // ... up to this many take expert tiles; more: row tiles
+  bool wide_rows = false;                // row tiles 256 x 512 (two MMAs per K step) or 256 x 256
   uint32_t* d_status = nullptr;
   void* static_scratch = nullptr;  // device address of the routing scratch array (moe_route_static)
   uint64_t launches = 0;
@@ -521,6 +524,12 @@ bool set_smem_attrs() {
   ok &= cudaFuncSetAttribute(grouped_gemm_2sm_kernel<MOE_GEMM_DOWN>,
                              cudaFuncAttributeMaxDynamicSharedMemorySize,
                              Gemm2Cfg<kGemmStages>::kSmem) == cudaSuccess;
+  ok &= cudaFuncSetAttribute(grouped_gemm_wide_kernel<0>,
+                             cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             WideCfg<0>::kSmem) == cudaSuccess;
+  ok &= cudaFuncSetAttribute(grouped_gemm_wide_kernel<1>,
+                             cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             WideCfg<1>::kSmem) == cudaSuccess;
   ok &= cudaFuncSetAttribute(expert_tile_kernel<0>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              kEtSmem) == cudaSuccess;
   ok &= cudaFuncSetAttribute(expert_tile_kernel<1>, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -671,6 +680,9 @@ moe_status expert_phase(moe_ctx* c, const Plan& p, const ExpertIO& io, const voi
     g.zero4 = reinterpret_cast<float4*>(io.out);
     g.n_zero4 = io.out_elems / 4;
     MOE_TRY(launch(c, kKindGateUpGemm, st, [&] {
+      if (c->wide_rows)
+        return launch_pdl(grouped_gemm_wide_kernel<0>, dim3(pair_grid), dim3(kWideThreads),
+                          WideCfg<0>::kSmem, st, g, *am, *wgu);
       return launch_pdl(grouped_gemm_2sm_kernel<MOE_GEMM_GATE_UP>, dim3(pair_grid),
                         dim3(kGemmThreads), Gemm2Cfg<kGemmStages>::kSmem, st, g, *am, *wgu);
     }));
@@ -757,6 +769,9 @@ moe_status expert_phase(moe_ctx* c, const Plan& p, const ExpertIO& io, const voi
     d.H = c->H;
     d.status = c->d_status;
     MOE_TRY(launch(c, kKindDownGemm, st, [&] {
+      if (c->wide_rows)
+        return launch_pdl(grouped_gemm_wide_kernel<1>, dim3(pair_grid), dim3(kWideThreads),
+                          WideCfg<1>::kSmem, st, d, *hm, *wdn);
       return launch_pdl(grouped_gemm_2sm_kernel<MOE_GEMM_DOWN>, dim3(pair_grid),
                         dim3(kGemmThreads), Gemm2Cfg<kGemmStages>::kSmem, st, d, *hm, *wdn);
     }));
@@ -889,6 +904,8 @@ moe_status moe_create(int E, int H, int I, int k, moe_t* out) {
   c->k = k;
   c->device = dev;
   c->num_sms = prop.multiProcessorCount;
+  // row-tile width of the grouped GEMM: MOE_ROW_TILE=512 or 256 (default below)
+  if (const char* v = getenv("MOE_ROW_TILE")) c->wide_rows = strcmp(v, "512") == 0;
   if (cudaMalloc(&c->d_status, sizeof(uint32_t)) != cudaSuccess ||
       cudaMemset(c->d_status, 0, sizeof(uint32_t)) != cudaSuccess) {
     cudaGetLastError();

@@ -5,11 +5,13 @@ hundreds of rows, many see tens, some a handful (hearth-lean-loomed-v1 card, "Wh
 streams can be slow on Vulkan").  Every case is checked against the fp64 oracle on all tokens.
 """
 import json
+import os
 
 import numpy as np
 import pytest
 import torch
 
+import moe_inputs as mi
 import oracle
 from parity_util import check_outputs, compare_routing, gpu_route, host_route, inputs_on_gpu
 
@@ -88,3 +90,56 @@ def test_thresholds_round_trip():
     assert layer.get_dispatch() == (4, 50)
     layer.set_path(moe.MOE_PATH_AUTO, 9)
     assert layer.get_path() == (moe.MOE_PATH_AUTO, 9) and layer.get_dispatch() == (9, 50)
+
+
+def _wide_layer(E, H, I, k):
+    """A handle whose row-tile GEMM uses 256 x 512 tiles (two MMAs per K step)."""
+    old = os.environ.get("MOE_ROW_TILE")
+    os.environ["MOE_ROW_TILE"] = "512"
+    try:
+        return moe.Moe(E, H, I, k)
+    finally:
+        if old is None:
+            del os.environ["MOE_ROW_TILE"]
+        else:
+            os.environ["MOE_ROW_TILE"] = old
+
+
+@pytest.mark.parametrize("T", [1, 65, 300, 520])
+def test_wide_row_tiles_ragged(T):
+    """The 256 x 512 row tiles: one or several 256-row chunks, a half-filled last column block
+    (I = 320: 256 + 64 gate/up columns; H = 256: one down tile of which only the first half has
+    columns), the next tile's first-half MMAs running while the second half drains."""
+    E, H, I, k = 8, 256, 320, 2
+    d, h = inputs_on_gpu(T, H, E, k, I, seed=2500 + T)
+    layer = _wide_layer(E, H, I, k)
+    layer.set_path(moe.MOE_PATH_GEMM)
+    ref_route = host_route(h, k)
+    g = gpu_route(layer, d)
+    compare_routing(g, ref_route, k, E)
+    out = layer.forward(d["x"], d["W_router"], d["b_router"], d["W_gate_up"], d["W_down"])
+    assert layer.sync_status() == moe.MOE_OK
+    ref = oracle.moe_forward_ref(h["x"], h["W_router"], h["b_router"], h["W_gate_up"],
+                                 h["W_down"], k, route=ref_route)
+    check_outputs(out.double().cpu().numpy(), np.arange(T), h, ref_route, g, ref)
+
+
+@pytest.mark.parametrize("T,path", [(300, "gemm"), (2048, "auto")])
+def test_wide_row_tiles_gpt_oss_shape(T, path):
+    """H = I = 2880: 12 gate/up tiles per chunk (the last with 64 columns, no second half) and
+    6 down tiles (the last with 320 columns)."""
+    E, H, I, k = 32, 2880, 2880, 4
+    d, h = inputs_on_gpu(T, H, E, k, I, seed=2600 + T)
+    layer = _wide_layer(E, H, I, k)
+    if path == "gemm":
+        layer.set_path(moe.MOE_PATH_GEMM)
+    ref_route = host_route(h, k)
+    g = gpu_route(layer, d)
+    compare_routing(g, ref_route, k, E)
+    out = layer.forward(d["x"], d["W_router"], d["b_router"], d["W_gate_up"], d["W_down"])
+    assert layer.sync_status() == moe.MOE_OK
+    tokens = np.arange(T) if T <= 300 else mi.sample_tokens(T, 512, 2600)
+    got = out[torch.from_numpy(tokens).cuda()].double().cpu().numpy()
+    ref = oracle.moe_forward_ref(h["x"], h["W_router"], h["b_router"], h["W_gate_up"],
+                                 h["W_down"], k, tokens=tokens, route=ref_route)
+    check_outputs(got, tokens, h, ref_route, g, ref)
