@@ -191,23 +191,58 @@ KERNEL_NAMES = {  # the gate/up kernel of each family, as ncu lists it
     "gemm": "grouped_gemm_kernel<gate_up>"}
 
 
-def split_families(counts, path: str, stream_rows: int, tile_rows: int) -> dict:
+MX_STREAM_T = 512   # MXFP4 layers stream in calls of at most this many tokens
+
+
+def split_families(counts, path: str, T: int, stream_T: int, stream_rows: int, tile_rows: int,
+                   weights: str = "bf16") -> dict:
     """Row counts of the experts each kernel family multiplies, as the library dispatches them
-    (moe_path in include/moe.h): with "auto", an expert with c rows streams if c <= stream_rows,
-    takes expert tiles if c <= tile_rows, else row tiles."""
+    (moe_path in include/moe.h): with "auto", in calls of at most stream_T tokens an expert with
+    c <= stream_rows rows streams; the others take expert tiles up to tile_rows and row tiles
+    above, and a side of a boundary that the call's counts barely populate joins its neighbour
+    (the library's snap rule)."""
     out = {f: [] for f in FAMILIES}
-    for c in counts:
-        if c <= 0:
-            continue
-        if path in FAMILIES:
-            f = path
-        elif c <= stream_rows:
-            f = "stream"
-        elif c <= max(stream_rows, tile_rows):
-            f = "tile"
-        else:
-            f = "gemm"
-        out[f].append(int(c))
+    cs = [int(c) for c in counts if c > 0]
+    if weights == "mxfp4":
+        f = "stream" if path == "stream" or (path == "auto" and T <= MX_STREAM_T) else "tile"
+        out[f] = cs
+        return out
+    if path in FAMILIES:
+        out[path] = cs
+        return out
+    s_on = T <= stream_T and stream_rows > 0
+    lists = []                                   # (family, upper bound), launched families only
+    lo = stream_rows if s_on else 0
+    if s_on:
+        lists.append(["stream", stream_rows])
+    if T > lo and tile_rows > lo:
+        lists.append(["tile", tile_rows])
+    if T > max(lo, tile_rows):
+        lists.append(["gemm", None])
+    lists[-1][1] = None                          # the last family takes everything above
+    fam = {}
+    for i, c in enumerate(cs):
+        for f, ub in lists:
+            if ub is None or c <= ub:
+                fam[i] = f
+                break
+    for l in range(len(lists) - 1):
+        b = lists[l][1]
+        lo_f, hi_f = lists[l][0], lists[l + 1][0]
+        lo_c = [cs[i] for i in fam if fam[i] == lo_f]
+        hi_c = [cs[i] for i in fam if fam[i] == hi_f]
+        if lo_c and hi_c:
+            if len(hi_c) <= len(lo_c) and max(hi_c) <= 2 * b:
+                src, dst = hi_f, lo_f
+            elif len(lo_c) < len(hi_c) and min(lo_c) > b // 2:
+                src, dst = lo_f, hi_f
+            else:
+                continue
+            for i in fam:
+                if fam[i] == src:
+                    fam[i] = dst
+    for i, f in fam.items():
+        out[f].append(cs[i])
     return out
 
 
@@ -438,11 +473,11 @@ def run_ours(args, w: mi.Workload, T: int) -> None:
     # ---- roofline of the dominant kernel: the gate/up projection (2/3 of bytes and FLOPs) of
     # the kernel family that spent the most time ----
     hbm, bf16, bf16_sus, peak_src = measured_peaks()
-    path_setting, _ = layer.get_path()
+    path_setting, stream_T = layer.get_path()
     stream_rows, tile_rows = layer.get_dispatch()
-    path = "stream" if mx else {moe.MOE_PATH_STREAM: "stream", moe.MOE_PATH_GEMM: "gemm",
-                                moe.MOE_PATH_TILE: "tile"}.get(path_setting, "auto")
-    fams = split_families(counts, path, stream_rows, tile_rows)
+    path = {moe.MOE_PATH_STREAM: "stream", moe.MOE_PATH_GEMM: "gemm",
+            moe.MOE_PATH_TILE: "tile"}.get(path_setting, "auto")
+    fams = split_families(counts, path, T, stream_T, stream_rows, tile_rows, w.weights)
     work = {f: family_work(fams[f], w.H, w.I, w.weights) for f in FAMILIES}
     n_prof = prof_steps
     gu_ms = {f: prof["gate_up_" + f][0] / n_prof for f in FAMILIES}
@@ -451,10 +486,11 @@ def run_ours(args, w: mi.Workload, T: int) -> None:
     kernels_ms = {k_: round(v[0] / n_prof, 4) for k_, v in prof.items() if v[1]}
     roof = dominant_roofline(work, gu_ms, hbm, bf16, bf16_sus, peak_src)
     if mx:
-        roof["kernel"] = "stream_gate_up_mx_kernel"
+        roof["kernel"] = {"stream": "stream_gate_up_mx_kernel",
+                          "tile": "expert_tile_mx_kernel<0>"}.get(roof["family"], roof["kernel"])
     roof["traffic"] = ncu_traffic(roof["kernel"], w.name)
     down_rate = {f"down_{f}_ms": round(dn_ms[f], 4) for f in FAMILIES if dn_ms[f] > 0}
-    dispatch = dict(stream_rows=stream_rows, tile_rows=tile_rows,
+    dispatch = dict(stream_T=stream_T, stream_rows=stream_rows, tile_rows=tile_rows,
                     experts={f: len(fams[f]) for f in FAMILIES},
                     rows={f: int(sum(fams[f])) for f in FAMILIES})
 

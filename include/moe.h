@@ -80,18 +80,23 @@ typedef enum {
   MOE_ERR_DEVICE = 6        /* no usable sm_100 device */
 } moe_status;
 
-/* Which kernels multiply an expert's rows.  AUTO decides per expert, on the device, from the
- * expert's row count in this call's routing (no host synchronisation):
- *   rows <= stream_rows               weight streaming (tensor-core mma.sync, split over K
- *                                     across all SMs): the decode regime, ~1 row per expert
- *   stream_rows < rows <= tile_rows   expert tiles: tcgen05 MMAs with the expert's weight
- *                                     columns as the M operand and its rows as N, each weight
- *                                     block read once for up to 128 rows
- *   rows > tile_rows                  row tiles: 2-SM tcgen05 grouped GEMM, 256 rows x 256
- *                                     columns per CTA pair (prefill, long sequences)
- * This is the per-expert mat-vec / mat-mat choice of the hearth-lean-loomed-v1 card ("Why
- * 12-16 streams can be slow on Vulkan"), made per expert and per call.  The other values
- * force one kernel family for every expert. */
+/* Which kernels multiply an expert's rows.  Three kernel families:
+ *   weight streaming  tensor-core mma.sync with the weights split over K across all SMs
+ *                     (stream-K): balances best when only a few experts are touched
+ *   expert tiles      tcgen05 MMAs with an expert's weight columns as the M operand and its rows
+ *                     as N, each weight block read once for up to 128 rows
+ *   row tiles         2-SM tcgen05 grouped GEMM, 256 rows x 256 columns per CTA pair (prefill,
+ *                     long sequences)
+ * MOE_PATH_AUTO chooses per expert, on the device, from the call's histogram (no host sync):
+ * in calls of at most crossover_T tokens the experts with at most stream_rows rows stream; the
+ * others take expert tiles up to tile_rows rows and row tiles above.  When a call's counts put
+ * a few experts just across the tile_rows boundary (an almost uniform routing), they join the
+ * larger side instead of running as a second, half-filled launch: the upper side joins the lower
+ * one if it holds no more experts and none has more than 2 * tile_rows rows, else the lower side
+ * joins the upper one if it holds fewer experts and none has tile_rows / 2 rows or less.  This
+ * is the per-expert mat-vec / mat-mat choice of the hearth-lean-loomed-v1 card ("Why 12-16
+ * streams can be slow on Vulkan"), made per expert and per call.  The other values force one
+ * family for every expert. */
 typedef enum {
   MOE_PATH_AUTO = 0,    /* per-expert choice among the three families below */
   MOE_PATH_STREAM = 1,  /* every expert through the weight-streaming kernels */
@@ -148,9 +153,9 @@ MOE_API moe_status moe_forward(moe_t ctx, int T, const void* x_bf16, const void*
  * gu_codes [E, 2I, H/2] and gu_scales [E, H/32, 2I] hold W_gate_up [E, H, 2I] (gate columns
  * [0, I), up columns [I, 2I)); dn_codes [E, H, I/2] and dn_scales [E, I/32, H] hold W_down
  * [E, I, H].  x, W_router, b_router and out as in moe_forward; all pointers 16-byte aligned.
- * Experts are dispatched like the bf16 layer's (moe_path), with two kernel families: up to
- * stream_rows rows, the MXFP4 weight-streaming kernels; more rows, the MXFP4 expert-tile kernel
- * (MOE_PATH_GEMM and MOE_PATH_TILE both force the latter; there is no MXFP4 row-tile GEMM).
+ * Two kernel families: MOE_PATH_AUTO streams the weights in calls of at most 512 tokens and
+ * runs the MXFP4 expert-tile kernel above; MOE_PATH_STREAM forces streaming, MOE_PATH_TILE and
+ * MOE_PATH_GEMM expert tiles (there is no MXFP4 row-tile GEMM).
  *   - expert tiles: the codes are widened to bf16 weights in shared memory (exact: an E2M1 value
  *     times 2^(s - 127) has two significant bits; bf16 holds it for 2 <= s <= 252, and for
  *     smaller s as a subnormal down to 2^-133) and multiplied with the bf16 activations on
@@ -207,30 +212,31 @@ MOE_API moe_status moe_experts(moe_t ctx, int R, int S, const int32_t* seg_count
 MOE_API moe_status moe_combine(moe_t ctx, int T, const int32_t* inv_perm, const float* y_rows,
                                float* out, moe_stream_t stream);
 
-/* Choose the path.  stream_rows >= 0 also sets the AUTO threshold: experts with at most this
- * many rows in a call stream their weights (the built-in default is 16, one streaming chunk;
- * moe_tune measures it); stream_rows < 0 keeps the current one.  MOE_ERR_ARG for an unknown
- * path. */
-MOE_API moe_status moe_set_path(moe_t ctx, moe_path path, int stream_rows);
+/* Choose the path.  crossover_T >= 0 also sets the largest call (in tokens) in which AUTO uses
+ * the weight-streaming family (default: the largest T whose touched experts' tiles fill less
+ * than two waves of the GPU: 3 for the 20b and 120b shapes on 148 SMs; moe_tune measures it);
+ * crossover_T < 0 keeps the current one.  MOE_ERR_ARG for an unknown path. */
+MOE_API moe_status moe_set_path(moe_t ctx, moe_path path, int crossover_T);
 
-/* Current path setting and AUTO streaming threshold (rows per expert). */
-MOE_API moe_status moe_get_path(moe_t ctx, moe_path* path, int* stream_rows);
+/* Current path setting and streaming crossover (tokens). */
+MOE_API moe_status moe_get_path(moe_t ctx, moe_path* path, int* crossover_T);
 
-/* Both AUTO thresholds, in rows of one expert: stream_rows (see moe_set_path) and tile_rows
- * (experts with more rows than stream_rows and at most tile_rows take expert tiles, more rows
- * the row-tile GEMM; default 256).  A negative value keeps the current one. */
+/* The two per-expert AUTO thresholds, in rows of one expert: stream_rows (default 16, one
+ * streaming chunk) and tile_rows (default 128, one expert tile).  A negative value keeps the
+ * current one. */
 MOE_API moe_status moe_set_dispatch(moe_t ctx, int stream_rows, int tile_rows);
 MOE_API moe_status moe_get_dispatch(moe_t ctx, int* stream_rows, int* tile_rows);
 
-/* Measure the AUTO thresholds on this device with the caller's layer: times the whole layer
+/* Measure the AUTO settings on this device with the caller's layer: times the whole layer
  * (median of 5 calls after 2 warm-ups) with every expert forced through each family, at
  * T = 1, 2, 4, 8, 12, 16, 24, 32, 48, 64, ... up to T_max, streaming against expert tiles and
- * expert tiles against row tiles.  For each pair it takes the largest T at which the lower
- * family was not slower (stopping once the upper one has been faster for a doubling of T) and
- * stores the mean rows per expert at that T, ceil(T * k / E), as the threshold.  x must hold
- * T_max rows, out T_max rows; workspace at least moe_tune_workspace_bytes(ctx, T_max).
- * Synchronises `stream`; the path setting is left as it was.  *crossover_out (may be NULL)
- * receives stream_rows; moe_get_dispatch gives both. */
+ * expert tiles against row tiles.  For each pair it takes the largest T at which the first
+ * family was not slower (stopping once the second has been faster for a doubling of T): the
+ * first gives the streaming crossover (tokens), the second the tile_rows threshold as the mean
+ * rows per expert at that T, ceil(T * k / E).  x must hold T_max rows, out T_max rows;
+ * workspace at least moe_tune_workspace_bytes(ctx, T_max).  Synchronises `stream`; the path
+ * setting is left as it was.  *crossover_out (may be NULL) receives the streaming crossover;
+ * moe_get_dispatch gives tile_rows. */
 MOE_API size_t moe_tune_workspace_bytes(moe_t ctx, int T_max);
 MOE_API moe_status moe_tune(moe_t ctx, int T_max, const void* x_bf16, const void* W_router_bf16,
                     const float* b_router, const void* W_gate_up_bf16,

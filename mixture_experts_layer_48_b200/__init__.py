@@ -130,8 +130,9 @@ class Moe:
         return self._h
 
     # -- settings --------------------------------------------------------------------
-    def set_path(self, path: int, stream_rows: int = -1) -> None:
-        _check(moe_set_path(self._h, path, stream_rows), "moe_set_path")
+    def set_path(self, path: int, crossover_T: int = -1) -> None:
+        """Path; crossover_T >= 0 also sets the largest call AUTO streams (see include/moe.h)."""
+        _check(moe_set_path(self._h, path, crossover_T), "moe_set_path")
 
     def get_path(self) -> tuple[int, int]:
         p, c = _c_int(), _c_int()

@@ -12,8 +12,9 @@
 //                            routing weight (sent with the row)
 //   build_segment_lists_kernel   work lists of the received rows: they arrive as segments
 //                            (source GPU, expert), source-major; an expert's kernel family is
-//                            chosen from its rows over all sources, each segment makes its own
-//                            chunks; also the identity row map of the expert kernels' output
+//                            chosen from its rows over all sources (assign_families), each
+//                            segment makes its own chunks; also the identity row map of the
+//                            expert kernels' output
 //   combine_rows_kernel      out[t] = sum_j y[inv_perm[t, j]] in slot order j
 #pragma once
 
@@ -85,7 +86,7 @@ constexpr int kMaxSegments = 4096;  // sources x experts of one expert-half call
 // over all sources); every block writes part of the identity row map perm[r] = r and zeroes the
 // completion counters.  Counts that do not add up to R are reported in the status word; rows
 // past R are never listed.  Also zero-fills zero4[0, n_zero4).  block 1024; dynamic smem
-// (4*S*E + E) ints.
+// (4*S*E + 2*E) ints.
 __global__ void __launch_bounds__(1024)
     build_segment_lists_kernel(const int32_t* __restrict__ seg_counts, int S, int E, int R,
                                RouteOut o, int32_t* __restrict__ perm_iota, float4* zero4,
@@ -97,6 +98,7 @@ __global__ void __launch_bounds__(1024)
   int32_t* base = cnt + n;       // [n] first work-list entry of each segment
   int32_t* rbase = base + n;     // [n] first row of each segment among its list's rows
   int32_t* total = rbase + n;    // [E] rows of each expert over all sources
+  int32_t* fam = total + E;      // [E] work list of each expert
   const int tid = threadIdx.x;
   pdl_wait();
   pdl_launch_next();
@@ -122,13 +124,13 @@ __global__ void __launch_bounds__(1024)
     total[e] = s_;
   }
   __syncthreads();
+  assign_families(total, E, o, fam);  // an expert's family from its rows over all sources
   // thread l < n_lists: exclusive scan of list l's entries over the segments in order
   if (tid < o.n_lists) {
     const WorkList& L = o.wl[tid];
     int run = 0, rows = 0;
     for (int i = 0; i < n; ++i) {
-      const int tot = total[i % E];
-      if (tot > L.min_count && tot <= L.max_count) {
+      if (fam[i % E] == tid) {
         base[i] = run;
         rbase[i] = rows;
         run += (cnt[i] + L.chunk_rows - 1) / L.chunk_rows;
@@ -139,17 +141,12 @@ __global__ void __launch_bounds__(1024)
   }
   __syncthreads();
   for (int i = tid; i < n; i += blockDim.x) {
-    const int e = i % E, tot = total[e], c = cnt[i];
-    if (c == 0) continue;
-    for (int l = 0; l < o.n_lists; ++l) {
-      const WorkList& L = o.wl[l];
-      if (tot > L.min_count && tot <= L.max_count) {
-        int b = base[i];
-        for (int r0 = 0; r0 < c; r0 += L.chunk_rows)
-          L.chunks[b++] = make_int4(e, seg_off[i] + r0, min(L.chunk_rows, c - r0), rbase[i] + r0);
-        break;
-      }
-    }
+    const int e = i % E, c = cnt[i], l = fam[e];
+    if (c == 0 || l < 0) continue;
+    const WorkList& L = o.wl[l];
+    int b = base[i];
+    for (int r0 = 0; r0 < c; r0 += L.chunk_rows)
+      L.chunks[b++] = make_int4(e, seg_off[i] + r0, min(L.chunk_rows, c - r0), rbase[i] + r0);
   }
 }
 

@@ -13,7 +13,7 @@
 //   warp 0      TMA producer: per K stage of 64, the codes of two 128-column matrices ([128 rows
 //               x 32 bytes] boxes of the [columns, K/2] code layout) and their scales ([2 x 128]
 //               boxes of the [K/32, columns] layout) into a deep ring (8 stages of 8.5 KB)
-//   warps 6-9   converters: thread c widens column c of both matrices (64 codes each) to bf16 in
+//   warps 6-13  converters: four warps per matrix, thread c widens column c (64 codes) to bf16 in
 //               the 128-byte-swizzled K-major layout (the A operand), and one of them issues the
 //               TMA loads of the stage's activation rows (the B operand), into a 2-stage ring
 //   warp 1      TMEM owner and MMA issuer: two tcgen05.mma M = 128, N = rows per K step of 16
@@ -34,7 +34,8 @@ namespace moe {
 constexpr int kEmxRawStages = 8;
 constexpr int kEmxAbStages = 2;
 constexpr int kEmxConvWarp0 = 6;
-constexpr int kEmxThreads = 320;                              // 10 warps
+constexpr int kEmxConvWarps = 8;                              // one per matrix row of 64 codes
+constexpr int kEmxThreads = 32 * (kEmxConvWarp0 + kEmxConvWarps);   // 14 warps
 constexpr int kEmxCodesBytes = kEtM * (kEtBK / 2);            // 4 KB: 128 columns x 32 bytes
 constexpr int kEmxScaleBytes = (kEtBK / 32) * kEtM;           // 256 B: 2 blocks x 128 columns
 constexpr int kEmxRawBytes = 2 * kEmxCodesBytes + 2 * kEmxScaleBytes;   // 8.5 KB
@@ -45,8 +46,16 @@ constexpr int kEmxSmem = 1024 + kEmxAbStages * kEmxAbBytes + kEmxRawStages * kEm
 static_assert(kEmxRawBytes % 128 == 0, "TMA destinations stay 128-byte aligned");
 static_assert(kEmxSmem <= 227 * 1024, "shared memory");
 
+// Two fp32 values to a bf16 pair (hardware round to nearest even), first in the low half.
+MOE_DEVINL uint32_t cvt_bf16x2(float lo, float hi) {
+  uint32_t r;
+  asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
+  return r;
+}
+
 // Eight E2M1 codes (one 32-bit word, first element in the low nibble of byte 0) times the block
-// scale to eight bf16 values (16 bytes, K order).
+// scale to eight bf16 values (16 bytes, K order).  Every step is exact: E2M1 -> f16 -> fp32, a
+// product with a power of two, and bf16 holds the result (see the file comment).
 MOE_DEVINL uint4 e2m1x8_scaled_bf16(uint32_t w, float scale) {
   uint32_t h[4];
   e2m1x8_to_f16x2(w, h);
@@ -57,7 +66,7 @@ MOE_DEVINL uint4 e2m1x8_scaled_bf16(uint32_t w, float scale) {
     asm("{\n .reg .f16 a, b;\n mov.b32 {a, b}, %2;\n cvt.f32.f16 %0, a;\n cvt.f32.f16 %1, b;\n}"
         : "=f"(lo), "=f"(hi)
         : "r"(h[i]));
-    o[i] = pack_bf16x2(lo * scale, hi * scale);
+    o[i] = cvt_bf16x2(lo * scale, hi * scale);
   }
   return make_uint4(o[0], o[1], o[2], o[3]);
 }
@@ -94,10 +103,10 @@ __global__ void __launch_bounds__(kEmxThreads, 1)
   if (tid == 0) {
     for (int s = 0; s < kEmxRawStages; ++s) {
       mbar_init(&raw_full[s], 1);
-      mbar_init(&raw_empty[s], 4);        // the four converter warps
+      mbar_init(&raw_empty[s], kEmxConvWarps);
     }
     for (int s = 0; s < kEmxAbStages; ++s) {
-      mbar_init(&ab_full[s], 1 + 4);      // the row loads' expect_tx + four converter warps
+      mbar_init(&ab_full[s], 1 + kEmxConvWarps);  // the row loads' expect_tx + the converters
       mbar_init(&ab_empty[s], 1);
     }
     for (int b = 0; b < 2; ++b) {
@@ -174,7 +183,8 @@ __global__ void __launch_bounds__(kEmxThreads, 1)
     }
   } else if (warp >= kEmxConvWarp0) {
     // ------------------------------ converters (+ activation rows) ------------------------------
-    const int ct = tid - kEmxConvWarp0 * 32;                        // weight column 0..127
+    const int cti = tid - kEmxConvWarp0 * 32;                       // 0..255
+    const int j = cti / kEtM, ct = cti % kEtM;                      // matrix, weight column
     uint32_t it = 0;
     int last_ab[kEmxAbStages] = {-1, -1};
     bool aborted = false;
@@ -197,7 +207,7 @@ __global__ void __launch_bounds__(kEmxThreads, 1)
           break;
         }
         uint8_t* abs_ = ab + as * kEmxAbBytes;
-        if (ct == 0) {  // this stage's activation rows (the B operand)
+        if (cti == 0) {  // this stage's activation rows (the B operand)
           mbar_arrive_expect_tx(&ab_full[as], xbytes);
           for (int r = 0; r < nrb; ++r)
             tma_load_2d(abs_ + kEmxABytes + r * (kEtRowBox * kEtBK * 2), &xmap, kst * kEtBK,
@@ -205,9 +215,7 @@ __global__ void __launch_bounds__(kEmxThreads, 1)
           last_ab[as] = (int)it;
         }
         const uint8_t* rst = raw + rs * kEmxRawBytes;
-#pragma unroll
-        for (int j = 0; j < 2; ++j) {
-          if (j == 0 ? !m0 : !m1) continue;
+        if (j == 0 ? m0 : m1) {  // warp-uniform: four warps per matrix
           const uint4* codes = reinterpret_cast<const uint4*>(rst + j * kEmxCodesBytes + ct * 32);
           const uint8_t* sc = rst + 2 * kEmxCodesBytes + j * kEmxScaleBytes;
           const float s0 = e8m0_to_f32(sc[ct]), s1 = e8m0_to_f32(sc[kEtM + ct]);
@@ -228,7 +236,7 @@ __global__ void __launch_bounds__(kEmxThreads, 1)
       }
     }
     // never leave the CTA with row copies in flight
-    if (ct == 0)
+    if (cti == 0)
       for (int s = 0; s < kEmxAbStages; ++s)
         if (last_ab[s] >= 0 &&
             !mbar_wait_bounded(&ab_full[s], (last_ab[s] / kEmxAbStages) & 1u, kWaitLimitNs))

@@ -31,11 +31,13 @@ namespace {
 constexpr int kMaxE = 256;
 constexpr int kMaxHI = 16384;
 constexpr int kMaxT = 1 << 20;
-// Per-expert dispatch thresholds (rows of one expert) until moe_tune measures them: up to one
-// streaming chunk streams, up to two expert tiles take the expert-tile kernel, more rows the
-// row-tile grouped GEMM.
+// Dispatch defaults until moe_tune measures them.  The weight-streaming family runs only in calls
+// so small that expert tiles could not fill the GPU (see default_stream_T); there it takes the
+// experts with up to one streaming chunk of rows.  Experts with up to one expert tile of rows take
+// the expert-tile kernel, more rows the row-tile grouped GEMM.
 constexpr int kDefaultStreamRows = 16;
-constexpr int kDefaultTileRows = 256;
+constexpr int kDefaultTileRows = 128;
+constexpr int kMxStreamT = 512;  // MXFP4: streaming for calls of at most this many tokens
 constexpr int kMaxKernelsPerCall = 12;
 
 moe_status static_scratch_address(void** out);  // defined beside the array, at the end
@@ -69,8 +71,10 @@ struct moe_ctx {
   int device = 0;
   int num_sms = 148;
   moe_path path = MOE_PATH_AUTO;
-  int stream_rows = kDefaultStreamRows;  // AUTO: experts with at most this many rows stream
-  int tile_rows = kDefaultTileRows;      // ... up to this many take expert tiles; more: row tiles
+  int stream_T = 0;                      // AUTO streams only in calls of at most this many tokens
+  int stream_rows = kDefaultStreamRows;  // ... the experts with at most this many rows
+  int tile_rows = kDefaultTileRows;      // experts up to this many rows take expert tiles; more:
+                                         // row tiles (moved across by the call's counts: snap)
   bool wide_rows = false;                // row tiles 256 x 512 (two MMAs per K step) or 256 x 256
   uint32_t* d_status = nullptr;
   void* static_scratch = nullptr;  // device address of the routing scratch array (moe_route_static)
@@ -228,6 +232,7 @@ constexpr int kFamChunkRows[kFamilies] = {kStreamRB, kEtRows, kGemmChunkRows};
 struct Plan {
   bool has[kFamilies] = {false, false, false};
   int max_count[kFamilies] = {0, 0, 0};   // family f takes counts in (max_count[f-1], max_count[f]]
+  bool snap = false;                      // the call's counts may move experts across a boundary
   int min_count(int f) const {
     int m = 0;
     for (int g = 0; g < f; ++g)
@@ -242,18 +247,10 @@ Plan make_plan(const moe_ctx* c, int T, bool mx, moe_path path) {
     p.has[f] = true;
     p.max_count[f] = INT_MAX;
   };
-  if (mx) {  // MXFP4 experts: weight streaming and expert tiles (no MXFP4 row-tile GEMM)
-    if (path == MOE_PATH_STREAM) {
-      only(kFamStream);
-    } else if (path == MOE_PATH_TILE || path == MOE_PATH_GEMM) {
-      only(kFamTile);
-    } else {
-      const int s = c->stream_rows;
-      p.has[kFamStream] = s > 0;
-      p.max_count[kFamStream] = T > s ? s : INT_MAX;
-      p.has[kFamTile] = T > s;
-      p.max_count[kFamTile] = INT_MAX;
-    }
+  if (mx) {  // MXFP4 experts: weight streaming or expert tiles (no MXFP4 row-tile GEMM)
+    if (path == MOE_PATH_STREAM) only(kFamStream);
+    else if (path == MOE_PATH_TILE || path == MOE_PATH_GEMM) only(kFamTile);
+    else only(T <= kMxStreamT ? kFamStream : kFamTile);
     return p;
   }
   switch (path) {
@@ -261,26 +258,44 @@ Plan make_plan(const moe_ctx* c, int T, bool mx, moe_path path) {
     case MOE_PATH_GEMM: only(kFamGemm); break;
     case MOE_PATH_TILE: only(kFamTile); break;
     default: {
-      const int s = c->stream_rows, t = std::max(c->stream_rows, c->tile_rows);
-      p.has[kFamStream] = s > 0;
-      p.max_count[kFamStream] = s;
-      p.has[kFamTile] = T > s && t > s;
-      p.max_count[kFamTile] = t;
-      p.has[kFamGemm] = T > t;
+      const bool s_on = T <= c->stream_T && c->stream_rows > 0;
+      const int lo = s_on ? c->stream_rows : 0;
+      p.has[kFamStream] = s_on;
+      p.has[kFamTile] = T > lo && c->tile_rows > lo;
+      p.has[kFamGemm] = T > std::max(lo, c->tile_rows);
+      p.max_count[kFamStream] = (p.has[kFamTile] || p.has[kFamGemm]) ? c->stream_rows : INT_MAX;
+      p.max_count[kFamTile] = p.has[kFamGemm] ? c->tile_rows : INT_MAX;
       p.max_count[kFamGemm] = INT_MAX;
-      if (!p.has[kFamTile] && !p.has[kFamGemm]) p.max_count[kFamStream] = INT_MAX;
-      else if (!p.has[kFamGemm]) p.max_count[kFamTile] = INT_MAX;
+      p.snap = true;
     }
   }
   return p;
+}
+
+// Largest T for which the expert tiles of every expert T tokens can touch fill less than two
+// waves of the GPU's SMs: below it the stream-K weight streaming balances better.
+int default_stream_T(const moe_ctx* c) {
+  const long long tiles_per_expert = (c->I + kEtM - 1) / kEtM;
+  int T = 0;
+  while (T < kMaxT &&
+         std::min<long long>(c->E, (long long)(T + 1) * c->k) * tiles_per_expert < 2LL * c->num_sms)
+    ++T;
+  return T;
+}
+
+// Rows an expert of family f can hold in a call: its upper threshold, twice that when the call's
+// counts may move neighbours in (snap), unbounded for the last family.
+long long family_row_bound(const Plan& p, int f) {
+  if (p.max_count[f] == INT_MAX) return LLONG_MAX;
+  return (long long)p.max_count[f] * (p.snap ? 2 : 1);
 }
 
 // Work-list entries family f can need for T tokens.
 int max_chunks(const moe_ctx* c, int T, const Plan& p, int f) {
   const long long R = (long long)T * c->k, rows = kFamChunkRows[f];
   long long n = R / rows + c->E;
-  if (p.max_count[f] != INT_MAX)
-    n = std::min(n, (long long)c->E * ((p.max_count[f] + rows - 1) / rows));
+  const long long b = family_row_bound(p, f);
+  if (b != LLONG_MAX) n = std::min(n, (long long)c->E * ((b + rows - 1) / rows));
   return (int)n;
 }
 
@@ -316,9 +331,8 @@ Layout make_layout(const moe_ctx* c, int T, const Plan& p, bool mx) {
     L.n_done = n * ((c->I + tile_cols - 1) / tile_cols);
     L.done = cv.take(4 * (size_t)L.n_done);
     // split-K sums of the streaming family's rows (each entry carries its rows' first index)
-    const long long srows = p.max_count[kFamStream] == INT_MAX
-                                ? (long long)R
-                                : std::min((long long)R, (long long)c->E * p.max_count[kFamStream]);
+    const long long sb = family_row_bound(p, kFamStream);
+    const long long srows = sb == LLONG_MAX ? (long long)R : std::min((long long)R, c->E * sb);
     L.acc_floats = (size_t)srows * 2 * c->I;
     L.acc = cv.take(sizeof(float) * L.acc_floats);
   }
@@ -338,17 +352,16 @@ Layout make_expert_layout(const moe_ctx* c, int R, int S, const Plan& p) {
     if (p.has[f]) {
       const long long rows = kFamChunkRows[f], segs = (long long)S * c->E;
       long long n = R / rows + segs;
-      if (p.max_count[f] != INT_MAX)  // every expert's segments together hold <= max_count rows
-        n = std::min(n, (long long)c->E * ((p.max_count[f] + rows - 1) / rows + S));
+      const long long b = family_row_bound(p, f);
+      if (b != LLONG_MAX)  // every expert's segments together hold <= b rows
+        n = std::min(n, (long long)c->E * ((b + rows - 1) / rows + S));
       L.sched[f] = cv.take(16);
       L.chunks[f] = cv.take(16 * (size_t)n);
       if (f == kFamStream) {
         const int tile_cols = std::min(kStreamCols, kMxTileCols);
         L.n_done = (int)(n * ((c->I + tile_cols - 1) / tile_cols));
         L.done = cv.take(4 * (size_t)L.n_done);
-        const long long srows = p.max_count[f] == INT_MAX
-                                    ? (long long)R
-                                    : std::min((long long)R, (long long)c->E * p.max_count[f]);
+        const long long srows = b == LLONG_MAX ? (long long)R : std::min((long long)R, c->E * b);
         L.acc_floats = (size_t)srows * 2 * c->I;
         L.acc = cv.take(sizeof(float) * L.acc_floats);
       }
@@ -441,7 +454,7 @@ moe_status launch_route(moe_ctx* c, int T, const uint16_t* x, const uint16_t* Wr
       return launch_router_tc<32>(1, st, x, Wr, b, T, H, E, k, o, nullptr, zero4, n_zero4, rt, partial);
     }));
     const size_t smem_f = (size_t)T * E * 4 + (size_t)T * k * 4 + (size_t)T * 8 * 4 +
-                          (256 + 257 + 512) * 4;
+                          (256 + 257 + 768) * 4;
     MOE_TRY(launch(c, kKindRouteFin, st, [&] {
       return launch_pdl(route_small_finalize_kernel, dim3(1), dim3(1024), smem_f, st,
                         (const float*)partial, rt.splits, b, T, E, k, o);
@@ -480,7 +493,7 @@ moe_status launch_route(moe_ctx* c, int T, const uint16_t* x, const uint16_t* Wr
   MOE_TRY(launch(c, kKindRouteFin, st, [&] {
     return launch_pdl(route_scan_kernel, dim3(E), dim3(256), 0, st, block_counts, NB, E, totals);
   }));
-  const size_t smem_s = (256 + 257 + 512) * 4 + (size_t)kRouterTcTokens * 8 * 4 +
+  const size_t smem_s = (256 + 257 + 768) * 4 + (size_t)kRouterTcTokens * 8 * 4 +
                         (size_t)kRouterTcTokens * E;
   MOE_TRY(launch(c, kKindRouteFin, st, [&] {
     return launch_pdl(route_scatter_kernel, dim3(NB), dim3(256), smem_s, st,
@@ -540,7 +553,7 @@ bool set_smem_attrs() {
                              cudaFuncAttributeMaxDynamicSharedMemorySize, kEmxSmem) == cudaSuccess;
   ok &= cudaFuncSetAttribute(build_segment_lists_kernel,
                              cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             (4 * kMaxSegments + kMaxE) * 4) == cudaSuccess;
+                             (4 * kMaxSegments + 2 * kMaxE) * 4) == cudaSuccess;
   return ok;
 }
 
@@ -795,6 +808,7 @@ void plan_lists(const Plan& p, const Layout& L, uint8_t* ws, RouteOut& o, Expert
     io.chunks[f] = wl.chunks;
     io.sched[f] = wl.sched;
   }
+  o.snap = p.snap ? 1 : 0;
   o.zero_i32 = p.has[kFamStream] ? reinterpret_cast<int32_t*>(ws + L.done) : nullptr;
   o.n_zero = p.has[kFamStream] ? L.n_done : 0;
   io.acc = p.has[kFamStream] ? reinterpret_cast<float*>(ws + L.acc) : nullptr;
@@ -904,6 +918,7 @@ moe_status moe_create(int E, int H, int I, int k, moe_t* out) {
   c->k = k;
   c->device = dev;
   c->num_sms = prop.multiProcessorCount;
+  c->stream_T = default_stream_T(c);
   // row-tile width of the grouped GEMM: MOE_ROW_TILE=512 or 256 (default below)
   if (const char* v = getenv("MOE_ROW_TILE")) c->wide_rows = strcmp(v, "512") == 0;
   if (cudaMalloc(&c->d_status, sizeof(uint32_t)) != cudaSuccess ||
@@ -1082,7 +1097,7 @@ moe_status moe_experts(moe_t c, int R, int S, const int32_t* seg_counts, const v
   plan_lists(p, L, ws, o, io);
   int32_t* iota = reinterpret_cast<int32_t*>(ws + L.perm);
   const int grid = (int)std::max<long long>(1, std::min<long long>(c->num_sms, (R + 1023) / 1024));
-  const size_t smem = (size_t)(4 * S * c->E + c->E) * 4;
+  const size_t smem = (size_t)(4 * S * c->E + 2 * c->E) * 4;
   moe_status s = launch(c, kKindRouteFin, st, [&] {
     return launch_pdl(build_segment_lists_kernel, dim3(grid), dim3(1024), smem, st, seg_counts,
                       S, c->E, R, o, iota, reinterpret_cast<float4*>(io.acc), L.acc_floats / 4,
@@ -1103,20 +1118,20 @@ moe_status moe_experts(moe_t c, int R, int S, const int32_t* seg_counts, const v
   return s;
 }
 
-moe_status moe_set_path(moe_t c, moe_path path, int stream_rows) {
+moe_status moe_set_path(moe_t c, moe_path path, int crossover_T) {
   if (!c) return MOE_ERR_ARG;
   if (path != MOE_PATH_AUTO && path != MOE_PATH_STREAM && path != MOE_PATH_GEMM &&
       path != MOE_PATH_TILE)
     return MOE_ERR_ARG;
   c->path = path;
-  if (stream_rows >= 0) c->stream_rows = stream_rows;
+  if (crossover_T >= 0) c->stream_T = crossover_T;
   return MOE_OK;
 }
 
-moe_status moe_get_path(moe_t c, moe_path* path, int* stream_rows) {
+moe_status moe_get_path(moe_t c, moe_path* path, int* crossover_T) {
   if (!c) return MOE_ERR_ARG;
   if (path) *path = c->path;
-  if (stream_rows) *stream_rows = c->stream_rows;
+  if (crossover_T) *crossover_T = c->stream_T;
   return MOE_OK;
 }
 
@@ -1196,8 +1211,8 @@ moe_status moe_tune(moe_t c, int T_max, const void* x_bf16, const void* W_router
     *T_out = cross;
     return MOE_OK;
   };
-  // A family boundary measured at T tokens becomes a per-expert row count: the mean rows per
-  // expert at that T (uniform routing: T*k/E), at least the token count itself when E <= k.
+  // The expert-tile / row-tile boundary measured at T tokens becomes a per-expert row count:
+  // the mean rows per expert at that T (uniform routing: T*k/E).
   auto rows_at = [&](int T) {
     return T == 0 ? 0 : std::max(1, (int)(((long long)T * c->k + c->E - 1) / c->E));
   };
@@ -1209,12 +1224,11 @@ moe_status moe_tune(moe_t c, int T_max, const void* x_bf16, const void* W_router
   c->path = saved_path;
   c->prof_max = saved_prof;
   if (s != MOE_OK) return s;
-  c->stream_rows = rows_at(Ts);
-  // the tile family ends where the row-tile GEMM wins; never below the streaming threshold,
-  // and where T_max never let the GEMM win the measured band is kept
-  c->tile_rows = std::max(c->stream_rows, Tt >= T_max ? std::max(c->tile_rows, rows_at(Tt))
-                                                       : rows_at(Tt));
-  if (crossover_out) *crossover_out = c->stream_rows;
+  // streaming runs in calls of at most Ts tokens; the tile family ends where the row-tile GEMM
+  // wins (if T_max never let it win, the measured band is kept as the lower bound)
+  c->stream_T = Ts;
+  c->tile_rows = Tt >= T_max ? std::max(c->tile_rows, rows_at(Tt)) : std::max(1, rows_at(Tt));
+  if (crossover_out) *crossover_out = c->stream_T;
   return MOE_OK;
 }
 

@@ -16,6 +16,8 @@
 //                  block, two 32-token ballot passes).
 #pragma once
 
+#include <climits>
+
 #include "common.cuh"
 
 namespace moe {
@@ -58,7 +60,7 @@ MOE_DEVINL int warp_exclusive_scan(int n, Val val, Put put) {
 // its own list, so the kernel that multiplies an expert's rows is chosen per expert on the
 // device, from the histogram.
 struct WorkList {
-  int4* chunks;        // {expert, first row, rows, 0}
+  int4* chunks;        // {expert, first row, rows, first row among the list's rows}
   int32_t* sched;      // [0] number of chunks
   int chunk_rows;
   int min_count, max_count;
@@ -75,6 +77,7 @@ struct RouteOut {
   float* row_w;        // [T * k] routing weight of each row (may be null)
   WorkList wl[kMaxWorkLists];
   int n_lists;         // work lists to build (0: routing only)
+  int snap;            // 1: let the call's counts move a barely-populated side of a boundary
   int32_t* zero_i32;   // region zeroed by the chain (completion counters), may be null
   int n_zero;
   const uint16_t* x;   // with x_perm non-null: copy token rows into expert order
@@ -251,23 +254,79 @@ MOE_DEVINL void zero_fill_f4(float4* z, size_t n4) {
     z[i] = make_float4(0.f, 0.f, 0.f, 0.f);
 }
 
-// Work lists of one routing: expert e (with count c > 0) belongs to the list whose
-// (min_count, max_count] holds c, and its rows are split there into entries of at most
-// chunk_rows rows, in expert order.  Each entry is {expert, first row, rows, first row among
-// the list's rows} (the last field lets a kernel keep per-row scratch for its own rows only).
-// Called by all threads of a block with count/off in shared memory (E <= 256 entries);
-// scratch holds [512] ints of shared memory.
+// Which work list takes each expert (fam[e], -1 for an expert without rows): the list whose
+// (min_count, max_count] holds its count.  With o.snap, the call's own counts then move experts
+// across a boundary between neighbouring lists l (lower) and l + 1, so that an almost uniform
+// routing does not split the experts over two half-filled launches:
+//   - if the upper side holds no more experts than the lower one and none of them has more than
+//     twice the boundary, they all join the lower list;
+//   - else, if the lower side holds fewer experts and none of them has half the boundary or
+//     less, they all join the upper list.
+// A skewed routing (counts far on both sides) keeps the per-expert choice.  Called by all
+// threads of a block; cnt and fam in shared memory (E <= 256).
+MOE_DEVINL void assign_families(const int32_t* cnt, int E, const RouteOut& o, int32_t* fam) {
+  const int tid = threadIdx.x;
+  for (int e = tid; e < E; e += blockDim.x) {
+    int f = -1;
+    const int c = cnt[e];
+    for (int l = 0; l < o.n_lists && c > 0; ++l)
+      if (c > o.wl[l].min_count && c <= o.wl[l].max_count) f = l;
+    fam[e] = f;
+  }
+  __syncthreads();
+  if (o.snap && tid < 32) {
+    const int lane = tid;
+    for (int l = 0; l + 1 < o.n_lists; ++l) {
+      const int b = o.wl[l].max_count;  // the boundary: lower list takes counts <= b
+      int n_lo = 0, n_hi = 0, max_hi = 0, min_lo = INT_MAX;
+      for (int e = lane; e < E; e += 32) {
+        if (fam[e] == l) {
+          ++n_lo;
+          min_lo = min(min_lo, cnt[e]);
+        } else if (fam[e] == l + 1) {
+          ++n_hi;
+          max_hi = max(max_hi, cnt[e]);
+        }
+      }
+#pragma unroll
+      for (int off = 16; off > 0; off >>= 1) {
+        n_lo += __shfl_xor_sync(0xffffffffu, n_lo, off);
+        n_hi += __shfl_xor_sync(0xffffffffu, n_hi, off);
+        max_hi = max(max_hi, __shfl_xor_sync(0xffffffffu, max_hi, off));
+        min_lo = min(min_lo, __shfl_xor_sync(0xffffffffu, min_lo, off));
+      }
+      int from = -1, to = -1;
+      if (n_lo > 0 && n_hi > 0) {
+        if (n_hi <= n_lo && max_hi <= 2 * b) from = l + 1, to = l;
+        else if (n_lo < n_hi && min_lo > b / 2) from = l, to = l + 1;
+      }
+      if (from >= 0)
+        for (int e = lane; e < E; e += 32)
+          if (fam[e] == from) fam[e] = to;
+      __syncwarp();
+    }
+  }
+  __syncthreads();
+}
+
+// Work lists of one routing: each expert with rows goes to its list (assign_families), its rows
+// split there into entries of at most chunk_rows rows, in expert order.  Each entry is {expert,
+// first row, rows, first row among the list's rows} (the last field lets a kernel keep per-row
+// scratch for its own rows only).  Called by all threads of a block with count/off in shared
+// memory (E <= 256 entries); scratch holds [768] ints of shared memory.
 MOE_DEVINL void build_work_lists(const int32_t* cnt, const int32_t* off, int E,
                                  const RouteOut& o, int32_t* scratch) {
   const int tid = threadIdx.x;
   if (o.n_lists == 0) return;
   int32_t* chunk_base = scratch;        // [256] first entry of each expert in its list
   int32_t* row_base = scratch + 256;    // [256] first row of each expert among its list's rows
+  int32_t* fam = scratch + 512;         // [256] list of each expert
+  assign_families(cnt, E, o, fam);
   // warp l < n_lists: exclusive scans of list l's entries and rows, in expert order
   const int warp = tid >> 5;
   if (warp < o.n_lists) {
     const WorkList& L = o.wl[warp];
-    auto member = [&](int e) { return cnt[e] > L.min_count && cnt[e] <= L.max_count; };
+    auto member = [&](int e) { return fam[e] == warp; };
     const int total = warp_exclusive_scan(
         E, [&](int e) { return member(e) ? (cnt[e] + L.chunk_rows - 1) / L.chunk_rows : 0; },
         [&](int e, int pre) {
@@ -281,17 +340,12 @@ MOE_DEVINL void build_work_lists(const int32_t* cnt, const int32_t* off, int E,
   }
   __syncthreads();
   for (int e = tid; e < E; e += blockDim.x) {
-    const int c = cnt[e];
-    if (c == 0) continue;
-    for (int i = 0; i < o.n_lists; ++i) {
-      const WorkList& L = o.wl[i];
-      if (c > L.min_count && c <= L.max_count) {
-        int base = chunk_base[e];
-        for (int r0 = 0; r0 < c; r0 += L.chunk_rows)
-          L.chunks[base++] = make_int4(e, off[e] + r0, min(L.chunk_rows, c - r0), row_base[e] + r0);
-        break;
-      }
-    }
+    const int c = cnt[e], l = fam[e];
+    if (l < 0) continue;
+    const WorkList& L = o.wl[l];
+    int base = chunk_base[e];
+    for (int r0 = 0; r0 < c; r0 += L.chunk_rows)
+      L.chunks[base++] = make_int4(e, off[e] + r0, min(L.chunk_rows, c - r0), row_base[e] + r0);
   }
 }
 
@@ -308,7 +362,7 @@ __global__ void __launch_bounds__(1024)
   uint32_t* bits = reinterpret_cast<uint32_t*>(sel + T * k);         // [T][8]
   int32_t* cnt = reinterpret_cast<int32_t*>(bits + T * 8);           // [256]
   int32_t* off = cnt + 256;                                          // [257]
-  int32_t* scratch = off + 257;                                      // [512]
+  int32_t* scratch = off + 257;                                      // [768]
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5, nwarps = blockDim.x >> 5;
   pdl_wait();
   pdl_launch_next();
@@ -652,8 +706,8 @@ __global__ void __launch_bounds__(256)
   extern __shared__ __align__(128) uint8_t smem_raw[];
   int32_t* cnt = reinterpret_cast<int32_t*>(smem_raw);  // [256]
   int32_t* off = cnt + 256;                             // [257]
-  int32_t* scratch = off + 257;                         // [512]
-  uint32_t* bits = reinterpret_cast<uint32_t*>(scratch + 512);  // [64][8]
+  int32_t* scratch = off + 257;                         // [768]
+  uint32_t* bits = reinterpret_cast<uint32_t*>(scratch + 768);  // [64][8]
   uint8_t* slot = reinterpret_cast<uint8_t*>(bits + TT * 8);    // [64][E] (k <= 256)
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int t0 = blockIdx.x * TT, nt = min(TT, T - t0);

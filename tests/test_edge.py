@@ -173,11 +173,11 @@ def test_tune_measures_the_dispatch_thresholds_and_auto_follows_them():
     d, h = inputs_on_gpu(1024, H, E, k, I, seed=1200)
     layer = moe.Moe(E, H, I, k)
     c = layer.tune(d["x"], d["W_router"], d["b_router"], d["W_gate_up"], d["W_down"])
-    path, stream_rows = layer.get_path()
+    path, crossover = layer.get_path()
     s, t = layer.get_dispatch()
-    assert path == moe.MOE_PATH_AUTO and stream_rows == c == s
-    assert 0 <= s <= t
-    print("measured dispatch thresholds: stream_rows", s, "tile_rows", t)
+    assert path == moe.MOE_PATH_AUTO and crossover == c
+    assert 0 <= c <= 1024 and t >= 1
+    print("measured: streaming in calls of <=", c, "tokens; tile_rows", t)
     assert layer.sync_status() == moe.MOE_OK
     # the layer with the measured thresholds still matches the oracle
     d2 = dict(d, x=d["x"][:300].contiguous())

@@ -21,17 +21,20 @@ if torch.cuda.is_available():
     import mixture_experts_layer_48_b200 as moe
 
 
-def _families(counts, stream_rows, tile_rows):
-    c = np.asarray(counts)
-    return (int(((c > 0) & (c <= stream_rows)).sum()),
-            int(((c > stream_rows) & (c <= tile_rows)).sum()), int((c > tile_rows).sum()))
+def _families(layer, T, counts):
+    """Experts per family as the library dispatches them (the bench's mirror of the rule)."""
+    import bench
+    _, stream_T = layer.get_path()
+    s, t = layer.get_dispatch()
+    f = bench.split_families(counts, "auto", T, stream_T, s, t)
+    return tuple(len(f[k]) for k in ("stream", "tile", "gemm"))
 
 
-def _run(T, E, H, I, k, seed, zipf=False, path=None, dispatch=None):
+def _run(T, E, H, I, k, seed, zipf=False, path=None, dispatch=None, crossover=-1):
     d, h = inputs_on_gpu(T, H, E, k, I, seed, zipf=zipf)
     layer = moe.Moe(E, H, I, k)
-    if path is not None:
-        layer.set_path(path)
+    if path is not None or crossover >= 0:
+        layer.set_path(moe.MOE_PATH_AUTO if path is None else path, crossover)
     if dispatch is not None:
         layer.set_dispatch(*dispatch)
     ref_route = host_route(h, k)
@@ -45,16 +48,46 @@ def _run(T, E, H, I, k, seed, zipf=False, path=None, dispatch=None):
     return layer, g, rep
 
 
-@pytest.mark.parametrize("T,dispatch", [(1024, None), (512, (16, 128)), (256, (8, 40))])
-def test_skewed_mid_T_mixes_all_three_families(T, dispatch):
-    """20b-shaped layer, Zipf-skewed routing: streaming, expert tiles and row tiles all take
-    experts in the same call."""
-    layer, g, rep = _run(T, 32, 2880, 2880, 4, seed=3, zipf=True, dispatch=dispatch)
-    s, t = layer.get_dispatch()
-    fam = _families(np.diff(g["expert_offsets"]), s, t)
-    print("hybrid T=%d thresholds=%s experts per family %s %s" % (T, (s, t), fam, json.dumps(
+@pytest.mark.parametrize("T,dispatch,expect", [(256, (8, 40), (8, 15, 9)),
+                                               (512, (16, 100), (6, 20, 6)),
+                                               (1024, (16, 128), (0, 22, 10))])
+def test_skewed_mid_T_mixes_the_families(T, dispatch, expect):
+    """20b-shaped layer, Zipf-skewed routing, streaming allowed at this T: streaming, expert
+    tiles and row tiles take experts in the same call.  At 1024 tokens the two experts with 13
+    and 14 rows are too few, with too many rows, to stream on their own: they join the expert
+    tiles (the snap rule), while the skew across the tile boundary keeps row tiles for the ten
+    largest experts."""
+    layer, g, rep = _run(T, 32, 2880, 2880, 4, seed=3, zipf=True, dispatch=dispatch, crossover=T)
+    fam = _families(layer, T, np.diff(g["expert_offsets"]).tolist())
+    print("hybrid T=%d dispatch=%s experts per family %s %s" % (T, dispatch, fam, json.dumps(
         {k: v for k, v in rep.items() if k != "set_changed"})))
-    assert all(n > 0 for n in fam), fam
+    assert fam == expect, fam
+
+
+@pytest.mark.parametrize("T", [1024, 1500])
+def test_tight_loads_do_not_split_across_the_tile_boundary(T):
+    """With no router bias the experts' loads sit close to T*k/E (128 and 188 rows here), on
+    both sides of tile_rows = 128: the call's counts move them all to one family (one launch
+    per projection); the layer stays exact."""
+    E, H, I, k = 32, 2880, 2880, 4
+    d, h = inputs_on_gpu(T, H, E, k, I, seed=2700 + T)
+    d["b_router"].zero_()
+    h = mi.host_inputs(d)
+    layer = moe.Moe(E, H, I, k)
+    ref_route = host_route(h, k)
+    g = gpu_route(layer, d)
+    compare_routing(g, ref_route, k, E)
+    counts = np.diff(g["expert_offsets"]).tolist()
+    fam = _families(layer, T, counts)
+    print("tight loads T=%d counts %d..%d experts per family %s" % (T, min(counts), max(counts), fam))
+    assert sum(1 for n in fam if n) == 1, (fam, counts)
+    out = layer.forward(d["x"], d["W_router"], d["b_router"], d["W_gate_up"], d["W_down"])
+    assert layer.sync_status() == moe.MOE_OK
+    tokens = mi.sample_tokens(T, 256, 2700 + T)
+    got = out[torch.from_numpy(tokens).cuda()].double().cpu().numpy()
+    ref = oracle.moe_forward_ref(h["x"], h["W_router"], h["b_router"], h["W_gate_up"],
+                                 h["W_down"], k, tokens=tokens, route=ref_route)
+    check_outputs(got, tokens, h, ref_route, g, ref)
 
 
 @pytest.mark.parametrize("T", [17, 40, 129, 300, 777])
@@ -82,14 +115,18 @@ def test_auto_20b_mid_T(T):
 
 
 def test_thresholds_round_trip():
-    layer = moe.Moe(8, 256, 256, 2)
-    assert layer.get_dispatch() == (16, 256)
+    layer = moe.Moe(32, 2880, 2880, 4)
+    # streaming by default only while the touched experts' tiles fill < 2 waves of the SMs
+    sms = torch.cuda.get_device_properties(0).multi_processor_count
+    T0 = layer.get_path()[1]
+    assert min(32, (T0 + 1) * 4) * 23 >= 2 * sms > min(32, T0 * 4) * 23
+    assert layer.get_dispatch() == (16, 128)
     layer.set_dispatch(4, 100)
     assert layer.get_dispatch() == (4, 100)
     layer.set_dispatch(-1, 50)
     assert layer.get_dispatch() == (4, 50)
     layer.set_path(moe.MOE_PATH_AUTO, 9)
-    assert layer.get_path() == (moe.MOE_PATH_AUTO, 9) and layer.get_dispatch() == (9, 50)
+    assert layer.get_path() == (moe.MOE_PATH_AUTO, 9) and layer.get_dispatch() == (4, 50)
 
 
 def _wide_layer(E, H, I, k):

@@ -151,19 +151,33 @@ def test_gemm_path_means_expert_tiles_for_mxfp4():
 
 def test_inputs_beyond_f16_range():
     """|x| > 65504: the streaming kernels' f16 activations cannot hold it; the call reports it
-    (moe_sync_status: MOE_ERR_UNSUPPORTED) and the expert-tile kernel, whose activations stay
-    bf16, computes the layer exactly as the oracle does."""
-    def edit(d):
-        d["x"][3, 5] = 1.0e5
-        d["x"][7, 100] = -3.0e6
-
+    (moe_sync_status: MOE_ERR_UNSUPPORTED).  The expert-tile kernel keeps the activations in
+    bf16: every ordinary token matches the oracle element by element, and the two tokens that
+    carry the huge inputs match it relative to their row's largest output -- their h reaches
+    ~1e9, and the GPU's bf16 rounding of h (which the oracle does not do) is relative to that
+    scale, so outputs that cancel to a small value keep an error of the row's scale times 2^-8."""
     E, H, I, k, T = 8, 256, 256, 2, 12
     d = mi.make_inputs(T, H, E, k, I, 660, device="cuda", weights="mxfp4")
-    edit(d)
+    d["x"][3, 5] = 1.0e5
+    d["x"][7, 100] = -3.0e6
     layer = moe.Moe(E, H, I, k)
     layer.set_path(moe.MOE_PATH_STREAM)
-    layer.forward_mxfp4(d["x"], d["W_router"], d["b_router"], d["gu_codes"], d["gu_scales"],
-                        d["dn_codes"], d["dn_scales"])
+    args = (d["x"], d["W_router"], d["b_router"], d["gu_codes"], d["gu_scales"], d["dn_codes"],
+            d["dn_scales"])
+    layer.forward_mxfp4(*args)
     assert layer.sync_status() == moe.MOE_ERR_UNSUPPORTED
     assert layer.sync_status() == moe.MOE_OK
-    _run_mx(T, H, E, k, I, 660, edit=edit, path=moe.MOE_PATH_TILE)
+    layer.set_path(moe.MOE_PATH_TILE)
+    out = layer.forward_mxfp4(*args).double().cpu().numpy()
+    assert layer.sync_status() == moe.MOE_OK
+    assert np.isfinite(out).all()
+    h = mi.host_inputs(d)
+    ref = oracle.moe_forward_mxfp4_ref(h["x"], h["W_router"], h["b_router"], h["gu_codes"],
+                                       h["gu_scales"], h["dn_codes"], h["dn_scales"], k)
+    big = [3, 7]
+    rest = [t for t in range(T) if t not in big]
+    err = np.abs(out - ref)
+    assert np.all(err[rest] <= 1e-2 + 2e-2 * np.abs(ref[rest]))
+    for t in big:
+        scale = np.abs(ref[t]).max()
+        assert scale > 1e6 and err[t].max() <= 2e-2 * scale, (t, err[t].max(), scale)
