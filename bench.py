@@ -191,16 +191,17 @@ KERNEL_NAMES = {  # the gate/up kernel of each family, as ncu lists it
     "gemm": "grouped_gemm_kernel<gate_up>"}
 
 
-MX_STREAM_T = 512   # MXFP4 layers stream in calls of at most this many tokens
+MX_STREAM_T = 256   # MXFP4 layers stream in calls of at most this many tokens
 
 
 def split_families(counts, path: str, T: int, stream_T: int, stream_rows: int, tile_rows: int,
                    weights: str = "bf16") -> dict:
     """Row counts of the experts each kernel family multiplies, as the library dispatches them
     (moe_path in include/moe.h): with "auto", in calls of at most stream_T tokens an expert with
-    c <= stream_rows rows streams; the others take expert tiles up to tile_rows and row tiles
-    above, and a side of a boundary that the call's counts barely populate joins its neighbour
-    (the library's snap rule)."""
+    c <= stream_rows rows streams; the others take expert tiles up to tile_rows (unless the mean
+    load is at least 8 * tile_rows) and row tiles above, and a side of a boundary that the call's
+    counts barely populate joins its neighbour (the library's snap rule).  `counts` is the
+    call's full histogram (one entry per expert)."""
     out = {f: [] for f in FAMILIES}
     cs = [int(c) for c in counts if c > 0]
     if weights == "mxfp4":
@@ -213,9 +214,10 @@ def split_families(counts, path: str, T: int, stream_T: int, stream_rows: int, t
     s_on = T <= stream_T and stream_rows > 0
     lists = []                                   # (family, upper bound), launched families only
     lo = stream_rows if s_on else 0
+    mean = sum(int(c) for c in counts) // max(1, len(counts))   # T * k / E for a full histogram
     if s_on:
         lists.append(["stream", stream_rows])
-    if T > lo and tile_rows > lo:
+    if T > lo and tile_rows > lo and mean < 8 * tile_rows:
         lists.append(["tile", tile_rows])
     if T > max(lo, tile_rows):
         lists.append(["gemm", None])

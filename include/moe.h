@@ -36,10 +36,13 @@
  *     W_gate_up  [E, H, 2I]  bf16   (per expert: gate columns [0,I), up columns [I,2I))
  *     W_down     [E, I, H]   bf16
  *     out        [T, H]      fp32   (fully overwritten)
- * - Work is only enqueued on `stream` (a cudaStream_t; NULL = legacy default stream).  No
- *   call below synchronises, allocates device memory or reads device memory on the host,
- *   except moe_create / moe_destroy (allocate / free the handle's 4-byte device status word),
- *   moe_sync_status and moe_tune (which synchronise) and moe_profile_* (events).
+ * - Work is only enqueued on `stream` (a cudaStream_t; NULL = legacy default stream).  A call
+ *   whose experts take more than one kernel family may run the row tiles on a second stream
+ *   of the handle, forked from and joined back into `stream` with events, so the call stays
+ *   ordered on `stream`.  No call below synchronises, allocates device memory or reads device
+ *   memory on the host, except moe_create / moe_destroy (allocate / free the handle's 4-byte
+ *   device status word, its second stream and two events), moe_sync_status, moe_tune and
+ *   moe_last_dispatch (which synchronise) and moe_profile_* (events).
  * - Errors are returned, never thrown or aborted on.  Argument errors are found on the host
  *   before anything is enqueued and leave every buffer untouched.  A failed launch returns
  *   MOE_ERR_CUDA.  Faults detected on the device (a bounded wait that ran out) set the
@@ -153,7 +156,7 @@ MOE_API moe_status moe_forward(moe_t ctx, int T, const void* x_bf16, const void*
  * gu_codes [E, 2I, H/2] and gu_scales [E, H/32, 2I] hold W_gate_up [E, H, 2I] (gate columns
  * [0, I), up columns [I, 2I)); dn_codes [E, H, I/2] and dn_scales [E, I/32, H] hold W_down
  * [E, I, H].  x, W_router, b_router and out as in moe_forward; all pointers 16-byte aligned.
- * Two kernel families: MOE_PATH_AUTO streams the weights in calls of at most 512 tokens and
+ * Two kernel families: MOE_PATH_AUTO streams the weights in calls of at most 256 tokens and
  * runs the MXFP4 expert-tile kernel above; MOE_PATH_STREAM forces streaming, MOE_PATH_TILE and
  * MOE_PATH_GEMM expert tiles (there is no MXFP4 row-tile GEMM).
  *   - expert tiles: the codes are widened to bf16 weights in shared memory (exact: an E2M1 value
@@ -242,6 +245,15 @@ MOE_API moe_status moe_tune(moe_t ctx, int T_max, const void* x_bf16, const void
                     const float* b_router, const void* W_gate_up_bf16,
                     const void* W_down_bf16, float* out, void* workspace, size_t ws_bytes,
                     moe_stream_t stream, int* crossover_out);
+
+/* Which kernels the last moe_forward (mxfp4 = 0) or moe_forward_mxfp4 (mxfp4 = 1) call of T
+ * tokens on this workspace ran: synchronises `stream`, then writes for each family (0 weight
+ * streaming, 1 expert tiles, 2 row tiles) the number of work-list entries it processed, or -1
+ * if the call did not launch that family.  An entry is a row chunk of one expert (up to 16, 128
+ * or 256 rows).  The handle's path and thresholds must be those of that call.  For
+ * diagnostics and tests; reads device memory. */
+MOE_API moe_status moe_last_dispatch(moe_t ctx, int T, int mxfp4, const void* workspace,
+                                     size_t ws_bytes, int32_t* entries, moe_stream_t stream);
 
 /* Synchronise `stream`, then read and clear the handle's device status word.  Returns
  * MOE_ERR_TIMEOUT if a device-side bounded wait gave up since the last call, MOE_ERR_ARG if a

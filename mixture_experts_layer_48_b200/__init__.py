@@ -62,6 +62,7 @@ _SIGS = {
     "moe_experts_workspace_bytes": (_sz, [_vp, _c_int, _c_int]),
     "moe_experts": (_c_int, [_vp, _c_int, _c_int, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _sz, _vp]),
     "moe_combine": (_c_int, [_vp, _c_int, _vp, _vp, _vp, _vp]),
+    "moe_last_dispatch": (_c_int, [_vp, _c_int, _c_int, _vp, _sz, _vp, _vp]),
     "moe_route_static_max_bytes": (_sz, []),
     "moe_route_static": (_c_int, [_vp, _c_int, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp]),
 }
@@ -285,6 +286,15 @@ class Moe:
                       _stream(stream), ctypes.byref(c))
         _check(st, "moe_tune")
         return c.value
+
+    def last_dispatch(self, T: int, workspace=None, mxfp4: bool = False, stream=None) -> tuple:
+        """Work-list entries per family (streaming, expert tiles, row tiles; -1: not launched)
+        of the last forward call of T tokens on `workspace` (default: the layer's own)."""
+        ws = self._ws if workspace is None else workspace
+        out = (ctypes.c_int32 * 3)()
+        _check(moe_last_dispatch(self._h, T, int(mxfp4), ws.data_ptr(), ws.numel(), out,
+                                 _stream(stream)), "moe_last_dispatch")
+        return tuple(out)
 
     # -- status and measurement --------------------------------------------------------
     def sync_status(self, stream=None) -> int:

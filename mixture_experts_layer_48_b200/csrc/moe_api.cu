@@ -37,7 +37,7 @@ constexpr int kMaxT = 1 << 20;
 // the expert-tile kernel, more rows the row-tile grouped GEMM.
 constexpr int kDefaultStreamRows = 16;
 constexpr int kDefaultTileRows = 128;
-constexpr int kMxStreamT = 512;  // MXFP4: streaming for calls of at most this many tokens
+constexpr int kMxStreamT = 256;  // MXFP4: streaming for calls of at most this many tokens
 constexpr int kMaxKernelsPerCall = 12;
 
 moe_status static_scratch_address(void** out);  // defined beside the array, at the end
@@ -77,6 +77,8 @@ struct moe_ctx {
                                          // row tiles (moved across by the call's counts: snap)
   bool wide_rows = false;                // row tiles 256 x 512 (two MMAs per K step) or 256 x 256
   uint32_t* d_status = nullptr;
+  cudaStream_t aux = nullptr;            // second stream for a call whose families fork
+  cudaEvent_t ev_fork = nullptr, ev_join = nullptr;
   void* static_scratch = nullptr;  // device address of the routing scratch array (moe_route_static)
   uint64_t launches = 0;
   // profiling
@@ -260,8 +262,11 @@ Plan make_plan(const moe_ctx* c, int T, bool mx, moe_path path) {
     default: {
       const bool s_on = T <= c->stream_T && c->stream_rows > 0;
       const int lo = s_on ? c->stream_rows : 0;
+      // expert tiles are left out when the mean load is far above their range: an expert
+      // that small would be a rare outlier, and row tiles handle it (padded)
+      const long long mean = (long long)T * c->k / c->E;
       p.has[kFamStream] = s_on;
-      p.has[kFamTile] = T > lo && c->tile_rows > lo;
+      p.has[kFamTile] = T > lo && c->tile_rows > lo && mean < 8LL * c->tile_rows;
       p.has[kFamGemm] = T > std::max(lo, c->tile_rows);
       p.max_count[kFamStream] = (p.has[kFamTile] || p.has[kFamGemm]) ? c->stream_rows : INT_MAX;
       p.max_count[kFamTile] = p.has[kFamGemm] ? c->tile_rows : INT_MAX;
@@ -591,10 +596,27 @@ struct ExpertIO {
 moe_status expert_phase(moe_ctx* c, const Plan& p, const ExpertIO& io, const void* W_gate_up_bf16,
                         const void* W_down_bf16, const MxWeights* mx, cudaStream_t st) {
   const size_t R = (size_t)io.R;
-  // `out` is zero-filled once, by one gate/up kernel: the row-tile GEMM's epilogue warps while
-  // its tensor cores run, else the first other gate/up kernel before its dependency wait.
-  const int zero_owner = p.has[kFamGemm] ? kFamGemm : p.has[kFamStream] ? kFamStream : kFamTile;
   const int pair_grid = c->num_sms & ~1;  // whole CTA pairs
+  // With more than one family the row tiles run on the handle's second stream, concurrently
+  // with the other families: a family with little or no work is then off the critical path,
+  // and families that share a call share the SMs.  `out` is zero-filled before the fork.
+  const int n_fam = (int)p.has[kFamStream] + (int)p.has[kFamTile] + (int)p.has[kFamGemm];
+  const bool fork = n_fam >= 2 && p.has[kFamGemm] && c->aux != nullptr;
+  const cudaStream_t gst = fork ? c->aux : st;   // stream of the row-tile family
+  // `out` is zero-filled once: before the fork, else by one gate/up kernel (the row-tile GEMM's
+  // epilogue warps while its tensor cores run, or the first other one before its dependency wait)
+  int zero_owner = p.has[kFamGemm] ? kFamGemm : p.has[kFamStream] ? kFamStream : kFamTile;
+  if (fork) {
+    zero_owner = -1;
+    const size_t n4 = io.out_elems / 4;
+    MOE_TRY(launch(c, kKindGather, st, [&] {
+      return launch_pdl(zero_out_kernel, dim3(2 * c->num_sms), dim3(256), 0, st,
+                        reinterpret_cast<float4*>(io.out), n4);
+    }));
+    if (cudaEventRecord(c->ev_fork, st) != cudaSuccess ||
+        cudaStreamWaitEvent(c->aux, c->ev_fork, 0) != cudaSuccess)
+      return MOE_ERR_CUDA;
+  }
 
   // ---------------------------- gate/up projection + SwiGLU ----------------------------
   if (p.has[kFamStream]) {
@@ -690,14 +712,16 @@ moe_status expert_phase(moe_ctx* c, const Plan& p, const ExpertIO& io, const voi
     g.H = c->H;
     g.status = c->d_status;
     // the epilogue warps zero-fill `out`, which the down projections accumulate into
-    g.zero4 = reinterpret_cast<float4*>(io.out);
-    g.n_zero4 = io.out_elems / 4;
-    MOE_TRY(launch(c, kKindGateUpGemm, st, [&] {
+    if (zero_owner == kFamGemm) {
+      g.zero4 = reinterpret_cast<float4*>(io.out);
+      g.n_zero4 = io.out_elems / 4;
+    }
+    MOE_TRY(launch(c, kKindGateUpGemm, gst, [&] {
       if (c->wide_rows)
         return launch_pdl(grouped_gemm_wide_kernel<0>, dim3(pair_grid), dim3(kWideThreads),
-                          WideCfg<0>::kSmem, st, g, *am, *wgu);
+                          WideCfg<0>::kSmem, gst, g, *am, *wgu);
       return launch_pdl(grouped_gemm_2sm_kernel<MOE_GEMM_GATE_UP>, dim3(pair_grid),
-                        dim3(kGemmThreads), Gemm2Cfg<kGemmStages>::kSmem, st, g, *am, *wgu);
+                        dim3(kGemmThreads), Gemm2Cfg<kGemmStages>::kSmem, gst, g, *am, *wgu);
     }));
   }
 
@@ -781,14 +805,17 @@ moe_status expert_phase(moe_ctx* c, const Plan& p, const ExpertIO& io, const voi
     d.out = io.out;
     d.H = c->H;
     d.status = c->d_status;
-    MOE_TRY(launch(c, kKindDownGemm, st, [&] {
+    MOE_TRY(launch(c, kKindDownGemm, gst, [&] {
       if (c->wide_rows)
         return launch_pdl(grouped_gemm_wide_kernel<1>, dim3(pair_grid), dim3(kWideThreads),
-                          WideCfg<1>::kSmem, st, d, *hm, *wdn);
+                          WideCfg<1>::kSmem, gst, d, *hm, *wdn);
       return launch_pdl(grouped_gemm_2sm_kernel<MOE_GEMM_DOWN>, dim3(pair_grid),
-                        dim3(kGemmThreads), Gemm2Cfg<kGemmStages>::kSmem, st, d, *hm, *wdn);
+                        dim3(kGemmThreads), Gemm2Cfg<kGemmStages>::kSmem, gst, d, *hm, *wdn);
     }));
   }
+  if (fork && (cudaEventRecord(c->ev_join, c->aux) != cudaSuccess ||
+               cudaStreamWaitEvent(st, c->ev_join, 0) != cudaSuccess))
+    return MOE_ERR_CUDA;
   return MOE_OK;
 }
 
@@ -928,8 +955,15 @@ moe_status moe_create(int E, int H, int I, int k, moe_t* out) {
     delete c;
     return MOE_ERR_CUDA;
   }
-  // the routing scratch of moe_route_static, looked up with this handle's device current
-  if (static_scratch_address(&c->static_scratch) != MOE_OK) {
+  // the routing scratch of moe_route_static, looked up with this handle's device current;
+  // the second stream and its fork / join events for calls whose kernel families fork
+  if (static_scratch_address(&c->static_scratch) != MOE_OK ||
+      cudaStreamCreateWithFlags(&c->aux, cudaStreamNonBlocking) != cudaSuccess ||
+      cudaEventCreateWithFlags(&c->ev_fork, cudaEventDisableTiming) != cudaSuccess ||
+      cudaEventCreateWithFlags(&c->ev_join, cudaEventDisableTiming) != cudaSuccess) {
+    cudaGetLastError();
+    if (c->ev_fork) cudaEventDestroy(c->ev_fork);
+    if (c->aux) cudaStreamDestroy(c->aux);
     cudaFree(c->d_status);
     delete c;
     return MOE_ERR_CUDA;
@@ -941,6 +975,9 @@ moe_status moe_create(int E, int H, int I, int k, moe_t* out) {
 moe_status moe_destroy(moe_t c) {
   if (!c) return MOE_OK;
   for (cudaEvent_t e : c->ev) cudaEventDestroy(e);
+  if (c->ev_fork) cudaEventDestroy(c->ev_fork);
+  if (c->ev_join) cudaEventDestroy(c->ev_join);
+  if (c->aux) cudaStreamDestroy(c->aux);
   if (c->d_status) cudaFree(c->d_status);
   delete c;
   return MOE_OK;
@@ -1116,6 +1153,26 @@ moe_status moe_experts(moe_t c, int R, int S, const int32_t* seg_counts, const v
   if (c->in_call) ++c->prof_calls;
   c->in_call = false;
   return s;
+}
+
+moe_status moe_last_dispatch(moe_t c, int T, int mxfp4, const void* workspace, size_t ws_bytes,
+                             int32_t* entries, moe_stream_t stream) {
+  if (!c || !entries || T < 1 || T > kMaxT || !workspace) return MOE_ERR_ARG;
+  const Plan p = make_plan(c, T, mxfp4 != 0, c->path);
+  const Layout L = make_layout(c, T, p, mxfp4 != 0);
+  if (ws_bytes < L.total) return MOE_ERR_WORKSPACE;
+  if (cudaStreamSynchronize(reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess)
+    return MOE_ERR_CUDA;
+  for (int f = 0; f < kFamilies; ++f) {
+    entries[f] = -1;
+    if (!p.has[f]) continue;
+    int32_t v = 0;
+    if (cudaMemcpy(&v, static_cast<const uint8_t*>(workspace) + L.sched[f], sizeof(v),
+                   cudaMemcpyDeviceToHost) != cudaSuccess)
+      return MOE_ERR_CUDA;
+    entries[f] = v;
+  }
+  return MOE_OK;
 }
 
 moe_status moe_set_path(moe_t c, moe_path path, int crossover_T) {

@@ -769,6 +769,14 @@ __global__ void __launch_bounds__(256)
   }
 }
 
+// Zero-fill of the layer output before its kernel families fork onto two streams (every down
+// kernel adds into it).  grid-stride, float4 stores.
+__global__ void __launch_bounds__(256) zero_out_kernel(float4* __restrict__ z, size_t n4) {
+  pdl_wait();  // the previous call's down kernels may still add into `out`
+  pdl_launch_next();
+  zero_fill_f4(z, n4);
+}
+
 // Rows in expert order for the grouped GEMM when T is small: x_perm[r] = x[perm[r]].
 // One warp per row, 16-byte copies.  grid ceil(R/8), block 256.
 __global__ void __launch_bounds__(256) gather_rows_kernel(const uint16_t* __restrict__ x,

@@ -146,7 +146,7 @@ def test_family_split_follows_the_dispatch_rule():
     assert f == {"stream": [], "tile": [20, 30, 40], "gemm": [500, 600]}
     assert bench.split_families([5, 40], "gemm", 8, 3, 16, 128) == {"stream": [], "tile": [], "gemm": [5, 40]}
     assert bench.split_families([5, 40], "auto", 16, 3, 16, 128, "mxfp4")["stream"] == [5, 40]
-    assert bench.split_families([5, 40], "auto", 600, 3, 16, 128, "mxfp4")["tile"] == [5, 40]
+    assert bench.split_families([5, 40], "auto", 300, 3, 16, 128, "mxfp4")["tile"] == [5, 40]
 
 
 def test_family_work_and_dominant_roofline():

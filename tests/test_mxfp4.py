@@ -141,7 +141,8 @@ def test_expert_tiles_extreme_scales():
 
 @pytest.mark.parametrize("T", [64, 512])
 def test_auto_mixes_streaming_and_expert_tiles_gpt_oss_shape(T):
-    """20b shape: at 64 tokens most experts stream and a few take tiles; at 512 all take tiles."""
+    """20b shape with MXFP4 experts: AUTO streams the 64-token call and runs the 512-token call
+    on expert tiles."""
     _run_mx(T, 2880, 32, 4, 2880, 600 + T, sample=48)
 
 
