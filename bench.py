@@ -94,16 +94,19 @@ def source_digest(paths) -> str:
     return h.hexdigest()[:16]
 
 
-def ncu_traffic(kernel_key: str, workload: str) -> float | None:
-    """DRAM bytes per launch from the committed ncu summary, if the kernel is unchanged."""
+def ncu_traffic(kernel_key: str, workload: str, T: int) -> float | None:
+    """DRAM bytes per launch of a kernel on a workload and token count, from the committed ncu
+    summaries (profiles/traffic.json), if the kernel's sources are unchanged since."""
     try:
         with open(TRAFFIC_FILE) as f:
-            t = json.load(f)[kernel_key]
+            entries = json.load(f)[kernel_key]
     except (OSError, KeyError, ValueError):
         return None
-    if t.get("workload") != workload or t.get("sources_sha") != source_digest(t["sources"]):
-        return None
-    return float(t["dram_bytes_per_launch"])
+    for t in entries:
+        if (t.get("workload") == workload and t.get("T") == T
+                and t.get("sources_sha") == source_digest(t["sources"])):
+            return float(t["dram_bytes_per_launch"])
+    return None
 
 
 def parse_clocks(csv_text: str) -> dict:
@@ -490,7 +493,7 @@ def run_ours(args, w: mi.Workload, T: int) -> None:
     if mx:
         roof["kernel"] = {"stream": "stream_gate_up_mx_kernel",
                           "tile": "expert_tile_mx_kernel<0>"}.get(roof["family"], roof["kernel"])
-    roof["traffic"] = ncu_traffic(roof["kernel"], w.name)
+    roof["traffic"] = ncu_traffic(roof["kernel"], w.name, T)
     down_rate = {f"down_{f}_ms": round(dn_ms[f], 4) for f in FAMILIES if dn_ms[f] > 0}
     dispatch = dict(stream_T=stream_T, stream_rows=stream_rows, tile_rows=tile_rows,
                     experts={f: len(fams[f]) for f in FAMILIES},

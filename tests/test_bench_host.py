@@ -168,3 +168,19 @@ def test_family_work_and_dominant_roofline():
                                 1661.1, 1383.9, "measured")
     assert r["family"] == "gemm" and r["bound"] == "tensor" and r["unit"] == "TFLOP/s"
     assert r["achieved"] == pytest.approx(2 * 4096 * 32 * 2880 * 5760 / 12e-3 / 1e12)
+
+
+def test_traffic_lookup_matches_workload_T_and_sources():
+    import json
+    entries = json.load(open(bench.TRAFFIC_FILE))
+    for kernel, caps in entries.items():
+        for c in caps:
+            for p in c["sources"]:
+                assert os.path.exists(os.path.join(ROOT, p)), p
+            assert os.path.exists(os.path.join(ROOT, c["capture"])), c["capture"]
+            got = bench.ncu_traffic(kernel, c["workload"], c["T"])
+            # a committed capture stays valid only while its kernel's sources are unchanged
+            fresh = c["sources_sha"] == bench.source_digest(c["sources"])
+            assert (got == c["dram_bytes_per_launch"]) if fresh else got is None
+            assert bench.ncu_traffic(kernel, c["workload"], c["T"] + 1) is None
+    assert bench.ncu_traffic("no_such_kernel", "tiny", 64) is None
