@@ -198,13 +198,15 @@ MX_STREAM_T = 256   # MXFP4 layers stream in calls of at most this many tokens
 
 
 def split_families(counts, path: str, T: int, stream_T: int, stream_rows: int, tile_rows: int,
-                   weights: str = "bf16") -> dict:
+                   weights: str = "bf16", per_expert: bool = False) -> dict:
     """Row counts of the experts each kernel family multiplies, as the library dispatches them
     (moe_path in include/moe.h): with "auto", in calls of at most stream_T tokens an expert with
     c <= stream_rows rows streams; the others take expert tiles up to tile_rows (unless the mean
     load is at least 8 * tile_rows) and row tiles above, and a side of a boundary that the call's
-    counts barely populate joins its neighbour (the library's snap rule).  `counts` is the
-    call's full histogram (one entry per expert)."""
+    counts barely populate joins its neighbour (the library's snap rule).  Without per_expert,
+    the experts of expert tiles and row tiles then all go to one of the two, row tiles if their
+    mean count is at least tile_rows.  `counts` is the call's full histogram (one entry per
+    expert)."""
     out = {f: [] for f in FAMILIES}
     cs = [int(c) for c in counts if c > 0]
     if weights == "mxfp4":
@@ -246,6 +248,13 @@ def split_families(counts, path: str, T: int, stream_T: int, stream_rows: int, t
             for i in fam:
                 if fam[i] == src:
                     fam[i] = dst
+    names = [f for f, _ in lists]
+    if not per_expert and "tile" in names and "gemm" in names:
+        both = [i for i in fam if fam[i] in ("tile", "gemm")]
+        rows = sum(cs[i] for i in both)
+        dst = "gemm" if rows >= tile_rows * len(both) else "tile"
+        for i in both:
+            fam[i] = dst
     for i, f in fam.items():
         out[f].append(cs[i])
     return out
@@ -479,10 +488,10 @@ def run_ours(args, w: mi.Workload, T: int) -> None:
     # the kernel family that spent the most time ----
     hbm, bf16, bf16_sus, peak_src = measured_peaks()
     path_setting, stream_T = layer.get_path()
-    stream_rows, tile_rows = layer.get_dispatch()
+    stream_rows, tile_rows, per_expert = layer.get_dispatch()
     path = {moe.MOE_PATH_STREAM: "stream", moe.MOE_PATH_GEMM: "gemm",
             moe.MOE_PATH_TILE: "tile"}.get(path_setting, "auto")
-    fams = split_families(counts, path, T, stream_T, stream_rows, tile_rows, w.weights)
+    fams = split_families(counts, path, T, stream_T, stream_rows, tile_rows, w.weights, per_expert)
     work = {f: family_work(fams[f], w.H, w.I, w.weights) for f in FAMILIES}
     n_prof = prof_steps
     gu_ms = {f: prof["gate_up_" + f][0] / n_prof for f in FAMILIES}
@@ -496,6 +505,7 @@ def run_ours(args, w: mi.Workload, T: int) -> None:
     roof["traffic"] = ncu_traffic(roof["kernel"], w.name, T)
     down_rate = {f"down_{f}_ms": round(dn_ms[f], 4) for f in FAMILIES if dn_ms[f] > 0}
     dispatch = dict(stream_T=stream_T, stream_rows=stream_rows, tile_rows=tile_rows,
+                    per_expert=per_expert,
                     experts={f: len(fams[f]) for f in FAMILIES},
                     rows={f: int(sum(fams[f])) for f in FAMILIES})
 
@@ -542,7 +552,7 @@ def main(argv=None):
     ap.add_argument("--T", type=int, default=None)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--path", default="auto", choices=["auto", "stream", "tile", "gemm"],
-                    help="kernel family for every expert (default: chosen per expert)")
+                    help="kernel family for every expert (default: chosen from the call's counts)")
     args = ap.parse_args(argv)
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")

@@ -90,18 +90,21 @@ typedef enum {
  *                     as N, each weight block read once for up to 128 rows
  *   row tiles         2-SM tcgen05 grouped GEMM, 256 rows x 256 columns per CTA pair (prefill,
  *                     long sequences)
- * MOE_PATH_AUTO chooses per expert, on the device, from the call's histogram (no host sync):
- * in calls of at most crossover_T tokens the experts with at most stream_rows rows stream; the
- * others take expert tiles up to tile_rows rows and row tiles above.  When a call's counts put
- * a few experts just across the tile_rows boundary (an almost uniform routing), they join the
- * larger side instead of running as a second, half-filled launch: the upper side joins the lower
- * one if it holds no more experts and none has more than 2 * tile_rows rows, else the lower side
- * joins the upper one if it holds fewer experts and none has tile_rows / 2 rows or less.  This
- * is the per-expert mat-vec / mat-mat choice of the hearth-lean-loomed-v1 card ("Why 12-16
- * streams can be slow on Vulkan"), made per expert and per call.  The other values force one
- * family for every expert. */
+ * MOE_PATH_AUTO chooses on the device, from the call's histogram (no host sync): in calls of at
+ * most crossover_T tokens the experts with at most stream_rows rows stream.  The other experts
+ * take one tcgen05 family for the whole call by default: expert tiles if their mean row count
+ * is below tile_rows, row tiles otherwise (the two persistent kernels cannot share an SM, so a
+ * call that runs both pays for two partly filled passes over the GPU).  With per-expert
+ * dispatch on (moe_set_dispatch) each of them takes expert tiles up to tile_rows rows and row
+ * tiles above; when a call's counts put a few experts just across that boundary (an almost
+ * uniform routing), they join the larger side instead of running as a second, half-filled
+ * launch: the upper side joins the lower one if it holds no more experts and none has more
+ * than 2 * tile_rows rows, else the lower side joins the upper one if it holds fewer experts
+ * and none has tile_rows / 2 rows or less.  This is the mat-vec / mat-mat choice of the
+ * hearth-lean-loomed-v1 card ("Why 12-16 streams can be slow on Vulkan"), made per call (and
+ * per expert on request).  The other values force one family for every expert. */
 typedef enum {
-  MOE_PATH_AUTO = 0,    /* per-expert choice among the three families below */
+  MOE_PATH_AUTO = 0,    /* choice among the three families below from the call's counts */
   MOE_PATH_STREAM = 1,  /* every expert through the weight-streaming kernels */
   MOE_PATH_GEMM = 2,    /* every expert through the 2-SM row-tile grouped GEMM */
   MOE_PATH_TILE = 3     /* every expert through the expert-tile kernels */
@@ -224,11 +227,14 @@ MOE_API moe_status moe_set_path(moe_t ctx, moe_path path, int crossover_T);
 /* Current path setting and streaming crossover (tokens). */
 MOE_API moe_status moe_get_path(moe_t ctx, moe_path* path, int* crossover_T);
 
-/* The two per-expert AUTO thresholds, in rows of one expert: stream_rows (default 16, one
- * streaming chunk) and tile_rows (default 128, one expert tile).  A negative value keeps the
- * current one. */
-MOE_API moe_status moe_set_dispatch(moe_t ctx, int stream_rows, int tile_rows);
-MOE_API moe_status moe_get_dispatch(moe_t ctx, int* stream_rows, int* tile_rows);
+/* The AUTO thresholds, in rows of one expert: stream_rows (default 16, one streaming chunk) and
+ * tile_rows (default 128, one expert tile), and per_expert (default 0): 1 lets one call run
+ * expert tiles and row tiles side by side (each expert by its own count, the row tiles on the
+ * handle's second stream), 0 keeps the call's non-streamed experts in one of the two by their
+ * mean count.  A negative value keeps the current setting. */
+MOE_API moe_status moe_set_dispatch(moe_t ctx, int stream_rows, int tile_rows, int per_expert);
+MOE_API moe_status moe_get_dispatch(moe_t ctx, int* stream_rows, int* tile_rows,
+                                    int* per_expert);
 
 /* Measure the AUTO settings on this device with the caller's layer: times the whole layer
  * (median of 5 calls after 2 warm-ups) with every expert forced through each family, at

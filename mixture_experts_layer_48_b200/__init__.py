@@ -45,8 +45,9 @@ _SIGS = {
                                    _sz, _vp]),
     "moe_set_path": (_c_int, [_vp, _c_int, _c_int]),
     "moe_get_path": (_c_int, [_vp, ctypes.POINTER(_c_int), ctypes.POINTER(_c_int)]),
-    "moe_set_dispatch": (_c_int, [_vp, _c_int, _c_int]),
-    "moe_get_dispatch": (_c_int, [_vp, ctypes.POINTER(_c_int), ctypes.POINTER(_c_int)]),
+    "moe_set_dispatch": (_c_int, [_vp, _c_int, _c_int, _c_int]),
+    "moe_get_dispatch": (_c_int, [_vp, ctypes.POINTER(_c_int), ctypes.POINTER(_c_int),
+                                  ctypes.POINTER(_c_int)]),
     "moe_tune_workspace_bytes": (_sz, [_vp, _c_int]),
     "moe_tune": (_c_int, [_vp, _c_int, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _sz, _vp,
                           ctypes.POINTER(_c_int)]),
@@ -140,14 +141,18 @@ class Moe:
         _check(moe_get_path(self._h, ctypes.byref(p), ctypes.byref(c)), "moe_get_path")
         return p.value, c.value
 
-    def set_dispatch(self, stream_rows: int = -1, tile_rows: int = -1) -> None:
-        """AUTO thresholds in rows of one expert (negative: keep); see include/moe.h."""
-        _check(moe_set_dispatch(self._h, stream_rows, tile_rows), "moe_set_dispatch")
+    def set_dispatch(self, stream_rows: int = -1, tile_rows: int = -1, per_expert: int = -1) -> None:
+        """AUTO thresholds in rows of one expert and the per-expert switch (negative: keep);
+        see include/moe.h."""
+        _check(moe_set_dispatch(self._h, stream_rows, tile_rows, int(per_expert)),
+               "moe_set_dispatch")
 
-    def get_dispatch(self) -> tuple[int, int]:
-        s_, t_ = _c_int(), _c_int()
-        _check(moe_get_dispatch(self._h, ctypes.byref(s_), ctypes.byref(t_)), "moe_get_dispatch")
-        return s_.value, t_.value
+    def get_dispatch(self) -> tuple[int, int, bool]:
+        """(stream_rows, tile_rows, per_expert)."""
+        s_, t_, p_ = _c_int(), _c_int(), _c_int()
+        _check(moe_get_dispatch(self._h, ctypes.byref(s_), ctypes.byref(t_), ctypes.byref(p_)),
+               "moe_get_dispatch")
+        return s_.value, t_.value, bool(p_.value)
 
     def workspace_bytes(self, T: int) -> int:
         return moe_workspace_bytes(self._h, T)

@@ -75,6 +75,7 @@ struct moe_ctx {
   int stream_rows = kDefaultStreamRows;  // ... the experts with at most this many rows
   int tile_rows = kDefaultTileRows;      // experts up to this many rows take expert tiles; more:
                                          // row tiles (moved across by the call's counts: snap)
+  bool per_expert = false;               // expert tiles and row tiles side by side in a call
   bool wide_rows = false;                // row tiles 256 x 512 (two MMAs per K step) or 256 x 256
   uint32_t* d_status = nullptr;
   cudaStream_t aux = nullptr;            // second stream for a call whose families fork
@@ -188,11 +189,14 @@ struct RouteTmp {
   int splits = 1, kc_per_split = 0;  // large-T router: hidden-dimension slices per token block
 };
 
-// Large-T router split: enough (token block, hidden slice) blocks for about two per SM.
+constexpr int kTopkMaxSlices = 8;  // partial-logit slices topk_from_partials sums itself
+
+// Large-T router split: enough (token block, hidden slice) blocks for about two per SM, at most
+// kTopkMaxSlices slices (so the top-k kernel sums them without a separate pass).
 void router_split(const moe_ctx* c, int T, int* splits, int* kc_per_split) {
   const int NB = (T + kRouterTcTokens - 1) / kRouterTcTokens;
   const int nk = c->H / kRouterHSlice;
-  int S = std::max(1, std::min(nk, (2 * c->num_sms + NB - 1) / NB));
+  int S = std::max(1, std::min(std::min(nk, kTopkMaxSlices), (2 * c->num_sms + NB - 1) / NB));
   const int kcps = (nk + S - 1) / S;
   *kc_per_split = kcps;
   *splits = (nk + kcps - 1) / kcps;
@@ -235,6 +239,7 @@ struct Plan {
   bool has[kFamilies] = {false, false, false};
   int max_count[kFamilies] = {0, 0, 0};   // family f takes counts in (max_count[f-1], max_count[f]]
   bool snap = false;                      // the call's counts may move experts across a boundary
+  bool one_tc = false;                    // expert tiles or row tiles, not both, in one call
   int min_count(int f) const {
     int m = 0;
     for (int g = 0; g < f; ++g)
@@ -272,6 +277,7 @@ Plan make_plan(const moe_ctx* c, int T, bool mx, moe_path path) {
       p.max_count[kFamTile] = p.has[kFamGemm] ? c->tile_rows : INT_MAX;
       p.max_count[kFamGemm] = INT_MAX;
       p.snap = true;
+      p.one_tc = !c->per_expert && p.has[kFamTile] && p.has[kFamGemm];
     }
   }
   return p;
@@ -289,9 +295,10 @@ int default_stream_T(const moe_ctx* c) {
 }
 
 // Rows an expert of family f can hold in a call: its upper threshold, twice that when the call's
-// counts may move neighbours in (snap), unbounded for the last family.
+// counts may move neighbours in (snap), unbounded for the last family and for expert tiles that
+// may take every non-streamed expert (one_tc).
 long long family_row_bound(const Plan& p, int f) {
-  if (p.max_count[f] == INT_MAX) return LLONG_MAX;
+  if (p.max_count[f] == INT_MAX || (p.one_tc && f == kFamTile)) return LLONG_MAX;
   return (long long)p.max_count[f] * (p.snap ? 2 : 1);
 }
 
@@ -435,8 +442,6 @@ cudaError_t launch_router_tc(int NB, cudaStream_t st, const uint16_t* x, const u
                     RouterTcCfg<NT8>::smem(k), st, x, Wr, b, T, H, E, k, o.topk_idx, o.topk_w,
                     block_counts, zero4, n_zero4, rt.kc_per_split, partial);
 }
-
-constexpr int kTopkMaxSlices = 8;  // partial-logit slices topk_from_partials sums itself
 
 // Routing chain.  zero4/n_zero4: a float scratch region the router kernel zero-fills.
 moe_status launch_route(moe_ctx* c, int T, const uint16_t* x, const uint16_t* Wr,
@@ -600,8 +605,9 @@ moe_status expert_phase(moe_ctx* c, const Plan& p, const ExpertIO& io, const voi
   // With more than one family the row tiles run on the handle's second stream, concurrently
   // with the other families: a family with little or no work is then off the critical path,
   // and families that share a call share the SMs.  `out` is zero-filled before the fork.
-  const int n_fam = (int)p.has[kFamStream] + (int)p.has[kFamTile] + (int)p.has[kFamGemm];
-  const bool fork = n_fam >= 2 && p.has[kFamGemm] && c->aux != nullptr;
+  // Expert tiles and row tiles that exclude each other (one_tc) stay on one stream.
+  const bool fork = p.has[kFamGemm] && c->aux != nullptr &&
+                    (p.has[kFamStream] || (p.has[kFamTile] && !p.one_tc));
   const cudaStream_t gst = fork ? c->aux : st;   // stream of the row-tile family
   // `out` is zero-filled once: before the fork, else by one gate/up kernel (the row-tile GEMM's
   // epilogue warps while its tensor cores run, or the first other one before its dependency wait)
@@ -836,6 +842,7 @@ void plan_lists(const Plan& p, const Layout& L, uint8_t* ws, RouteOut& o, Expert
     io.sched[f] = wl.sched;
   }
   o.snap = p.snap ? 1 : 0;
+  o.one_of = p.one_tc ? (p.has[kFamStream] ? 1 : 0) : -1;  // the expert-tile list's index
   o.zero_i32 = p.has[kFamStream] ? reinterpret_cast<int32_t*>(ws + L.done) : nullptr;
   o.n_zero = p.has[kFamStream] ? L.n_done : 0;
   io.acc = p.has[kFamStream] ? reinterpret_cast<float*>(ws + L.acc) : nullptr;
@@ -1192,17 +1199,19 @@ moe_status moe_get_path(moe_t c, moe_path* path, int* crossover_T) {
   return MOE_OK;
 }
 
-moe_status moe_set_dispatch(moe_t c, int stream_rows, int tile_rows) {
+moe_status moe_set_dispatch(moe_t c, int stream_rows, int tile_rows, int per_expert) {
   if (!c) return MOE_ERR_ARG;
   if (stream_rows >= 0) c->stream_rows = stream_rows;
   if (tile_rows >= 0) c->tile_rows = tile_rows;
+  if (per_expert >= 0) c->per_expert = per_expert != 0;
   return MOE_OK;
 }
 
-moe_status moe_get_dispatch(moe_t c, int* stream_rows, int* tile_rows) {
+moe_status moe_get_dispatch(moe_t c, int* stream_rows, int* tile_rows, int* per_expert) {
   if (!c) return MOE_ERR_ARG;
   if (stream_rows) *stream_rows = c->stream_rows;
   if (tile_rows) *tile_rows = c->tile_rows;
+  if (per_expert) *per_expert = c->per_expert ? 1 : 0;
   return MOE_OK;
 }
 

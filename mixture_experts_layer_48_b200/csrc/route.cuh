@@ -78,6 +78,8 @@ struct RouteOut {
   WorkList wl[kMaxWorkLists];
   int n_lists;         // work lists to build (0: routing only)
   int snap;            // 1: let the call's counts move a barely-populated side of a boundary
+  int one_of = -1;     // >= 0: the experts of lists one_of and one_of + 1 all go to one of the
+                       // two, the upper one if their mean count reaches the boundary
   int32_t* zero_i32;   // region zeroed by the chain (completion counters), may be null
   int n_zero;
   const uint16_t* x;   // with x_perm non-null: copy token rows into expert order
@@ -262,6 +264,8 @@ MOE_DEVINL void zero_fill_f4(float4* z, size_t n4) {
 //     twice the boundary, they all join the lower list;
 //   - else, if the lower side holds fewer experts and none of them has half the boundary or
 //     less, they all join the upper list.
+// With o.one_of = l, the experts of lists l and l + 1 then all go to one of the two: the upper
+// one if their mean count is at least the boundary, else the lower one.
 // A skewed routing (counts far on both sides) keeps the per-expert choice.  Called by all
 // threads of a block; cnt and fam in shared memory (E <= 256).
 MOE_DEVINL void assign_families(const int32_t* cnt, int E, const RouteOut& o, int32_t* fam) {
@@ -305,6 +309,25 @@ MOE_DEVINL void assign_families(const int32_t* cnt, int E, const RouteOut& o, in
           if (fam[e] == from) fam[e] = to;
       __syncwarp();
     }
+  }
+  if (o.one_of >= 0 && tid < 32) {
+    const int lane = tid, l = o.one_of;
+    const int b = o.wl[l].max_count;
+    long long rows = 0;
+    int n = 0;
+    for (int e = lane; e < E; e += 32)
+      if (fam[e] == l || fam[e] == l + 1) {
+        ++n;
+        rows += cnt[e];
+      }
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) {
+      n += __shfl_xor_sync(0xffffffffu, n, off);
+      rows += __shfl_xor_sync(0xffffffffu, rows, off);
+    }
+    const int to = rows >= (long long)b * n ? l + 1 : l;
+    for (int e = lane; e < E; e += 32)
+      if (fam[e] == l || fam[e] == l + 1) fam[e] = to;
   }
   __syncthreads();
 }

@@ -88,8 +88,8 @@ def test_null_handle_calls(lib):
     assert lib.moe_forward(None, 1, None, None, None, None, None, None, None, 0, None) == lib.MOE_ERR_ARG
     assert lib.moe_route(None, 1, None, None, None, None, None, None, None, None, None, 0, None) == lib.MOE_ERR_ARG
     assert lib.moe_set_path(None, 0, -1) == lib.MOE_ERR_ARG
-    assert lib.moe_set_dispatch(None, 16, 256) == lib.MOE_ERR_ARG
-    assert lib.moe_get_dispatch(None, None, None) == lib.MOE_ERR_ARG
+    assert lib.moe_set_dispatch(None, 16, 256, 0) == lib.MOE_ERR_ARG
+    assert lib.moe_get_dispatch(None, None, None, None) == lib.MOE_ERR_ARG
     assert lib.moe_sync_status(None, None) == lib.MOE_ERR_ARG
     assert lib.moe_profile_begin(None, 4) == lib.MOE_ERR_ARG
     assert lib.moe_selftest_timeout(None, 10, None) == lib.MOE_ERR_ARG

@@ -133,17 +133,26 @@ def test_peak_labels_for_measured_and_fallback_peaks():
 
 
 def test_family_split_follows_the_dispatch_rule():
-    # a call allowed to stream: each expert by its own count, skew keeps three families
-    f = bench.split_families([0, 3, 4, 5, 16, 17, 40, 128, 300, 900], "auto", 1024, 1024, 16, 128)
+    # a call allowed to stream: each expert by its own count, skew keeps three families when the
+    # dispatch is per expert; by default the non-streamed experts take one tcgen05 family by
+    # their mean count (1385 rows / 5 experts >= 128: row tiles)
+    counts = [0, 3, 4, 5, 16, 17, 40, 128, 300, 900]
+    f = bench.split_families(counts, "auto", 1024, 1024, 16, 128, per_expert=True)
     assert f == {"stream": [3, 4, 5, 16], "tile": [17, 40, 128], "gemm": [300, 900]}
+    f = bench.split_families(counts, "auto", 1024, 1024, 16, 128)
+    assert f == {"stream": [3, 4, 5, 16], "tile": [], "gemm": [17, 40, 128, 300, 900]}
+    f = bench.split_families([0, 20, 30, 40, 200], "auto", 1024, 3, 16, 128)
+    assert f == {"stream": [], "tile": [20, 30, 40, 200], "gemm": []}
     # larger calls do not stream; uniform counts around the boundary snap to one family
     f = bench.split_families([100, 110, 120, 130, 140], "auto", 1024, 3, 16, 128)
     assert f == {"stream": [], "tile": [100, 110, 120, 130, 140], "gemm": []}
     f = bench.split_families([120, 130, 140, 150, 160], "auto", 1024, 3, 16, 128)
     assert f == {"stream": [], "tile": [], "gemm": [120, 130, 140, 150, 160]}
-    # skew across the boundary keeps the per-expert choice
-    f = bench.split_families([20, 30, 40, 500, 600], "auto", 1024, 3, 16, 128)
+    # skew across the boundary keeps the per-expert choice when asked for
+    f = bench.split_families([20, 30, 40, 500, 600], "auto", 1024, 3, 16, 128, per_expert=True)
     assert f == {"stream": [], "tile": [20, 30, 40], "gemm": [500, 600]}
+    f = bench.split_families([20, 30, 40, 500, 600], "auto", 1024, 3, 16, 128)
+    assert f == {"stream": [], "tile": [], "gemm": [20, 30, 40, 500, 600]}
     assert bench.split_families([5, 40], "gemm", 8, 3, 16, 128) == {"stream": [], "tile": [], "gemm": [5, 40]}
     assert bench.split_families([5, 40], "auto", 16, 3, 16, 128, "mxfp4")["stream"] == [5, 40]
     assert bench.split_families([5, 40], "auto", 300, 3, 16, 128, "mxfp4")["tile"] == [5, 40]

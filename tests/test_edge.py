@@ -174,7 +174,7 @@ def test_tune_measures_the_dispatch_thresholds_and_auto_follows_them():
     layer = moe.Moe(E, H, I, k)
     c = layer.tune(d["x"], d["W_router"], d["b_router"], d["W_gate_up"], d["W_down"])
     path, crossover = layer.get_path()
-    s, t = layer.get_dispatch()
+    s, t, _ = layer.get_dispatch()
     assert path == moe.MOE_PATH_AUTO and crossover == c
     assert 0 <= c <= 1024 and t >= 1
     print("measured: streaming in calls of <=", c, "tokens; tile_rows", t)

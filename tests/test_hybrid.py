@@ -28,8 +28,8 @@ def _families(layer, T, counts):
     """Experts per family as the dispatch rule assigns them (the bench's mirror of the rule)."""
     import bench
     _, stream_T = layer.get_path()
-    s, t = layer.get_dispatch()
-    f = bench.split_families(counts, "auto", T, stream_T, s, t)
+    s, t, per_expert = layer.get_dispatch()
+    f = bench.split_families(counts, "auto", T, stream_T, s, t, per_expert=per_expert)
     return tuple(len(f[k]) for k in ("stream", "tile", "gemm")), f
 
 
@@ -61,23 +61,30 @@ def _run(T, E, H, I, k, seed, zipf=False, path=None, dispatch=None, crossover=-1
     return layer, g, rep
 
 
-@pytest.mark.parametrize("T,dispatch,expect", [(256, (8, 40), (True, True, True)),
-                                               (512, (16, 100), (True, True, True)),
-                                               (1024, (16, 128), (False, True, True))])
+@pytest.mark.parametrize("T,dispatch,expect", [(256, (8, 40, 1), (True, True, True)),
+                                               (512, (16, 100, 1), (True, True, True)),
+                                               (1024, (16, 128, 1), (False, True, True)),
+                                               (256, (8, 40, 0), (True, None, None)),
+                                               (1024, (16, 128, 0), (False, False, True)),
+                                               (1024, (16, 1000, 0), (False, True, False))])
 def test_skewed_mid_T_mixes_the_families(T, dispatch, expect):
-    """20b-shaped layer, Zipf-skewed routing, streaming allowed at this T: streaming, expert
-    tiles and row tiles take experts in the same call, and the work lists built on the device
-    are the ones the rule gives for the call's histogram.  At 1024 tokens the few experts under
-    16 rows are too few, with too many rows, to stream on their own: they join the expert tiles
-    (the snap rule), while the skew across the tile boundary keeps row tiles for the largest
-    experts."""
+    """20b-shaped layer, Zipf-skewed routing, streaming allowed at this T.  With per-expert
+    dispatch, streaming, expert tiles and row tiles take experts in the same call, and the work
+    lists built on the device are the ones the rule gives for the call's histogram.  At 1024
+    tokens the few experts under 16 rows are too few, with too many rows, to stream on their
+    own: they join the expert tiles (the snap rule), while the skew across the tile boundary
+    keeps row tiles for the largest experts.  Without it, the non-streamed experts take one
+    tcgen05 family by their mean count (row tiles here, expert tiles once tile_rows is above
+    that mean)."""
     layer, g, rep = _run(T, 32, 2880, 2880, 4, seed=3, zipf=True, dispatch=dispatch, crossover=T)
     counts = np.diff(g["expert_offsets"]).tolist()
     fam, _ = _families(layer, T, counts)
     entries = _check_device_dispatch(layer, T, counts)
     print("hybrid T=%d dispatch=%s experts per family %s entries %s %s" % (
         T, dispatch, fam, entries, json.dumps({k: v for k, v in rep.items() if k != "set_changed"})))
-    assert all((n > 0) == want for n, want in zip(fam, expect)), (fam, sorted(counts))
+    assert all(want is None or (n > 0) == want for n, want in zip(fam, expect)), (fam, sorted(counts))
+    if not dispatch[2]:
+        assert fam[1] == 0 or fam[2] == 0, fam
 
 
 @pytest.mark.parametrize("T", [1024, 1500])
@@ -137,13 +144,15 @@ def test_thresholds_round_trip():
     sms = torch.cuda.get_device_properties(0).multi_processor_count
     T0 = layer.get_path()[1]
     assert min(32, (T0 + 1) * 4) * 23 >= 2 * sms > min(32, T0 * 4) * 23
-    assert layer.get_dispatch() == (16, 128)
-    layer.set_dispatch(4, 100)
-    assert layer.get_dispatch() == (4, 100)
+    assert layer.get_dispatch() == (16, 128, False)
+    layer.set_dispatch(4, 100, 1)
+    assert layer.get_dispatch() == (4, 100, True)
     layer.set_dispatch(-1, 50)
-    assert layer.get_dispatch() == (4, 50)
+    assert layer.get_dispatch() == (4, 50, True)
+    layer.set_dispatch(-1, -1, 0)
+    assert layer.get_dispatch() == (4, 50, False)
     layer.set_path(moe.MOE_PATH_AUTO, 9)
-    assert layer.get_path() == (moe.MOE_PATH_AUTO, 9) and layer.get_dispatch() == (4, 50)
+    assert layer.get_path() == (moe.MOE_PATH_AUTO, 9) and layer.get_dispatch() == (4, 50, False)
 
 
 def _wide_layer(E, H, I, k):
