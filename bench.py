@@ -391,6 +391,33 @@ def default_steps(step, stream, world: int) -> int:
     return int(reduce_max(float(k), world))
 
 
+def graph_timing(step, steps: int, world: int) -> dict:
+    """The same call captured once in a CUDA graph and replayed K times: no host launch work in
+    the timed region, so the difference from `us_per_layer` is what launching from the host
+    costs (it matters only at a few tokens per call)."""
+    g = torch.cuda.CUDAGraph()
+    try:
+        with torch.cuda.graph(g):
+            step()
+    except RuntimeError as e:      # capture refused: report it, the eager numbers stand
+        return dict(error=str(e).splitlines()[0][:200])
+    for _ in range(3):
+        g.replay()
+    torch.cuda.synchronize()
+    stream = torch.cuda.current_stream()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    if world > 1:
+        torch.distributed.barrier()
+    e0.record(stream)
+    for _ in range(steps):
+        g.replay()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    secs = reduce_max(e0.elapsed_time(e1) / 1e3, world)
+    del g
+    return dict(us_per_layer=secs / steps * 1e6, steps=steps)
+
+
 def run_ours(args, w: mi.Workload, T: int) -> None:
     rank, world, local = dist_env()
     if not torch.cuda.is_available():
@@ -483,6 +510,8 @@ def run_ours(args, w: mi.Workload, T: int) -> None:
     e1.record(stream)
     torch.cuda.synchronize()
     e2e_secs = reduce_max(e0.elapsed_time(e1) / 1e3, world)
+    graph = graph_timing(step, steps, world)
+    assert layer.sync_status() == moe.MOE_OK
 
     # ---- roofline of the dominant kernel: the gate/up projection (2/3 of bytes and FLOPs) of
     # the kernel family that spent the most time ----
@@ -531,6 +560,7 @@ def run_ours(args, w: mi.Workload, T: int) -> None:
                  h2d_bytes_per_step=T * w.H * 2, d2h_bytes_per_step=T * w.H * 4),
         gpu_launches=gpu_launches,
         clocks=clk.result(),
+        graph=graph,
     )
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         h = mi.host_inputs(d)

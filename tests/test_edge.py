@@ -216,3 +216,40 @@ def test_wide_hidden_and_intermediate(path):
     """H = I = 8192: long K loops and many column tiles in every path."""
     d, h = inputs_on_gpu(24, 8192, 2, 1, 8192, seed=1500)
     _check_layer(d, h, 2, 8192, 8192, 1, path=_path(path))
+
+
+@pytest.mark.parametrize("T,per_expert", [(3, 0), (40, 0), (300, 0), (300, 1)])
+def test_forward_replays_in_a_cuda_graph(T, per_expert):
+    """One call captured in a CUDA graph, replayed on new tokens written into the captured
+    input: the replay reads them and matches the oracle (streaming at 3 tokens, expert tiles at
+    40, row tiles at 300; the per-expert dispatch at 300 may fork the row tiles onto the handle's
+    second stream inside the capture)."""
+    E, H, I, k = 8, 256, 320, 2
+    d, _ = inputs_on_gpu(T, H, E, k, I, seed=2800 + T)
+    layer = moe.Moe(E, H, I, k)
+    layer.set_path(moe.MOE_PATH_AUTO, T)
+    layer.set_dispatch(-1, 64, per_expert)
+    x = d["x"].clone()
+    out = torch.empty((T, H), dtype=torch.float32, device="cuda")
+    ws = torch.empty(layer.workspace_bytes(T), dtype=torch.uint8, device="cuda")
+    fwd = lambda: layer.forward(x, d["W_router"], d["b_router"], d["W_gate_up"], d["W_down"],
+                                out=out, workspace=ws)
+    fwd()  # tensor maps built outside the capture
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        fwd()
+    x.copy_(mi.draw_x(T, H, 2900 + T, "cuda"))
+    out.fill_(float("nan"))
+    g.replay()
+    torch.cuda.synchronize()
+    assert layer.sync_status() == moe.MOE_OK
+    d2 = dict(d, x=x.clone())
+    h2 = mi.host_inputs(d2)
+    ref_route = host_route(h2, k)
+    gr = gpu_route(layer, d2)
+    compare_routing(gr, ref_route, k, E)
+    ref = oracle.moe_forward_ref(h2["x"], h2["W_router"], h2["b_router"], h2["W_gate_up"],
+                                 h2["W_down"], k, route=ref_route)
+    check_outputs(out.double().cpu().numpy(), np.arange(T), h2, ref_route, gr, ref)
+    del g
