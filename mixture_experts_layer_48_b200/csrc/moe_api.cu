@@ -273,6 +273,11 @@ Plan make_plan(const moe_ctx* c, int T, bool mx, moe_path path) {
       p.has[kFamStream] = s_on;
       p.has[kFamTile] = T > lo && c->tile_rows > lo && mean < 8LL * c->tile_rows;
       p.has[kFamGemm] = T > std::max(lo, c->tile_rows);
+      // one family per call: a mean load of tile_rows over all E experts already puts the call
+      // on row tiles (the touched experts' mean is at least that), so no expert-tile launch
+      if (!c->per_expert && !s_on && p.has[kFamGemm] &&
+          (long long)T * c->k >= (long long)c->tile_rows * c->E)
+        p.has[kFamTile] = false;
       p.max_count[kFamStream] = (p.has[kFamTile] || p.has[kFamGemm]) ? c->stream_rows : INT_MAX;
       p.max_count[kFamTile] = p.has[kFamGemm] ? c->tile_rows : INT_MAX;
       p.max_count[kFamGemm] = INT_MAX;
@@ -609,9 +614,10 @@ moe_status expert_phase(moe_ctx* c, const Plan& p, const ExpertIO& io, const voi
   const bool fork = p.has[kFamGemm] && c->aux != nullptr &&
                     (p.has[kFamStream] || (p.has[kFamTile] && !p.one_tc));
   const cudaStream_t gst = fork ? c->aux : st;   // stream of the row-tile family
-  // `out` is zero-filled once: before the fork, else by one gate/up kernel (the row-tile GEMM's
-  // epilogue warps while its tensor cores run, or the first other one before its dependency wait)
-  int zero_owner = p.has[kFamGemm] ? kFamGemm : p.has[kFamStream] ? kFamStream : kFamTile;
+  // `out` is zero-filled once: before the fork, else by one gate/up kernel (the expert-tile or
+  // streaming kernel before its dependency wait, while routing runs; the row-tile GEMM's epilogue
+  // warps while its tensor cores run when it is the only family)
+  int zero_owner = p.has[kFamTile] ? kFamTile : p.has[kFamStream] ? kFamStream : kFamGemm;
   if (fork) {
     zero_owner = -1;
     const size_t n4 = io.out_elems / 4;
