@@ -449,9 +449,12 @@ cudaError_t launch_router_tc(int NB, cudaStream_t st, const uint16_t* x, const u
 }
 
 // Routing chain.  zero4/n_zero4: a float scratch region the router kernel zero-fills.
+// finalize = false (T <= kSmallT only): stop after the partial logits; the streaming gate/up
+// kernel finishes the routing (StreamRoute).
 moe_status launch_route(moe_ctx* c, int T, const uint16_t* x, const uint16_t* Wr,
                         const float* b, const RouteOut& o, uint8_t* ws, const RouteTmp& rt,
-                        cudaStream_t st, float* zero = nullptr, size_t n_zero_floats = 0) {
+                        cudaStream_t st, float* zero = nullptr, size_t n_zero_floats = 0,
+                        bool finalize = true) {
   float4* zero4 = reinterpret_cast<float4*>(zero);
   const size_t n_zero4 = n_zero_floats / 4;
   const int E = c->E, H = c->H, k = c->k;
@@ -468,6 +471,7 @@ moe_status launch_route(moe_ctx* c, int T, const uint16_t* x, const uint16_t* Wr
       if (nt8 <= 16) return launch_router_tc<16>(1, st, x, Wr, b, T, H, E, k, o, nullptr, zero4, n_zero4, rt, partial);
       return launch_router_tc<32>(1, st, x, Wr, b, T, H, E, k, o, nullptr, zero4, n_zero4, rt, partial);
     }));
+    if (!finalize) return MOE_OK;
     const size_t smem_f = (size_t)T * E * 4 + (size_t)T * k * 4 + (size_t)T * 8 * 4 +
                           (256 + 257 + 768) * 4;
     MOE_TRY(launch(c, kKindRouteFin, st, [&] {
@@ -601,6 +605,7 @@ struct ExpertIO {
   float* acc;                         // streaming family: split-K sums, zero on entry
   int32_t* done;                      // streaming family: completion counters, zero on entry
   uint16_t* h;                        // [R, I] SwiGLU output
+  StreamRoute sr{};                   // routing finished by the streaming gate/up kernel, if set
 };
 
 moe_status expert_phase(moe_ctx* c, const Plan& p, const ExpertIO& io, const void* W_gate_up_bf16,
@@ -665,7 +670,7 @@ moe_status expert_phase(moe_ctx* c, const Plan& p, const ExpertIO& io, const voi
       if (!m) return MOE_ERR_CUDA;
       MOE_TRY(launch(c, kKindGateUp, st, [&] {
         return launch_pdl(stream_gate_up_kernel, dim3(c->num_sms), dim3(kStreamThreads),
-                          kGateUpSmem, st, ga, *m);
+                          kGateUpSmem, st, ga, io.sr, *m);
       }));
     }
   }
@@ -895,8 +900,26 @@ moe_status forward_plan(moe_ctx* c, int T, const void* x_bf16, const void* W_rou
     o.x_perm = x_perm;
     o.H = c->H;
   }
-  MOE_TRY(launch_route(c, T, x, static_cast<const uint16_t*>(W_router_bf16), b_router, o, ws,
-                       L.rt, st, io.acc, L.acc_floats));
+  // A few tokens on the streaming family alone: the gate/up kernel finishes the routing from
+  // the partial logits (no finalize kernel in between); the router zero-fills the completion
+  // counters and the split-K sums that follow them.
+  const bool fuse = !mx && p.has[kFamStream] && !p.has[kFamTile] && !p.has[kFamGemm] &&
+                    T <= kFusedRouteT && R <= (size_t)kFusedRouteRows && T <= kSmallT;
+  if (fuse) {
+    io.sr.partial = reinterpret_cast<const float*>(ws + L.rt.partial);
+    io.sr.S = L.rt.splits;
+    io.sr.b_router = b_router;
+    io.sr.T = T;
+    io.sr.E = c->E;
+    io.sr.k = c->k;
+    io.sr.o = o;
+    MOE_TRY(launch_route(c, T, x, static_cast<const uint16_t*>(W_router_bf16), b_router, o, ws,
+                         L.rt, st, reinterpret_cast<float*>(ws + L.done),
+                         (L.acc - L.done) / 4 + L.acc_floats, /*finalize=*/false));
+  } else {
+    MOE_TRY(launch_route(c, T, x, static_cast<const uint16_t*>(W_router_bf16), b_router, o, ws,
+                         L.rt, st, io.acc, L.acc_floats));
+  }
   if (x_perm && !fused_copy)
     MOE_TRY(launch(c, kKindGather, st, [&] {
       return launch_pdl(gather_rows_kernel, dim3((unsigned)((R + 7) / 8)), dim3(256), 0, st, x,

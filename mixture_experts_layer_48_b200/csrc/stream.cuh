@@ -30,6 +30,7 @@
 #pragma once
 
 #include "common.cuh"
+#include "route.cuh"
 
 namespace moe {
 
@@ -51,7 +52,11 @@ constexpr int kGUXPitch = kGateUpKC * 2 + 16;                      // activation
 constexpr int kDNXPitch = kDownKC * 2 + 16;                        // padded: conflict-free ldmatrix
 constexpr int kGUStageX = kStreamRB * kGUXPitch;
 constexpr int kDNStageX = kStreamRB * kDNXPitch;
-constexpr int kGateUpSmem = 1024 + kStreamStages * (kGUStageW + kGUStageX) + 2 * kStreamStages * 8;
+constexpr int kFusedRouteT = 8;       // largest call whose routing the gate/up kernel finishes
+constexpr int kFusedRouteRows = 64;   // ... with at most this many routed rows
+constexpr int kFusedRouteSmem = kFusedRouteRows * (16 + 4) + 16;  // its work list and row map
+constexpr int kGateUpSmem = 1024 + kStreamStages * (kGUStageW + kGUStageX) + 2 * kStreamStages * 8 +
+                            kFusedRouteSmem;
 constexpr int kDownSmem = 1024 + kStreamStages * (kDNStageW + kDNStageX) + 2 * kStreamStages * 8;
 static_assert(kGUStageW % 1024 == 0 && kDNStageW % 1024 == 0, "128B-swizzle atoms need 1 KB");
 static_assert(kGUXPitch % 16 == 0 && kDNXPitch % 16 == 0, "bulk copy alignment");
@@ -80,6 +85,21 @@ struct GateUpArgs {
   float* out;            // [T, H] zero-filled here
   size_t out_elems;
   uint32_t* status;
+};
+
+// Routing of a call of at most kFusedRouteT tokens (and T*k <= kFusedRouteRows rows), done by
+// every CTA of the gate/up kernel from the router's partial logits instead of by a finalize
+// kernel between them: the sum of the slices in slice order, top-k, softmax, histogram, scan,
+// the stable permutation and the work list, in shared memory, with the same functions and the
+// same order of operations as route_small_finalize_kernel (so the results are identical).  Every
+// CTA needs the work list before its first copy; CTA 0 also writes the routing results for the
+// caller and the down kernel.  Each touched expert holds at most T <= 16 rows: one entry.
+struct StreamRoute {
+  const float* partial;   // [S][T][E] partial logits; null: the routing kernels built the list
+  int S;
+  const float* b_router;  // [E]
+  int T, E, k;
+  RouteOut o;             // topk_idx, topk_w, offsets, perm, inv_perm, row_w, wl[0]
 };
 
 struct DownArgs {
@@ -146,15 +166,118 @@ MOE_DEVINL void gateup_stage_mma(uint32_t wbase, uint32_t xbase, int warp_c, int
   }
 }
 
+// What the fused routing keeps in shared memory past the prologue (its scratch is the ring).
+struct FusedRouteSmem {
+  int4 chunks[kFusedRouteRows];     // the streaming work list
+  int32_t perm[kFusedRouteRows];    // row -> token
+  int32_t n_chunks;
+};
+static_assert(sizeof(FusedRouteSmem) <= kFusedRouteSmem, "fused routing shared memory");
+
+// The routing finish of StreamRoute, by every thread of the block.  scratch: at least
+// (T*E + T*k + 256 + 257 + 256) * 4 bytes of shared memory that nothing else uses until the
+// barrier this function ends with.
+MOE_DEVINL void fused_route_cta(const StreamRoute& r, uint8_t* scratch, FusedRouteSmem& fs) {
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5, nwarps = blockDim.x >> 5;
+  const int T = r.T, E = r.E, k = r.k, S = r.S;
+  const bool writer = blockIdx.x == 0;
+  const RouteOut& o = r.o;
+  float* lg = reinterpret_cast<float*>(scratch);           // [T][E]
+  int32_t* sel = reinterpret_cast<int32_t*>(lg + T * E);   // [T][k]
+  int32_t* cnt = sel + T * k;                              // [256]
+  int32_t* off = cnt + 256;                                // [257]
+  int32_t* first = off + 257;                              // [256] list entry of each expert
+  for (int i = tid; i < T * E; i += blockDim.x) {
+    const int e = i % E;
+    float v = 0.f;  // slices added in order, as the finalize kernel does
+    int s = 0;
+    for (; s + 8 <= S; s += 8) {
+      float p[8];
+#pragma unroll
+      for (int q = 0; q < 8; ++q) p[q] = __ldcg(r.partial + (size_t)(s + q) * T * E + i);
+#pragma unroll
+      for (int q = 0; q < 8; ++q) v += p[q];
+    }
+    for (; s < S; ++s) v += __ldcg(r.partial + (size_t)s * T * E + i);
+    lg[i] = v + r.b_router[e];
+  }
+  for (int i = tid; i < 256; i += blockDim.x) cnt[i] = 0;
+  __syncthreads();
+  for (int t = warp; t < T; t += nwarps) {
+    float* row = lg + t * E;
+    int32_t* srow = sel + t * k;
+    warp_topk(row, E, k, srow);
+    const float denom = warp_softmax_denominator(row, k);
+    float wv[8];  // k <= 256: at most 8 slots per lane
+#pragma unroll
+    for (int q = 0; q < 8; ++q) {
+      const int j = lane + 32 * q;
+      wv[q] = (j < k) ? expf(row[j] - row[0]) / denom : 0.f;
+    }
+    __syncwarp();  // every lane has read row[0] before any weight overwrites it
+#pragma unroll
+    for (int q = 0; q < 8; ++q) {
+      const int j = lane + 32 * q;
+      if (j < k) {
+        if (writer) {
+          o.topk_idx[t * k + j] = srow[j];
+          o.topk_w[t * k + j] = wv[q];
+        }
+        row[j] = wv[q];  // the weight, for the row map below
+        atomicAdd(&cnt[srow[j]], 1);
+      }
+    }
+  }
+  __syncthreads();
+  if (warp == 0) {
+    const int total = warp_exclusive_scan(E, [&](int e) { return cnt[e]; },
+                                          [&](int e, int pre) { off[e] = pre; });
+    const int n = warp_exclusive_scan(E, [&](int e) { return cnt[e] > 0 ? 1 : 0; },
+                                      [&](int e, int pre) { first[e] = pre; });
+    if (lane == 0) {
+      off[E] = total;
+      fs.n_chunks = n;
+    }
+  }
+  __syncthreads();
+  // stable permutation: rank of (t, e) = earlier tokens that chose e (a token's k are distinct)
+  for (int i = tid; i < T * k; i += blockDim.x) {
+    const int t = i / k, e = sel[i];
+    int rank = 0;
+    for (int i2 = 0; i2 < t * k; ++i2) rank += sel[i2] == e ? 1 : 0;
+    const int rw = off[e] + rank;
+    fs.perm[rw] = t;
+    if (writer) {
+      o.perm[rw] = t;
+      o.inv_perm[i] = rw;
+      if (o.row_w) o.row_w[rw] = lg[t * E + (i - t * k)];
+    }
+  }
+  for (int e = tid; e < E; e += blockDim.x)
+    if (cnt[e] > 0) {  // one entry per touched expert (at most T <= 16 rows)
+      const int4 ch = make_int4(e, off[e], cnt[e], off[e]);
+      fs.chunks[first[e]] = ch;
+      if (writer) o.wl[0].chunks[first[e]] = ch;
+    }
+  if (writer) {
+    for (int e = tid; e <= E; e += blockDim.x) o.offsets[e] = off[e];
+    if (tid == 0) o.wl[0].sched[0] = fs.n_chunks;
+  }
+  fence_proxy_async_smem();  // the ring's copies overwrite the scratch next
+  __syncthreads();
+}
+
 // The weight tensor map views W_gate_up as [E*H rows, 2I columns], box [32 x 64], 128B swizzle.
 __global__ void __launch_bounds__(kStreamThreads, 1)
-    stream_gate_up_kernel(const GateUpArgs a, const __grid_constant__ CUtensorMap wmap) {
+    stream_gate_up_kernel(const GateUpArgs a, const StreamRoute r,
+                          const __grid_constant__ CUtensorMap wmap) {
   extern __shared__ __align__(128) uint8_t smem_raw[];
   __shared__ int s_last;
   uint8_t* wring = align1k(smem_raw);
   uint8_t* xring = wring + kStreamStages * kGUStageW;
   uint64_t* full = reinterpret_cast<uint64_t*>(xring + kStreamStages * kGUStageX);
   uint64_t* empty = full + kStreamStages;
+  FusedRouteSmem* fs = reinterpret_cast<FusedRouteSmem*>(empty + kStreamStages);
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   if (tid == 0) {
     for (int s = 0; s < kStreamStages; ++s) {
@@ -176,10 +299,21 @@ __global__ void __launch_bounds__(kStreamThreads, 1)
   pdl_wait();  // the routing results below come from the previous kernels
   pdl_launch_next();
 
+  const int4* chunks = a.chunks;
+  const int32_t* perm = a.perm;
+  int n_chunks;
+  if (r.partial != nullptr) {  // finish the routing here (every CTA the same way)
+    fused_route_cta(r, wring, *fs);
+    chunks = fs->chunks;
+    perm = fs->perm;
+    n_chunks = fs->n_chunks;
+  } else {
+    n_chunks = a.sched[0];
+  }
   const int I2 = 2 * a.I;
   const int NT = (a.I + kStreamCols - 1) / kStreamCols;
   const int nk = a.H / kGateUpKC;
-  const StreamKRange rng = stream_k_range((long long)a.sched[0] * NT, nk);
+  const StreamKRange rng = stream_k_range((long long)n_chunks * NT, nk);
 
   if (warp == kStreamWarps) {
     // ---------------- producer ----------------
@@ -192,9 +326,9 @@ __global__ void __launch_bounds__(kStreamThreads, 1)
       const int unit = (int)(g / nk), kb = (int)(g % nk);
       const int ke = (int)min((long long)nk, kb + (rng.g1 - g));
       g += ke - kb;
-      const int4 ch = a.chunks[unit / NT];
+      const int4 ch = chunks[unit / NT];
       const int col0 = (unit % NT) * kStreamCols;
-      const int tok = (lane < ch.z) ? a.perm[ch.y + lane] : 0;
+      const int tok = (lane < ch.z) ? perm[ch.y + lane] : 0;
       // lanes 0-4 load gate boxes, lanes 5-9 the matching up boxes
       const int box_col = lane < kStreamWarps ? col0 + kBox * lane
                                               : a.I + col0 + kBox * (lane - kStreamWarps);
@@ -239,7 +373,7 @@ __global__ void __launch_bounds__(kStreamThreads, 1)
     const int unit = (int)(g / nk), kb = (int)(g % nk);
     const int ke = (int)min((long long)nk, kb + (rng.g1 - g));
     g += ke - kb;
-    const int4 ch = a.chunks[unit / NT];
+    const int4 ch = chunks[unit / NT];
     const int col0 = (unit % NT) * kStreamCols;
     const int wg = min(kStreamCols, a.I - col0);
     const int nrows = ch.z;

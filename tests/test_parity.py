@@ -97,3 +97,28 @@ def test_120b_above_the_crossover(layer_120b, T, path):
                                      h["W_down"], w.k, route=ref_route)
     rep.update(check_outputs(out.double().cpu().numpy(), tokens, h, ref_route, g, ref_out))
     print("120b", path, T, json.dumps({k: v for k, v in rep.items() if k != "set_changed"}))
+
+
+@pytest.mark.parametrize("T", [1, 2, 3, 5, 8])
+def test_120b_streaming_finishes_its_routing(layer_120b, T):
+    """Calls of at most 8 tokens on the streaming family alone: the gate/up kernel finishes the
+    routing from the router's partial logits in every CTA (no finalize kernel).  Outputs against
+    the oracle, and the work list it left in the workspace has one entry per touched expert."""
+    w, d0, h0 = layer_120b
+    d = dict(d0, x=d0["x"][:T].contiguous())
+    h = dict(h0, x=h0["x"][:T])
+    layer = moe.Moe(w.E, w.H, w.I, w.k)
+    layer.set_path(moe.MOE_PATH_STREAM)
+    ref_route = host_route(h, w.k)
+    g = gpu_route(layer, d)
+    rep = compare_routing(g, ref_route, w.k, w.E)
+    ws = torch.empty(layer.workspace_bytes(T), dtype=torch.uint8, device="cuda")
+    out = layer.forward(d["x"], d["W_router"], d["b_router"], d["W_gate_up"], d["W_down"],
+                        workspace=ws)
+    assert layer.sync_status() == moe.MOE_OK
+    touched = int((np.diff(g["expert_offsets"]) > 0).sum())
+    assert layer.last_dispatch(T, workspace=ws)[0] == touched
+    ref_out = oracle.moe_forward_ref(h["x"], h["W_router"], h["b_router"], h["W_gate_up"],
+                                     h["W_down"], w.k, route=ref_route)
+    rep.update(check_outputs(out.double().cpu().numpy(), np.arange(T), h, ref_route, g, ref_out))
+    print("120b stream", T, json.dumps({k: v for k, v in rep.items() if k != "set_changed"}))
