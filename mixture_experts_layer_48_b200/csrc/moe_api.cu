@@ -773,7 +773,7 @@ moe_status expert_phase(moe_ctx* c, const Plan& p, const ExpertIO& io, const voi
       if (!m) return MOE_ERR_CUDA;
       MOE_TRY(launch(c, kKindDown, st, [&] {
         return launch_pdl(stream_down_kernel, dim3(c->num_sms), dim3(kStreamThreads),
-                          kDownSmem, st, da, io.sr, *m);
+                          kDownSmem, st, da, *m);
       }));
     }
   }

@@ -54,12 +54,10 @@ constexpr int kGUStageX = kStreamRB * kGUXPitch;
 constexpr int kDNStageX = kStreamRB * kDNXPitch;
 constexpr int kFusedRouteT = 8;       // largest call whose routing the gate/up kernel finishes
 constexpr int kFusedRouteRows = 64;   // ... with at most this many routed rows
-constexpr int kFusedRouteSmem = kFusedRouteRows * (16 + 4 + 4) + 16;  // work list, rows, weights
-constexpr int kFusedRouteStage = 16384;  // partial logits staged in shared memory (floats)
+constexpr int kFusedRouteSmem = kFusedRouteRows * (16 + 4) + 16;  // its work list and row map
 constexpr int kGateUpSmem = 1024 + kStreamStages * (kGUStageW + kGUStageX) + 2 * kStreamStages * 8 +
                             kFusedRouteSmem;
-constexpr int kDownSmem = 1024 + kStreamStages * (kDNStageW + kDNStageX) + 2 * kStreamStages * 8 +
-                          kFusedRouteSmem;
+constexpr int kDownSmem = 1024 + kStreamStages * (kDNStageW + kDNStageX) + 2 * kStreamStages * 8;
 static_assert(kGUStageW % 1024 == 0 && kDNStageW % 1024 == 0, "128B-swizzle atoms need 1 KB");
 static_assert(kGUXPitch % 16 == 0 && kDNXPitch % 16 == 0, "bulk copy alignment");
 
@@ -172,50 +170,36 @@ MOE_DEVINL void gateup_stage_mma(uint32_t wbase, uint32_t xbase, int warp_c, int
 struct FusedRouteSmem {
   int4 chunks[kFusedRouteRows];     // the streaming work list
   int32_t perm[kFusedRouteRows];    // row -> token
-  float row_w[kFusedRouteRows];     // row -> routing weight
   int32_t n_chunks;
 };
 static_assert(sizeof(FusedRouteSmem) <= kFusedRouteSmem, "fused routing shared memory");
 
-// The routing finish of StreamRoute, by every thread of the block; block 0 also writes the
-// results when `write` is set.  scratch: at least (T*E + T*k + 769 + S*T*E) * 4 bytes of shared
-// memory that nothing else uses until the barrier this function ends with.
-MOE_DEVINL void fused_route_cta(const StreamRoute& r, uint8_t* scratch, FusedRouteSmem& fs,
-                                bool write) {
+// The routing finish of StreamRoute, by every thread of the block.  scratch: at least
+// (T*E + T*k + 256 + 257 + 256) * 4 bytes of shared memory that nothing else uses until the
+// barrier this function ends with.
+MOE_DEVINL void fused_route_cta(const StreamRoute& r, uint8_t* scratch, FusedRouteSmem& fs) {
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5, nwarps = blockDim.x >> 5;
   const int T = r.T, E = r.E, k = r.k, S = r.S;
-  const bool writer = write && blockIdx.x == 0;
+  const bool writer = blockIdx.x == 0;
   const RouteOut& o = r.o;
   float* lg = reinterpret_cast<float*>(scratch);           // [T][E]
   int32_t* sel = reinterpret_cast<int32_t*>(lg + T * E);   // [T][k]
   int32_t* cnt = sel + T * k;                              // [256]
   int32_t* off = cnt + 256;                                // [257]
   int32_t* first = off + 257;                              // [256] list entry of each expert
-  float* stage = reinterpret_cast<float*>(first + 256);    // [S][T][E] when it fits
-  const int n = S * T * E;
-  if (n <= kFusedRouteStage) {
-    // every slice in flight at once (coalesced), then each logit's slices added in order
-    for (int i = tid; i < n; i += blockDim.x) stage[i] = __ldcg(r.partial + i);
-    __syncthreads();
-    for (int i = tid; i < T * E; i += blockDim.x) {
-      float v = 0.f;  // slice order, as the finalize kernel adds them
-      for (int s = 0; s < S; ++s) v += stage[s * T * E + i];
-      lg[i] = v + r.b_router[i % E];
-    }
-  } else {
-    for (int i = tid; i < T * E; i += blockDim.x) {
-      float v = 0.f;
-      int s = 0;
-      for (; s + 8 <= S; s += 8) {
-        float p[8];
+  for (int i = tid; i < T * E; i += blockDim.x) {
+    const int e = i % E;
+    float v = 0.f;  // slices added in order, as the finalize kernel does
+    int s = 0;
+    for (; s + 8 <= S; s += 8) {
+      float p[8];
 #pragma unroll
-        for (int q = 0; q < 8; ++q) p[q] = __ldcg(r.partial + (size_t)(s + q) * T * E + i);
+      for (int q = 0; q < 8; ++q) p[q] = __ldcg(r.partial + (size_t)(s + q) * T * E + i);
 #pragma unroll
-        for (int q = 0; q < 8; ++q) v += p[q];
-      }
-      for (; s < S; ++s) v += __ldcg(r.partial + (size_t)s * T * E + i);
-      lg[i] = v + r.b_router[i % E];
+      for (int q = 0; q < 8; ++q) v += p[q];
     }
+    for (; s < S; ++s) v += __ldcg(r.partial + (size_t)s * T * E + i);
+    lg[i] = v + r.b_router[e];
   }
   for (int i = tid; i < 256; i += blockDim.x) cnt[i] = 0;
   __syncthreads();
@@ -263,7 +247,6 @@ MOE_DEVINL void fused_route_cta(const StreamRoute& r, uint8_t* scratch, FusedRou
     for (int i2 = 0; i2 < t * k; ++i2) rank += sel[i2] == e ? 1 : 0;
     const int rw = off[e] + rank;
     fs.perm[rw] = t;
-    fs.row_w[rw] = lg[t * E + (i - t * k)];
     if (writer) {
       o.perm[rw] = t;
       o.inv_perm[i] = rw;
@@ -320,7 +303,7 @@ __global__ void __launch_bounds__(kStreamThreads, 1)
   const int32_t* perm = a.perm;
   int n_chunks;
   if (r.partial != nullptr) {  // finish the routing here (every CTA the same way)
-    fused_route_cta(r, wring, *fs, /*write=*/true);
+    fused_route_cta(r, wring, *fs);
     chunks = fs->chunks;
     perm = fs->perm;
     n_chunks = fs->n_chunks;
@@ -502,14 +485,12 @@ MOE_DEVINL void down_stage_mma(uint32_t wbase, uint32_t xbase, int warp_c, int l
 
 // The weight tensor map views W_down as [E*I rows, H columns], box [64 x 64], 128B swizzle.
 __global__ void __launch_bounds__(kStreamThreads, 1)
-    stream_down_kernel(const DownArgs a, const StreamRoute r,
-                       const __grid_constant__ CUtensorMap wmap) {
+    stream_down_kernel(const DownArgs a, const __grid_constant__ CUtensorMap wmap) {
   extern __shared__ __align__(128) uint8_t smem_raw[];
   uint8_t* wring = align1k(smem_raw);
   uint8_t* xring = wring + kStreamStages * kDNStageW;
   uint64_t* full = reinterpret_cast<uint64_t*>(xring + kStreamStages * kDNStageX);
   uint64_t* empty = full + kStreamStages;
-  FusedRouteSmem* fs = reinterpret_cast<FusedRouteSmem*>(empty + kStreamStages);
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   if (tid == 0) {
     for (int s = 0; s < kStreamStages; ++s) {
@@ -521,30 +502,12 @@ __global__ void __launch_bounds__(kStreamThreads, 1)
   __syncthreads();
 
   if (tid == 32 * kStreamWarps) tma_prefetch_desc(&wmap);
-  // With StreamRoute the work list comes from the router's partial logits, which the router
-  // finished writing before the gate/up kernel could start (and so before this one): the
-  // routing and the first weight stages run before the wait, while gate/up ends.  Otherwise
-  // the work list comes from the routing kernels, after the wait.
-  const bool early = r.partial != nullptr;
-  const int4* chunks = a.chunks;
-  const int32_t* perm = a.perm;
-  const float* row_w = a.row_w;
-  int n_chunks;
-  if (early) {
-    fused_route_cta(r, wring, *fs, /*write=*/false);
-    chunks = fs->chunks;
-    perm = fs->perm;
-    row_w = fs->row_w;
-    n_chunks = fs->n_chunks;
-  } else {
-    pdl_wait();  // h and the work list come from the previous kernels
-    pdl_launch_next();
-    n_chunks = a.sched[0];
-  }
+  pdl_wait();  // h and the work list come from the previous kernels
+  pdl_launch_next();
 
   const int NT = (a.H + kStreamCols - 1) / kStreamCols;
   const int nk = a.I / kDownKC;
-  const StreamKRange rng = stream_k_range((long long)n_chunks * NT, nk);
+  const StreamKRange rng = stream_k_range((long long)a.sched[0] * NT, nk);
 
   if (warp == kStreamWarps) {
     bool aborted = false;
@@ -552,29 +515,13 @@ __global__ void __launch_bounds__(kStreamThreads, 1)
     int last_it[kStreamStages];
 #pragma unroll
     for (int s = 0; s < kStreamStages; ++s) last_it[s] = -1;
-    // early: the weight boxes of the first stages (the ring is empty: no slot to wait for)
-    const int n_pre = early ? (int)min((long long)kStreamStages, rng.g1 - rng.g0) : 0;
-    for (int i = 0; i < n_pre; ++i) {
-      const long long g = rng.g0 + i;
-      const int unit = (int)(g / nk), kst = (int)(g % nk);
-      const int4 ch = chunks[unit / NT];
-      if (lane == 0) mbar_expect_tx(&full[i], (uint32_t)kDNStageW);
-      __syncwarp();
-      if (lane < kStreamWarps)
-        tma_load_2d(wring + i * kDNStageW + lane * kDNBoxBytes, &wmap,
-                    (unit % NT) * kStreamCols + kBox * lane, ch.x * a.I + kst * kDownKC, &full[i]);
-    }
-    if (early) {
-      pdl_wait();  // h comes from the gate/up kernel
-      pdl_launch_next();
-    }
     for (long long g = rng.g0; g < rng.g1;) {
       const int unit = (int)(g / nk), kb = (int)(g % nk);
       const int ke = (int)min((long long)nk, kb + (rng.g1 - g));
       g += ke - kb;
-      const int4 ch = chunks[unit / NT];
+      const int4 ch = a.chunks[unit / NT];
       const int col0 = (unit % NT) * kStreamCols;
-      const uint32_t hbytes = (uint32_t)ch.z * kDownKC * 2u;
+      const uint32_t bytes = (uint32_t)kDNStageW + (uint32_t)ch.z * kDownKC * 2u;
       for (int kst = kb; kst < ke; ++kst, ++it) {
         const int slot = it % kStreamStages;
         const uint32_t ph = (it / kStreamStages) & 1u;
@@ -584,11 +531,10 @@ __global__ void __launch_bounds__(kStreamThreads, 1)
         }
         aborted = __shfl_sync(0xffffffffu, aborted, 0);
         if (aborted) continue;
-        const bool pre = (int)it < n_pre;  // its weight boxes are already on the way
-        if (lane == 0) mbar_arrive_expect_tx(&full[slot], hbytes + (pre ? 0u : (uint32_t)kDNStageW));
+        if (lane == 0) mbar_arrive_expect_tx(&full[slot], bytes);
         __syncwarp();
         const int k0 = kst * kDownKC;
-        if (lane < kStreamWarps && !pre)
+        if (lane < kStreamWarps)
           tma_load_2d(wring + slot * kDNStageW + lane * kDNBoxBytes, &wmap, col0 + kBox * lane,
                       ch.x * a.I + k0, &full[slot]);
         if (lane < ch.z)
@@ -606,10 +552,6 @@ __global__ void __launch_bounds__(kStreamThreads, 1)
     return;
   }
 
-  if (early) {
-    pdl_wait();  // `out` is zero-filled by the gate/up kernel
-    pdl_launch_next();
-  }
   const uint32_t wring_s = smem_u32(wring), xring_s = smem_u32(xring);
   bool aborted = false;
   uint32_t it = 0;
@@ -617,7 +559,7 @@ __global__ void __launch_bounds__(kStreamThreads, 1)
     const int unit = (int)(g / nk), kb = (int)(g % nk);
     const int ke = (int)min((long long)nk, kb + (rng.g1 - g));
     g += ke - kb;
-    const int4 ch = chunks[unit / NT];
+    const int4 ch = a.chunks[unit / NT];
     const int col0 = (unit % NT) * kStreamCols;
     const int wc = min(kStreamCols, a.H - col0);
     const int nrows = ch.z;
@@ -654,8 +596,8 @@ __global__ void __launch_bounds__(kStreamThreads, 1)
 #pragma unroll
       for (int q = 0; q < 2; ++q) {
         const int r = nb * 8 + 2 * (lane & 3) + q;
-        tok[nb][q] = r < nrows ? perm[ch.y + r] : -1;
-        wt[nb][q] = r < nrows ? row_w[ch.y + r] : 0.f;
+        tok[nb][q] = r < nrows ? a.perm[ch.y + r] : -1;
+        wt[nb][q] = r < nrows ? a.row_w[ch.y + r] : 0.f;
       }
 #pragma unroll
     for (int mt = 0; mt < 4; ++mt)
