@@ -113,15 +113,17 @@ MOE_DEVINL void tma_load_2d_hint(void* smem_dst, const CUtensorMap* map, int c0,
       "l"(reinterpret_cast<uint64_t>(map)), "r"(c0), "r"(c1), "r"(smem_u32(bar)), "l"(policy)
       : "memory");
 }
-// L2 policies: bytes read once (leave first) and bytes that another kernel reads next (keep).
+// L2 policies: bytes read once (they leave first) and bytes with the normal priority (a
+// prefetch for the next kernel: it outlives evict-first lines, and nothing of it stays pinned
+// after the call, as evict-last lines would).
 MOE_DEVINL uint64_t l2_policy_evict_first() {
   uint64_t p;
   asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(p));
   return p;
 }
-MOE_DEVINL uint64_t l2_policy_evict_last() {
+MOE_DEVINL uint64_t l2_policy_evict_normal() {
   uint64_t p;
-  asm volatile("createpolicy.fractional.L2::evict_last.b64 %0, 1.0;" : "=l"(p));
+  asm volatile("createpolicy.fractional.L2::evict_normal.b64 %0, 1.0;" : "=l"(p));
   return p;
 }
 // Bring `bytes` (a multiple of 16, 16-byte aligned address) of global memory into L2.

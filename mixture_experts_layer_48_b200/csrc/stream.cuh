@@ -86,8 +86,9 @@ struct GateUpArgs {
   size_t out_elems;
   uint32_t* status;
   // When the touched experts' W_down fits in L2 (n_chunks * down_bytes <= down_l2_limit): the
-  // kernel brings it into L2 (kept) while it streams W_gate_up (read once, left first), so the
-  // down kernel reads it from L2.  down_w null: no prefetch.
+  // kernel brings it into L2 while it streams W_gate_up (read with the evict-first policy, so
+  // it leaves L2 before the prefetched lines do), and the down kernel reads it from L2.
+  // down_w null: no prefetch.
   const uint8_t* down_w;  // W_down [E, I, H] bf16
   size_t down_bytes;      // bytes of one expert's W_down
   size_t down_l2_limit;
@@ -332,7 +333,7 @@ __global__ void __launch_bounds__(kStreamThreads, 1)
     // (pieces blockIdx.x, blockIdx.x + gridDim.x, ...), while W_gate_up is read evict-first
     const bool pf = a.down_w != nullptr && (size_t)n_chunks * a.down_bytes <= a.down_l2_limit;
     const uint64_t pol_first = pf ? l2_policy_evict_first() : 0ull;
-    const uint64_t pol_last = pf ? l2_policy_evict_last() : 0ull;
+    const uint64_t pol_keep = pf ? l2_policy_evict_normal() : 0ull;
     constexpr uint32_t kPiece = 65536;
     const long long per_chunk = pf ? (long long)((a.down_bytes + kPiece - 1) / kPiece) : 0;
     const long long pf_end = per_chunk * n_chunks;
@@ -342,7 +343,7 @@ __global__ void __launch_bounds__(kStreamThreads, 1)
       if (lane == 0) {
         const long long c = pf_next / per_chunk, off = (pf_next % per_chunk) * kPiece;
         const uint32_t nb = (uint32_t)min((long long)kPiece, (long long)a.down_bytes - off);
-        prefetch_l2_bulk(a.down_w + (size_t)chunks[c].x * a.down_bytes + off, nb, pol_last);
+        prefetch_l2_bulk(a.down_w + (size_t)chunks[c].x * a.down_bytes + off, nb, pol_keep);
       }
       pf_next += gridDim.x;
     };
