@@ -10,7 +10,8 @@
 // mma.sync streaming kernel and too few rows to fill a 256-row MMA tile.  So the roles swap:
 //
 //   D[w, n] = sum_k W[k, w] * X[n, k]       w: 128 weight columns (TMEM lanes)
-//                                           n: the chunk's rows, rounded up to 16 (MMA N <= 128)
+//                                           n: the chunk's rows, rounded up to 16 (MMA N <= 128,
+//                                              or <= 256 in the 256-row variant)
 //
 // and each tile streams a [K x 128]-column block of one expert's weights exactly once for all of
 // that expert's rows (up to 128 per tile).  Work: tiles = (row chunk of one expert, column
@@ -52,11 +53,28 @@ constexpr int kEtSmem = 1024 + kEtStages * kEtStageBytes + 256 + kEtEpiBytes;
 constexpr int kEtTmemCols = 512;
 static_assert(kEtSmem <= 227 * 1024, "shared memory");
 
+// Tile shapes by rows per tile (the MMA's largest N): 128 rows keep two accumulator buffers of
+// 2 x 128 TMEM columns (the epilogue of one tile overlaps the MMAs of the next) and four stages;
+// 256 rows fill the 512 columns with one buffer (gate 256 | up 256) and take three stages of
+// 64 KB.  Per K step a 256-row tile reads the weight blocks once for twice the rows: the same
+// operand bytes per FLOP as the 2-SM row tiles, with rows padded to 16 instead of 256.
+template <int ROWS>
+struct EtCfg {
+  static_assert(ROWS == 128 || ROWS == 256, "rows per tile");
+  static constexpr int kStages = ROWS == 128 ? 4 : 3;
+  static constexpr int kBBytes = ROWS * kEtBK * 2;
+  static constexpr int kStageBytes = kEtABytes + kBBytes;
+  static constexpr int kAccBufs = kEtTmemCols / (2 * ROWS);
+  static constexpr int kSmem = 1024 + kStages * kStageBytes + 256 + kEtEpiBytes;
+  static_assert(kSmem <= 227 * 1024, "shared memory");
+  static_assert(kStageBytes % 1024 == 0, "128-byte swizzle atoms");
+};
+
 struct EtArgs {
   int K;                 // reduction length: H (gate/up) or I (down)
   int Ncols;             // gate/up: I (columns of each of gate and up); down: H
   int w_rows;            // weight rows per expert (= K)
-  const int4* chunks;    // {expert, first row, rows <= 128}
+  const int4* chunks;    // {expert, first row, rows <= ROWS}
   const int32_t* sched;  // [0] number of chunks
   uint16_t* h;           // gate/up output [R, I] bf16
   const int32_t* perm;   // down: token of each row
@@ -84,31 +102,32 @@ MOE_DEVINL int et_boxes(int j, int n0, int Ncols) {
 // Epilogue of the expert-tile kernels (warps 2-5, one TMEM lane quarter each): waits for each
 // tile's accumulators, writes h = silu(g) * u (gate/up) or adds w * y into out (down) through a
 // shared-memory transpose, and hands the accumulator buffer back.
-template <int MODE>
+template <int MODE, int ROWS>
 MOE_DEVINL void et_epilogue(const EtArgs& a, uint32_t tmem_base, uint64_t* acc_full,
                             uint64_t* acc_empty, float* epi, int tiles, int NT,
                             volatile int* abort_flag) {
+  using C = EtCfg<ROWS>;
   constexpr int TW = MODE == 0 ? kEtM : 2 * kEtM;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int q = warp & 3;                       // TMEM lanes 32q .. 32q + 31
   float* stage = epi + (warp - 2) * 32 * kEtPitch;
   int tile_i = 0;
   for (int t = blockIdx.x; t < tiles; t += gridDim.x, ++tile_i) {
-    const int buf = tile_i & 1;
-    const uint32_t aph = (tile_i >> 1) & 1u;
+    const int buf = tile_i % C::kAccBufs;
+    const uint32_t aph = (tile_i / C::kAccBufs) & 1u;
     if (!wait_or_abort(&acc_full[buf], aph, abort_flag, a.status)) break;
     tc_fence_after();
     const int4 ch = a.chunks[t / NT];
     const int n0 = (t % NT) * TW;
     const int nrows = ch.z;
-    const uint32_t tbase = tmem_base + ((uint32_t)(32 * q) << 16) + buf * 2 * kEtM;
+    const uint32_t tbase = tmem_base + ((uint32_t)(32 * q) << 16) + buf * 2 * ROWS;
     if constexpr (MODE == 0) {
       // this warp's 32 columns of gate and up: valid when the tile's last box is
       const bool cols_ok = n0 + 32 * q < a.Ncols;  // warp-uniform
       for (int r0 = 0; cols_ok && r0 < nrows; r0 += 32) {
         float g[32], u[32];
         tmem_ld32(tbase + r0, g);
-        tmem_ld32(tbase + kEtM + r0, u);
+        tmem_ld32(tbase + ROWS + r0, u);
 #pragma unroll
         for (int i = 0; i < 32; ++i) stage[i * kEtPitch + lane] = silu_fast(g[i]) * u[i];
         __syncwarp();
@@ -132,7 +151,7 @@ MOE_DEVINL void et_epilogue(const EtArgs& a, uint32_t tmem_base, uint64_t* acc_f
         if (col0 >= a.Ncols) continue;  // warp-uniform: columns past H
         for (int r0 = 0; r0 < nrows; r0 += 32) {
           float y[32];
-          tmem_ld32(tbase + j * kEtM + r0, y);
+          tmem_ld32(tbase + j * ROWS + r0, y);
           const bool rv = r0 + lane < nrows;
           const int tok = rv ? a.perm[ch.y + r0 + lane] : -1;
           const float w = rv ? a.row_w[ch.y + r0 + lane] : 0.f;
@@ -162,21 +181,23 @@ MOE_DEVINL void et_epilogue(const EtArgs& a, uint32_t tmem_base, uint64_t* acc_f
 // MODE 0: gate/up projection with the SwiGLU epilogue.  MODE 1: down projection with the
 // routing-weight + combine epilogue.  wmap: the weights as [E*K rows, columns], box 64 x 64,
 // 128-byte swizzle.  xmap: the activation rows [R, K], box 16 x 64, 128-byte swizzle.
-template <int MODE>
+template <int MODE, int ROWS = kEtRows>
 __global__ void __launch_bounds__(kEtThreads, 1)
     expert_tile_kernel(const EtArgs a, const __grid_constant__ CUtensorMap wmap,
                        const __grid_constant__ CUtensorMap xmap) {
+  using C = EtCfg<ROWS>;
+  constexpr int kStages = C::kStages, kStageBytes = C::kStageBytes, kBufs = C::kAccBufs;
   extern __shared__ __align__(128) uint8_t smem_raw[];
   __shared__ uint32_t s_tmem;
   __shared__ int s_abort;
   uint8_t* ring = align1k(smem_raw);
-  uint64_t* bars = reinterpret_cast<uint64_t*>(ring + kEtStages * kEtStageBytes);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(ring + kStages * kStageBytes);
   uint64_t* full = bars;
-  uint64_t* empty = full + kEtStages;
-  uint64_t* acc_full = empty + kEtStages;
+  uint64_t* empty = full + kStages;
+  uint64_t* acc_full = empty + kStages;
   uint64_t* acc_empty = acc_full + 2;
   uint64_t* drain = acc_empty + 2;
-  float* epi = reinterpret_cast<float*>(ring + kEtStages * kEtStageBytes + 256);
+  float* epi = reinterpret_cast<float*>(ring + kStages * kStageBytes + 256);
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
 
   if (warp == 1) {
@@ -184,11 +205,11 @@ __global__ void __launch_bounds__(kEtThreads, 1)
     tmem_relinquish();
   }
   if (tid == 0) {
-    for (int s = 0; s < kEtStages; ++s) {
+    for (int s = 0; s < kStages; ++s) {
       mbar_init(&full[s], 1);
       mbar_init(&empty[s], 1);
     }
-    for (int b = 0; b < 2; ++b) {
+    for (int b = 0; b < kBufs; ++b) {
       mbar_init(&acc_full[b], 1);
       mbar_init(&acc_empty[b], 128);
     }
@@ -221,9 +242,9 @@ __global__ void __launch_bounds__(kEtThreads, 1)
     // ------------------------------ TMA producer ------------------------------
     if (lane == 0) {
       uint32_t it = 0;
-      int last_it[kEtStages];
+      int last_it[kStages];
 #pragma unroll
-      for (int s = 0; s < kEtStages; ++s) last_it[s] = -1;
+      for (int s = 0; s < kStages; ++s) last_it[s] = -1;
       for (int t = blockIdx.x; t < tiles && !*abort_flag; t += gridDim.x) {
         const int4 ch = a.chunks[t / NT];
         const int n0 = (t % NT) * TW;
@@ -235,14 +256,14 @@ __global__ void __launch_bounds__(kEtThreads, 1)
         const int wrow0 = ch.x * a.w_rows;
         bool ok = true;
         for (int kst = 0; kst < nk; ++kst, ++it) {
-          const int slot = it % kEtStages;
-          const uint32_t ph = (it / kEtStages) & 1u;
+          const int slot = it % kStages;
+          const uint32_t ph = (it / kStages) & 1u;
           if (!wait_or_abort(&empty[slot], ph ^ 1u, abort_flag, a.status)) {
             ok = false;
             break;
           }
           mbar_arrive_expect_tx(&full[slot], bytes);
-          uint8_t* st = ring + slot * kEtStageBytes;
+          uint8_t* st = ring + slot * kStageBytes;
           const int k0 = kst * kEtBK;
           for (int b = 0; b < nb0; ++b)
             tma_load_2d(st + b * kEtBoxBytes, &wmap, c0 + 64 * b, wrow0 + k0, &full[slot]);
@@ -256,9 +277,9 @@ __global__ void __launch_bounds__(kEtThreads, 1)
         if (!ok) break;
       }
       // never leave the CTA with copies in flight
-      for (int s = 0; s < kEtStages; ++s)
+      for (int s = 0; s < kStages; ++s)
         if (last_it[s] >= 0 &&
-            !mbar_wait_bounded(&full[s], (last_it[s] / kEtStages) & 1u, kWaitLimitNs))
+            !mbar_wait_bounded(&full[s], (last_it[s] / kStages) & 1u, kWaitLimitNs))
           atomicOr(a.status, kStatusTimeout);
     }
   } else if (warp == 1) {
@@ -278,21 +299,21 @@ __global__ void __launch_bounds__(kEtThreads, 1)
         const int nb0 = et_boxes<MODE>(0, n0, a.Ncols), nb1 = et_boxes<MODE>(1, n0, a.Ncols);
         const int N = ((ch.z + kEtRowBox - 1) / kEtRowBox) * kEtRowBox;
         const uint32_t idesc = idesc_bf16_f32(kEtM, N, /*a_mn_major=*/true, /*b_mn_major=*/false);
-        const int buf = tile_i & 1;
-        const uint32_t aph = (tile_i >> 1) & 1u;
+        const int buf = tile_i % kBufs;
+        const uint32_t aph = (tile_i / kBufs) & 1u;
         if (!wait_or_abort(&acc_empty[buf], aph ^ 1u, abort_flag, a.status)) break;
         tc_fence_after();
-        const uint32_t d0 = tmem_base + buf * 2 * kEtM, d1 = d0 + kEtM;
+        const uint32_t d0 = tmem_base + buf * 2 * ROWS, d1 = d0 + ROWS;
         bool ok = true;
         for (int kst = 0; kst < nk; ++kst, ++it) {
-          const int slot = it % kEtStages;
-          const uint32_t ph = (it / kEtStages) & 1u;
+          const int slot = it % kStages;
+          const uint32_t ph = (it / kStages) & 1u;
           if (!wait_or_abort(&full[slot], ph, abort_flag, a.status)) {
             ok = false;
             break;
           }
           tc_fence_after();
-          const uint64_t soff = (uint64_t)((slot * kEtStageBytes) >> 4);
+          const uint64_t soff = (uint64_t)((slot * kStageBytes) >> 4);
 #pragma unroll
           for (int k16 = 0; k16 < kEtBK / 16; ++k16) {
             const uint64_t ak = adesc0 + soff + ((k16 * 16 * 128) >> 4);
@@ -314,7 +335,7 @@ __global__ void __launch_bounds__(kEtThreads, 1)
     }
   } else {
     // ------------------------------ epilogue ------------------------------
-    et_epilogue<MODE>(a, tmem_base, acc_full, acc_empty, epi, tiles, NT, abort_flag);
+    et_epilogue<MODE, ROWS>(a, tmem_base, acc_full, acc_empty, epi, tiles, NT, abort_flag);
   }
 
   tc_fence_before();

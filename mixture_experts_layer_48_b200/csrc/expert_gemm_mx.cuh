@@ -292,7 +292,7 @@ __global__ void __launch_bounds__(kEmxThreads, 1)
     }
   } else {
     // ------------------------------ epilogue (warps 2-5) ------------------------------
-    et_epilogue<MODE>(a, tmem_base, acc_full, acc_empty, epi, tiles, NT, abort_flag);
+    et_epilogue<MODE, kEtRows>(a, tmem_base, acc_full, acc_empty, epi, tiles, NT, abort_flag);
   }
 
   tc_fence_before();

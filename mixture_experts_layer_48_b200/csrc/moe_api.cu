@@ -77,6 +77,7 @@ struct moe_ctx {
   int tile_rows = kDefaultTileRows;      // experts up to this many rows take expert tiles; more:
                                          // row tiles (moved across by the call's counts: snap)
   bool per_expert = false;               // expert tiles and row tiles side by side in a call
+  int tile_n = 0;                        // rows per expert tile: 0 by the call's mean load, 128, 256
   bool wide_rows = false;                // row tiles 256 x 512 (two MMAs per K step) or 256 x 256
   uint32_t* d_status = nullptr;
   cudaStream_t aux = nullptr;            // second stream for a call whose families fork
@@ -235,12 +236,15 @@ RouteTmp carve_route_tmp(Carver& cv, const moe_ctx* c, int T, bool allow_split =
 // token picks an expert at most once), so families above T are not launched.
 enum Family { kFamStream = 0, kFamTile = 1, kFamGemm = 2, kFamilies = 3 };
 constexpr int kFamChunkRows[kFamilies] = {kStreamRB, kEtRows, kGemmChunkRows};
+constexpr int kEtWideRows = 256;   // rows per entry of the 256-row expert tiles
 
 struct Plan {
   bool has[kFamilies] = {false, false, false};
   int max_count[kFamilies] = {0, 0, 0};   // family f takes counts in (max_count[f-1], max_count[f]]
   bool snap = false;                      // the call's counts may move experts across a boundary
   bool one_tc = false;                    // expert tiles or row tiles, not both, in one call
+  int tile_entry_rows = kEtRows;          // rows per expert-tile entry: 128 or 256 (bf16 only)
+  int chunk_rows(int f) const { return f == kFamTile ? tile_entry_rows : kFamChunkRows[f]; }
   int min_count(int f) const {
     int m = 0;
     for (int g = 0; g < f; ++g)
@@ -286,6 +290,10 @@ Plan make_plan(const moe_ctx* c, int T, bool mx, moe_path path) {
       p.one_tc = !c->per_expert && p.has[kFamTile] && p.has[kFamGemm];
     }
   }
+  // bf16 expert tiles of 256 rows when the call's mean load reaches 128 rows per expert
+  const bool wide = c->tile_n == 256 ||
+                    (c->tile_n == 0 && (long long)T * c->k >= (long long)kEtRows * c->E);
+  if (p.has[kFamTile] && wide) p.tile_entry_rows = kEtWideRows;
   return p;
 }
 
@@ -310,7 +318,7 @@ long long family_row_bound(const Plan& p, int f) {
 
 // Work-list entries family f can need for T tokens.
 int max_chunks(const moe_ctx* c, int T, const Plan& p, int f) {
-  const long long R = (long long)T * c->k, rows = kFamChunkRows[f];
+  const long long R = (long long)T * c->k, rows = p.chunk_rows(f);
   long long n = R / rows + c->E;
   const long long b = family_row_bound(p, f);
   if (b != LLONG_MAX) n = std::min(n, (long long)c->E * ((b + rows - 1) / rows));
@@ -368,7 +376,7 @@ Layout make_expert_layout(const moe_ctx* c, int R, int S, const Plan& p) {
   Carver cv;
   for (int f = 0; f < kFamilies; ++f)
     if (p.has[f]) {
-      const long long rows = kFamChunkRows[f], segs = (long long)S * c->E;
+      const long long rows = p.chunk_rows(f), segs = (long long)S * c->E;
       long long n = R / rows + segs;
       const long long b = family_row_bound(p, f);
       if (b != LLONG_MAX)  // every expert's segments together hold <= b rows
@@ -567,6 +575,12 @@ bool set_smem_attrs() {
                              kEtSmem) == cudaSuccess;
   ok &= cudaFuncSetAttribute(expert_tile_kernel<1>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              kEtSmem) == cudaSuccess;
+  ok &= cudaFuncSetAttribute(expert_tile_kernel<0, kEtWideRows>,
+                             cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             EtCfg<kEtWideRows>::kSmem) == cudaSuccess;
+  ok &= cudaFuncSetAttribute(expert_tile_kernel<1, kEtWideRows>,
+                             cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             EtCfg<kEtWideRows>::kSmem) == cudaSuccess;
   ok &= cudaFuncSetAttribute(expert_tile_mx_kernel<0>,
                              cudaFuncAttributeMaxDynamicSharedMemorySize, kEmxSmem) == cudaSuccess;
   ok &= cudaFuncSetAttribute(expert_tile_mx_kernel<1>,
@@ -719,6 +733,9 @@ moe_status expert_phase(moe_ctx* c, const Plan& p, const ExpertIO& io, const voi
       if (mx)
         return launch_pdl(expert_tile_mx_kernel<0>, dim3(c->num_sms), dim3(kEmxThreads),
                           kEmxSmem, st, e, *cm, *sm, *xm);
+      if (p.tile_entry_rows == kEtWideRows)
+        return launch_pdl(expert_tile_kernel<0, kEtWideRows>, dim3(c->num_sms), dim3(kEtThreads),
+                          EtCfg<kEtWideRows>::kSmem, st, e, *wgu, *xm);
       return launch_pdl(expert_tile_kernel<0>, dim3(c->num_sms), dim3(kEtThreads), kEtSmem, st,
                         e, *wgu, *xm);
     }));
@@ -811,6 +828,9 @@ moe_status expert_phase(moe_ctx* c, const Plan& p, const ExpertIO& io, const voi
       if (mx)
         return launch_pdl(expert_tile_mx_kernel<1>, dim3(c->num_sms), dim3(kEmxThreads),
                           kEmxSmem, st, e, *cm, *sm, *hm);
+      if (p.tile_entry_rows == kEtWideRows)
+        return launch_pdl(expert_tile_kernel<1, kEtWideRows>, dim3(c->num_sms), dim3(kEtThreads),
+                          EtCfg<kEtWideRows>::kSmem, st, e, *wdn, *hm);
       return launch_pdl(expert_tile_kernel<1>, dim3(c->num_sms), dim3(kEtThreads), kEtSmem, st,
                         e, *wdn, *hm);
     }));
@@ -854,7 +874,7 @@ void plan_lists(const Plan& p, const Layout& L, uint8_t* ws, RouteOut& o, Expert
     WorkList& wl = o.wl[o.n_lists++];
     wl.chunks = reinterpret_cast<int4*>(ws + L.chunks[f]);
     wl.sched = reinterpret_cast<int32_t*>(ws + L.sched[f]);
-    wl.chunk_rows = kFamChunkRows[f];
+    wl.chunk_rows = p.chunk_rows(f);
     wl.min_count = p.min_count(f);
     wl.max_count = p.max_count[f];
     io.chunks[f] = wl.chunks;
@@ -993,6 +1013,8 @@ moe_status moe_create(int E, int H, int I, int k, moe_t* out) {
   c->stream_T = default_stream_T(c);
   // row-tile width of the grouped GEMM: MOE_ROW_TILE=512 or 256 (default below)
   if (const char* v = getenv("MOE_ROW_TILE")) c->wide_rows = strcmp(v, "512") == 0;
+  // rows per expert tile: MOE_TILE_ROWS=128 or 256 (default: by each call's mean load)
+  if (const char* v = getenv("MOE_TILE_ROWS")) c->tile_n = atoi(v) == 256 ? 256 : atoi(v) == 128 ? 128 : 0;
   if (cudaMalloc(&c->d_status, sizeof(uint32_t)) != cudaSuccess ||
       cudaMemset(c->d_status, 0, sizeof(uint32_t)) != cudaSuccess) {
     cudaGetLastError();

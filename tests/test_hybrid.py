@@ -206,3 +206,55 @@ def test_wide_row_tiles_gpt_oss_shape(T, path):
     ref = oracle.moe_forward_ref(h["x"], h["W_router"], h["b_router"], h["W_gate_up"],
                                  h["W_down"], k, tokens=tokens, route=ref_route)
     check_outputs(got, tokens, h, ref_route, g, ref)
+
+
+def _tile_rows_layer(E, H, I, k, rows):
+    """A handle whose expert tiles take `rows` rows per tile (MOE_TILE_ROWS at creation)."""
+    old = os.environ.get("MOE_TILE_ROWS")
+    os.environ["MOE_TILE_ROWS"] = str(rows)
+    try:
+        return moe.Moe(E, H, I, k)
+    finally:
+        if old is None:
+            del os.environ["MOE_TILE_ROWS"]
+        else:
+            os.environ["MOE_TILE_ROWS"] = old
+
+
+def _check_tile_layer(layer, d, h, k, tokens):
+    ref_route = host_route(h, k)
+    g = gpu_route(layer, d)
+    compare_routing(g, ref_route, k, layer.E)
+    out = layer.forward(d["x"], d["W_router"], d["b_router"], d["W_gate_up"], d["W_down"])
+    assert layer.sync_status() == moe.MOE_OK
+    got = out[torch.from_numpy(tokens).cuda()].double().cpu().numpy()
+    ref = oracle.moe_forward_ref(h["x"], h["W_router"], h["b_router"], h["W_gate_up"],
+                                 h["W_down"], k, tokens=tokens, route=ref_route)
+    check_outputs(got, tokens, h, ref_route, g, ref)
+    return g
+
+
+@pytest.mark.parametrize("T", [3, 40, 300, 1200])
+def test_expert_tiles_of_256_rows_ragged(T):
+    """256-row expert tiles (one accumulator buffer of 2 x 256 TMEM columns, 3 stages): rows 1..16
+    per box, up to 16 boxes, experts of more than 256 rows split over two or three entries, a
+    half-filled last column block (I = 320)."""
+    E, H, I, k = 8, 256, 320, 2
+    d, h = inputs_on_gpu(T, H, E, k, I, seed=3000 + T)
+    layer = _tile_rows_layer(E, H, I, k, 256)
+    layer.set_path(moe.MOE_PATH_TILE)
+    g = _check_tile_layer(layer, d, h, k, np.arange(T))
+    counts = np.diff(g["expert_offsets"])
+    want = int(sum(-(-c // 256) for c in counts if c > 0))
+    assert layer.last_dispatch(T)[1] == want
+
+
+@pytest.mark.parametrize("T", [512, 2048])
+def test_expert_tiles_of_256_rows_gpt_oss_shape(T):
+    """H = I = 2880 with 256-row expert tiles: 45 K stages, 23 gate/up and 12 down column blocks
+    (the last ones 64 wide)."""
+    E, H, I, k = 32, 2880, 2880, 4
+    d, h = inputs_on_gpu(T, H, E, k, I, seed=3100 + T)
+    layer = _tile_rows_layer(E, H, I, k, 256)
+    layer.set_path(moe.MOE_PATH_TILE)
+    _check_tile_layer(layer, d, h, k, mi.sample_tokens(T, 384, 3100 + T))
