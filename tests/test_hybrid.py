@@ -24,6 +24,13 @@ if torch.cuda.is_available():
 FAMILY_ROWS = (16, 128, 256)   # rows per work-list entry: streaming, expert tiles, row tiles
 
 
+def _entry_rows(layer, T):
+    """Rows per work-list entry of each family in a T-token call: expert tiles take 256 rows
+    once the mean load reaches 128 rows per expert (handles created without MOE_TILE_ROWS)."""
+    wide = T * layer.k >= 128 * layer.E
+    return (FAMILY_ROWS[0], 256 if wide else 128, FAMILY_ROWS[2])
+
+
 def _families(layer, T, counts):
     """Experts per family as the dispatch rule assigns them (the bench's mirror of the rule)."""
     import bench
@@ -37,8 +44,9 @@ def _check_device_dispatch(layer, T, counts):
     """The work lists the last forward call built on the device agree with the rule."""
     _, f = _families(layer, T, counts)
     entries = layer.last_dispatch(T)
+    rows = _entry_rows(layer, T)
     for i, k in enumerate(("stream", "tile", "gemm")):
-        want = sum(-(-c // FAMILY_ROWS[i]) for c in f[k])
+        want = sum(-(-c // rows[i]) for c in f[k])
         assert entries[i] == want or (entries[i] == -1 and want == 0), (k, entries, want)
     return entries
 
