@@ -87,7 +87,8 @@ typedef enum {
  *   weight streaming  tensor-core mma.sync with the weights split over K across all SMs
  *                     (stream-K): balances best when only a few experts are touched
  *   expert tiles      tcgen05 MMAs with an expert's weight columns as the M operand and its rows
- *                     as N, each weight block read once for up to 128 rows
+ *                     as N, each weight block read once for up to 128 rows (256 rows per
+ *                     tile once a call's mean load reaches 128 rows per expert)
  *   row tiles         2-SM tcgen05 grouped GEMM, 256 rows x 256 columns per CTA pair (prefill,
  *                     long sequences)
  * MOE_PATH_AUTO chooses on the device, from the call's histogram (no host sync): in calls of at
@@ -227,8 +228,9 @@ MOE_API moe_status moe_set_path(moe_t ctx, moe_path path, int crossover_T);
 /* Current path setting and streaming crossover (tokens). */
 MOE_API moe_status moe_get_path(moe_t ctx, moe_path* path, int* crossover_T);
 
-/* The AUTO thresholds, in rows of one expert: stream_rows (default 16, one streaming chunk) and
- * tile_rows (default 128, one expert tile), and per_expert (default 0): 1 lets one call run
+/* The AUTO thresholds, in rows of one expert: stream_rows (default 16, one streaming chunk),
+ * tile_rows (default 192: up to there the expert tiles, with 256 rows per tile once a call's mean
+ * load reaches 128 rows, beat the row tiles) and per_expert (default 0): 1 lets one call run
  * expert tiles and row tiles side by side (each expert by its own count, the row tiles on the
  * handle's second stream), 0 keeps the call's non-streamed experts in one of the two by their
  * mean count.  A negative value keeps the current setting. */

@@ -97,9 +97,9 @@ def test_skewed_mid_T_mixes_the_families(T, dispatch, expect):
 
 @pytest.mark.parametrize("T", [1024, 1500])
 def test_tight_loads_do_not_split_across_the_tile_boundary(T):
-    """With no router bias the experts' loads sit close to T*k/E (128 and 188 rows here), on
-    both sides of tile_rows = 128: the call's counts move them all to one family (one launch
-    per projection); the layer stays exact."""
+    """With no router bias the experts' loads sit close to T*k/E (128 and 188 rows here), the
+    second call just below tile_rows = 192: the call's counts keep them all in one family (one
+    launch per projection); the layer stays exact."""
     E, H, I, k = 32, 2880, 2880, 4
     d, h = inputs_on_gpu(T, H, E, k, I, seed=2700 + T)
     d["b_router"].zero_()
@@ -152,7 +152,7 @@ def test_thresholds_round_trip():
     sms = torch.cuda.get_device_properties(0).multi_processor_count
     T0 = layer.get_path()[1]
     assert min(32, (T0 + 1) * 4) * 23 >= 2 * sms > min(32, T0 * 4) * 23
-    assert layer.get_dispatch() == (16, 128, False)
+    assert layer.get_dispatch() == (16, 192, False)
     layer.set_dispatch(4, 100, 1)
     assert layer.get_dispatch() == (4, 100, True)
     layer.set_dispatch(-1, 50)
