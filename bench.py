@@ -391,31 +391,45 @@ def default_steps(step, stream, world: int) -> int:
     return int(reduce_max(float(k), world))
 
 
-def graph_timing(step, steps: int, world: int) -> dict:
-    """The same call captured once in a CUDA graph and replayed K times: no host launch work in
-    the timed region, so the difference from `us_per_layer` is what launching from the host
-    costs (it matters only at a few tokens per call)."""
+def graph_timing(step, steps: int, world: int, per_graph: int = 1) -> dict:
+    """The same calls captured once in a CUDA graph (per_graph consecutive steps: one per input
+    batch) and replayed: no host launch work in the timed region, so the difference from
+    `us_per_layer` is what launching from the host costs (it matters only at a few tokens)."""
     g = torch.cuda.CUDAGraph()
     try:
         with torch.cuda.graph(g):
-            step()
+            for _ in range(per_graph):
+                step()
     except RuntimeError as e:      # capture refused: report it, the eager numbers stand
         return dict(error=str(e).splitlines()[0][:200])
     for _ in range(3):
         g.replay()
     torch.cuda.synchronize()
     stream = torch.cuda.current_stream()
+    replays = max(1, steps // per_graph)
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     if world > 1:
         torch.distributed.barrier()
     e0.record(stream)
-    for _ in range(steps):
+    for _ in range(replays):
         g.replay()
     e1.record(stream)
     torch.cuda.synchronize()
     secs = reduce_max(e0.elapsed_time(e1) / 1e3, world)
     del g
-    return dict(us_per_layer=secs / steps * 1e6, steps=steps)
+    return dict(us_per_layer=secs / (replays * per_graph) * 1e6, steps=replays * per_graph)
+
+
+# A step whose touched expert weights are less than this many L2 sizes would keep part of them in
+# L2 for the next step if every step routed the same tokens; such workloads cycle through
+# ROTATE_BATCHES seeded token batches instead, so that consecutive steps touch other experts.
+ROTATE_L2_FACTOR = 4
+ROTATE_BATCHES = 16
+
+
+def mean_dicts(ds: list) -> dict:
+    """Field-wise mean of dicts with the same numeric fields."""
+    return {k_: sum(d_[k_] for d_ in ds) / len(ds) for k_ in ds[0]}
 
 
 def run_ours(args, w: mi.Workload, T: int) -> None:
@@ -436,8 +450,19 @@ def run_ours(args, w: mi.Workload, T: int) -> None:
     layer = moe.Moe(w.E, w.H, w.I, w.k)
     layer.set_path({"auto": moe.MOE_PATH_AUTO, "stream": moe.MOE_PATH_STREAM,
                     "tile": moe.MOE_PATH_TILE, "gemm": moe.MOE_PATH_GEMM}[args.path])
-    counts = torch.diff(layer.route(d["x"], d["W_router"], d["b_router"])["expert_offsets"]).cpu().tolist()
+    def route_counts(x):
+        r = layer.route(x, d["W_router"], d["b_router"])
+        return torch.diff(r["expert_offsets"]).cpu().tolist()
+
+    counts = route_counts(d["x"])
     alg = algorithmic(T, w.H, w.E, w.k, w.I, counts, w.weights)
+    xs = [d["x"]]
+    l2_bytes = torch.cuda.get_device_properties(local).L2_cache_size
+    rotate = alg["layer_bytes"] < ROTATE_L2_FACTOR * l2_bytes
+    if rotate:
+        xs += [mi.draw_x(T, w.H, seed + 104729 * j, "cuda") for j in range(1, ROTATE_BATCHES)]
+    counts_all = [counts] + [route_counts(x) for x in xs[1:]]
+    alg = mean_dicts([algorithmic(T, w.H, w.E, w.k, w.I, c_, w.weights) for c_ in counts_all])
     out = torch.empty((T, w.H), dtype=torch.float32, device="cuda")
     mx = w.weights == "mxfp4"
     if mx:
@@ -451,8 +476,12 @@ def run_ours(args, w: mi.Workload, T: int) -> None:
         args_fwd = (d["x"], d["W_router"], d["b_router"], d["W_gate_up"], d["W_down"])
     stream = torch.cuda.current_stream()
 
-    def step():
-        fwd(*args_fwd, out=out, workspace=ws)
+    cur = [0]
+
+    def step():  # one layer call on the next input batch
+        x = xs[cur[0] % len(xs)]
+        cur[0] += 1
+        fwd(x, *args_fwd[1:], out=out, workspace=ws)
 
     for _ in range(args.warmup):
         step()
@@ -489,12 +518,14 @@ def run_ours(args, w: mi.Workload, T: int) -> None:
     prof = layer.profile_end()
     assert layer.sync_status() == moe.MOE_OK
     # ---- e2e: the same call with host buffers, copies inside the timed region ----
-    x_host = d["x"].cpu().pin_memory()
+    x_hosts = [x.cpu().pin_memory() for x in xs]
     out_host = torch.empty((T, w.H), dtype=torch.float32).pin_memory()
     x_dev = torch.empty_like(d["x"])
+    cur_e = [0]
 
     def e2e_step():
-        x_dev.copy_(x_host, non_blocking=True)
+        x_dev.copy_(x_hosts[cur_e[0] % len(x_hosts)], non_blocking=True)
+        cur_e[0] += 1
         fwd(x_dev, *args_fwd[1:], out=out, workspace=ws)
         out_host.copy_(out, non_blocking=True)
 
@@ -510,7 +541,7 @@ def run_ours(args, w: mi.Workload, T: int) -> None:
     e1.record(stream)
     torch.cuda.synchronize()
     e2e_secs = reduce_max(e0.elapsed_time(e1) / 1e3, world)
-    graph = graph_timing(step, steps, world)
+    graph = graph_timing(step, steps, world, per_graph=len(xs))
     assert layer.sync_status() == moe.MOE_OK
 
     # ---- roofline of the dominant kernel: the gate/up projection (2/3 of bytes and FLOPs) of
@@ -520,8 +551,11 @@ def run_ours(args, w: mi.Workload, T: int) -> None:
     stream_rows, tile_rows, per_expert = layer.get_dispatch()
     path = {moe.MOE_PATH_STREAM: "stream", moe.MOE_PATH_GEMM: "gemm",
             moe.MOE_PATH_TILE: "tile"}.get(path_setting, "auto")
-    fams = split_families(counts, path, T, stream_T, stream_rows, tile_rows, w.weights, per_expert)
-    work = {f: family_work(fams[f], w.H, w.I, w.weights) for f in FAMILIES}
+    fams_all = [split_families(c_, path, T, stream_T, stream_rows, tile_rows, w.weights,
+                               per_expert) for c_ in counts_all]
+    fams = fams_all[0]
+    work = {f: mean_dicts([family_work(fa[f], w.H, w.I, w.weights) for fa in fams_all])
+            for f in FAMILIES}
     n_prof = prof_steps
     gu_ms = {f: prof["gate_up_" + f][0] / n_prof for f in FAMILIES}
     dn_ms = {f: prof["down_" + f][0] / n_prof for f in FAMILIES}
@@ -535,8 +569,10 @@ def run_ours(args, w: mi.Workload, T: int) -> None:
     down_rate = {f"down_{f}_ms": round(dn_ms[f], 4) for f in FAMILIES if dn_ms[f] > 0}
     dispatch = dict(stream_T=stream_T, stream_rows=stream_rows, tile_rows=tile_rows,
                     per_expert=per_expert,
-                    experts={f: len(fams[f]) for f in FAMILIES},
-                    rows={f: int(sum(fams[f])) for f in FAMILIES})
+                    experts={f: round(sum(len(fa[f]) for fa in fams_all) / len(fams_all), 2)
+                             for f in FAMILIES},
+                    rows={f: round(sum(sum(fa[f]) for fa in fams_all) / len(fams_all), 1)
+                          for f in FAMILIES})
 
     line = dict(
         metric=METRIC, value=agg["value"], unit=UNIT, n_gpus=world, steps=steps,
@@ -547,8 +583,12 @@ def run_ours(args, w: mi.Workload, T: int) -> None:
         config=dict(workload=w.name, T=T, H=w.H, E=w.E, k=w.k, I=w.I, path=path,
                     weights=w.weights, dispatch=dispatch,
                     parallelism=f"replicas{world}" if world > 1 else "single",
-                    l2="inputs larger than L2: %.2f GB of touched expert weights and tokens per "
-                       "step vs 126 MB L2" % ((alg["layer_bytes"]) / 1e9)),
+                    l2=("steps cycle through %d seeded token batches, so consecutive steps "
+                        "touch other experts (%.2f GB of touched expert weights and tokens per "
+                        "step vs %d MB L2)" % (len(xs), alg["layer_bytes"] / 1e9, l2_bytes >> 20))
+                    if rotate else
+                    ("inputs larger than L2: %.2f GB of touched expert weights and tokens per "
+                     "step vs %d MB L2" % (alg["layer_bytes"] / 1e9, l2_bytes >> 20))),
         roofline=roof,
         layer_roofline=dict(touched_experts=alg["touched"], alg_bytes=alg["layer_bytes"],
                             alg_flops=alg["flops"], roofline_us=layer_roof_s * 1e6,

@@ -193,3 +193,12 @@ def test_traffic_lookup_matches_workload_T_and_sources():
             assert (got == c["dram_bytes_per_launch"]) if fresh else got is None
             assert bench.ncu_traffic(kernel, c["workload"], c["T"] + 1) is None
     assert bench.ncu_traffic("no_such_kernel", "tiny", 64) is None
+
+
+def test_small_steps_rotate_their_input_batches():
+    # field-wise means of the per-batch work, and the size below which steps rotate batches
+    assert bench.mean_dicts([{"a": 1, "b": 2}, {"a": 3, "b": 6}]) == {"a": 2.0, "b": 4.0}
+    l2 = 126 << 20
+    one_token_120b = bench.algorithmic(1, 2880, 128, 4, 2880, [1, 1, 1, 1] + [0] * 124)
+    decode_20b = bench.algorithmic(16, 2880, 32, 4, 2880, [3] * 21 + [1] * 1 + [0] * 10)
+    assert one_token_120b["layer_bytes"] < bench.ROTATE_L2_FACTOR * l2 <= decode_20b["layer_bytes"]
