@@ -104,34 +104,6 @@ MOE_DEVINL void tma_load_2d(void* smem_dst, const CUtensorMap* map, int c0, int 
       "l"(reinterpret_cast<uint64_t>(map)), "r"(c0), "r"(c1), "r"(smem_u32(bar))
       : "memory");
 }
-// The same copy with an L2 cache policy (createpolicy) for the bytes it reads.
-MOE_DEVINL void tma_load_2d_hint(void* smem_dst, const CUtensorMap* map, int c0, int c1,
-                                 uint64_t* bar, uint64_t policy) {
-  asm volatile(
-      "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
-      ".L2::cache_hint [%0], [%1, {%2, %3}], [%4], %5;" ::"r"(smem_u32(smem_dst)),
-      "l"(reinterpret_cast<uint64_t>(map)), "r"(c0), "r"(c1), "r"(smem_u32(bar)), "l"(policy)
-      : "memory");
-}
-// L2 policies: bytes read once (they leave first) and bytes with the normal priority (a
-// prefetch for the next kernel: it outlives evict-first lines, and nothing of it stays pinned
-// after the call, as evict-last lines would).
-MOE_DEVINL uint64_t l2_policy_evict_first() {
-  uint64_t p;
-  asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(p));
-  return p;
-}
-MOE_DEVINL uint64_t l2_policy_evict_normal() {
-  uint64_t p;
-  asm volatile("createpolicy.fractional.L2::evict_normal.b64 %0, 1.0;" : "=l"(p));
-  return p;
-}
-// Bring `bytes` (a multiple of 16, 16-byte aligned address) of global memory into L2.
-MOE_DEVINL void prefetch_l2_bulk(const void* g, uint32_t bytes, uint64_t policy) {
-  asm volatile("cp.async.bulk.prefetch.L2.global.L2::cache_hint [%0], %1, %2;" ::"l"(g),
-               "r"(bytes), "l"(policy)
-               : "memory");
-}
 MOE_DEVINL void tma_prefetch_desc(const CUtensorMap* map) {
   asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");
 }

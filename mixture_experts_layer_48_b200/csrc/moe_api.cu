@@ -73,7 +73,6 @@ struct moe_ctx {
   MapCache gu_codes_t, gu_scales_t, dn_codes_t, dn_scales_t;  // MXFP4 weights (expert tiles)
   int device = 0;
   int num_sms = 148;
-  size_t l2_bytes = 0;                   // L2 size of the device
   moe_path path = MOE_PATH_AUTO;
   int stream_T = 0;                      // AUTO streams only in calls of at most this many tokens
   int stream_rows = kDefaultStreamRows;  // ... the experts with at most this many rows
@@ -669,13 +668,6 @@ moe_status expert_phase(moe_ctx* c, const Plan& p, const ExpertIO& io, const voi
     ga.out = io.out;
     ga.out_elems = zero_owner == kFamStream ? io.out_elems : 0;
     ga.status = c->d_status;
-    if (!mx && !p.has[kFamTile] && !p.has[kFamGemm]) {
-      // the down kernel follows on the same SMs: its weights into L2 when they take at most
-      // 60 % of it (the gate/up stream is read with the evict-first policy meanwhile)
-      ga.down_w = static_cast<const uint8_t*>(W_down_bf16);
-      ga.down_bytes = (size_t)c->I * c->H * 2;
-      ga.down_l2_limit = c->l2_bytes * 3 / 5;
-    }
     if (mx) {
       const CUtensorMap* cm = cached_map_u8(c->gu_codes, mx->gu_codes, 2ull * c->I * c->E,
                                             (uint64_t)c->H / 2, kMxBoxRows, kMxKC / 2,
@@ -1012,7 +1004,6 @@ moe_status moe_create(int E, int H, int I, int k, moe_t* out) {
   c->k = k;
   c->device = dev;
   c->num_sms = prop.multiProcessorCount;
-  c->l2_bytes = (size_t)prop.l2CacheSize;
   c->stream_T = default_stream_T(c);
   // row-tile width of the grouped GEMM: MOE_ROW_TILE=512 or 256 (default below)
   if (const char* v = getenv("MOE_ROW_TILE")) c->wide_rows = strcmp(v, "512") == 0;

@@ -85,13 +85,6 @@ struct GateUpArgs {
   float* out;            // [T, H] zero-filled here
   size_t out_elems;
   uint32_t* status;
-  // When the touched experts' W_down fits in L2 (n_chunks * down_bytes <= down_l2_limit): the
-  // kernel brings it into L2 while it streams W_gate_up (read with the evict-first policy, so
-  // it leaves L2 before the prefetched lines do), and the down kernel reads it from L2.
-  // down_w null: no prefetch.
-  const uint8_t* down_w;  // W_down [E, I, H] bf16
-  size_t down_bytes;      // bytes of one expert's W_down
-  size_t down_l2_limit;
 };
 
 // Routing of a call of at most kFusedRouteT tokens (and T*k <= kFusedRouteRows rows), done by
@@ -329,24 +322,6 @@ __global__ void __launch_bounds__(kStreamThreads, 1)
     int last_it[kStreamStages];
 #pragma unroll
     for (int s = 0; s < kStreamStages; ++s) last_it[s] = -1;
-    // W_down of the touched experts into L2, one 64 KB piece after each stage this CTA issues
-    // (pieces blockIdx.x, blockIdx.x + gridDim.x, ...), while W_gate_up is read evict-first
-    const bool pf = a.down_w != nullptr && (size_t)n_chunks * a.down_bytes <= a.down_l2_limit;
-    const uint64_t pol_first = pf ? l2_policy_evict_first() : 0ull;
-    const uint64_t pol_keep = pf ? l2_policy_evict_normal() : 0ull;
-    constexpr uint32_t kPiece = 65536;
-    const long long per_chunk = pf ? (long long)((a.down_bytes + kPiece - 1) / kPiece) : 0;
-    const long long pf_end = per_chunk * n_chunks;
-    long long pf_next = blockIdx.x;
-    auto prefetch_next = [&]() {
-      if (pf_next >= pf_end) return;
-      if (lane == 0) {
-        const long long c = pf_next / per_chunk, off = (pf_next % per_chunk) * kPiece;
-        const uint32_t nb = (uint32_t)min((long long)kPiece, (long long)a.down_bytes - off);
-        prefetch_l2_bulk(a.down_w + (size_t)chunks[c].x * a.down_bytes + off, nb, pol_keep);
-      }
-      pf_next += gridDim.x;
-    };
     for (long long g = rng.g0; g < rng.g1;) {
       const int unit = (int)(g / nk), kb = (int)(g % nk);
       const int ke = (int)min((long long)nk, kb + (rng.g1 - g));
@@ -370,22 +345,15 @@ __global__ void __launch_bounds__(kStreamThreads, 1)
         if (lane == 0) mbar_arrive_expect_tx(&full[slot], bytes);
         __syncwarp();
         const int k0 = kst * kGateUpKC;
-        if (lane < 2 * kStreamWarps) {
-          if (pf)
-            tma_load_2d_hint(wring + slot * kGUStageW + lane * kGUBoxBytes, &wmap, box_col,
-                             ch.x * a.H + k0, &full[slot], pol_first);
-          else
-            tma_load_2d(wring + slot * kGUStageW + lane * kGUBoxBytes, &wmap, box_col,
-                        ch.x * a.H + k0, &full[slot]);
-        }
+        if (lane < 2 * kStreamWarps)
+          tma_load_2d(wring + slot * kGUStageW + lane * kGUBoxBytes, &wmap, box_col,
+                      ch.x * a.H + k0, &full[slot]);
         if (lane < ch.z)
           bulk_g2s(xring + slot * kGUStageX + lane * kGUXPitch, a.x + (size_t)tok * a.H + k0,
                    kGateUpKC * 2, &full[slot]);
         last_it[slot] = it;
-        prefetch_next();
       }
     }
-    while (pf_next < pf_end) prefetch_next();  // the rest of this CTA's pieces
     // never leave the CTA with copies in flight
     if (lane == 0) {
       for (int s = 0; s < kStreamStages; ++s)
