@@ -113,8 +113,12 @@ typedef enum {
 
 /* Create a handle for a layer of shape (E, H, I, k) on the current device.  Validates the
  * shape (see conventions; MOE_ERR_ARG otherwise), checks for an sm_100 device
- * (MOE_ERR_DEVICE), allocates the 4-byte device status word and looks up the device address
- * of the library's routing scratch array (moe_route_static).  *out receives the handle. */
+ * (MOE_ERR_DEVICE), allocates the 4-byte device status word, creates a second stream and two
+ * events (for calls whose kernel families run side by side) and looks up the device address of
+ * the library's routing scratch array (moe_route_static).  *out receives the handle.
+ * Two environment variables, read here, select kernel variants for measurement: MOE_ROW_TILE=512
+ * (row tiles of 256 x 512 instead of 256 x 256) and MOE_TILE_ROWS=128 or 256 (rows per expert
+ * tile for every call instead of by the call's mean load). */
 MOE_API moe_status moe_create(int E, int H, int I, int k, moe_t* out);
 
 /* Free the handle and its status word.  NULL is accepted.  Work still queued on a stream
