@@ -14,9 +14,9 @@
 //                                              or <= 256 in the 256-row variant)
 //
 // and each tile streams a [K x 128]-column block of one expert's weights exactly once for all of
-// that expert's rows (up to 128 per tile).  Work: tiles = (row chunk of one expert, column
-// block); per K stage of 64 a tile loads two 128-column weight blocks (gate and up, or two
-// neighbouring blocks of W_down: 32 KB) and the chunk's rows (16 rows per box, up to 16 KB).
+// that expert's rows (up to 128 or 256 per tile).  Work: tiles = (row chunk of one expert,
+// column block); per K stage of 64 a tile loads two 128-column weight blocks (gate and up, or two
+// neighbouring blocks of W_down: 32 KB) and the chunk's rows (16 rows per box, up to 16 or 32 KB).
 //
 //   warp 0      TMA producer (weights as 64 x 64 boxes with the 128-byte swizzle: the MN-major
 //               A operand; activation rows as 16 x 64 boxes: the K-major B operand)

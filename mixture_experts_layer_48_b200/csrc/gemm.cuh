@@ -37,7 +37,7 @@ struct GemmArgs {
   int Ncols;             // output columns of one matrix: I (gate/up) or H (down)
   int sub_stride;        // column offset between sub-tiles in the weight (I for gate/up)
   int w_rows;            // weight rows per expert (= K)
-  const int4* chunks;    // {expert, first row, rows}, rows <= 128
+  const int4* chunks;    // {expert, first row, rows}, rows <= 256 (one chunk per CTA pair)
   const int32_t* sched;  // [0] number of chunks
   uint16_t* h;           // gate/up output [R, I] bf16
   const int32_t* perm;   // down: token of each row

@@ -228,14 +228,16 @@ RouteTmp carve_route_tmp(Carver& cv, const moe_ctx* c, int T, bool allow_split =
   return r;
 }
 
-// ---- per-expert dispatch --------------------------------------------------------------
-// Three kernel families multiply an expert's rows, chosen per expert on the device from its
-// row count (the routing kernels build one work list per family):
+// ---- dispatch -------------------------------------------------------------------------
+// Three kernel families multiply an expert's rows, chosen on the device from the call's row
+// counts (the routing kernels build one work list per family):
 //   stream  rows <= stream_rows:      weight streaming on mma.sync, stream-K split (decode)
 //   tile    up to tile_rows:          tcgen05 expert tiles, weights as the M operand
 //   gemm    more than tile_rows:      2-SM tcgen05 row tiles (prefill, long sequences)
-// The host only decides which families may receive rows: an expert holds at most T rows (a
-// token picks an expert at most once), so families above T are not launched.
+// By default (one_tc) the experts past the streaming bound then all take expert tiles or all
+// take row tiles, by their mean count; per_expert keeps each expert's own choice.  The host
+// only decides which families may receive rows: an expert holds at most T rows (a token picks
+// an expert at most once), so families above T are not launched.
 enum Family { kFamStream = 0, kFamTile = 1, kFamGemm = 2, kFamilies = 3 };
 constexpr int kFamChunkRows[kFamilies] = {kStreamRB, kEtRows, kGemmChunkRows};
 constexpr int kEtWideRows = 256;   // rows per entry of the 256-row expert tiles
