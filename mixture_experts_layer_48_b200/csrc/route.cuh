@@ -513,9 +513,8 @@ __global__ void __launch_bounds__(128)
   const int nk = min(H / kRouterHSlice - kc0, kc_per_split);
   const bool vec_w = (E % 8) == 0;
 
-  pdl_wait();
-  pdl_launch_next();
-  zero_fill_f4(zero4, n_zero4);
+  // x and W_router are the caller's inputs, which no kernel of this library writes: the loads
+  // and the products run before the dependency wait, everything this kernel writes after it
   for (int i = tid; i < EP; i += blockDim.x) cnt[i] = 0;
   for (int i = tid; i < C::kStages * kRouterHSlice * WP; i += blockDim.x)
     wsm[i] = 0;  // padding experts stay zero
@@ -589,6 +588,9 @@ __global__ void __launch_bounds__(128)
     }
   }
   cp_async_wait<0>();
+  pdl_wait();
+  pdl_launch_next();
+  zero_fill_f4(zero4, n_zero4);
   // C fragment: c0,c1 -> token 16w + lane/4, experts 8n + 2(lane%4) + {0,1}; c2,c3 -> token + 8
   if (partial != nullptr) {  // one slice of the hidden dimension: partial logits, no bias
 #pragma unroll
