@@ -229,52 +229,22 @@ __global__ void __launch_bounds__(kEtThreads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = s_tmem;
-  // The down projection's producer fetches the weight boxes of its first stages before the
-  // dependency wait: the weights are the caller's, and the work list comes from the routing
-  // kernels, which finished before the gate/up kernel (the kernel before this one) could start.
-  // Only h, from the gate/up kernel, waits.
-  constexpr bool kEarly = MODE == 1;
-  if (!kEarly || warp != 0) {
-    pdl_wait();  // work list, activation rows and (down) h come from the previous kernels
-    pdl_launch_next();
-  }
+  pdl_wait();  // work list, activation rows and (down) h come from the previous kernels
+  pdl_launch_next();
 
   constexpr int TW = MODE == 0 ? kEtM : 2 * kEtM;
   const int NT = (a.Ncols + TW - 1) / TW;
-  const int tiles = __ldcg(a.sched) * NT;
+  const int tiles = a.sched[0] * NT;
   const int nk = a.K / kEtBK;
   volatile int* abort_flag = &s_abort;
 
   if (warp == 0) {
     // ------------------------------ TMA producer ------------------------------
-    int n_pre = 0;  // stages whose weight boxes went out before the wait (first tile only)
-    if (kEarly && lane == 0 && (int)blockIdx.x < tiles) {
-      const int t = blockIdx.x;
-      const int4 ch = __ldcg(a.chunks + t / NT);
-      const int n0 = (t % NT) * TW;
-      const int nb0 = et_boxes<MODE>(0, n0, a.Ncols), nb1 = et_boxes<MODE>(1, n0, a.Ncols);
-      const int c0 = n0, c1 = n0 + kEtM;
-      const int wrow0 = ch.x * a.w_rows;
-      n_pre = min(kStages, nk);
-      for (int s = 0; s < n_pre; ++s) {  // the ring is empty: no slot to wait for
-        mbar_expect_tx(&full[s], (uint32_t)(nb0 + nb1) * kEtBoxBytes);
-        uint8_t* st = ring + s * kStageBytes;
-        for (int b = 0; b < nb0; ++b)
-          tma_load_2d(st + b * kEtBoxBytes, &wmap, c0 + 64 * b, wrow0 + s * kEtBK, &full[s]);
-        for (int b = 0; b < nb1; ++b)
-          tma_load_2d(st + (2 + b) * kEtBoxBytes, &wmap, c1 + 64 * b, wrow0 + s * kEtBK, &full[s]);
-      }
-    }
-    if (kEarly) {
-      pdl_wait();  // h comes from the gate/up kernel
-      pdl_launch_next();
-    }
     if (lane == 0) {
       uint32_t it = 0;
       int last_it[kStages];
 #pragma unroll
       for (int s = 0; s < kStages; ++s) last_it[s] = -1;
-      for (int s = 0; s < n_pre; ++s) last_it[s] = s;  // drained below even after an abort
       for (int t = blockIdx.x; t < tiles && !*abort_flag; t += gridDim.x) {
         const int4 ch = a.chunks[t / NT];
         const int n0 = (t % NT) * TW;
@@ -292,14 +262,12 @@ __global__ void __launch_bounds__(kEtThreads, 1)
             ok = false;
             break;
           }
-          const bool pre = (int)it < n_pre;  // weight boxes already on the way
-          mbar_arrive_expect_tx(&full[slot],
-                                pre ? bytes - (uint32_t)(nb0 + nb1) * kEtBoxBytes : bytes);
+          mbar_arrive_expect_tx(&full[slot], bytes);
           uint8_t* st = ring + slot * kStageBytes;
           const int k0 = kst * kEtBK;
-          for (int b = 0; b < nb0 && !pre; ++b)
+          for (int b = 0; b < nb0; ++b)
             tma_load_2d(st + b * kEtBoxBytes, &wmap, c0 + 64 * b, wrow0 + k0, &full[slot]);
-          for (int b = 0; b < nb1 && !pre; ++b)
+          for (int b = 0; b < nb1; ++b)
             tma_load_2d(st + (2 + b) * kEtBoxBytes, &wmap, c1 + 64 * b, wrow0 + k0, &full[slot]);
           for (int r = 0; r < nrb; ++r)
             tma_load_2d(st + kEtABytes + r * (kEtRowBox * kEtBK * 2), &xmap, k0,
