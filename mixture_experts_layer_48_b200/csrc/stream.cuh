@@ -402,7 +402,8 @@ __global__ void __launch_bounds__(kStreamThreads, 1)
       __syncwarp();
       if (lane == 0 && !aborted) mbar_arrive(&empty[slot]);
     }
-    if (aborted) continue;
+    // every consumer warp walks the same units and takes the barriers below even after giving
+    // up on a wait (skipping only the data work), so no warp is left at a barrier
 
     // ---- epilogue: C fragment (m = weight column, n = row) ----
     // value v of tile (mt, nb): column 64*warp + 16*mt + (lane>>2) + 8*(v>>1),
@@ -416,7 +417,7 @@ __global__ void __launch_bounds__(kStreamThreads, 1)
           for (int v = 0; v < 4; ++v) {
             const int cl = kBox * warp + 16 * mt + (lane >> 2) + 8 * (v >> 1);
             const int r = nb * 8 + 2 * (lane & 3) + (v & 1);
-            if (r < nrows && cl < wg) {
+            if (!aborted && r < nrows && cl < wg) {
               const float hv = silu_f32(accg[mt][nb][v]) * accu[mt][nb][v];
               a.h[(size_t)(ch.y + r) * a.I + col0 + cl] = (uint16_t)f32_to_bf16_bits(hv);
             }
@@ -431,7 +432,7 @@ __global__ void __launch_bounds__(kStreamThreads, 1)
         for (int v = 0; v < 4; ++v) {
           const int cl = kBox * warp + 16 * mt + (lane >> 2) + 8 * (v >> 1);
           const int r = nb * 8 + 2 * (lane & 3) + (v & 1);
-          if (r < nrows && cl < wg) {
+          if (!aborted && r < nrows && cl < wg) {
             float* p = a.acc + ((size_t)ch.w + r) * I2 + col0 + cl;
             atomicAdd(p, accg[mt][nb][v]);
             atomicAdd(p + a.I, accu[mt][nb][v]);
@@ -441,7 +442,8 @@ __global__ void __launch_bounds__(kStreamThreads, 1)
     // barrier orders every thread's atomics before thread 0's release; thread 0's acquire
     // and the second barrier order the last piece's reads after all other pieces' atomics.
     named_bar_sync(1, kStreamConsumers);
-    if (ctid == 0) s_last = (atom_add_acq_rel_gpu(&a.done[unit], ke - kb) + (ke - kb) == nk);
+    if (ctid == 0)
+      s_last = !aborted && atom_add_acq_rel_gpu(&a.done[unit], ke - kb) + (ke - kb) == nk;
     named_bar_sync(1, kStreamConsumers);
     if (s_last) {
       for (int i = ctid; i < nrows * (wg / 2); i += kStreamConsumers) {
