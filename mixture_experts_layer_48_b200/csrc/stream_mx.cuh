@@ -36,13 +36,9 @@
 
 namespace moe {
 
-constexpr int kMxWarps = 10;                        // m-tiles of 16 columns per tile and matrix
-// gate/up: one consumer warp per (matrix, m-tile) -- gate and up on different warps, so that
-// twice the warps hide the latency of the code conversion
-constexpr int kMxGuWarps = 2 * kMxWarps;
-constexpr int kMxConsumers = 32 * kMxGuWarps;
+constexpr int kMxWarps = 10;                        // consumer warps, one m-tile each
+constexpr int kMxConsumers = 32 * kMxWarps;
 constexpr int kMxThreads = kMxConsumers + 32;       // + 1 producer warp
-constexpr int kMxXchgBytes = kMxWarps * 32 * 8 * 4; // up sums handed to the gate warps (10 KB)
 constexpr int kMxKC = 256;                          // K per stage (8 scale blocks)
 constexpr int kMxBoxRows = 32;                      // weight columns per box (two warps)
 constexpr int kMxTileCols = 160;                    // weight columns per tile and matrix
@@ -66,7 +62,7 @@ constexpr int kMxGUStage = (kMxGUW + kMxGUS + kMxX + 1023) / 1024 * 1024;  // 53
 constexpr int kMxDNStage = (kMxDNW + kMxDNS + kMxX + 1023) / 1024 * 1024;  // 53 KB
 constexpr int kMxGUStages = 4;
 constexpr int kMxDNStages = 4;
-constexpr int kMxGateUpSmem = 1024 + kMxGUStages * kMxGUStage + 2 * kMxGUStages * 8 + kMxXchgBytes;
+constexpr int kMxGateUpSmem = 1024 + kMxGUStages * kMxGUStage + 2 * kMxGUStages * 8;
 constexpr int kMxDownSmem = 1024 + kMxDNStages * kMxDNStage + 2 * kMxDNStages * 8;
 static_assert(kMxGateUpSmem <= 227 * 1024 && kMxDownSmem <= 227 * 1024, "shared memory");
 
@@ -230,12 +226,11 @@ __global__ void __launch_bounds__(kMxThreads, 1)
   uint8_t* ring = align1k(smem_raw);
   uint64_t* full = reinterpret_cast<uint64_t*>(ring + kMxGUStages * kMxGUStage);
   uint64_t* empty = full + kMxGUStages;
-  float* xchg = reinterpret_cast<float*>(empty + kMxGUStages);  // [kMxWarps][8][32]
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   if (tid == 0) {
     for (int s = 0; s < kMxGUStages; ++s) {
       mbar_init(&full[s], 1);
-      mbar_init(&empty[s], kMxGuWarps);
+      mbar_init(&empty[s], kMxWarps);
     }
     fence_barrier_init();
   }
@@ -260,7 +255,7 @@ __global__ void __launch_bounds__(kMxThreads, 1)
   const int nk = (a.H + kMxKC - 1) / kMxKC;
   const StreamKRange rng = stream_k_range((long long)a.sched[0] * NT, nk);
 
-  if (warp == kMxGuWarps) {
+  if (warp == kMxWarps) {
     // ---------------- producer ----------------
     bool aborted = false;
     uint32_t it = 0;
@@ -317,10 +312,8 @@ __global__ void __launch_bounds__(kMxThreads, 1)
   }
 
   // ---------------- consumers ----------------
-  const int ctid = tid;                       // 0..639
-  const int mat = warp / kMxWarps;            // this warp's matrix: 0 gate, 1 up
-  const int wl = warp % kMxWarps;
-  const int box = wl >> 1, mt = wl & 1;       // ... and its m-tile mt of box `box`
+  const int ctid = tid;                       // 0..319
+  const int box = warp >> 1, mt = warp & 1;   // this warp: m-tile mt of box `box`
   const uint32_t ring_s = smem_u32(ring);
   bool aborted = false;
   uint32_t it = 0;
@@ -332,11 +325,13 @@ __global__ void __launch_bounds__(kMxThreads, 1)
     const int col0 = (unit % NT) * kMxTileCols;
     const int wg = min(kMxTileCols, a.I - col0);
     const int nrows = ch.z;
-    float acc[1][2][4];  // this warp's matrix: [nb][v]
+    float acc[2][2][4];  // [gate / up][nb][v]
 #pragma unroll
-    for (int nb = 0; nb < 2; ++nb)
+    for (int m = 0; m < 2; ++m)
 #pragma unroll
-      for (int v = 0; v < 4; ++v) acc[0][nb][v] = 0.f;
+      for (int nb = 0; nb < 2; ++nb)
+#pragma unroll
+        for (int v = 0; v < 4; ++v) acc[m][nb][v] = 0.f;
 
     for (int kst = kb0; kst < ke; ++kst, ++it) {
       const int slot = it % kMxGUStages;
@@ -347,14 +342,15 @@ __global__ void __launch_bounds__(kMxThreads, 1)
       }
       if (!aborted) {
         const uint32_t st = ring_s + slot * kMxGUStage;
-        const uint32_t boxes[1] = {st + (mat * kMxBoxes + box) * kMxBoxBytes};
-        const uint32_t scs[1] = {st + kMxGUW + (mat * kMxBoxes + box) * kMxScaleBytes};
+        const uint32_t boxes[2] = {st + box * kMxBoxBytes, st + (kMxBoxes + box) * kMxBoxBytes};
+        const uint32_t scs[2] = {st + kMxGUW + box * kMxScaleBytes,
+                                 st + kMxGUW + (kMxBoxes + box) * kMxScaleBytes};
         const uint32_t xb = st + kMxGUW + kMxGUS;
         const int nkb = mx_stage_blocks(a.H, kst * kMxKC);
         if (nrows <= 8)
-          mx_stage<1, 1>(boxes, scs, xb, mt, nkb, lane, acc);
+          mx_stage<1, 2>(boxes, scs, xb, mt, nkb, lane, acc);
         else
-          mx_stage<2, 1>(boxes, scs, xb, mt, nkb, lane, acc);
+          mx_stage<2, 2>(boxes, scs, xb, mt, nkb, lane, acc);
       }
       __syncwarp();
       if (lane == 0 && !aborted) mbar_arrive(&empty[slot]);
@@ -364,28 +360,18 @@ __global__ void __launch_bounds__(kMxThreads, 1)
 
     // ---- epilogue: as in stream_gate_up_kernel; value v of n-tile nb: column
     //      32*box + 16*mt + (lane>>2) + 8*(v>>1), row nb*8 + 2*(lane&3) + (v&1)
-    if (kb0 == 0 && ke == nk) {  // this CTA holds the whole K range: SwiGLU from registers,
-                                 // the up warps' sums handed over through shared memory
-      float* xw = xchg + wl * 8 * 32;
-      if (mat == 1) {
+    if (kb0 == 0 && ke == nk) {  // this CTA holds the whole K range: SwiGLU from registers
 #pragma unroll
-        for (int q = 0; q < 8; ++q) xw[q * 32 + lane] = acc[0][q >> 2][q & 3];
-      }
-      named_bar_sync(2, kMxConsumers);
-      if (mat == 0) {
+      for (int nb = 0; nb < 2; ++nb)
 #pragma unroll
-        for (int nb = 0; nb < 2; ++nb)
-#pragma unroll
-          for (int v = 0; v < 4; ++v) {
-            const int cl = kMxBoxRows * box + 16 * mt + (lane >> 2) + 8 * (v >> 1);
-            const int r = nb * 8 + 2 * (lane & 3) + (v & 1);
-            if (!aborted && r < nrows && cl < wg) {
-              const float hv = silu_f32(acc[0][nb][v]) * xw[(nb * 4 + v) * 32 + lane];
-              a.h[(size_t)(ch.y + r) * a.I + col0 + cl] = (uint16_t)pack_f16x2(hv, 0.f);
-            }
+        for (int v = 0; v < 4; ++v) {
+          const int cl = kMxBoxRows * box + 16 * mt + (lane >> 2) + 8 * (v >> 1);
+          const int r = nb * 8 + 2 * (lane & 3) + (v & 1);
+          if (!aborted && r < nrows && cl < wg) {
+            const float hv = silu_f32(acc[0][nb][v]) * acc[1][nb][v];
+            a.h[(size_t)(ch.y + r) * a.I + col0 + cl] = (uint16_t)pack_f16x2(hv, 0.f);
           }
-      }
-      named_bar_sync(2, kMxConsumers);  // read before the next hand-over overwrites it
+        }
       continue;
     }
 #pragma unroll
@@ -394,8 +380,11 @@ __global__ void __launch_bounds__(kMxThreads, 1)
       for (int v = 0; v < 4; ++v) {
         const int cl = kMxBoxRows * box + 16 * mt + (lane >> 2) + 8 * (v >> 1);
         const int r = nb * 8 + 2 * (lane & 3) + (v & 1);
-        if (!aborted && r < nrows && cl < wg)
-          atomicAdd(a.acc + ((size_t)ch.w + r) * I2 + mat * a.I + col0 + cl, acc[0][nb][v]);
+        if (!aborted && r < nrows && cl < wg) {
+          float* p = a.acc + ((size_t)ch.w + r) * I2 + col0 + cl;
+          atomicAdd(p, acc[0][nb][v]);
+          atomicAdd(p + a.I, acc[1][nb][v]);
+        }
       }
     // Completion count in K stages: the piece that brings it to nk applies SwiGLU.  The
     // barrier orders every thread's atomics before thread 0's release; thread 0's acquire
