@@ -207,13 +207,19 @@ void router_split(const moe_ctx* c, int T, int* splits, int* kc_per_split) {
 }
 
 // allow_split = false keeps the large-T router unsplit (the fixed-scratch routing entry point).
-RouteTmp carve_route_tmp(Carver& cv, const moe_ctx* c, int T, bool allow_split = true) {
+// fused: the streaming gate/up kernel finishes the routing (StreamRoute).  Its CTAs sum the
+// slices cheaply, so each router block takes only as many 64-row chunks as its ring holds (all
+// in flight at once: two for more than 64 experts, whose ring has two stages); the finalize
+// kernel sums them in one block, so without fusion the blocks take kSmallTChunks chunks.
+RouteTmp carve_route_tmp(Carver& cv, const moe_ctx* c, int T, bool allow_split = true,
+                         bool fused = false) {
   RouteTmp r;
   if (T <= kSmallT) {
-    // partial logits of each group of kSmallTChunks 64-row slices of W_router
+    // partial logits of each group of kc 64-row slices of W_router
     const int nk = c->H / kRouterHSlice;
-    r.kc_per_split = kSmallTChunks;
-    r.splits = (nk + kSmallTChunks - 1) / kSmallTChunks;
+    const int kc = fused && c->E > 64 ? RouterTcCfg<16>::kStages : kSmallTChunks;
+    r.kc_per_split = kc;
+    r.splits = (nk + kc - 1) / kc;
     r.partial = cv.take(sizeof(float) * (size_t)r.splits * T * c->E);
   } else {
     const size_t NB = (T + kRouterTcTokens - 1) / kRouterTcTokens;
@@ -248,6 +254,7 @@ struct Plan {
   bool snap = false;                      // the call's counts may move experts across a boundary
   bool one_tc = false;                    // expert tiles or row tiles, not both, in one call
   int tile_entry_rows = kEtRows;          // rows per expert-tile entry: 128 or 256 (bf16 only)
+  bool fused_route = false;               // the streaming gate/up kernel finishes the routing
   int chunk_rows(int f) const { return f == kFamTile ? tile_entry_rows : kFamChunkRows[f]; }
   int min_count(int f) const {
     int m = 0;
@@ -298,6 +305,9 @@ Plan make_plan(const moe_ctx* c, int T, bool mx, moe_path path) {
   const bool wide = c->tile_n == 256 ||
                     (c->tile_n == 0 && (long long)T * c->k >= (long long)kEtRows * c->E);
   if (p.has[kFamTile] && wide) p.tile_entry_rows = kEtWideRows;
+  // a few tokens on the streaming family alone: its gate/up kernel finishes the routing
+  p.fused_route = p.has[kFamStream] && !p.has[kFamTile] && !p.has[kFamGemm] &&
+                  T <= kFusedRouteT && (long long)T * c->k <= kFusedRouteRows && T <= kSmallT;
   return p;
 }
 
@@ -369,7 +379,7 @@ Layout make_layout(const moe_ctx* c, int T, const Plan& p, bool mx) {
   L.h = cv.take(2 * R * c->I);
   if (mx) L.x16 = cv.take(2 * (size_t)T * c->H);  // the layer input in f16
   if (p.has[kFamTile] || p.has[kFamGemm]) L.x_perm = cv.take(2 * R * c->H);
-  L.rt = carve_route_tmp(cv, c, T);
+  L.rt = carve_route_tmp(cv, c, T, true, p.fused_route);
   L.total = cv.cur;
   return L;
 }
@@ -928,8 +938,7 @@ moe_status forward_plan(moe_ctx* c, int T, const void* x_bf16, const void* W_rou
   // A few tokens on the streaming family alone: the gate/up kernel finishes the routing from
   // the partial logits (no finalize kernel in between); the router zero-fills the completion
   // counters and the split-K sums that follow them.
-  const bool fuse = !mx && p.has[kFamStream] && !p.has[kFamTile] && !p.has[kFamGemm] &&
-                    T <= kFusedRouteT && R <= (size_t)kFusedRouteRows && T <= kSmallT;
+  const bool fuse = p.fused_route;
   if (fuse) {
     io.sr.partial = reinterpret_cast<const float*>(ws + L.rt.partial);
     io.sr.S = L.rt.splits;
