@@ -58,25 +58,16 @@ static_assert(kEtSmem <= 227 * 1024, "shared memory");
 // 256 rows fill the 512 columns with one buffer (gate 256 | up 256) and take three stages of
 // 64 KB.  Per K step a 256-row tile reads the weight blocks once for twice the rows: the same
 // operand bytes per FLOP as the 2-SM row tiles, with rows padded to 16 instead of 256.
-//
-// The 256-row tiles keep the weights and the rows in separate rings: four stages of weight boxes
-// (128 KB in flight per SM, as many as the 128-row tiles keep) and two of rows, which come from
-// L2.  One stage ring for both would hold three stages, 96 KB of weights: too few bytes in flight
-// to keep the SM's share of HBM busy.  Producer lane 0 feeds the weight ring, lane 1 the row ring.
 template <int ROWS>
 struct EtCfg {
   static_assert(ROWS == 128 || ROWS == 256, "rows per tile");
-  static constexpr bool kSplit = ROWS == 256;     // separate weight and row rings
-  static constexpr int kStages = 4;               // (weight) ring stages
-  static constexpr int kBStages = kSplit ? 2 : kStages;
+  static constexpr int kStages = ROWS == 128 ? 4 : 3;
   static constexpr int kBBytes = ROWS * kEtBK * 2;
-  static constexpr int kStageBytes = kSplit ? kEtABytes : kEtABytes + kBBytes;
-  static constexpr int kRingBytes = kStages * kStageBytes + (kSplit ? kBStages * kBBytes : 0);
+  static constexpr int kStageBytes = kEtABytes + kBBytes;
   static constexpr int kAccBufs = kEtTmemCols / (2 * ROWS);
-  static constexpr int kSmem = 1024 + kRingBytes + 256 + kEtEpiBytes;
+  static constexpr int kSmem = 1024 + kStages * kStageBytes + 256 + kEtEpiBytes;
   static_assert(kSmem <= 227 * 1024, "shared memory");
-  static_assert(kStageBytes % 1024 == 0 && kBBytes % 1024 == 0, "128-byte swizzle atoms");
-  static_assert(kRingBytes <= 240 * 1024, "descriptor start addresses stay below 256 KB");
+  static_assert(kStageBytes % 1024 == 0, "128-byte swizzle atoms");
 };
 
 struct EtArgs {
@@ -196,21 +187,17 @@ __global__ void __launch_bounds__(kEtThreads, 1)
                        const __grid_constant__ CUtensorMap xmap) {
   using C = EtCfg<ROWS>;
   constexpr int kStages = C::kStages, kStageBytes = C::kStageBytes, kBufs = C::kAccBufs;
-  constexpr int kBStages = C::kBStages;
   extern __shared__ __align__(128) uint8_t smem_raw[];
   __shared__ uint32_t s_tmem;
   __shared__ int s_abort;
   uint8_t* ring = align1k(smem_raw);
-  uint8_t* bring = ring + kStages * kStageBytes;   // split rings: the rows' ring
-  uint64_t* bars = reinterpret_cast<uint64_t*>(ring + C::kRingBytes);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(ring + kStages * kStageBytes);
   uint64_t* full = bars;
   uint64_t* empty = full + kStages;
   uint64_t* acc_full = empty + kStages;
   uint64_t* acc_empty = acc_full + 2;
   uint64_t* drain = acc_empty + 2;
-  uint64_t* bfull = drain + 1;                     // split rings: the rows' barriers
-  uint64_t* bempty = bfull + kBStages;
-  float* epi = reinterpret_cast<float*>(ring + C::kRingBytes + 256);
+  float* epi = reinterpret_cast<float*>(ring + kStages * kStageBytes + 256);
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
 
   if (warp == 1) {
@@ -227,11 +214,6 @@ __global__ void __launch_bounds__(kEtThreads, 1)
       mbar_init(&acc_empty[b], 128);
     }
     mbar_init(drain, 1);
-    if constexpr (C::kSplit)
-      for (int s = 0; s < kBStages; ++s) {
-        mbar_init(&bfull[s], 1);
-        mbar_init(&bempty[s], 1);
-      }
     s_abort = 0;
     fence_barrier_init();
     tma_prefetch_desc(&wmap);
@@ -258,61 +240,7 @@ __global__ void __launch_bounds__(kEtThreads, 1)
 
   if (warp == 0) {
     // ------------------------------ TMA producer ------------------------------
-    if constexpr (C::kSplit) {
-      // lane 0: weight boxes into the weight ring; lane 1: row boxes into the row ring.  Each
-      // lane walks the same (tile, K stage) sequence with its own slots and phases.
-      if (lane < 2) {
-        const bool wl = lane == 0;
-        const int nst = wl ? kStages : kBStages;
-        uint32_t it = 0;
-        int last_it[kStages];
-#pragma unroll
-        for (int s = 0; s < kStages; ++s) last_it[s] = -1;
-        for (int t = blockIdx.x; t < tiles && !*abort_flag; t += gridDim.x) {
-          const int4 ch = a.chunks[t / NT];
-          const int n0 = (t % NT) * TW;
-          const int nb0 = et_boxes<MODE>(0, n0, a.Ncols), nb1 = et_boxes<MODE>(1, n0, a.Ncols);
-          const int c0 = n0, c1 = MODE == 0 ? a.Ncols + n0 : n0 + kEtM;
-          const int nrb = (ch.z + kEtRowBox - 1) / kEtRowBox;
-          const uint32_t bytes = wl ? (uint32_t)(nb0 + nb1) * kEtBoxBytes
-                                    : (uint32_t)nrb * kEtRowBox * kEtBK * 2;
-          const int wrow0 = ch.x * a.w_rows;
-          uint64_t* fb = wl ? full : bfull;
-          uint64_t* eb = wl ? empty : bempty;
-          bool ok = true;
-          for (int kst = 0; kst < nk; ++kst, ++it) {
-            const int slot = it % nst;
-            const uint32_t ph = (it / nst) & 1u;
-            if (!wait_or_abort(&eb[slot], ph ^ 1u, abort_flag, a.status)) {
-              ok = false;
-              break;
-            }
-            mbar_arrive_expect_tx(&fb[slot], bytes);
-            const int k0 = kst * kEtBK;
-            if (wl) {
-              uint8_t* st = ring + slot * kStageBytes;
-              for (int b = 0; b < nb0; ++b)
-                tma_load_2d(st + b * kEtBoxBytes, &wmap, c0 + 64 * b, wrow0 + k0, &fb[slot]);
-              for (int b = 0; b < nb1; ++b)
-                tma_load_2d(st + (2 + b) * kEtBoxBytes, &wmap, c1 + 64 * b, wrow0 + k0, &fb[slot]);
-            } else {
-              uint8_t* st = bring + slot * C::kBBytes;
-              for (int r = 0; r < nrb; ++r)
-                tma_load_2d(st + r * (kEtRowBox * kEtBK * 2), &xmap, k0, ch.y + r * kEtRowBox,
-                            &fb[slot]);
-            }
-            last_it[slot] = it;
-          }
-          if (!ok) break;
-        }
-        // never leave the CTA with copies in flight
-        uint64_t* fb = wl ? full : bfull;
-        for (int s = 0; s < nst; ++s)
-          if (last_it[s] >= 0 &&
-              !mbar_wait_bounded(&fb[s], (last_it[s] / nst) & 1u, kWaitLimitNs))
-            atomicOr(a.status, kStatusTimeout);
-      }
-    } else if (lane == 0) {
+    if (lane == 0) {
       uint32_t it = 0;
       int last_it[kStages];
 #pragma unroll
@@ -361,9 +289,7 @@ __global__ void __launch_bounds__(kEtThreads, 1)
       // slot 0's descriptors; a slot / K-step offset only moves the 14-bit start address
       // (addresses stay below 256 KB, so adding (offset >> 4) never carries out of the field)
       const uint64_t adesc0 = smem_desc_sw128(ring_s, kEtBoxBytes, 1024);          // MN-major
-      // K-major rows: after the weight boxes of a stage, or in their own ring
-      const uint64_t bdesc0 =
-          smem_desc_sw128(ring_s + (C::kSplit ? kStages * kStageBytes : kEtABytes), 16, 1024);
+      const uint64_t bdesc0 = smem_desc_sw128(ring_s + kEtABytes, 16, 1024);       // K-major
       uint32_t it = 0;
       int tile_i = 0;
       bool issued = false;
@@ -382,26 +308,21 @@ __global__ void __launch_bounds__(kEtThreads, 1)
         for (int kst = 0; kst < nk; ++kst, ++it) {
           const int slot = it % kStages;
           const uint32_t ph = (it / kStages) & 1u;
-          const int bslot = it % kBStages;
-          const uint32_t bph = (it / kBStages) & 1u;
-          if (!wait_or_abort(&full[slot], ph, abort_flag, a.status) ||
-              (C::kSplit && !wait_or_abort(&bfull[bslot], bph, abort_flag, a.status))) {
+          if (!wait_or_abort(&full[slot], ph, abort_flag, a.status)) {
             ok = false;
             break;
           }
           tc_fence_after();
           const uint64_t soff = (uint64_t)((slot * kStageBytes) >> 4);
-          const uint64_t boff = C::kSplit ? (uint64_t)((bslot * C::kBBytes) >> 4) : soff;
 #pragma unroll
           for (int k16 = 0; k16 < kEtBK / 16; ++k16) {
             const uint64_t ak = adesc0 + soff + ((k16 * 16 * 128) >> 4);
-            const uint64_t bk = bdesc0 + boff + ((k16 * 32) >> 4);
+            const uint64_t bk = bdesc0 + soff + ((k16 * 32) >> 4);
             const uint32_t acc = (kst | k16) != 0;
             if (nb0) tc_mma_bf16(d0, ak, bk, idesc, acc);
             if (nb1) tc_mma_bf16(d1, ak + ((2 * kEtBoxBytes) >> 4), bk, idesc, acc);
           }
           tc_commit(&empty[slot]);
-          if constexpr (C::kSplit) tc_commit(&bempty[bslot]);
           issued = true;
         }
         if (!ok) break;
