@@ -225,8 +225,8 @@ MOE_API moe_status moe_combine(moe_t ctx, int T, const int32_t* inv_perm, const 
 
 /* Choose the path.  crossover_T >= 0 also sets the largest call (in tokens) in which AUTO uses
  * the weight-streaming family (default: the largest T whose touched experts' tiles fill less
- * than two waves of the GPU or leave their last wave under 80 % full: 4 for the 20b and 120b
- * shapes on 148 SMs; moe_tune measures it);
+ * than two waves of the GPU or leave their last wave under 85 % full: 5 for the 20b and 4 for
+ * the 120b shape on 148 SMs; moe_tune measures it);
  * crossover_T < 0 keeps the current one.  MOE_ERR_ARG for an unknown path. */
 MOE_API moe_status moe_set_path(moe_t ctx, moe_path path, int crossover_T);
 

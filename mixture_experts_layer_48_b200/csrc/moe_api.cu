@@ -314,10 +314,10 @@ Plan make_plan(const moe_ctx* c, int T, bool mx, moe_path path) {
 
 // Largest T up to which AUTO streams by default: while the expert tiles of the experts T tokens
 // are expected to touch (E * (1 - (1 - k/E)^T), uniform routing) fill less than two waves of the
-// GPU's SMs, or fill their last wave to less than 80 %.  A tile wave that is mostly empty costs
-// as much as a full one, while the stream-K split balances any number of experts: measured on the
-// 20b and 120b layers (rotating token batches), streaming wins at 4 tokens (2.05 and 2.35 waves of
-// tiles) and the tiles from 5 (120b, 2.9 waves) or 8 tokens (20b).
+// GPU's SMs, or fill their last wave to less than 85 %.  A tile wave that is mostly empty costs
+// as much as a full one, while the stream-K split balances any number of experts.  Measured on the
+// 20b and 120b layers (rotating token batches): streaming wins at 4 tokens (2.05 and 2.35 waves of
+// tiles) and, on the 20b layer, at 5 (2.43 waves); the 120b tiles win from 5 tokens (2.9 waves).
 int default_stream_T(const moe_ctx* c) {
   const double tiles_per_expert = (double)((c->I + kEtM - 1) / kEtM);
   // a layer whose tiles cannot fill two waves even with every expert touched always streams
@@ -328,7 +328,7 @@ int default_stream_T(const moe_ctx* c) {
   while (T < kMaxT) {
     miss_T *= miss;
     const double waves = c->E * (1.0 - miss_T) * tiles_per_expert / c->num_sms;
-    if (!(waves < 2.0 || waves / std::ceil(waves) < 0.8)) break;
+    if (!(waves < 2.0 || waves / std::ceil(waves) < 0.85)) break;
     ++T;
     if (miss_T < 1e-6) break;  // the touched count no longer grows
   }
