@@ -194,7 +194,7 @@ KERNEL_NAMES = {  # the gate/up kernel of each family, as ncu lists it
     "gemm": "grouped_gemm_kernel<gate_up>"}
 
 
-MX_STREAM_T = 256   # MXFP4 layers stream in calls of at most this many tokens
+MX_STREAM_T = 176   # MXFP4 layers stream in calls of at most this many tokens
 
 
 def split_families(counts, path: str, T: int, stream_T: int, stream_rows: int, tile_rows: int,

@@ -164,7 +164,7 @@ MOE_API moe_status moe_forward(moe_t ctx, int T, const void* x_bf16, const void*
  * gu_codes [E, 2I, H/2] and gu_scales [E, H/32, 2I] hold W_gate_up [E, H, 2I] (gate columns
  * [0, I), up columns [I, 2I)); dn_codes [E, H, I/2] and dn_scales [E, I/32, H] hold W_down
  * [E, I, H].  x, W_router, b_router and out as in moe_forward; all pointers 16-byte aligned.
- * Two kernel families: MOE_PATH_AUTO streams the weights in calls of at most 256 tokens and
+ * Two kernel families: MOE_PATH_AUTO streams the weights in calls of at most 176 tokens and
  * runs the MXFP4 expert-tile kernel above; MOE_PATH_STREAM forces streaming, MOE_PATH_TILE and
  * MOE_PATH_GEMM expert tiles (there is no MXFP4 row-tile GEMM).
  *   - expert tiles: the codes are widened to bf16 weights in shared memory (exact: an E2M1 value

@@ -41,7 +41,9 @@ constexpr int kDefaultStreamRows = 16;
 // 256-row expert tiles beat the row tiles (20b layer 452 vs 461 us at 1024 tokens, 120b layer
 // 1711 vs 1976 us at 4096), at 256 rows the row tiles win (593 vs 632 us; 2565 vs 2707 us).
 constexpr int kDefaultTileRows = 192;
-constexpr int kMxStreamT = 256;  // MXFP4: streaming for calls of at most this many tokens
+// MXFP4: streaming for calls of at most this many tokens (20b layer, rotating token batches:
+// streaming 283 vs tiles 308 us at 160 tokens, a tie at 192, tiles 336 vs 390 us at 256)
+constexpr int kMxStreamT = 176;
 constexpr int kMaxKernelsPerCall = 12;
 
 moe_status static_scratch_address(void** out);  // defined beside the array, at the end
