@@ -561,16 +561,7 @@ def run_ours(args, w: mi.Workload, T: int) -> None:
     dn_ms = {f: prof["down_" + f][0] / n_prof for f in FAMILIES}
     layer_roof_s = max(alg["layer_bytes"] / (hbm * 1e9), alg["flops"] / (bf16 * 1e12))
     kernels_ms = {k_: round(v[0] / n_prof, 4) for k_, v in prof.items() if v[1]}
-    # a streaming call whose gate/up kernel finishes the routing runs both projections in one
-    # launch (profiled as gate/up): its roofline counts both projections' work
-    one_launch = gu_ms["stream"] > 0 and dn_ms["stream"] == 0 and not mx
-    if one_launch:
-        ws_ = work["stream"]
-        work["stream"] = dict(ws_, gate_up_bytes=ws_["gate_up_bytes"] + ws_["down_bytes"],
-                              gate_up_flops=ws_["gate_up_flops"] + ws_["down_flops"])
     roof = dominant_roofline(work, gu_ms, hbm, bf16, bf16_sus, peak_src)
-    if one_launch and roof["family"] == "stream":
-        roof["kernel"] = "stream_layer_kernel"
     if mx:
         roof["kernel"] = {"stream": "stream_gate_up_mx_kernel",
                           "tile": "expert_tile_mx_kernel<0>"}.get(roof["family"], roof["kernel"])

@@ -311,14 +311,6 @@ MOE_DEVINL void red_add_f32x4(float* p, float a, float b, float c, float d) {
 }
 
 // gpu-scope release / acquire-release atomics for cross-CTA completion counters.
-MOE_DEVINL int ld_acquire_gpu(const int* p) {
-  int v;
-  asm volatile("ld.acquire.gpu.global.b32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
-  return v;
-}
-MOE_DEVINL void mbar_inval(uint64_t* bar) {
-  asm volatile("mbarrier.inval.shared::cta.b64 [%0];" ::"r"(smem_u32(bar)) : "memory");
-}
 MOE_DEVINL int atom_add_acq_rel_gpu(int* p, int v) {
   int old;
   asm volatile("atom.acq_rel.gpu.global.add.s32 %0, [%1], %2;" : "=r"(old) : "l"(p), "r"(v) : "memory");

@@ -384,7 +384,7 @@ Layout make_layout(const moe_ctx* c, int T, const Plan& p, bool mx) {
     // one completion counter per (chunk, column tile); the MXFP4 kernels' tiles are narrower
     const int tile_cols = std::min(kStreamCols, kMxTileCols);
     L.n_done = n * ((c->I + tile_cols - 1) / tile_cols);
-    L.done = cv.take(4 * ((size_t)L.n_done + 1));  // + the one-launch layer's grid barrier
+    L.done = cv.take(4 * (size_t)L.n_done);
     // split-K sums of the streaming family's rows (each entry carries its rows' first index)
     const long long sb = family_row_bound(p, kFamStream);
     const long long srows = sb == LLONG_MAX ? (long long)R : std::min((long long)R, c->E * sb);
@@ -588,8 +588,6 @@ bool set_smem_attrs() {
                              kMxGateUpSmem) == cudaSuccess;
   ok &= cudaFuncSetAttribute(stream_down_mx_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              kMxDownSmem) == cudaSuccess;
-  ok &= cudaFuncSetAttribute(stream_layer_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             kLayerSmem) == cudaSuccess;
   ok &= cudaFuncSetAttribute(grouped_gemm_2sm_kernel<MOE_GEMM_GATE_UP>,
                              cudaFuncAttributeMaxDynamicSharedMemorySize,
                              Gemm2Cfg<kGemmStages>::kSmem) == cudaSuccess;
@@ -650,25 +648,9 @@ struct ExpertIO {
   const int32_t* sched[kFamilies];
   float* acc;                         // streaming family: split-K sums, zero on entry
   int32_t* done;                      // streaming family: completion counters, zero on entry
-  int* grid_bar = nullptr;            // with sr: the one-launch layer's barrier, zero on entry
   uint16_t* h;                        // [R, I] SwiGLU output
   StreamRoute sr{};                   // routing finished by the streaming gate/up kernel, if set
 };
-
-DownArgs stream_down_args(const moe_ctx* c, const ExpertIO& io) {
-  DownArgs da{};
-  da.h = io.h;
-  da.H = c->H;
-  da.I = c->I;
-  da.R = io.R;
-  da.perm = io.perm;
-  da.row_w = io.row_w;
-  da.chunks = io.chunks[kFamStream];
-  da.sched = io.sched[kFamStream];
-  da.out = io.out;
-  da.status = c->d_status;
-  return da;
-}
 
 moe_status expert_phase(moe_ctx* c, const Plan& p, const ExpertIO& io, const void* W_gate_up_bf16,
                         const void* W_down_bf16, const MxWeights* mx, cudaStream_t st) {
@@ -696,10 +678,6 @@ moe_status expert_phase(moe_ctx* c, const Plan& p, const ExpertIO& io, const voi
         cudaStreamWaitEvent(c->aux, c->ev_fork, 0) != cudaSuccess)
       return MOE_ERR_CUDA;
   }
-
-  // a call whose gate/up kernel finishes the routing runs its whole expert half in one launch
-  const bool layer_fused = !mx && io.sr.partial != nullptr && io.grid_bar != nullptr &&
-                           p.has[kFamStream] && !p.has[kFamTile] && !p.has[kFamGemm];
 
   // ---------------------------- gate/up projection + SwiGLU ----------------------------
   if (p.has[kFamStream]) {
@@ -734,21 +712,10 @@ moe_status expert_phase(moe_ctx* c, const Plan& p, const ExpertIO& io, const voi
                                         (uint64_t)c->E * c->H, 2ull * c->I, kGateUpKC, kBox,
                                         /*promote_256=*/false);
       if (!m) return MOE_ERR_CUDA;
-      if (layer_fused) {  // gate/up, grid barrier and down in one launch
-        const CUtensorMap* dm = cached_map(c->down_stream, W_down_bf16, (uint64_t)c->E * c->I,
-                                           (uint64_t)c->H, kDownKC, kBox, /*promote_256=*/false);
-        if (!dm) return MOE_ERR_CUDA;
-        const DownArgs da = stream_down_args(c, io);
-        MOE_TRY(launch(c, kKindGateUp, st, [&] {
-          return launch_pdl(stream_layer_kernel, dim3(c->num_sms), dim3(kStreamThreads),
-                            kLayerSmem, st, ga, io.sr, da, io.grid_bar, *m, *dm);
-        }));
-      } else {
-        MOE_TRY(launch(c, kKindGateUp, st, [&] {
-          return launch_pdl(stream_gate_up_kernel, dim3(c->num_sms), dim3(kStreamThreads),
-                            kGateUpSmem, st, ga, io.sr, *m);
-        }));
-      }
+      MOE_TRY(launch(c, kKindGateUp, st, [&] {
+        return launch_pdl(stream_gate_up_kernel, dim3(c->num_sms), dim3(kStreamThreads),
+                          kGateUpSmem, st, ga, io.sr, *m);
+      }));
     }
   }
   const CUtensorMap* wgu = nullptr;
@@ -823,8 +790,18 @@ moe_status expert_phase(moe_ctx* c, const Plan& p, const ExpertIO& io, const voi
   }
 
   // ---------------------------- down projection + weighted combine ----------------------------
-  if (p.has[kFamStream] && !layer_fused) {
-    const DownArgs da = stream_down_args(c, io);
+  if (p.has[kFamStream]) {
+    DownArgs da{};
+    da.h = io.h;
+    da.H = c->H;
+    da.I = c->I;
+    da.R = io.R;
+    da.perm = io.perm;
+    da.row_w = io.row_w;
+    da.chunks = io.chunks[kFamStream];
+    da.sched = io.sched[kFamStream];
+    da.out = io.out;
+    da.status = c->d_status;
     if (mx) {
       const CUtensorMap* cm = cached_map_u8(c->dn_codes, mx->dn_codes, (uint64_t)c->H * c->E,
                                             (uint64_t)c->I / 2, kMxBoxRows, kMxKC / 2,
@@ -985,7 +962,6 @@ moe_status forward_plan(moe_ctx* c, int T, const void* x_bf16, const void* W_rou
     io.sr.E = c->E;
     io.sr.k = c->k;
     io.sr.o = o;
-    io.grid_bar = reinterpret_cast<int*>(ws + L.done) + L.n_done;
     MOE_TRY(launch_route(c, T, x, static_cast<const uint16_t*>(W_router_bf16), b_router, o, ws,
                          L.rt, st, reinterpret_cast<float*>(ws + L.done),
                          (L.acc - L.done) / 4 + L.acc_floats, /*finalize=*/false));

@@ -267,35 +267,17 @@ MOE_DEVINL void fused_route_cta(const StreamRoute& r, uint8_t* scratch, FusedRou
   __syncthreads();
 }
 
-// Shared-memory layout of the gate/up phase (also its mbarriers' addresses).
-struct GateUpSmem {
-  uint8_t* wring;
-  uint8_t* xring;
-  uint64_t* full;
-  uint64_t* empty;
-  FusedRouteSmem* fs;
-  MOE_DEVINL explicit GateUpSmem(uint8_t* smem_raw) {
-    wring = align1k(smem_raw);
-    xring = wring + kStreamStages * kGUStageW;
-    full = reinterpret_cast<uint64_t*>(xring + kStreamStages * kGUStageX);
-    empty = full + kStreamStages;
-    fs = reinterpret_cast<FusedRouteSmem*>(empty + kStreamStages);
-  }
-};
-
-// The gate/up kernel's work, by every thread of a block of kStreamThreads (the producer warp
-// returns early).  The weight tensor map views W_gate_up as [E*H rows, 2I columns], box
-// [32 x 64], 128B swizzle.
-MOE_DEVINL void stream_gate_up_body(const GateUpArgs& a, const StreamRoute& r,
-                                    const CUtensorMap* wmapp, uint8_t* smem_raw) {
-  const CUtensorMap& wmap = *wmapp;
+// The weight tensor map views W_gate_up as [E*H rows, 2I columns], box [32 x 64], 128B swizzle.
+__global__ void __launch_bounds__(kStreamThreads, 1)
+    stream_gate_up_kernel(const GateUpArgs a, const StreamRoute r,
+                          const __grid_constant__ CUtensorMap wmap) {
+  extern __shared__ __align__(128) uint8_t smem_raw[];
   __shared__ int s_last;
-  const GateUpSmem sm(smem_raw);
-  uint8_t* wring = sm.wring;
-  uint8_t* xring = sm.xring;
-  uint64_t* full = sm.full;
-  uint64_t* empty = sm.empty;
-  FusedRouteSmem* fs = sm.fs;
+  uint8_t* wring = align1k(smem_raw);
+  uint8_t* xring = wring + kStreamStages * kGUStageW;
+  uint64_t* full = reinterpret_cast<uint64_t*>(xring + kStreamStages * kGUStageX);
+  uint64_t* empty = full + kStreamStages;
+  FusedRouteSmem* fs = reinterpret_cast<FusedRouteSmem*>(empty + kStreamStages);
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   if (tid == 0) {
     for (int s = 0; s < kStreamStages; ++s) {
@@ -476,13 +458,6 @@ MOE_DEVINL void stream_gate_up_body(const GateUpArgs& a, const StreamRoute& r,
   }
 }
 
-__global__ void __launch_bounds__(kStreamThreads, 1)
-    stream_gate_up_kernel(const GateUpArgs a, const StreamRoute r,
-                          const __grid_constant__ CUtensorMap wmap) {
-  extern __shared__ __align__(128) uint8_t smem_raw[];
-  stream_gate_up_body(a, r, &wmap, smem_raw);
-}
-
 // ------------------------------------------------------------------------------------------
 // down projection + routing weight + combine
 // ------------------------------------------------------------------------------------------
@@ -510,11 +485,10 @@ MOE_DEVINL void down_stage_mma(uint32_t wbase, uint32_t xbase, int warp_c, int l
   }
 }
 
-// The down kernel's work, by every thread of a block of kStreamThreads (the producer warp
-// returns early).  The weight tensor map views W_down as [E*I rows, H columns], box [64 x 64],
-// 128B swizzle.
-MOE_DEVINL void stream_down_body(const DownArgs& a, const CUtensorMap* wmapp, uint8_t* smem_raw) {
-  const CUtensorMap& wmap = *wmapp;
+// The weight tensor map views W_down as [E*I rows, H columns], box [64 x 64], 128B swizzle.
+__global__ void __launch_bounds__(kStreamThreads, 1)
+    stream_down_kernel(const DownArgs a, const __grid_constant__ CUtensorMap wmap) {
+  extern __shared__ __align__(128) uint8_t smem_raw[];
   uint8_t* wring = align1k(smem_raw);
   uint8_t* xring = wring + kStreamStages * kDNStageW;
   uint64_t* full = reinterpret_cast<uint64_t*>(xring + kStreamStages * kDNStageX);
@@ -639,54 +613,6 @@ MOE_DEVINL void stream_down_body(const DownArgs& a, const CUtensorMap* wmapp, ui
             atomicAdd(a.out + (size_t)t * a.H + col0 + cl, wt[nb][v & 1] * acc[mt][nb][v]);
         }
   }
-}
-
-__global__ void __launch_bounds__(kStreamThreads, 1)
-    stream_down_kernel(const DownArgs a, const __grid_constant__ CUtensorMap wmap) {
-  extern __shared__ __align__(128) uint8_t smem_raw[];
-  stream_down_body(a, &wmap, smem_raw);
-}
-
-// A call of a few tokens on the streaming family whose gate/up phase finishes the routing
-// (StreamRoute): gate/up, a grid-wide barrier, then down, in one launch, so that the second
-// kernel's launch, CTA placement and pipeline fill leave the critical path.  One CTA per SM
-// (each takes most of its SM's shared memory; nothing else of the call runs meanwhile), so every
-// CTA is resident when the barrier is reached.  grid_bar: a counter zeroed by the router kernel;
-// the wait is bounded, and on a timeout the down phase is skipped and the status word says so.
-constexpr int kLayerSmem = kGateUpSmem > kDownSmem ? kGateUpSmem : kDownSmem;
-
-__global__ void __launch_bounds__(kStreamThreads, 1)
-    stream_layer_kernel(const GateUpArgs ga, const StreamRoute r, const DownArgs da,
-                        int* grid_bar, const __grid_constant__ CUtensorMap gmap,
-                        const __grid_constant__ CUtensorMap dmap) {
-  extern __shared__ __align__(128) uint8_t smem_raw[];
-  __shared__ int s_go;
-  stream_gate_up_body(ga, r, &gmap, smem_raw);
-  // every thread's h, routing results and zero-filled output are visible GPU-wide before its
-  // CTA arrives; the down phase reuses this shared memory, so the gate/up mbarriers (quiet: the
-  // producer drained its copies) are invalidated first
-  __threadfence();
-  __syncthreads();
-  if (threadIdx.x == 0) {
-    const GateUpSmem sm(smem_raw);
-    for (int s = 0; s < kStreamStages; ++s) {
-      mbar_inval(&sm.full[s]);
-      mbar_inval(&sm.empty[s]);
-    }
-    atomicAdd(grid_bar, 1);
-    bool ok = true;
-    const uint64_t t0 = globaltimer_ns();
-    while (ld_acquire_gpu(grid_bar) < (int)gridDim.x) {
-      if (globaltimer_ns() - t0 > kWaitLimitNs) {
-        ok = false;
-        record_timeout(ga.status);
-        break;
-      }
-    }
-    s_go = ok;
-  }
-  __syncthreads();
-  if (s_go) stream_down_body(da, &dmap, smem_raw);
 }
 
 }  // namespace moe

@@ -153,23 +153,6 @@ def test_profile_counts_kernels():
     assert all(v[0] >= 0 for v in prof.values())
 
 
-def test_few_tokens_run_the_expert_half_in_one_launch():
-    """At 4 tokens on the streaming kernels the routing finishes in the gate/up phase and gate/up,
-    a grid barrier and down run as one kernel: per call the router and that kernel only (the
-    profile files it under gate/up), and the result matches the oracle."""
-    d, h = inputs_on_gpu(4, 256, 8, 2, 256, seed=902)
-    layer = moe.Moe(8, 256, 256, 2)
-    layer.set_path(moe.MOE_PATH_STREAM)
-    layer.profile_begin(3)
-    for _ in range(3):
-        layer.forward(d["x"], d["W_router"], d["b_router"], d["W_gate_up"], d["W_down"])
-    prof = layer.profile_end()
-    assert layer.sync_status() == moe.MOE_OK
-    assert prof["router"][1] == 3 and prof["gate_up_stream"][1] == 3
-    assert prof["route_finalize"][1] == 0 and prof["down_stream"][1] == 0
-    _check_layer(d, h, 8, 256, 256, 2, layer=layer)
-
-
 @pytest.mark.parametrize("T", [1, 5, 16, 64, 65, 200, 520])
 @pytest.mark.parametrize("path", ["stream", "gemm", "tile"])
 def test_every_path_matches_the_oracle(T, path):
