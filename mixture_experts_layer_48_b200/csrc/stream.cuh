@@ -187,20 +187,8 @@ MOE_DEVINL void fused_route_cta(const StreamRoute& r, uint8_t* scratch, FusedRou
   int32_t* cnt = sel + T * k;                              // [256]
   int32_t* off = cnt + 256;                                // [257]
   int32_t* first = off + 257;                              // [256] list entry of each expert
-  for (int i = tid; i < T * E; i += blockDim.x) {
-    const int e = i % E;
-    float v = 0.f;  // slices added in order, as the finalize kernel does
-    int s = 0;
-    for (; s + 8 <= S; s += 8) {
-      float p[8];
-#pragma unroll
-      for (int q = 0; q < 8; ++q) p[q] = __ldcg(r.partial + (size_t)(s + q) * T * E + i);
-#pragma unroll
-      for (int q = 0; q < 8; ++q) v += p[q];
-    }
-    for (; s < S; ++s) v += __ldcg(r.partial + (size_t)s * T * E + i);
-    lg[i] = v + r.b_router[e];
-  }
+  for (int i = tid; i < T * E; i += blockDim.x)  // slices in order, as the finalize kernel
+    lg[i] = sum_slices(r.partial + i, (size_t)T * E, S) + r.b_router[i % E];
   for (int i = tid; i < 256; i += blockDim.x) cnt[i] = 0;
   __syncthreads();
   for (int t = warp; t < T; t += nwarps) {
