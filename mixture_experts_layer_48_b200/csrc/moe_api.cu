@@ -486,6 +486,15 @@ cudaError_t launch_router_tc(int NB, cudaStream_t st, const uint16_t* x, const u
                     block_counts, zero4, n_zero4, rt.kc_per_split, partial);
 }
 
+template <int NT8>
+cudaError_t launch_router_small(cudaStream_t st, const uint16_t* x, const uint16_t* Wr, int T,
+                                int H, int E, float4* zero4, size_t n_zero4, const RouteTmp& rt,
+                                float* partial) {
+  return launch_pdl(router_partial_small_kernel<NT8>, dim3(1, rt.splits), dim3(128),
+                    (size_t)RouterSmallCfg<NT8>::kSmem, st, x, Wr, T, H, E, zero4, n_zero4,
+                    rt.kc_per_split, partial);
+}
+
 // Routing chain.  zero4/n_zero4: a float scratch region the router kernel zero-fills.
 // finalize = false (T <= kSmallT only): stop after the partial logits; the streaming gate/up
 // kernel finishes the routing (StreamRoute).
@@ -502,6 +511,14 @@ moe_status launch_route(moe_ctx* c, int T, const uint16_t* x, const uint16_t* Wr
     // tensor cores, then one block finishes the routing
     float* partial = reinterpret_cast<float*>(ws + rt.partial);
     MOE_TRY(launch(c, kKindRouter, st, [&] {
+      if (T <= kRouterSmallT) {  // small enough to run beside the previous call's down kernel
+        if (nt8 <= 1) return launch_router_small<1>(st, x, Wr, T, H, E, zero4, n_zero4, rt, partial);
+        if (nt8 <= 2) return launch_router_small<2>(st, x, Wr, T, H, E, zero4, n_zero4, rt, partial);
+        if (nt8 <= 4) return launch_router_small<4>(st, x, Wr, T, H, E, zero4, n_zero4, rt, partial);
+        if (nt8 <= 8) return launch_router_small<8>(st, x, Wr, T, H, E, zero4, n_zero4, rt, partial);
+        if (nt8 <= 16) return launch_router_small<16>(st, x, Wr, T, H, E, zero4, n_zero4, rt, partial);
+        return launch_router_small<32>(st, x, Wr, T, H, E, zero4, n_zero4, rt, partial);
+      }
       if (nt8 <= 1) return launch_router_tc<1>(1, st, x, Wr, b, T, H, E, k, o, nullptr, zero4, n_zero4, rt, partial);
       if (nt8 <= 2) return launch_router_tc<2>(1, st, x, Wr, b, T, H, E, k, o, nullptr, zero4, n_zero4, rt, partial);
       if (nt8 <= 4) return launch_router_tc<4>(1, st, x, Wr, b, T, H, E, k, o, nullptr, zero4, n_zero4, rt, partial);

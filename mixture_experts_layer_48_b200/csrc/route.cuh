@@ -620,6 +620,122 @@ __global__ void __launch_bounds__(128)
   topk_block_epilogue(lg, EP + 1, nt, t0, E, k, sel, cnt, topk_idx, topk_w, block_counts);
 }
 
+// Partial logits of a call of at most 16 tokens (grid (1, slices), one hidden-dimension slice
+// per block) in little shared memory: one 16-token tile that all four warps share, the experts
+// split over the warps (n-tile n on warp n % 4), and pipeline stages of one 16-deep K step (four
+// stages, 12 KB, up to 64 experts; two, 10 KB, at 128).  A block this small fits on an SM beside
+// a CTA of the streaming
+// or expert-tile kernels, so its loads and products run while the previous call's down kernel
+// still holds the SMs, instead of after it.  Every (token, expert) sum takes the same MMAs, on the
+// same operands and in the same K order, as in router_topk_kernel, so the partial logits are
+// the same numbers.
+constexpr int kRouterSmallT = 16;
+constexpr int kRouterSmallXPitch = 24;  // elements; 48-byte rows keep ldmatrix conflict-free
+template <int NT8>
+struct RouterSmallCfg {
+  static constexpr int kStages = NT8 <= 8 ? 4 : 2;
+  static constexpr int EP = NT8 * 8;
+  static constexpr int WP = EP + 8;
+  static constexpr int kXStage = kRouterSmallT * kRouterSmallXPitch;  // elements
+  static constexpr int kWStage = 16 * WP;                              // elements
+  static constexpr int kSmem = kStages * (kXStage + kWStage) * 2;
+};
+
+template <int NT8>
+__global__ void __launch_bounds__(128)
+    router_partial_small_kernel(const uint16_t* __restrict__ x, const uint16_t* __restrict__ Wr,
+                                int T, int H, int E, float4* zero4, size_t n_zero4,
+                                int kc_per_split, float* __restrict__ partial) {
+  using C = RouterSmallCfg<NT8>;
+  constexpr int WP = C::WP, XP = kRouterSmallXPitch;
+  constexpr int NW = (NT8 + 3) / 4;  // n-tiles per warp
+  extern __shared__ __align__(128) uint8_t smem_raw[];
+  uint16_t* xs = reinterpret_cast<uint16_t*>(smem_raw);  // [stages][16][XP]
+  uint16_t* wsm = xs + C::kStages * C::kXStage;           // [stages][16][WP]
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  // this block's slice of the hidden dimension: K steps of 16 rows from h_first
+  const int kc0 = blockIdx.y * kc_per_split;
+  const int nsteps = min(H / kRouterHSlice - kc0, kc_per_split) * (kRouterHSlice / 16);
+  const int h_first = kc0 * kRouterHSlice;
+  const bool vec_w = (E % 8) == 0;
+
+  // x and W_router are the caller's inputs, which no kernel of this library writes: the loads
+  // and the products run before the dependency wait, everything this kernel writes after it
+  for (int i = tid; i < C::kStages * C::kWStage; i += blockDim.x) wsm[i] = 0;  // padding experts
+  __syncthreads();
+
+  auto load_step = [&](int s, int buf) {
+    const int h0 = h_first + 16 * s;
+    uint16_t* xb = xs + buf * C::kXStage;
+    if (tid < 2 * kRouterSmallT) {  // 16 rows x 2 pieces of 16 B; rows past T are zero-filled
+      const int r = tid >> 1, c = tid & 1;
+      const bool ok = r < T;
+      cp_async16(xb + r * XP + c * 8, x + (size_t)(ok ? r : 0) * H + h0 + c * 8, ok);
+    }
+    uint16_t* wb = wsm + buf * C::kWStage;
+    if (vec_w) {
+      const int per_row = E / 8;
+      for (int i = tid; i < 16 * per_row; i += blockDim.x) {
+        const int r = i / per_row, c = i - r * per_row;
+        cp_async16(wb + r * WP + c * 8, Wr + (size_t)(h0 + r) * E + c * 8, true);
+      }
+    } else {
+      for (int i = tid; i < 16 * E; i += blockDim.x) {
+        const int r = i / E, c = i - r * E;
+        wb[r * WP + c] = Wr[(size_t)(h0 + r) * E + c];
+      }
+    }
+  };
+
+  float acc[NW][4];
+#pragma unroll
+  for (int j = 0; j < NW; ++j) acc[j][0] = acc[j][1] = acc[j][2] = acc[j][3] = 0.f;
+  // prologue: stages-1 steps in flight; every iteration commits one group (maybe empty)
+#pragma unroll
+  for (int p = 0; p < C::kStages - 1; ++p) {
+    if (p < nsteps) load_step(p, p);
+    cp_async_commit();
+  }
+  for (int s = 0; s < nsteps; ++s) {
+    const int buf = s % C::kStages;
+    cp_async_wait<C::kStages - 2>();  // step s has landed
+    __syncthreads();                   // ... for every thread; buffer s-1 is free again
+    {
+      const int nx = s + C::kStages - 1;
+      if (nx < nsteps) load_step(nx, nx % C::kStages);
+      cp_async_commit();
+    }
+    const uint32_t xb = smem_u32(xs + buf * C::kXStage);
+    const uint32_t wb = smem_u32(wsm + buf * C::kWStage);
+    const int i = lane >> 3, j8 = lane & 7;
+    uint32_t a0, a1, a2, a3;
+    ldsm_x4(xb + (((i & 1) * 8 + j8) * XP + (i >> 1) * 8) * 2, a0, a1, a2, a3);
+#pragma unroll
+    for (int j = 0; j < NW; ++j) {
+      const int n = warp + 4 * j;
+      if (n < NT8) {  // matrices 0/1: experts [8n, 8n+8) at k 0-7 / 8-15
+        uint32_t b0, b1;
+        ldsm_x2_trans(wb + (((i & 1) * 8 + j8) * WP + 8 * n) * 2, b0, b1);
+        mma_bf16_16816(acc[j], a0, a1, a2, a3, b0, b1);
+      }
+    }
+  }
+  cp_async_wait<0>();
+  pdl_wait();
+  pdl_launch_next();
+  zero_fill_f4(zero4, n_zero4);
+  // C fragment: c0,c1 -> token lane/4, experts 8n + 2(lane%4) + {0,1}; c2,c3 -> token + 8
+#pragma unroll
+  for (int j = 0; j < NW; ++j)
+#pragma unroll
+    for (int v = 0; v < 4; ++v) {
+      const int n = warp + 4 * j;
+      const int tt = (lane >> 2) + 8 * (v >> 1);
+      const int e = 8 * n + 2 * (lane & 3) + (v & 1);
+      if (n < NT8 && e < E && tt < T) partial[((size_t)blockIdx.y * T + tt) * E + e] = acc[j][v];
+    }
+}
+
 // Sum of the S partial-logit slices of every (token, expert), in slice order, written in place
 // into slice 0 (each thread owns one element).  grid ceil(n/256), block 256.
 __global__ void __launch_bounds__(256) sum_partials_kernel(float* __restrict__ partial, int S,
