@@ -7,9 +7,11 @@
 //
 // Two chains:
 //   T <= kSmallT : router_topk_kernel split over the hidden dimension (one block per
-//                  kSmallTChunks 64-row slices of W_router, partial logits on the tensor cores)
-//                  -> route_small_finalize_kernel (one block: sum of the slices, top-k,
-//                     softmax, histogram, scan, permutation, work lists).
+//                  kSmallTChunks 64-row slices of W_router, partial logits on the tensor cores;
+//                  router_partial_small_kernel, the same products in less shared memory, for
+//                  T <= 16) -> route_small_finalize_kernel (one block: sum of the slices, top-k,
+//                  softmax, histogram, scan, permutation, work lists), or the streaming gate/up
+//                  kernel itself for a few tokens.
 //   T >  kSmallT : router_topk_kernel (64 tokens per block, all experts on the tensor cores;
 //                  top-k and a block histogram) -> route_scan_kernel (one block per expert:
 //                  prefix over blocks) -> route_scatter_kernel (permutation, 64 tokens per
@@ -623,12 +625,11 @@ __global__ void __launch_bounds__(128)
 // Partial logits of a call of at most 16 tokens (grid (1, slices), one hidden-dimension slice
 // per block) in little shared memory: one 16-token tile that all four warps share, the experts
 // split over the warps (n-tile n on warp n % 4), and pipeline stages of one 16-deep K step (four
-// stages, 12 KB, up to 64 experts; two, 10 KB, at 128).  A block this small fits on an SM beside
-// a CTA of the streaming
-// or expert-tile kernels, so its loads and products run while the previous call's down kernel
-// still holds the SMs, instead of after it.  Every (token, expert) sum takes the same MMAs, on the
-// same operands and in the same K order, as in router_topk_kernel, so the partial logits are
-// the same numbers.
+// stages, at most 12 KB, up to 64 experts; two, 10 KB, at 128; 18 KB at 256).  Up to 128
+// experts a block fits on an SM beside a CTA of the streaming or expert-tile kernels, so its
+// loads and products run while the previous call's down kernel still holds the SMs, instead of
+// after it.  Every (token, expert) sum takes the same MMAs, on the same operands and in the same
+// K order, as in router_topk_kernel, so the partial logits are the same numbers.
 constexpr int kRouterSmallT = 16;
 constexpr int kRouterSmallXPitch = 24;  // elements; 48-byte rows keep ldmatrix conflict-free
 template <int NT8>
